@@ -1,0 +1,157 @@
+"""MLA paged-decode oracle (fp64, CPU).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+bench's CPU-baseline leg may import this package; the product path
+(``mla_paged_decode_04_b200``) never does, and shares no code with it.
+
+``mla_decode`` wraps the C implementation in ``mla_oracle.c`` (plain
+definition, fp64, OpenMP over rows). ``brute.py`` holds an independent
+pure-Python restatement used to pin the C code on tiny inputs.
+
+Every function states the passage it follows; the definition is the one in
+``mla_oracle.c``'s header (tokenspeed-mla package card, "What it is and what
+it does"; TokenSpeed MLA article 最快MLA内核背后的秘密, sections 一, 二, 四, 六).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mla_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle_mla.so")
+_lock = threading.Lock()
+_lib = None
+
+DTYPE_CODES = {"bf16": 0, "fp16": 1, "fp8": 2}
+
+# Planted mistakes for the pin-sensitivity tests (see mla_oracle.c).
+MUTATIONS = {
+    "none": 0,
+    "drop_rope": 1,
+    "v_offset": 2,
+    "no_causal": 3,
+    "no_scale": 4,
+    "lse_log2": 5,
+    "page_index": 6,
+    "wrong_sign": 7,
+}
+
+
+def build(force: bool = False) -> str:
+    """Compile mla_oracle.c into liboracle_mla.so (gcc -O3 -fopenmp, no fast-math)."""
+    with _lock:
+        stale = (not os.path.exists(_LIB)) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC)
+        if force or stale:
+            tmp = _LIB + f".tmp{os.getpid()}"
+            cmd = ["gcc", "-O3", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                   "-o", tmp, _SRC, "-lm"]
+            subprocess.run(cmd, check=True)
+            os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        i32, i64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_double
+        vp = ctypes.c_void_p
+        lib.oracle_mla_decode_range.argtypes = [
+            i32, i32, i32, i32, i32, i32, vp, vp, i64, i32, vp, i32, vp,
+            f64, f64, f64, i64, vp, i64, i64, i32, vp, vp]
+        lib.oracle_mla_decode_range.restype = i32
+        lib.oracle_lse_merge.argtypes = [i32, i32, vp, vp, vp, vp]
+        lib.oracle_lse_merge.restype = None
+        lib.oracle_decode_buffer.argtypes = [i32, vp, ctypes.c_size_t, vp]
+        lib.oracle_decode_buffer.restype = None
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_num_threads.restype = i32
+        _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def _raw_bytes(t) -> np.ndarray:
+    """Raw element bytes of a CPU tensor / ndarray as a contiguous uint8 array."""
+    try:
+        import torch
+        if isinstance(t, torch.Tensor):
+            t = t.detach().contiguous().cpu()
+            return t.view(torch.uint8).numpy().reshape(-1)
+    except ImportError:  # pragma: no cover
+        pass
+    a = np.ascontiguousarray(t)
+    return a.view(np.uint8).reshape(-1)
+
+
+def decode_values(dtype: str, raw) -> np.ndarray:
+    """Decode raw element bytes (bf16 / fp16 / E4M3FN) to float64 with the oracle's own decoder."""
+    b = _raw_bytes(raw)
+    esize = 1 if dtype == "fp8" else 2
+    n = b.size // esize
+    out = np.empty(n, dtype=np.float64)
+    _load().oracle_decode_buffer(DTYPE_CODES[dtype], b.ctypes.data, n, out.ctypes.data)
+    return out
+
+
+def mla_decode(q, kv_cache, block_tables, seq_lens, softmax_scale, *, dtype,
+               q_scale=1.0, kv_scale=1.0, rows=None, key_range=None,
+               mutation="none"):
+    """Oracle MLA decode.
+
+    q: [B, q_len, H, D] and kv_cache: [num_pages, page_size, D] CPU tensors (bf16 /
+    fp16 / float8_e4m3fn, or their raw uint8/uint16 views); block_tables [B, P]
+    int32, seq_lens [B] int32. rows: optional flat row indices (b*q_len+t)*H+h.
+    key_range: optional (lo, hi) restriction of the keys (hi=-1: unbounded).
+    Returns (out [n_rows, Dv=512] float64, lse [n_rows] float64), natural log.
+    """
+    lib = _load()
+    B, T, H, D = (int(x) for x in q.shape)
+    num_pages, page_size, D2 = (int(x) for x in kv_cache.shape)
+    assert D2 == D
+    Dv = 512
+    bt = np.ascontiguousarray(np.asarray(block_tables, dtype=np.int32))
+    sl = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+    assert bt.ndim == 2 and bt.shape[0] == B and sl.shape == (B,)
+    qb = _raw_bytes(q)
+    cb = _raw_bytes(kv_cache)
+    if rows is None:
+        n_rows = B * T * H
+        rows_ptr = None
+        rows_arr = None
+    else:
+        rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1))
+        n_rows = rows_arr.size
+        rows_ptr = rows_arr.ctypes.data
+    out = np.zeros((n_rows, Dv), dtype=np.float64)
+    lse = np.zeros((n_rows,), dtype=np.float64)
+    lo, hi = (0, -1) if key_range is None else key_range
+    rc = lib.oracle_mla_decode_range(
+        DTYPE_CODES[dtype], B, T, H, D, Dv, qb.ctypes.data, cb.ctypes.data, num_pages,
+        page_size, bt.ctypes.data, bt.shape[1], sl.ctypes.data, float(softmax_scale),
+        float(q_scale), float(kv_scale), n_rows, rows_ptr, int(lo), int(hi),
+        MUTATIONS[mutation], out.ctypes.data, lse.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle_mla_decode_range failed with code {rc}")
+    return out, lse
+
+
+def lse_merge(o_parts, lse_parts):
+    """Merge per-split partials of one row: returns (out [Dv], lse)."""
+    o = np.ascontiguousarray(np.asarray(o_parts, dtype=np.float64))
+    l = np.ascontiguousarray(np.asarray(lse_parts, dtype=np.float64))
+    n, Dv = o.shape
+    out = np.zeros(Dv, dtype=np.float64)
+    lse = np.zeros(1, dtype=np.float64)
+    _load().oracle_lse_merge(n, Dv, o.ctypes.data, l.ctypes.data, out.ctypes.data,
+                             lse.ctypes.data)
+    return out, float(lse[0])
