@@ -1,0 +1,406 @@
+#!/usr/bin/env python
+"""Bench: MLA paged decode on B200 -- µs per decode step and effective KV GB/s.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one decode call (split-KV partial kernel + combine kernel) over a
+resident synthetic workload (default: FP8 E4M3 cache, q_len 4, 32 heads,
+81,920 keys, batch 16). Each timed step is bracketed by CUDA events on the
+launching stream; a 256 MiB buffer is rewritten between steps so no step
+starts from a warm L2 (the cache pool is larger than L2 anyway). With N > 1
+(torchrun) every rank runs an independent replica on its own GPU ("replicas
+only": the decode has no exchange step); the time is the max over ranks and
+the value the KV bytes of all ranks over that time.
+
+--impl reference times the fp64 CPU oracle (the only reference this build
+has) on the host cores, one bounded sample of the workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_HBM_GBS = 6650.0
+PUBLISHED_US = {"fp8_long_b4": 49.5, "fp8_long_b16": 148.1}  # TokenSpeed, article section 二
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="fp8_long_b16")
+    ap.add_argument("--kernel", default="auto", choices=["auto", "tcgen05", "simt"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+# ---------------------------------------------------------------- helpers
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mla_paged_decode_04_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h", ".cpp")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile(workload, kernel_name):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    e = d.get(workload, {}).get(kernel_name)
+    if not e or e.get("source_sha") != kernel_source_sha():
+        return None
+    return float(e["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed work runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.path = None
+        self.device_index = device_index
+
+    def start(self):
+        try:
+            import torch
+            sel = []
+            try:
+                uuid = str(torch.cuda.get_device_properties(self.device_index).uuid)
+                sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+            except Exception:
+                sel = []
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        try:
+            rows = [l.strip().split(", ") for l in open(self.path) if l.strip()]
+            os.unlink(self.path)
+        except Exception:
+            return None
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import mla_paged_decode_04_b200 as mla
+    from mla_paged_decode_04_b200.inputs import D_QK, D_V, WORKLOADS, make_inputs
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(args.workload, device=dev)
+    g = inp.to(dev)
+    B, T, H = g.batch, g.q_len, g.heads
+    dec = mla.MlaDecoder(B, T, H, g.max_seq_len, g.dtype, dev, kernel=args.kernel)
+    plan = dec.plan
+    out = torch.empty((B, T, H, D_V), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, T, H), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    esize = 1 if g.dtype == "fp8" else 2
+    kv_tokens = int(inp.seq_lens.clamp(min=0).sum())
+    kv_bytes = kv_tokens * D_QK * esize
+    q_bytes = g.q.numel() * esize
+    table_bytes = sum((int(n) + 63) // 64 for n in inp.seq_lens.tolist()) * 4 + B * 4
+    out_bytes = out.numel() * 2 + lse.numel() * 4
+    alg_bytes_step = kv_bytes + q_bytes + table_bytes + out_bytes
+    alg_bytes_partial = kv_bytes + q_bytes + table_bytes + (out_bytes if plan.split_kv == 1 else 0)
+    call = (g.q, g.kv_cache, g.block_tables, g.seq_lens, g.softmax_scale, out, lse, dec.workspace,
+            g.q_scale, g.kv_scale)
+    kernels_per_step = 1 + (1 if plan.split_kv > 1 else 0)
+
+    def step():
+        mla.mla_decode_partial(plan, *call)
+        mla.mla_decode_combine(plan, *call)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if dec.status() != 0:
+        raise RuntimeError("device status word set during warm-up")
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    # keep the GPU busy for ~1.5 s so the clock samples see the kernel under load
+    t_end = time.perf_counter() + 1.5
+    while time.perf_counter() < t_end:
+        for _ in range(20):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for k in range(args.steps):
+        flush.zero_()
+        e0, e1, e2 = evs[k]
+        e0.record()
+        mla.mla_decode_partial(plan, *call)
+        e1.record()
+        mla.mla_decode_combine(plan, *call)
+        e2.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    wall1 = time.perf_counter()
+    clocks = sampler.stop()
+    step_ms = [e0.elapsed_time(e2) for e0, _, e2 in evs]
+    part_ms = [e0.elapsed_time(e1) for e0, e1, _ in evs]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * kv_bytes * args.steps / (total_ms / 1e3) / 1e9
+
+    # end to end through the public API: inputs from pinned host memory each step,
+    # result read back to pinned host memory, all inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        hq = inp.q.cpu().pin_memory() if not inp.q.is_cuda else inp.q.cpu().pin_memory()
+        hbt = inp.block_tables.cpu().pin_memory()
+        hsl = inp.seq_lens.cpu().pin_memory()
+        dq, dbt, dsl = torch.empty_like(g.q), torch.empty_like(g.block_tables), torch.empty_like(g.seq_lens)
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        h2d = hq.numel() * hq.element_size() + hbt.numel() * 4 + hsl.numel() * 4
+        d2h = hout.numel() * 2 + hlse.numel() * 4
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dbt.copy_(hbt, non_blocking=True)
+            dsl.copy_(hsl, non_blocking=True)
+            dec(dq, g.kv_cache, dbt, dsl, g.softmax_scale, g.q_scale, g.kv_scale, out=out, lse=lse)
+            hout.copy_(out, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        for k in range(args.steps):
+            flush.zero_()
+            ev2[k][0].record()
+            e2e_step()
+            ev2[k][1].record()
+        torch.cuda.synchronize()
+        e2e_ms = sum(a.elapsed_time(b) for a, b in ev2)
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": round(world * kv_bytes * args.steps / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+               "us_per_step": round(e2e_ms / args.steps * 1e3, 2),
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+        if not torch.equal(hout, out.cpu()):
+            raise RuntimeError("e2e read-back differs from the device result")
+
+    peak, peak_kind = measured_peak()
+    part_avg_s = statistics.mean(part_ms) / 1e3
+    achieved = alg_bytes_partial / part_avg_s / 1e9
+    kname = "mla_tc_partial" if plan.kernel == 1 else "mla_simt_partial"
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_source": peak_kind,
+                "traffic": traffic_from_profile(args.workload, kname), "kernel": kname,
+                "alg_bytes_per_launch": int(alg_bytes_partial),
+                "partial_us": round(statistics.mean(part_ms) * 1e3, 2),
+                "combine_us": round((statistics.mean(step_ms) - statistics.mean(part_ms)) * 1e3, 2)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.workload, rows_per_sample=64, repeats=1)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    us = ms_per_step * 1e3
+    vs = None
+    if args.workload in PUBLISHED_US:
+        vs = round(PUBLISHED_US[args.workload] / us, 3)  # >1: faster than the published figure
+    line = {
+        "metric": "MLA decode effective KV GB/s (us/step in ms_per_step) on 1 B200",
+        "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "us_per_step": round(us, 2),
+        "us_p10": round(sorted(step_ms)[len(step_ms) // 10] * 1e3, 2),
+        "us_p90": round(sorted(step_ms)[(9 * len(step_ms)) // 10] * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": vs,
+        "dtype": {"fp8": "fp8_e4m3", "bf16": "bf16", "fp16": "fp16"}[g.dtype],
+        "data": "synthetic (seeded, generated on device)",
+        "config": {"workload": args.workload, "batch": B, "q_len": T, "heads": H,
+                   "seq_len_max": g.max_seq_len, "kv_tokens": kv_tokens, "page_size": 64,
+                   "split_kv": plan.split_kv, "fold": plan.fold, "kernel": kname,
+                   "kv_bytes_per_step": kv_bytes, "l2": "256 MiB buffer rewritten between steps; "
+                   "cache pool larger than L2", "parallelism": f"replicas x{world}"},
+        "gpu_launches": kernels_per_step * args.steps,
+        "wall_s_timed": round(wall1 - wall0, 4),
+        "roofline": roofline, "e2e": e2e, "clocks": clocks, "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- oracle timing
+
+def _oracle_sample_inputs(workload):
+    """One batch entry of the workload, same shape and distributions, drawn on the CPU."""
+    from mla_paged_decode_04_b200.inputs import WORKLOADS, make_inputs_custom
+    w = WORKLOADS[workload]
+    n = w.max_seq_len if w.seq[0] == "fixed" else int(w.seq[1]) if w.seq[0] == "lognormal" else (w.seq[1] + w.seq[2]) // 2
+    return make_inputs_custom(1, w.q_len, w.heads, w.dtype, [n], seed=2000 + w.config,
+                              pool="exact", q_std=w.q_std, kv_std=w.kv_std), n
+
+
+def cpu_baseline(workload, rows_per_sample, repeats):
+    import oracle
+    inp, n = _oracle_sample_inputs(workload)
+    rows_total = inp.q_len * inp.heads
+    rows = list(range(0, rows_total, max(1, rows_total // rows_per_sample)))[:rows_per_sample]
+    esize = 1 if inp.dtype == "fp8" else 2
+    t0 = time.perf_counter()
+    for _ in range(repeats):
+        oracle.mla_decode(inp.q, inp.kv_cache, inp.block_tables, inp.seq_lens, inp.softmax_scale,
+                          dtype=inp.dtype, q_scale=inp.q_scale, kv_scale=inp.kv_scale, rows=rows)
+    dt = (time.perf_counter() - t0) / repeats
+    work_bytes = n * 576 * esize * len(rows) / rows_total
+    return {"value": round(work_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "seconds": round(dt, 3),
+            "sample": f"{len(rows)} of the {rows_total} query rows of one batch entry "
+                      f"({n} keys, {inp.dtype}); KV bytes scaled by the row fraction"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    from mla_paged_decode_04_b200.inputs import WORKLOADS
+    inp, n = _oracle_sample_inputs(args.workload)
+    rows_total = inp.q_len * inp.heads
+    rows = list(range(0, rows_total, rows_total // 8))[:8]
+    esize = 1 if inp.dtype == "fp8" else 2
+
+    def one():
+        oracle.mla_decode(inp.q, inp.kv_cache, inp.block_tables, inp.seq_lens, inp.softmax_scale,
+                          dtype=inp.dtype, q_scale=inp.q_scale, kv_scale=inp.kv_scale, rows=rows)
+
+    for _ in range(args.warmup):
+        one()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        one()
+        times.append(time.perf_counter() - t0)
+    dt = sum(times)
+    work_bytes = n * 576 * esize * len(rows) / rows_total
+    value = work_bytes * args.steps / dt / 1e9
+    w = WORKLOADS[args.workload]
+    sample = (f"{len(rows)} of the {rows_total} query rows of one batch entry ({n} keys, "
+              f"{inp.dtype}) per step; KV bytes scaled by the row fraction")
+    line = {"impl": "reference", "metric": "MLA decode effective KV GB/s (us/step in ms_per_step) on 1 B200",
+            "value": round(value, 5), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": {"fp8": "fp8_e4m3", "bf16": "bf16", "fp16": "fp16"}[w.dtype],
+            "data": "synthetic (seeded)",
+            "config": {"workload": args.workload, "batch": w.batch, "q_len": w.q_len,
+                       "heads": w.heads, "seq_len_max": w.max_seq_len, "page_size": 64},
+            "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,195 @@
+/*
+ * mla_decode.h -- C ABI of the B200 (sm_100a) MLA paged-decode library.
+ *
+ * Multi-head Latent Attention decode over a paged latent KV cache: every
+ * batch entry's q_len x H query rows (576 = 512 latent + 64 rope dims) attend
+ * through a block table to one per-token latent cache shared by all heads
+ * (K = all 576 dims of a cached row, V = its first 512 dims), causally among
+ * the q_len tokens of the step. Output: BF16 rows plus an fp32 per-row LSE.
+ *
+ * Sources (prose only; the pages print no formulas or code):
+ *   - tokenspeed-mla package card, "What it is and what it does": a decode
+ *     path over FP16, BF16 or FP8 inputs that always writes BF16 output, run
+ *     as two kernels (split-KV partials, then a reduction) with the split
+ *     count and workspace size derived at run time.
+ *   - TokenSpeed MLA article (最快MLA内核背后的秘密), section 二: split_kv and
+ *     the workspace size follow from batch_size, q_len and max_seq_len;
+ *     section 三: query-token folding (largest F with q_len % F == 0 and
+ *     H * F <= 128); section 四: causal and LSE outputs; section 六: tensor
+ *     layouts query [B, q_len, H, D_qk], kv_cache [num_pages, page_size,
+ *     D_total] plus block_tables.
+ *
+ * Conventions for every entry point:
+ *   - Return 0 (MLA_OK) on success, a negative mla_status otherwise. Host-side
+ *     argument errors are detected before anything is enqueued.
+ *   - Device pointers are raw CUDA device addresses owned by the caller (in
+ *     practice allocated by PyTorch). The library allocates no device memory
+ *     and never synchronises the stream in mla_decode.
+ *   - `stream` is a cudaStream_t passed as void*; NULL means the legacy
+ *     default stream. All device work is enqueued on it, asynchronously.
+ *   - Problems only the device can see (a block-table entry outside
+ *     [0, num_pages), a seq_len above the planned maximum, a pipeline wait
+ *     that ran out) are recorded as bits of a status word in the workspace
+ *     header and never trap; read them with mla_decode_status. The affected
+ *     rows' outputs are then unspecified but finite; no memory outside the
+ *     arguments is touched.
+ */
+#ifndef MLA_DECODE_H
+#define MLA_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_D_QK 576        /* latent (512) + rope (64) dims of q and of a cached row */
+#define MLA_D_V 512         /* V = first 512 dims of the cached row */
+#define MLA_PAGE_SIZE 64    /* tokens per cache page (the only page size supported) */
+#define MLA_MAX_ROWS 128    /* rows (heads x folded tokens) one CTA pair processes */
+
+typedef enum { MLA_BF16 = 0, MLA_FP16 = 1, MLA_FP8_E4M3 = 2 } mla_dtype;
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = -1,       /* null pointer, negative size, bad dtype, ... */
+  MLA_ERR_UNSUPPORTED_SHAPE = -2, /* e.g. page_size != 64, H > 128 */
+  MLA_ERR_WORKSPACE_TOO_SMALL = -3,
+  MLA_ERR_ARCH = -4,              /* current device is not sm_100 */
+  MLA_ERR_CUDA = -5,              /* a CUDA runtime call failed */
+  MLA_ERR_PLAN_MISMATCH = -6      /* plan fields inconsistent or not from mla_decode_plan */
+} mla_status;
+
+/* Bits of the device status word (workspace header). */
+#define MLA_DEV_BAD_PAGE 0x1     /* block-table entry outside [0, num_pages): keys masked */
+#define MLA_DEV_SEQ_TOO_LONG 0x2 /* seq_len above max_seq_len or the table width: clamped */
+#define MLA_DEV_TIMEOUT 0x4      /* a bounded pipeline wait gave up; outputs unspecified */
+
+typedef enum {
+  MLA_KERNEL_AUTO = 0,    /* the tcgen05 CTA-pair kernel */
+  MLA_KERNEL_TCGEN05 = 1, /* sm_100a tensor-core split-KV kernel (TMA + tcgen05 + TMEM) */
+  MLA_KERNEL_SIMT = 2     /* plain CUDA-core kernel: a slow, simple cross-check */
+} mla_kernel;
+
+/*
+ * Plan of one decode shape. Filled by mla_decode_plan; treat as read-only.
+ *   fold            F: query tokens folded into the row dimension
+ *   q_groups        G = q_len / F; each (batch entry, group) is one unit
+ *   rows_per_unit   M = H * F <= 128 query rows that share each K tile
+ *   split_kv        S: key chunks per unit processed in parallel
+ *   keys_per_split  chunk length in keys (multiple of 64); split s covers
+ *                   keys [s * keys_per_split, (s + 1) * keys_per_split)
+ *   num_ctas        CTAs of the partial kernel
+ *   workspace_bytes bytes the caller must pass as workspace (>= 256)
+ *   partial_offset, lse_offset  byte offsets of the fp32 partial O
+ *                   [B*q_len*H, S, 512] and partial LSE [B*q_len*H, S]
+ *                   inside the workspace (used when split_kv > 1)
+ */
+typedef struct {
+  int32_t batch, q_len, num_heads, max_seq_len, dtype;
+  int32_t fold, q_groups, rows_per_unit;
+  int32_t split_kv, keys_per_split;
+  int32_t kernel, num_ctas;
+  uint64_t workspace_bytes, partial_offset, lse_offset;
+  uint32_t magic; /* set by the planner; checked by mla_decode */
+  uint32_t reserved;
+} mla_plan;
+
+/*
+ * mla_decode_plan: choose F, split_kv and the workspace size for a shape
+ * (TokenSpeed MLA article, section 二 for split_kv and workspace sizing from
+ * batch, q_len and max_seq_len; section 三 for the fold factor).
+ * Pure host arithmetic on the 148-SM B200, deterministic and memoised; no
+ * device calls. batch >= 0, 1 <= q_len, 1 <= num_heads <= 128,
+ * max_seq_len >= 0, dtype an mla_dtype. Errors: MLA_ERR_INVALID_ARG,
+ * MLA_ERR_UNSUPPORTED_SHAPE. `plan` is written only on success.
+ */
+int mla_decode_plan(int batch, int q_len, int num_heads, int max_seq_len, int dtype,
+                    mla_plan* plan);
+
+/*
+ * mla_decode_plan_custom: as mla_decode_plan, with overrides for tests and
+ * tuning: split_kv > 0 forces S (clamped to the number of 64-key tiles),
+ * fold > 0 forces F (must divide q_len with H * F <= 128), kernel selects an
+ * mla_kernel. Zero means "choose automatically".
+ */
+int mla_decode_plan_custom(int batch, int q_len, int num_heads, int max_seq_len, int dtype,
+                           int split_kv, int fold, int kernel, mla_plan* plan);
+
+/*
+ * mla_decode: one decode step (tokenspeed-mla package card, "Quickstart":
+ * query, kv_cache, workspace, block_tables, seq_lens, max_seq_len,
+ * softmax_scale; layouts from the TokenSpeed MLA article, section 六).
+ *
+ *   plan            from mla_decode_plan for this batch/q_len/H/max_seq_len/dtype
+ *   q               device, [B, q_len, H, 576] of plan->dtype, contiguous,
+ *                   16-byte aligned
+ *   kv_cache        device, [num_pages, page_size, 576] of plan->dtype,
+ *                   contiguous, 16-byte aligned; page_size must be 64
+ *   block_tables    device int32 [B, max_pages_per_seq]; entry j of row b is
+ *                   the page holding keys 64j .. 64j+63 of entry b; entries
+ *                   past ceil(seq_len/64) are never read
+ *   seq_lens        device int32 [B]: keys in the cache for entry b, counting
+ *                   this step's q_len tokens; token t of the step sees keys
+ *                   0 .. seq_len - q_len + t (no key: out 0, lse -inf)
+ *   softmax_scale   applied to q.k (e.g. 576^-0.5)
+ *   q_scale, kv_scale  FP8 dequantisation: values are code * scale; the
+ *                   cache's one scale serves K and V. Ignored (1) for 16-bit
+ *   out             device bf16 [B, q_len, H, 512]
+ *   lse             device fp32 [B, q_len, H], natural log of the sum of
+ *                   exp(scaled scores); may be NULL
+ *   workspace       device buffer of >= plan->workspace_bytes, 256-byte
+ *                   aligned; holds the status word and the split partials.
+ *                   Calls that share a workspace must not overlap on the GPU.
+ *   stream          cudaStream_t as void*
+ * Errors: MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED_SHAPE,
+ * MLA_ERR_WORKSPACE_TOO_SMALL, MLA_ERR_PLAN_MISMATCH, MLA_ERR_ARCH,
+ * MLA_ERR_CUDA (launch failure). Nothing is enqueued when an error is
+ * returned before the first launch. Capturable in a CUDA graph.
+ */
+int mla_decode(const mla_plan* plan, const void* q, const void* kv_cache, int64_t num_pages,
+               int page_size, const int32_t* block_tables, int max_pages_per_seq,
+               const int32_t* seq_lens, float softmax_scale, float q_scale, float kv_scale,
+               void* out, float* lse, void* workspace, uint64_t workspace_bytes, void* stream);
+
+/*
+ * mla_decode_partial / mla_decode_combine: the two kernels of mla_decode,
+ * enqueued separately (TokenSpeed MLA article, section 二: a split-KV kernel
+ * writing partial outputs and LSEs, then a reduction kernel merging them).
+ * Same arguments, validation and errors as mla_decode; calling
+ * mla_decode_partial then mla_decode_combine on one stream equals one
+ * mla_decode. mla_decode_partial resets the status word and, when
+ * plan->split_kv == 1, writes out/lse itself; mla_decode_combine is then a
+ * no-op. Exposed so that each kernel can be timed on its own.
+ */
+int mla_decode_partial(const mla_plan* plan, const void* q, const void* kv_cache,
+                       int64_t num_pages, int page_size, const int32_t* block_tables,
+                       int max_pages_per_seq, const int32_t* seq_lens, float softmax_scale,
+                       float q_scale, float kv_scale, void* out, float* lse, void* workspace,
+                       uint64_t workspace_bytes, void* stream);
+int mla_decode_combine(const mla_plan* plan, const void* q, const void* kv_cache,
+                       int64_t num_pages, int page_size, const int32_t* block_tables,
+                       int max_pages_per_seq, const int32_t* seq_lens, float softmax_scale,
+                       float q_scale, float kv_scale, void* out, float* lse, void* workspace,
+                       uint64_t workspace_bytes, void* stream);
+
+/*
+ * mla_decode_status: synchronise `stream`, copy the device status word of
+ * `workspace` (MLA_DEV_* bits from the last mla_decode that used it) into
+ * *device_status, and clear it if `clear` is non-zero. For tests and debug
+ * tooling; it blocks. Errors: MLA_ERR_INVALID_ARG, MLA_ERR_CUDA.
+ */
+int mla_decode_status(void* workspace, void* stream, int clear, int32_t* device_status);
+
+/* Human-readable name of an mla_status code (static storage, never NULL). */
+const char* mla_status_string(int code);
+
+/* Library version string, e.g. "0.1.0". */
+const char* mla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_DECODE_H */

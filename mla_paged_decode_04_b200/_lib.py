@@ -1,0 +1,209 @@
+"""ctypes binding of libmla_decode.so (argument marshalling only).
+
+The functions carry the C ABI's names (include/mla_decode.h) and pass raw
+device pointers and the current CUDA stream; every step of the decode runs
+in the library's kernels. PyTorch is used only to own device memory and
+streams. If the shared library is missing this module raises at import: there
+is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmla_decode.so")
+
+MLA_BF16, MLA_FP16, MLA_FP8_E4M3 = 0, 1, 2
+DTYPES = {"bf16": MLA_BF16, "fp16": MLA_FP16, "fp8": MLA_FP8_E4M3}
+MLA_KERNEL_AUTO, MLA_KERNEL_TCGEN05, MLA_KERNEL_SIMT = 0, 1, 2
+KERNELS = {"auto": MLA_KERNEL_AUTO, "tcgen05": MLA_KERNEL_TCGEN05, "simt": MLA_KERNEL_SIMT}
+
+MLA_DEV_BAD_PAGE, MLA_DEV_SEQ_TOO_LONG, MLA_DEV_TIMEOUT = 0x1, 0x2, 0x4
+
+EXPORTED = ["mla_decode_plan", "mla_decode_plan_custom", "mla_decode", "mla_decode_partial",
+            "mla_decode_combine", "mla_decode_status", "mla_status_string", "mla_version"]
+
+
+class MlaPlan(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("q_len", ctypes.c_int32), ("num_heads", ctypes.c_int32),
+        ("max_seq_len", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("fold", ctypes.c_int32), ("q_groups", ctypes.c_int32), ("rows_per_unit", ctypes.c_int32),
+        ("split_kv", ctypes.c_int32), ("keys_per_split", ctypes.c_int32),
+        ("kernel", ctypes.c_int32), ("num_ctas", ctypes.c_int32),
+        ("workspace_bytes", ctypes.c_uint64), ("partial_offset", ctypes.c_uint64),
+        ("lse_offset", ctypes.c_uint64), ("magic", ctypes.c_uint32), ("reserved", ctypes.c_uint32),
+    ]
+
+    def as_dict(self):
+        return {f: getattr(self, f) for f, _ in self._fields_}
+
+
+class MlaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what} failed: {status_string(code)} ({code})")
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python mla_paged_decode_04_b200/build.py` "
+            "(there is no non-CUDA fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    i32, i64, u64, f32, vp = (ctypes.c_int, ctypes.c_int64, ctypes.c_uint64, ctypes.c_float,
+                              ctypes.c_void_p)
+    P = ctypes.POINTER(MlaPlan)
+    lib.mla_decode_plan.argtypes = [i32, i32, i32, i32, i32, P]
+    lib.mla_decode_plan.restype = i32
+    lib.mla_decode_plan_custom.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, P]
+    lib.mla_decode_plan_custom.restype = i32
+    for name in ("mla_decode", "mla_decode_partial", "mla_decode_combine"):
+        fn = getattr(lib, name)
+        fn.argtypes = [P, vp, vp, i64, i32, vp, i32, vp, f32, f32, f32, vp, vp, vp, u64, vp]
+        fn.restype = i32
+    lib.mla_decode_status.argtypes = [vp, vp, i32, ctypes.POINTER(ctypes.c_int32)]
+    lib.mla_decode_status.restype = i32
+    lib.mla_status_string.argtypes = [i32]
+    lib.mla_status_string.restype = ctypes.c_char_p
+    lib.mla_version.argtypes = []
+    lib.mla_version.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load()
+
+
+def lib():
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return _lib.mla_status_string(int(code)).decode()
+
+
+def mla_version() -> str:
+    return _lib.mla_version().decode()
+
+
+def _dtype_code(dtype) -> int:
+    if isinstance(dtype, str):
+        return DTYPES[dtype]
+    if dtype == torch.bfloat16:
+        return MLA_BF16
+    if dtype == torch.float16:
+        return MLA_FP16
+    if dtype == torch.float8_e4m3fn:
+        return MLA_FP8_E4M3
+    return int(dtype)
+
+
+def mla_decode_plan(batch, q_len, num_heads, max_seq_len, dtype) -> MlaPlan:
+    p = MlaPlan()
+    rc = _lib.mla_decode_plan(batch, q_len, num_heads, max_seq_len, _dtype_code(dtype), ctypes.byref(p))
+    if rc != 0:
+        raise MlaError(rc, "mla_decode_plan")
+    return p
+
+
+def mla_decode_plan_custom(batch, q_len, num_heads, max_seq_len, dtype, split_kv=0, fold=0,
+                           kernel="auto") -> MlaPlan:
+    p = MlaPlan()
+    k = KERNELS[kernel] if isinstance(kernel, str) else int(kernel)
+    rc = _lib.mla_decode_plan_custom(batch, q_len, num_heads, max_seq_len, _dtype_code(dtype),
+                                     split_kv, fold, k, ctypes.byref(p))
+    if rc != 0:
+        raise MlaError(rc, "mla_decode_plan_custom")
+    return p
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _call(name, plan, q, kv_cache, block_tables, seq_lens, softmax_scale, out, lse, workspace,
+          q_scale, kv_scale, stream):
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream if q.is_cuda else 0
+    elif isinstance(stream, torch.cuda.Stream):
+        stream = stream.cuda_stream
+    num_pages, page_size = int(kv_cache.shape[0]), int(kv_cache.shape[1])
+    rc = getattr(_lib, name)(ctypes.byref(plan), _ptr(q), _ptr(kv_cache), num_pages, page_size,
+                         _ptr(block_tables), int(block_tables.shape[1]), _ptr(seq_lens),
+                         float(softmax_scale), float(q_scale), float(kv_scale), _ptr(out),
+                         _ptr(lse), _ptr(workspace), int(workspace.numel() * workspace.element_size()),
+                         ctypes.c_void_p(stream))
+    if rc != 0:
+        raise MlaError(rc, name)
+
+
+def mla_decode(plan: MlaPlan, q, kv_cache, block_tables, seq_lens, softmax_scale, out, lse,
+               workspace, q_scale=1.0, kv_scale=1.0, stream=None) -> None:
+    """Enqueue one decode step on `stream` (default: torch's current stream).
+
+    Tensors are device tensors in the layouts of include/mla_decode.h; `out`
+    (bf16 [B, q_len, H, 512]), `lse` (fp32 [B, q_len, H] or None) and
+    `workspace` (uint8, >= plan.workspace_bytes, 256-byte aligned) are written.
+    """
+    _call("mla_decode", plan, q, kv_cache, block_tables, seq_lens, softmax_scale, out, lse,
+          workspace, q_scale, kv_scale, stream)
+
+
+def mla_decode_partial(plan: MlaPlan, q, kv_cache, block_tables, seq_lens, softmax_scale, out,
+                       lse, workspace, q_scale=1.0, kv_scale=1.0, stream=None) -> None:
+    """First kernel only (split-KV partials; writes out/lse itself when split_kv == 1)."""
+    _call("mla_decode_partial", plan, q, kv_cache, block_tables, seq_lens, softmax_scale, out,
+          lse, workspace, q_scale, kv_scale, stream)
+
+
+def mla_decode_combine(plan: MlaPlan, q, kv_cache, block_tables, seq_lens, softmax_scale, out,
+                       lse, workspace, q_scale=1.0, kv_scale=1.0, stream=None) -> None:
+    """Second kernel only (LSE merge of the partials; no-op when split_kv == 1)."""
+    _call("mla_decode_combine", plan, q, kv_cache, block_tables, seq_lens, softmax_scale, out,
+          lse, workspace, q_scale, kv_scale, stream)
+
+
+def mla_decode_status(workspace, clear=True, stream=None) -> int:
+    """Synchronise and read the device status word (MLA_DEV_* bits)."""
+    if stream is None:
+        stream = torch.cuda.current_stream(workspace.device).cuda_stream
+    v = ctypes.c_int32(0)
+    rc = _lib.mla_decode_status(_ptr(workspace), ctypes.c_void_p(stream), int(bool(clear)),
+                                ctypes.byref(v))
+    if rc != 0:
+        raise MlaError(rc, "mla_decode_status")
+    return int(v.value)
+
+
+def alloc_workspace(plan: MlaPlan, device) -> torch.Tensor:
+    """A zeroed workspace tensor of plan.workspace_bytes (torch allocations are 256-byte aligned)."""
+    return torch.zeros(int(plan.workspace_bytes), dtype=torch.uint8, device=device)
+
+
+class MlaDecoder:
+    """Plan + workspace for one decode shape; call it once per decode step."""
+
+    def __init__(self, batch, q_len, num_heads, max_seq_len, dtype, device, split_kv=0, fold=0,
+                 kernel="auto"):
+        self.plan = mla_decode_plan_custom(batch, q_len, num_heads, max_seq_len, dtype,
+                                           split_kv, fold, kernel)
+        self.device = torch.device(device)
+        self.workspace = alloc_workspace(self.plan, self.device)
+        self.batch, self.q_len, self.num_heads = batch, q_len, num_heads
+
+    def __call__(self, q, kv_cache, block_tables, seq_lens, softmax_scale, q_scale=1.0,
+                 kv_scale=1.0, out=None, lse=None, want_lse=True, stream=None):
+        B, T, H = self.batch, self.q_len, self.num_heads
+        if out is None:
+            out = torch.empty((B, T, H, 512), dtype=torch.bfloat16, device=self.device)
+        if lse is None and want_lse:
+            lse = torch.empty((B, T, H), dtype=torch.float32, device=self.device)
+        mla_decode(self.plan, q, kv_cache, block_tables, seq_lens, softmax_scale, out, lse,
+                   self.workspace, q_scale, kv_scale, stream)
+        return out, lse
+
+    def status(self, clear=True) -> int:
+        return mla_decode_status(self.workspace, clear)

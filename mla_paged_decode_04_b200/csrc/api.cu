@@ -1,0 +1,189 @@
+// C ABI: argument validation, workspace layout and kernel launches.
+#include <cmath>
+#include <mutex>
+
+#include "internal.h"
+
+namespace mla {
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+int check_device_arch() {
+  static std::mutex mu;
+  static int cached[64];
+  static bool init = false;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return MLA_ERR_ARCH;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!init) {
+    for (int i = 0; i < 64; ++i) cached[i] = 1;  // 1 = unknown
+    init = true;
+  }
+  if (cached[dev] == 1) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    cached[dev] = (major == 10 && minor == 0) ? MLA_OK : MLA_ERR_ARCH;
+  }
+  return cached[dev];
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// The plan must be one the planner could have produced for its own fields.
+int check_plan(const mla_plan* p) {
+  if (!p || p->magic != kPlanMagic) return MLA_ERR_PLAN_MISMATCH;
+  if (p->batch < 0 || p->q_len < 1 || p->num_heads < 1 || p->num_heads > MLA_MAX_ROWS ||
+      p->max_seq_len < 0)
+    return MLA_ERR_PLAN_MISMATCH;
+  if (p->dtype != MLA_BF16 && p->dtype != MLA_FP16 && p->dtype != MLA_FP8_E4M3) return MLA_ERR_PLAN_MISMATCH;
+  if (p->fold < 1 || p->q_len % p->fold != 0 || p->q_groups * p->fold != p->q_len ||
+      p->rows_per_unit != p->num_heads * p->fold || p->rows_per_unit > MLA_MAX_ROWS)
+    return MLA_ERR_PLAN_MISMATCH;
+  if (p->split_kv < 1 || p->keys_per_split < kTileKeys || p->keys_per_split % kTileKeys != 0)
+    return MLA_ERR_PLAN_MISMATCH;
+  if ((int64_t)p->split_kv * p->keys_per_split < (int64_t)p->max_seq_len) return MLA_ERR_PLAN_MISMATCH;
+  if (p->kernel != MLA_KERNEL_TCGEN05 && p->kernel != MLA_KERNEL_SIMT) return MLA_ERR_PLAN_MISMATCH;
+  const uint64_t rows = (uint64_t)p->batch * p->q_len * p->num_heads;
+  if (p->split_kv > 1) {
+    if (p->partial_offset < (uint64_t)kHeaderBytes || p->partial_offset % 256 != 0 ||
+        p->lse_offset < p->partial_offset + rows * (uint64_t)p->split_kv * MLA_D_V * 4 ||
+        p->lse_offset % 256 != 0 ||
+        p->workspace_bytes < p->lse_offset + rows * (uint64_t)p->split_kv * 4)
+      return MLA_ERR_PLAN_MISMATCH;
+  } else if (p->workspace_bytes < (uint64_t)kHeaderBytes) {
+    return MLA_ERR_PLAN_MISMATCH;
+  }
+  return MLA_OK;
+}
+
+}  // namespace
+
+namespace {
+
+// Validate the arguments and fill the launch description. Returns MLA_OK or
+// an error code; nothing is enqueued here.
+int prepare(const mla_plan* plan, const void* q, const void* kv_cache, int64_t num_pages,
+            int page_size, const int32_t* block_tables, int max_pages_per_seq,
+            const int32_t* seq_lens, float softmax_scale, float q_scale, float kv_scale, void* out,
+            float* lse, void* workspace, uint64_t workspace_bytes, DecodeArgs* a) {
+  int rc = check_plan(plan);
+  if (rc != MLA_OK) return rc;
+  const mla_plan& p = *plan;
+  if (page_size != MLA_PAGE_SIZE) return MLA_ERR_UNSUPPORTED_SHAPE;
+  if (!workspace || !aligned(workspace, 256)) return MLA_ERR_INVALID_ARG;
+  if (workspace_bytes < p.workspace_bytes) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
+  if (p.dtype == MLA_FP8_E4M3 &&
+      (!std::isfinite(q_scale) || !std::isfinite(kv_scale) || q_scale <= 0.f || kv_scale <= 0.f))
+    return MLA_ERR_INVALID_ARG;
+  if (p.batch > 0) {
+    if (!q || !kv_cache || !block_tables || !seq_lens || !out) return MLA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(kv_cache, 16) || !aligned(out, 16) || !aligned(block_tables, 4) ||
+        !aligned(seq_lens, 4) || (lse && !aligned(lse, 4)))
+      return MLA_ERR_INVALID_ARG;
+    if (num_pages < 1 || max_pages_per_seq < 1) return MLA_ERR_INVALID_ARG;
+    if (num_pages > (int64_t(1) << 31) / MLA_PAGE_SIZE) return MLA_ERR_UNSUPPORTED_SHAPE;
+  }
+  rc = check_device_arch();
+  if (rc != MLA_OK) return rc;
+
+  *a = DecodeArgs{};
+  a->plan = p;
+  a->q = q;
+  a->kv_cache = kv_cache;
+  a->num_pages = num_pages;
+  a->block_tables = block_tables;
+  a->max_pages_per_seq = max_pages_per_seq;
+  a->seq_lens = seq_lens;
+  const bool fp8 = p.dtype == MLA_FP8_E4M3;
+  a->score_scale_log2 =
+      (float)((double)softmax_scale * (fp8 ? (double)q_scale * kv_scale : 1.0) * (double)kLog2e);
+  a->v_scale = fp8 ? kv_scale : 1.f;
+  a->out = out;
+  a->lse = lse;
+  a->status = reinterpret_cast<int32_t*>(workspace);
+  char* ws = reinterpret_cast<char*>(workspace);
+  a->o_part = p.split_kv > 1 ? reinterpret_cast<float*>(ws + p.partial_offset) : nullptr;
+  a->lse_part = p.split_kv > 1 ? reinterpret_cast<float*>(ws + p.lse_offset) : nullptr;
+  return MLA_OK;
+}
+
+int run_partial(const DecodeArgs& a, cudaStream_t st) {
+  if (cudaMemsetAsync(a.status, 0, sizeof(int32_t), st) != cudaSuccess) return MLA_ERR_CUDA;
+  if (a.plan.batch == 0) return MLA_OK;
+  cudaError_t e = (a.plan.kernel == MLA_KERNEL_SIMT) ? launch_simt_partial(a, st) : launch_tc_partial(a, st);
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int run_combine(const DecodeArgs& a, cudaStream_t st) {
+  if (a.plan.batch == 0 || a.plan.split_kv == 1) return MLA_OK;
+  return launch_combine(a, st) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace mla
+
+#define MLA_ARGS_DECL                                                                            \
+  const mla_plan *plan, const void *q, const void *kv_cache, int64_t num_pages, int page_size, \
+      const int32_t *block_tables, int max_pages_per_seq, const int32_t *seq_lens,              \
+      float softmax_scale, float q_scale, float kv_scale, void *out, float *lse, void *workspace, \
+      uint64_t workspace_bytes, void *stream
+#define MLA_ARGS_FWD                                                                            \
+  plan, q, kv_cache, num_pages, page_size, block_tables, max_pages_per_seq, seq_lens,          \
+      softmax_scale, q_scale, kv_scale, out, lse, workspace, workspace_bytes
+
+using namespace mla;
+
+extern "C" int mla_decode(MLA_ARGS_DECL) {
+  DecodeArgs a;
+  int rc = prepare(MLA_ARGS_FWD, &a);
+  if (rc != MLA_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  rc = run_partial(a, st);
+  if (rc != MLA_OK) return rc;
+  return run_combine(a, st);
+}
+
+extern "C" int mla_decode_partial(MLA_ARGS_DECL) {
+  DecodeArgs a;
+  int rc = prepare(MLA_ARGS_FWD, &a);
+  if (rc != MLA_OK) return rc;
+  return run_partial(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int mla_decode_combine(MLA_ARGS_DECL) {
+  DecodeArgs a;
+  int rc = prepare(MLA_ARGS_FWD, &a);
+  if (rc != MLA_OK) return rc;
+  return run_combine(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int mla_decode_status(void* workspace, void* stream, int clear, int32_t* device_status) {
+  if (!workspace || !device_status) return MLA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, workspace, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return MLA_ERR_CUDA;
+  if (clear && cudaMemset(workspace, 0, sizeof v) != cudaSuccess) return MLA_ERR_CUDA;
+  *device_status = v;
+  return MLA_OK;
+}
+
+extern "C" const char* mla_status_string(int code) {
+  switch (code) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+    case MLA_ERR_UNSUPPORTED_SHAPE: return "MLA_ERR_UNSUPPORTED_SHAPE";
+    case MLA_ERR_WORKSPACE_TOO_SMALL: return "MLA_ERR_WORKSPACE_TOO_SMALL";
+    case MLA_ERR_ARCH: return "MLA_ERR_ARCH";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_PLAN_MISMATCH: return "MLA_ERR_PLAN_MISMATCH";
+    default: return "MLA_ERR_UNKNOWN";
+  }
+}
+
+extern "C" const char* mla_version(void) { return "0.1.0"; }

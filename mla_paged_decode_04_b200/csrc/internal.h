@@ -1,0 +1,41 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mla_decode.h"
+
+namespace mla {
+
+constexpr uint32_t kPlanMagic = 0x4d4c4131u;  // "MLA1"
+constexpr int kNumSMs = 148;                    // B200
+constexpr int kHeaderBytes = 256;               // workspace header (status word at offset 0)
+constexpr int kTileKeys = 64;                   // keys per tile = one cache page
+
+// Everything a launch needs, validated by the ABI layer.
+struct DecodeArgs {
+  mla_plan plan;
+  const void* q;
+  const void* kv_cache;
+  int64_t num_pages;
+  const int32_t* block_tables;
+  int max_pages_per_seq;
+  const int32_t* seq_lens;
+  float score_scale_log2;  // softmax_scale * q_scale * kv_scale * log2(e)
+  float v_scale;           // kv_scale (FP8) or 1
+  void* out;               // bf16 [B*T*H, 512]
+  float* lse;              // fp32 [B*T*H] or null
+  int32_t* status;         // device status word
+  float* o_part;           // fp32 [B*T*H, S, 512] (split_kv > 1)
+  float* lse_part;         // fp32 [B*T*H, S]       (split_kv > 1)
+};
+
+int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, int split_kv,
+              int fold, int kernel, mla_plan* plan);
+
+cudaError_t launch_simt_partial(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_tc_partial(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t stream);
+
+}  // namespace mla

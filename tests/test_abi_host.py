@@ -1,0 +1,106 @@
+"""C ABI: symbols and host-side argument checks (CPU only).
+
+Every mla_decode call here is invalid in a way the library detects before it
+touches the device, so the fake pointers are never dereferenced (this file is
+also safe to run on a GPU machine).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mla_paged_decode_04_b200 as mla
+from mla_paged_decode_04_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?\w+\s*\**\s*(mla_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared_functions()
+    assert "mla_decode" in names and "mla_decode_plan" in names
+    lib = ctypes.CDLL(_lib.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(_lib.EXPORTED)
+
+
+def test_library_is_built_for_sm100a():
+    # the build records ptxas reports per translation unit
+    build = os.path.join(ROOT, "_build")
+    logs = [f for f in os.listdir(build) if f.endswith(".ptxas.txt")]
+    assert logs
+    text = "".join(open(os.path.join(build, f)).read() for f in logs)
+    assert "for 'sm_100a'" in text and "spill stores" in text
+
+
+def test_status_strings_and_version():
+    assert mla.status_string(0) == "MLA_OK"
+    assert mla.status_string(-3) == "MLA_ERR_WORKSPACE_TOO_SMALL"
+    assert mla.status_string(-99) == "MLA_ERR_UNKNOWN"
+    assert mla.mla_version().count(".") == 2
+
+
+FAKE = 1 << 20  # 256-byte aligned, never dereferenced
+
+
+def _call(plan, **kw):
+    args = dict(q=FAKE, kv=FAKE, num_pages=8, page_size=64, bt=FAKE, maxp=4, sl=FAKE,
+                scale=0.04, qs=1.0, ks=1.0, out=FAKE, lse=FAKE, ws=FAKE, ws_bytes=1 << 30)
+    args.update(kw)
+    L = _lib.lib()
+    vp = ctypes.c_void_p
+    return L.mla_decode(ctypes.byref(plan) if plan is not None else None, vp(args["q"]),
+                        vp(args["kv"]), args["num_pages"], args["page_size"], vp(args["bt"]),
+                        args["maxp"], vp(args["sl"]), args["scale"], args["qs"], args["ks"],
+                        vp(args["out"]), vp(args["lse"]), vp(args["ws"]), args["ws_bytes"], None)
+
+
+def test_decode_rejects_bad_arguments_before_any_launch():
+    p = mla.mla_decode_plan(2, 4, 32, 256, "fp8")
+    assert _call(None) == -6
+    bad = _lib.MlaPlan.from_buffer_copy(p)
+    bad.magic = 0
+    assert _call(bad) == -6
+    bad = _lib.MlaPlan.from_buffer_copy(p)
+    bad.fold = 3
+    assert _call(bad) == -6
+    bad = _lib.MlaPlan.from_buffer_copy(p)
+    bad.keys_per_split = 64
+    bad.split_kv = 1  # no longer covers max_seq_len
+    assert _call(bad) == -6
+    assert _call(p, page_size=32) == -2
+    assert _call(p, ws=0) == -1
+    assert _call(p, ws=FAKE + 16) == -1           # workspace not 256-aligned
+    assert _call(p, ws_bytes=p.workspace_bytes - 1) == -3
+    assert _call(p, q=0) == -1
+    assert _call(p, kv=0) == -1
+    assert _call(p, bt=0) == -1
+    assert _call(p, sl=0) == -1
+    assert _call(p, out=0) == -1
+    assert _call(p, q=FAKE + 8) == -1             # q not 16-byte aligned
+    assert _call(p, num_pages=0) == -1
+    assert _call(p, maxp=0) == -1
+    assert _call(p, qs=0.0) == -1                 # FP8 scales must be positive
+    assert _call(p, ks=float("nan")) == -1
+    assert _call(p, scale=float("inf")) == -1
+
+
+def test_workspace_error_from_python_wrapper():
+    torch = pytest.importorskip("torch")
+    p = mla.mla_decode_plan(1, 1, 16, 256, "bf16")
+    t = torch.empty(0)
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_decode(p, t, torch.empty(1, 32, 576), torch.empty(1, 4, dtype=torch.int32), t,
+                       0.04, t, None, torch.empty(0, dtype=torch.uint8))
+    assert e.value.code in (-1, -2)

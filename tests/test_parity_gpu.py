@@ -1,0 +1,190 @@
+"""GPU parity: the CUDA path against the fp64 oracle, through the C ABI.
+
+Small cases are compared on every row; the full-size workloads run in the
+launch configuration the bench times (automatic plan) and are compared on
+sampled rows the oracle computes one by one.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import mla_paged_decode_04_b200 as mla
+from mla_paged_decode_04_b200.inputs import make_inputs, make_inputs_custom
+from helpers import compare, oracle_rows, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+KERNELS = ["simt"]
+
+
+def run(inp, kernel="auto", split_kv=0, fold=0, want_lse=True):
+    dev = torch.device("cuda", 0)
+    g = inp.to(dev)
+    dec = mla.MlaDecoder(g.batch, g.q_len, g.heads, max(g.max_seq_len, 0), g.dtype, dev,
+                         split_kv=split_kv, fold=fold, kernel=kernel)
+    out, lse = dec(g.q, g.kv_cache, g.block_tables, g.seq_lens, g.softmax_scale,
+                   g.q_scale, g.kv_scale, want_lse=want_lse)
+    torch.cuda.synchronize()
+    status = dec.status()
+    return out, lse, status, dec
+
+
+SMALL = [
+    # (B, T, H, dtype, seq_lens, pool, q_std, kv_std)
+    (1, 1, 16, "bf16", [256], "exact", 1.0, 1.0),
+    (2, 4, 32, "bf16", [1000, 77], 2.0, 1.0, 0.5),
+    (3, 4, 16, "fp16", [64, 65, 300], 2.0, 1.0, 1.0),
+    (2, 4, 64, "fp16", [513, 130], 2.0, 1.0, 1.0),
+    (2, 2, 128, "bf16", [700, 3], 2.0, 1.0, 0.5),
+    (2, 4, 32, "fp8", [900, 128], 2.0, 1.0, 1.0),
+    (1, 3, 40, "fp8", [200], 1.0, 1.0, 1.0),
+    (4, 1, 8, "bf16", [1, 2, 63, 64], 1.0, 1.0, 1.0),
+    (3, 4, 32, "fp16", [2, 0, 5], 1.0, 1.0, 1.0),   # seq_len < q_len and empty entries
+]
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("case", range(len(SMALL)))
+def test_small_cases_all_rows(case, kernel):
+    B, T, H, dt, sl, pool, qs, ks = SMALL[case]
+    inp = make_inputs_custom(B, T, H, dt, sl, seed=100 + case, pool=pool, q_std=qs, kv_std=ks)
+    out, lse, status, _ = run(inp, kernel)
+    assert status == 0
+    ref_o, ref_l = oracle_rows(inp)
+    compare(out, lse, ref_o, ref_l, dt, what=f"case {case}")
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("split_kv", [1, 2, 3, 7, 10 ** 6])
+def test_forced_splits_agree(split_kv, kernel):
+    inp = make_inputs_custom(2, 4, 32, "bf16", [1500, 640], seed=7, pool=2.0, kv_std=0.5)
+    out, lse, status, dec = run(inp, kernel, split_kv=split_kv)
+    assert status == 0
+    ref_o, ref_l = oracle_rows(inp)
+    compare(out, lse, ref_o, ref_l, "bf16", what=f"split {dec.plan.split_kv}")
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_fold_on_and_off_agree(kernel):
+    inp = make_inputs_custom(2, 4, 16, "fp16", [333, 1200], seed=8, pool=2.0)
+    ref_o, ref_l = oracle_rows(inp)
+    for fold in (1, 2, 4):
+        out, lse, status, dec = run(inp, kernel, fold=fold)
+        assert dec.plan.fold == fold and status == 0
+        compare(out, lse, ref_o, ref_l, "fp16", what=f"fold {fold}")
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_page_shuffle_is_bitwise_invariant(kernel):
+    inp = make_inputs_custom(2, 4, 32, "fp8", [777, 2000], seed=9, pool=2.0)
+    out1, lse1, _, _ = run(inp, kernel)
+    perm = torch.randperm(inp.num_pages, generator=torch.Generator().manual_seed(3))
+    inv = torch.empty_like(perm)
+    inv[perm] = torch.arange(inp.num_pages)
+    moved = make_inputs_custom(2, 4, 32, "fp8", [777, 2000], seed=9, pool=2.0)
+    moved.kv_cache = inp.kv_cache[perm].clone()
+    bt = inp.block_tables.clone()
+    bt[bt >= 0] = inv[bt[bt >= 0].long()].to(torch.int32)
+    moved.block_tables = bt
+    out2, lse2, _, _ = run(moved, kernel)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    assert torch.equal(lse1, lse2)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_keys_past_the_causal_limit_do_not_matter(kernel):
+    T, H = 4, 32
+    inp = make_inputs_custom(1, T, H, "bf16", [300], seed=10)
+    out1, lse1, _, _ = run(inp, kernel)
+    # key 298 is visible only to tokens 2 and 3 (limits 296, 297, 298, 299)
+    pert = make_inputs_custom(1, T, H, "bf16", [300], seed=10)
+    page = int(pert.block_tables[0, 298 // 64])
+    pert.kv_cache[page, 298 % 64] = 7.0
+    out2, lse2, _, _ = run(pert, kernel)
+    assert torch.equal(out1[:, :2], out2[:, :2]) and torch.equal(lse1[:, :2], lse2[:, :2])
+    assert not torch.equal(out1[:, 2:], out2[:, 2:])
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_lse_optional(kernel):
+    inp = make_inputs_custom(1, 2, 16, "bf16", [500], seed=11)
+    out1, _, _, _ = run(inp, kernel, want_lse=False)
+    out2, _, _, _ = run(inp, kernel)
+    assert torch.equal(out1, out2)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_cuda_graph_replay_matches_eager(kernel):
+    dev = torch.device("cuda", 0)
+    inp = make_inputs_custom(2, 4, 32, "bf16", [900, 2100], seed=12, pool=2.0).to(dev)
+    dec = mla.MlaDecoder(2, 4, 32, 2100, "bf16", dev, kernel=kernel)
+    out = torch.empty(2, 4, 32, 512, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(2, 4, 32, dtype=torch.float32, device=dev)
+    dec(inp.q, inp.kv_cache, inp.block_tables, inp.seq_lens, inp.softmax_scale, out=out, lse=lse)
+    torch.cuda.synchronize()
+    eager_o, eager_l = out.clone(), lse.clone()
+    out.zero_()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        dec(inp.q, inp.kv_cache, inp.block_tables, inp.seq_lens, inp.softmax_scale, out=out, lse=lse)
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, eager_o) and torch.equal(lse, eager_l)
+    del g
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_status_word_flags_bad_pages_and_long_sequences(kernel):
+    inp = make_inputs_custom(2, 1, 16, "bf16", [200, 100], seed=13, pool=1.0)
+    inp.block_tables[1, 0] = inp.num_pages + 5          # outside the pool
+    _, _, status, _ = run(inp, kernel)
+    assert status & mla.MLA_DEV_BAD_PAGE
+    inp2 = make_inputs_custom(1, 1, 16, "bf16", [200], seed=14, pool=1.0)
+    dev = torch.device("cuda", 0)
+    g = inp2.to(dev)
+    dec = mla.MlaDecoder(1, 1, 16, 100, "bf16", dev, kernel=kernel)   # planned for 100 keys
+    out, lse = dec(g.q, g.kv_cache, g.block_tables, g.seq_lens, g.softmax_scale)
+    torch.cuda.synchronize()
+    assert dec.status() & mla.MLA_DEV_SEQ_TOO_LONG
+    assert torch.isfinite(out.float()).all()
+    # a clean call clears the word again
+    g.seq_lens.fill_(90)
+    dec(g.q, g.kv_cache, g.block_tables, g.seq_lens, g.softmax_scale)
+    assert dec.status() == 0
+
+
+def test_batch_zero_is_a_no_op():
+    dev = torch.device("cuda", 0)
+    dec = mla.MlaDecoder(0, 1, 16, 0, "bf16", dev)
+    q = torch.empty(0, 1, 16, 576, dtype=torch.bfloat16, device=dev)
+    cache = torch.zeros(1, 64, 576, dtype=torch.bfloat16, device=dev)
+    bt = torch.zeros(0, 1, dtype=torch.int32, device=dev)
+    sl = torch.zeros(0, dtype=torch.int32, device=dev)
+    out, lse = dec(q, cache, bt, sl, 0.04)
+    torch.cuda.synchronize()
+    assert out.numel() == 0 and dec.status() == 0
+
+
+FULL = ["tiny_bf16", "mtp_bf16", "fp8_long_b4", "fp8_long_b16", "fold_fp16_h16", "fold_fp16_h64",
+        "highconc_bf16"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_workloads(name):
+    """Automatic plan (what the bench times); every row for the small ones, sampled rows otherwise."""
+    dev = torch.device("cuda", 0)
+    inp = make_inputs(name, device=dev)
+    out, lse, status, dec = run(inp)
+    assert status == 0
+    B, T, H = inp.batch, inp.q_len, inp.heads
+    rows = None if B * T * H * inp.max_seq_len <= 512 * 8192 else sample_rows(B, T, H, n=48)
+    ref_o, ref_l = oracle_rows(inp, rows)
+    compare(out, lse, ref_o, ref_l, inp.dtype, rows=rows, what=name)
+    # properties that hold at any size: finite outputs, LSE bounded by the closed form
+    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()

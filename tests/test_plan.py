@@ -1,0 +1,95 @@
+"""Host plan: fold factor, split_kv and workspace sizing (CPU only)."""
+import math
+
+import pytest
+
+import mla_paged_decode_04_b200 as mla
+from mla_paged_decode_04_b200.inputs import WORKLOADS
+
+
+def _fold_rule(q_len, heads):
+    # Largest F with q_len % F == 0 and H*F <= 128 (TokenSpeed MLA article, section 三).
+    return max(f for f in range(1, q_len + 1) if q_len % f == 0 and heads * f <= 128)
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_fold_per_workload(name):
+    w = WORKLOADS[name]
+    p = mla.mla_decode_plan(w.batch, w.q_len, w.heads, w.max_seq_len, w.dtype)
+    assert p.fold == _fold_rule(w.q_len, w.heads)
+    assert p.q_groups * p.fold == w.q_len and p.rows_per_unit == w.heads * p.fold <= 128
+
+
+def test_fold_examples_from_the_article():
+    # H=64, q_len=4 folds F=2 (H_eff=128, two query groups); section 三's example.
+    p = mla.mla_decode_plan(32, 4, 64, 65536, "fp16")
+    assert (p.fold, p.q_groups, p.rows_per_unit) == (2, 2, 128)
+    assert mla.mla_decode_plan(32, 4, 16, 65536, "fp16").fold == 4
+    assert mla.mla_decode_plan(4, 4, 32, 8192, "bf16").fold == 4
+    assert mla.mla_decode_plan(128, 2, 128, 81920, "bf16").fold == 1
+    assert mla.mla_decode_plan(1, 3, 48, 100, "bf16").fold == 1   # 48*3 > 128
+    assert mla.mla_decode_plan(1, 6, 20, 100, "bf16").fold == 6   # 120 <= 128
+
+
+@pytest.mark.parametrize("batch,q_len,heads,n", [(1, 1, 16, 256), (4, 4, 32, 8192), (4, 4, 32, 81920),
+                                                  (16, 4, 32, 81920), (32, 4, 64, 65536),
+                                                  (128, 2, 128, 81920), (3, 1, 8, 1), (2, 2, 2, 0)])
+def test_split_covers_all_keys(batch, q_len, heads, n):
+    p = mla.mla_decode_plan(batch, q_len, heads, n, "bf16")
+    tiles = math.ceil(n / 64)
+    assert p.keys_per_split % 64 == 0 and p.keys_per_split >= 64
+    assert p.split_kv * p.keys_per_split >= n
+    assert 1 <= p.split_kv <= max(1, tiles)
+    # no empty trailing split
+    assert (p.split_kv - 1) * p.keys_per_split < max(n, 1)
+
+
+def test_workspace_holds_the_partials():
+    for (b, t, h, n) in [(4, 4, 32, 81920), (16, 4, 32, 81920), (1, 1, 16, 256)]:
+        p = mla.mla_decode_plan(b, t, h, n, "fp8")
+        rows = b * t * h
+        if p.split_kv > 1:
+            assert p.partial_offset >= 256 and p.partial_offset % 256 == 0
+            assert p.lse_offset >= p.partial_offset + rows * p.split_kv * 512 * 4
+            assert p.workspace_bytes >= p.lse_offset + rows * p.split_kv * 4
+        assert p.workspace_bytes >= 256 and p.workspace_bytes % 256 == 0
+
+
+def test_split_fills_the_gpu_for_the_long_fp8_case():
+    p4 = mla.mla_decode_plan(4, 4, 32, 81920, "fp8")
+    assert p4.split_kv * 4 <= 74 and p4.split_kv * 4 >= 60  # one wave of CTA pairs
+    p16 = mla.mla_decode_plan(16, 4, 32, 81920, "fp8")
+    waves = math.ceil(p16.split_kv * 16 / 74)
+    assert p16.split_kv * 16 / (waves * 74) > 0.85  # little wave quantisation
+
+
+def test_plan_is_deterministic_and_forced_values_apply():
+    a = mla.mla_decode_plan(4, 4, 32, 8192, "bf16").as_dict()
+    b = mla.mla_decode_plan(4, 4, 32, 8192, "bf16").as_dict()
+    assert a == b
+    p = mla.mla_decode_plan_custom(4, 4, 32, 8192, "bf16", split_kv=3)
+    assert p.split_kv == 3 and p.keys_per_split == 64 * math.ceil(128 / 3)
+    p = mla.mla_decode_plan_custom(4, 4, 32, 8192, "bf16", split_kv=10 ** 6)
+    assert p.split_kv == 128 and p.keys_per_split == 64
+    p = mla.mla_decode_plan_custom(4, 4, 32, 8192, "bf16", fold=2)
+    assert (p.fold, p.q_groups, p.rows_per_unit) == (2, 2, 64)
+    p = mla.mla_decode_plan_custom(4, 4, 32, 8192, "bf16", kernel="simt")
+    assert p.kernel == 2
+
+
+@pytest.mark.parametrize("args,code", [
+    ((-1, 1, 16, 10, "bf16"), -1), ((1, 0, 16, 10, "bf16"), -1), ((1, 1, 0, 10, "bf16"), -1),
+    ((1, 1, 16, -5, "bf16"), -1), ((1, 1, 16, 10, 7), -1), ((1, 1, 129, 10, "bf16"), -2),
+])
+def test_plan_errors(args, code):
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_decode_plan(*args)
+    assert e.value.code == code
+
+
+def test_forced_fold_must_divide():
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_decode_plan_custom(1, 4, 16, 10, "bf16", fold=3)
+    assert e.value.code == -2
+    with pytest.raises(mla.MlaError):
+        mla.mla_decode_plan_custom(1, 4, 64, 10, "bf16", fold=4)  # 256 rows
