@@ -25,9 +25,22 @@ __global__ void __launch_bounds__(256) simt_partial_kernel(const DecodeArgs a) {
   const int b = idx / S;
   const int n = effective_seq_len(a, b, s == 0 && g == 0 && threadIdx.x == 0);
   const int key0 = s * p.keys_per_split;
-  if (key0 >= n) return;
-  const int key1 = min(n, key0 + p.keys_per_split);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (key0 >= n) {
+    // Only split 0 can be empty-and-final: with one split the outputs are
+    // written here, so an entry without keys still gets out = 0, lse = -inf.
+    // (With several splits the combine kernel writes those rows.)
+    if (S == 1) {
+      for (int m = warp; m < M; m += 8) {
+        const int64_t row = (int64_t)b * T * H + (int64_t)g * M + m;
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + row * MLA_D_V;
+        for (int i = lane; i < MLA_D_V; i += 32) out[i] = __float2bfloat16_rn(0.f);
+        if (a.lse && lane == 0) a.lse[row] = -INFINITY;
+      }
+    }
+    return;
+  }
+  const int key1 = min(n, key0 + p.keys_per_split);
   const int32_t* table = a.block_tables + (int64_t)b * a.max_pages_per_seq;
 
   for (int m = warp; m < M; m += 8) {
