@@ -46,6 +46,8 @@ def parse_args():
     ap.add_argument("--kernel", default="auto", choices=["auto", "tcgen05", "simt"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--clock-window-s", type=float, default=1.5,
+                    help="seconds of untimed decode steps run while clocks are sampled")
     return ap.parse_args()
 
 
@@ -200,7 +202,7 @@ def run_ours(args):
     sampler = ClockSampler(local)
     sampler.start()
     # keep the GPU busy for ~1.5 s so the clock samples see the kernel under load
-    t_end = time.perf_counter() + 1.5
+    t_end = time.perf_counter() + args.clock_window_s
     while time.perf_counter() < t_end:
         for _ in range(20):
             flush.zero_()

@@ -99,7 +99,7 @@ int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, i
   }
   const int G = q_len / F;
   const int M = num_heads * F;
-  const int kern = kernel == MLA_KERNEL_AUTO ? MLA_KERNEL_SIMT : kernel;
+  const int kern = kernel == MLA_KERNEL_AUTO ? MLA_KERNEL_TCGEN05 : kernel;
   const int64_t units = (int64_t)batch * G;
   const int64_t tiles = ceil_div(max_seq_len, kTileKeys);
   // The tcgen05 kernel runs one CTA pair per two SMs; the SIMT kernel uses

@@ -16,7 +16,7 @@ from helpers import compare, oracle_rows, sample_rows
 
 pytestmark = pytest.mark.gpu
 
-KERNELS = ["simt"]
+KERNELS = ["tcgen05", "simt"]
 
 
 def run(inp, kernel="auto", split_kv=0, fold=0, want_lse=True):
