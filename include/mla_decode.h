@@ -48,6 +48,7 @@ extern "C" {
 #define MLA_D_V 512         /* V = first 512 dims of the cached row */
 #define MLA_PAGE_SIZE 64    /* tokens per cache page (the only page size supported) */
 #define MLA_MAX_ROWS 128    /* rows (heads x folded tokens) one CTA pair processes */
+#define MLA_NO_ALLOC_SCRATCH_BYTES (32u << 20) /* scratch of mla_decode_no_alloc, per device */
 
 typedef enum { MLA_BF16 = 0, MLA_FP16 = 1, MLA_FP8_E4M3 = 2 } mla_dtype;
 
@@ -181,6 +182,33 @@ int mla_decode_combine(const mla_plan* plan, const void* q, const void* kv_cache
  * tooling; it blocks. Errors: MLA_ERR_INVALID_ARG, MLA_ERR_CUDA.
  */
 int mla_decode_status(void* workspace, void* stream, int clear, int32_t* device_status);
+
+/*
+ * mla_decode_no_alloc: mla_decode without a caller-provided workspace, for
+ * callers that cannot allocate device memory (no counterpart on the pages:
+ * an addition of this library). Examples: a plugin inside a serving engine
+ * that has reserved all device memory for its own pool and gives its kernels
+ * no allocator, or code where cudaMalloc is not allowed because it may
+ * synchronise the device. The workspace is instead a scratch array of
+ * MLA_NO_ALLOC_SCRATCH_BYTES in this library's own device memory, reserved on
+ * every GPU that loads the library and held until the process exits; the
+ * call itself allocates nothing (no cudaMalloc, no cudaFree).
+ *   - Arguments, layouts and errors as mla_decode, minus workspace and
+ *     workspace_bytes. A plan whose workspace_bytes exceeds
+ *     MLA_NO_ALLOC_SCRATCH_BYTES is rejected with MLA_ERR_WORKSPACE_TOO_SMALL
+ *     before anything is enqueued (use fewer splits or mla_decode).
+ *   - The first call on a device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture on the device.
+ *   - Every call on a device shares the one scratch array and it keeps the
+ *     last call's contents: calls that overlap on the GPU (different streams
+ *     without ordering) race on it and must not be issued. The status word
+ *     it holds is reset by each call.
+ */
+int mla_decode_no_alloc(const mla_plan* plan, const void* q, const void* kv_cache,
+                        int64_t num_pages, int page_size, const int32_t* block_tables,
+                        int max_pages_per_seq, const int32_t* seq_lens, float softmax_scale,
+                        float q_scale, float kv_scale, void* out, float* lse, void* stream);
 
 /* Human-readable name of an mla_status code (static storage, never NULL). */
 const char* mla_status_string(int code);

@@ -24,7 +24,9 @@ KERNELS = {"auto": MLA_KERNEL_AUTO, "tcgen05": MLA_KERNEL_TCGEN05, "simt": MLA_K
 MLA_DEV_BAD_PAGE, MLA_DEV_SEQ_TOO_LONG, MLA_DEV_TIMEOUT = 0x1, 0x2, 0x4
 
 EXPORTED = ["mla_decode_plan", "mla_decode_plan_custom", "mla_decode", "mla_decode_partial",
-            "mla_decode_combine", "mla_decode_status", "mla_status_string", "mla_version"]
+            "mla_decode_combine", "mla_decode_status", "mla_status_string", "mla_version",
+            "mla_decode_no_alloc"]
+MLA_NO_ALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class MlaPlan(ctypes.Structure):

@@ -1,0 +1,58 @@
+// Decode entry point for callers that cannot allocate device memory.
+//
+// mla_decode needs a workspace (status word plus the split-KV partials) that
+// the caller allocates. Some callers cannot do that: a plugin inside a
+// serving engine that has reserved all device memory for its own pool and
+// offers its kernels no allocator, or code running where cudaMalloc is not
+// allowed (it may synchronise the device, which a latency-critical decode loop
+// or another library's critical section must not do). mla_decode_no_alloc
+// serves them with a scratch buffer that lives in this library's own device
+// memory: a file-scope array of MLA_NO_ALLOC_SCRATCH_BYTES, reserved on every
+// GPU that loads the library and held until the process exits.
+//
+// The array's name is only a host-side stand-in; its device address is looked
+// up once per device with cudaGetSymbolAddress (with that device current, on
+// the first call on the device) and then passed to the kernels like any
+// workspace. Nothing here calls cudaMalloc or cudaFree.
+#include <mutex>
+
+#include "internal.h"
+
+namespace {
+
+__device__ __align__(256) unsigned char g_no_alloc_scratch[MLA_NO_ALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void* g_scratch_ptr[kMaxDevices] = {nullptr};
+
+// Device address of the scratch array on the current device (looked up once).
+int scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_no_alloc_scratch) != cudaSuccess || p == nullptr) return MLA_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" int mla_decode_no_alloc(const mla_plan* plan, const void* q, const void* kv_cache,
+                                   int64_t num_pages, int page_size, const int32_t* block_tables,
+                                   int max_pages_per_seq, const int32_t* seq_lens, float softmax_scale,
+                                   float q_scale, float kv_scale, void* out, float* lse, void* stream) {
+  if (!plan) return MLA_ERR_PLAN_MISMATCH;
+  if (plan->workspace_bytes > (uint64_t)MLA_NO_ALLOC_SCRATCH_BYTES) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = nullptr;
+  const int rc = scratch_address(&scratch);
+  if (rc != MLA_OK) return rc;
+  return mla_decode(plan, q, kv_cache, num_pages, page_size, block_tables, max_pages_per_seq, seq_lens,
+                    softmax_scale, q_scale, kv_scale, out, lse, scratch, (uint64_t)MLA_NO_ALLOC_SCRATCH_BYTES,
+                    stream);
+}
