@@ -115,7 +115,13 @@ int prepare(const mla_plan* plan, const void* q, const void* kv_cache, int64_t n
 int run_partial(const DecodeArgs& a, cudaStream_t st) {
   if (cudaMemsetAsync(a.status, 0, sizeof(int32_t), st) != cudaSuccess) return MLA_ERR_CUDA;
   if (a.plan.batch == 0) return MLA_OK;
-  cudaError_t e = (a.plan.kernel == MLA_KERNEL_SIMT) ? launch_simt_partial(a, st) : launch_tc_partial(a, st);
+  cudaError_t e;
+  if (a.plan.kernel == MLA_KERNEL_SIMT)
+    e = launch_simt_partial(a, st);
+  else if (a.plan.dtype == MLA_FP8_E4M3)
+    e = launch_tc_fp8_partial(a, st);
+  else
+    e = launch_tc_partial(a, st);
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

@@ -35,7 +35,8 @@ int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, i
               int fold, int kernel, mla_plan* plan);
 
 cudaError_t launch_simt_partial(const DecodeArgs& a, cudaStream_t stream);
-cudaError_t launch_tc_partial(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_tc_partial(const DecodeArgs& a, cudaStream_t stream);      // 16-bit inputs
+cudaError_t launch_tc_fp8_partial(const DecodeArgs& a, cudaStream_t stream);  // FP8 E4M3 inputs
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t stream);
 
 }  // namespace mla

@@ -1,0 +1,99 @@
+// Helpers shared by the tensor-core partial kernels: bounded waits, tensor
+// maps over [rows, 576] arrays, and the epilogue store of a 32-column chunk.
+#pragma once
+
+#include <cuda.h>
+
+#include "device_common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace mla {
+
+constexpr uint64_t kWaitLimitNs = 500ull * 1000 * 1000;  // per wait: 0.5 s
+
+// Bounded wait on an mbarrier phase. Returns false (after setting the abort
+// flag and MLA_DEV_TIMEOUT) when the limit passes, or when another role of
+// the CTA has already aborted.
+__device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                             int32_t* status) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((it & 127) == 0) {
+      if (*abort_flag) return false;
+      if (ptx::globaltimer() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        atomicOr(status, MLA_DEV_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Warp-uniform bounded wait: every lane waits (and so acquires); the warp
+// goes on only if all lanes saw the phase complete.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int32_t* status) {
+  const bool ok = bounded_wait(bar, parity, abort_flag, status);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void spin_ns(uint64_t ns) {
+  const uint64_t t0 = ptx::globaltimer();
+  while (ptx::globaltimer() - t0 < ns) {
+  }
+}
+
+// Before the producer returns: wait (bounded, even after an abort) for the
+// loads it issued into the last `stages` stages, so no copy lands after exit.
+__device__ __forceinline__ void drain_loads(uint32_t full_bar0, int stages, int n_tiles) {
+  for (int j = n_tiles - stages; j < n_tiles; ++j) {
+    if (j < 0) continue;
+    const uint32_t bar = full_bar0 + 8u * (uint32_t)(j % stages);
+    const uint64_t t0 = ptx::globaltimer();
+    while (!ptx::mbar_try_wait(bar, (j / stages) & 1) && ptx::globaltimer() - t0 < kWaitLimitNs) {
+    }
+  }
+}
+
+// Write 32 output columns [col, col + 32) of flat row `rg`: BF16 to `out`
+// when there is one split, else fp32 to the split's partial. inv = 0 means the
+// row saw no key (written as exact zeros).
+__device__ __forceinline__ void store_out_chunk(const DecodeArgs& a, int64_t rg, int s, int col,
+                                                const uint32_t (&o)[32], float inv) {
+  const int S = a.plan.split_kv;
+  if (S == 1) {
+    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + rg * MLA_D_V + col);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      uint32_t pk[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float f0 = inv > 0.f ? __uint_as_float(o[8 * u + 2 * k]) * inv : 0.f;
+        const float f1 = inv > 0.f ? __uint_as_float(o[8 * u + 2 * k + 1]) * inv : 0.f;
+        __nv_bfloat162 hb = __floats2bfloat162_rn(f0, f1);
+        pk[k] = *reinterpret_cast<uint32_t*>(&hb);
+      }
+      dst[u] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+  } else {
+    float4* dst = reinterpret_cast<float4*>(a.o_part + (rg * S + s) * MLA_D_V + col);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      float4 f;
+      f.x = inv > 0.f ? __uint_as_float(o[4 * u + 0]) * inv : 0.f;
+      f.y = inv > 0.f ? __uint_as_float(o[4 * u + 1]) * inv : 0.f;
+      f.z = inv > 0.f ? __uint_as_float(o[4 * u + 2]) * inv : 0.f;
+      f.w = inv > 0.f ? __uint_as_float(o[4 * u + 3]) * inv : 0.f;
+      dst[u] = f;
+    }
+  }
+}
+
+// 2-D tensor map over a row-major [rows, 576] array of 1- or 2-byte elements
+// (q or the cache viewed as [num_pages * 64, 576]); box = box_x x box_y.
+bool encode_rows_576(CUtensorMap* m, const void* base, int esize, uint64_t rows, uint32_t box_x, uint32_t box_y,
+                     CUtensorMapSwizzle sw);
+
+}  // namespace mla

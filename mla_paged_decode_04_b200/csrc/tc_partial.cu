@@ -31,6 +31,7 @@
 
 #include "device_common.cuh"
 #include "sm100_ptx.cuh"
+#include "tc_common.cuh"
 
 namespace mla {
 namespace {
@@ -97,39 +98,11 @@ struct Bar {
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kOCol = 0;      // O: columns [0, 256)
 constexpr uint32_t kSCol = 256;    // S buffers: [256, 320) and [320, 384)
-constexpr uint64_t kWaitNs = 500ull * 1000 * 1000;  // per-wait limit: 0.5 s
 
 struct TcParams {
   CUtensorMap tm_q_main, tm_q_rope, tm_kv_main, tm_kv_rope;
   DecodeArgs a;
 };
-
-// Bounded wait on an mbarrier phase. Returns false (and sets the abort flag
-// and the device status word) when the limit passes or another role aborted.
-__device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                             int32_t* status) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 127) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer() - t0 > kWaitNs) {
-        *abort_flag = 1;
-        atomicOr(status, MLA_DEV_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
-
-// Warp-uniform bounded wait: every lane waits (and so acquires); the warp
-// proceeds only if all lanes saw the phase complete.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int32_t* status) {
-  bool ok = bounded_wait(bar, parity, abort_flag, status);
-  return __all_sync(0xffffffffu, ok);
-}
 
 // P for 32 keys of a row, packed for the tensor core, plus two sums: the
 // exact fp32 sum of the weights (for the LSE) and the sum of the weights as
@@ -298,14 +271,7 @@ __global__ void __launch_bounds__(192, 1) tc_partial_kernel(const __grid_constan
         tma_load_2d(stage + C::STAGE_MAIN, &prm.tm_kv_rope, 512 + 32 * (int)c, page * kTileKeys,
                     bar(B::K_FULL + st), pol_kv);
       }
-      // wait (bounded, regardless of an abort) for our own loads in flight
-      const int last = n_tiles - 1;
-      for (int j = max(0, last - C::NS + 1); j <= last; ++j) {
-        const int st = j % C::NS;
-        const uint64_t t0 = globaltimer();
-        while (!mbar_try_wait(bar(B::K_FULL + st), (j / C::NS) & 1) && globaltimer() - t0 < kWaitNs) {
-        }
-      }
+      drain_loads(bar(B::K_FULL), C::NS, n_tiles);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -589,48 +555,10 @@ __global__ void __launch_bounds__(192, 1) tc_partial_kernel(const __grid_constan
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    if (*abort_flag) {
-      // let any MMA still in flight finish before TMEM is released
-      const uint64_t t0 = globaltimer();
-      while (globaltimer() - t0 < 1000000ull) {
-      }
-    }
+    if (*abort_flag) spin_ns(1000000ull);  // let any MMA still in flight finish
     tmem_dealloc(tmem, kTmemCols);
   }
   cluster_sync();
-}
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
-// 2-D map over a [rows, 576] row-major array of 1- or 2-byte elements.
-bool encode_2d(CUtensorMap* m, const void* base, int esize, uint64_t rows, uint32_t box_x, uint32_t box_y,
-               CUtensorMapSwizzle sw) {
-  EncodeTiledFn enc = get_encode();
-  if (!enc) return false;
-  const cuuint64_t dims[2] = {MLA_D_QK, rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)MLA_D_QK * esize};
-  const cuuint32_t box[2] = {box_x, box_y};
-  const cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
-                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
 }
 
 template <int DT>
@@ -642,11 +570,11 @@ cudaError_t launch_dt(const DecodeArgs& a, cudaStream_t stream) {
   const uint64_t q_rows = (uint64_t)p.batch * p.q_len * p.num_heads;
   const uint64_t kv_rows = (uint64_t)a.num_pages * kTileKeys;
   const CUtensorMapSwizzle rope_sw = C::E == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
-  if (!encode_2d(&prm.tm_q_main, a.q, C::E, q_rows, C::CHUNK_ELEMS, p.rows_per_unit, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_2d(&prm.tm_q_rope, a.q, C::E, q_rows, 32, p.rows_per_unit, rope_sw) ||
-      !encode_2d(&prm.tm_kv_main, a.kv_cache, C::E, kv_rows, C::CHUNK_ELEMS, kTileKeys,
+  if (!encode_rows_576(&prm.tm_q_main, a.q, C::E, q_rows, C::CHUNK_ELEMS, p.rows_per_unit, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_rows_576(&prm.tm_q_rope, a.q, C::E, q_rows, 32, p.rows_per_unit, rope_sw) ||
+      !encode_rows_576(&prm.tm_kv_main, a.kv_cache, C::E, kv_rows, C::CHUNK_ELEMS, kTileKeys,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_2d(&prm.tm_kv_rope, a.kv_cache, C::E, kv_rows, 32, kTileKeys, rope_sw))
+      !encode_rows_576(&prm.tm_kv_rope, a.kv_cache, C::E, kv_rows, 32, kTileKeys, rope_sw))
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
@@ -678,7 +606,7 @@ cudaError_t launch_tc_partial(const DecodeArgs& a, cudaStream_t stream) {
   switch (a.plan.dtype) {
     case MLA_BF16: return launch_dt<MLA_BF16>(a, stream);
     case MLA_FP16: return launch_dt<MLA_FP16>(a, stream);
-    default: return launch_dt<MLA_FP8_E4M3>(a, stream);
+    default: return cudaErrorInvalidValue;  // FP8 has its own kernel
   }
 }
 
