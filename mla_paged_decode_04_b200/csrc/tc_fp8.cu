@@ -48,46 +48,57 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kNS = 4;                     // cache-page stages
 constexpr int kTwoTermKeys = 16384;        // entries shorter than this use two-term P
 constexpr float kTau = 2.f;                // lazy-rescale threshold (log2 units)
 constexpr float kSigma = 6.f;              // P <= 2^(kTau + kSigma) = 256 <= 448
 
-// shared memory (bytes from a 1024-aligned base)
-constexpr uint32_t kQRope = 0;                              // 128 rows x 64 B (SW64)
-constexpr uint32_t kStage0 = 8192;                          // stages: 4 x 8 KB main (SW128) + 4 KB rope (SW64)
-constexpr uint32_t kStageMain = 4 * 8192;
-constexpr uint32_t kStageBytes = kStageMain + 64 * 64;      // 36 KB
-constexpr uint32_t kPOff = kStage0 + kNS * kStageBytes;     // P[2 buffers][2 planes][128 rows x 64 B]
-constexpr uint32_t kPPlane = 128 * 64;
-constexpr uint32_t kPBuf = 2 * kPPlane;
-constexpr uint32_t kMOff = kPOff + 2 * kPBuf;               // row reference maxima [2 tile parities][128]
-constexpr uint32_t kFinOff = kMOff + 1024;                  // final (l, m) per group [2][2][128]
-constexpr uint32_t kBarOff = kFinOff + 2048;
-// Q latent dims are staged (TMA, SW128, 4 chunks of 128 rows x 128 B) in the
-// P buffers (chunks 0, 1) and the last stage (chunks 2, 3) before either is used.
-constexpr uint32_t kQStage01 = kPOff;
-constexpr uint32_t kQStage23 = kStage0 + (kNS - 1) * kStageBytes;
-constexpr int kNBars = 2 * kNS + 16;
-constexpr uint32_t kMiscOff = kBarOff + 8 * kNBars;
-constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;
-static_assert(kStage0 % 1024 == 0 && kStageBytes % 1024 == 0 && kPOff % 1024 == 0, "alignment");
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+// Each cache page is split over two rings of shared-memory slots: the V ring
+// holds this CTA's half of the 512 latent dims (the V operand of its P.V, and
+// half of K), kept until that P.V completes; the K ring holds the other half
+// plus the 64 rope dims, freed as soon as S = Q.K^T has been computed. A K
+// slot is held for about the load latency, a V slot for that plus the
+// softmax, so splitting the page roughly doubles the pages in flight.
+template <bool kTwo>
+struct Fp8Layout {
+  static constexpr int NK = 4;                                  // K-ring slots
+  static constexpr int NV = kTwo ? 6 : 7;                       // V-ring slots
+  static constexpr uint32_t kQRope = 0;                         // 128 rows x 64 B (SW64)
+  static constexpr uint32_t kPPlane = 128 * 64;                 // one E4M3 plane of P (SW64)
+  static constexpr uint32_t kPBuf = (kTwo ? 2 : 1) * kPPlane;   // hi (and lo) plane
+  static constexpr uint32_t kPOff = 8192;                       // P[2 buffers]
+  static constexpr uint32_t kKSlot = 2 * 8192 + 64 * 64;        // 2 x 8 KB main (SW128) + 4 KB rope (SW64)
+  static constexpr uint32_t kKOff = kPOff + 2 * kPBuf;
+  static constexpr uint32_t kVSlot = 2 * 8192;                  // 2 x 8 KB main (SW128)
+  static constexpr uint32_t kVOff = kKOff + NK * kKSlot;
+  static constexpr uint32_t kMOff = kVOff + NV * kVSlot;        // row reference maxima [2 tile parities][128]
+  static constexpr uint32_t kFinOff = kMOff + 1024;             // final (l, m) per group [2][2][128]
+  static constexpr uint32_t kBarOff = kFinOff + 2048;
+  // Q latent dims are staged (TMA, SW128, 4 chunks of 128 rows x 128 B) in
+  // V slots NV-4 .. NV-1 before those are first filled with a page.
+  static constexpr uint32_t kQStage = kVOff + (NV - 4) * kVSlot;
+  // barriers
+  static constexpr int B_Q_ROPE = 0;
+  static constexpr int B_Q_TMEM = 1;
+  static constexpr int B_Q_MAIN = 2;
+  static constexpr int B_FULL = 3;                 // + V slot: all 36 KB of the page landed
+  static constexpr int B_V_EMPTY = B_FULL + NV;    // + V slot
+  static constexpr int B_K_EMPTY = B_V_EMPTY + NV; // + K slot
+  static constexpr int B_S_FULL = B_K_EMPTY + NK;  // + buffer
+  static constexpr int B_S_EMPTY = B_S_FULL + 2;   // + buffer
+  static constexpr int B_P_FULL = B_S_EMPTY + 2;   // + buffer
+  static constexpr int B_P_EMPTY = B_P_FULL + 2;   // + buffer
+  static constexpr int B_O_DONE = B_P_EMPTY + 2;
+  static constexpr int B_O_FINAL = B_O_DONE + 1;   // completes once, after the last P.V
+  static constexpr int B_M_READY = B_O_FINAL + 1;  // + tile parity: a group published its row maxima
+  static constexpr int B_FIN = B_M_READY + 2;      // both groups published their final (l, m)
+  static constexpr int kNBars = B_FIN + 1;
+  static_assert(8 * kNBars <= 512, "barrier area");
+  static constexpr uint32_t kMiscOff = kBarOff + 512;
+  static constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;
+  static_assert(kKOff % 1024 == 0 && kKSlot % 1024 == 0 && kVOff % 1024 == 0, "alignment");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
 
-// barriers
-constexpr int B_Q_ROPE = 0;
-constexpr int B_Q_TMEM = 1;
-constexpr int B_K_FULL = 2;                 // + stage
-constexpr int B_K_EMPTY = 2 + kNS;          // + stage
-constexpr int B_S_FULL = 2 + 2 * kNS;       // + buffer
-constexpr int B_S_EMPTY = 4 + 2 * kNS;      // + buffer
-constexpr int B_P_FULL = 6 + 2 * kNS;       // + buffer
-constexpr int B_P_EMPTY = 8 + 2 * kNS;      // + buffer
-constexpr int B_O_DONE = 10 + 2 * kNS;
-constexpr int B_Q_MAIN = 11 + 2 * kNS;
-constexpr int B_O_FINAL = 12 + 2 * kNS;     // completes once, after the last P.V
-constexpr int B_M_READY = 13 + 2 * kNS;     // + tile parity: a group published its row maxima
-constexpr int B_FIN = 15 + 2 * kNS;         // both groups published their final (l, m)
 constexpr int kSoftmaxWarps = 8;
 constexpr int kPvWarp = 10;                          // issues P.V (warp 1 issues S = Q.K^T)
 constexpr int kThreads = 32 * (3 + kSoftmaxWarps);
@@ -113,15 +124,22 @@ __device__ __forceinline__ float max32(const float (&x)[32]) {
   return m[0];
 }
 
-__global__ void __launch_bounds__(kThreads, 1) tc_fp8_partial_kernel(const __grid_constant__ Fp8Params prm) {
+// One CTA's work; kTwo selects two-term P and the matching shared-memory layout.
+template <bool kTwo>
+__device__ __forceinline__ void fp8_cta(const Fp8Params& prm, uint8_t* smem_raw) {
+  using L = Fp8Layout<kTwo>;
+  constexpr int NK = L::NK, NV = L::NV;
+  constexpr int B_Q_ROPE = L::B_Q_ROPE, B_Q_TMEM = L::B_Q_TMEM, B_Q_MAIN = L::B_Q_MAIN, B_FULL = L::B_FULL,
+                B_V_EMPTY = L::B_V_EMPTY, B_K_EMPTY = L::B_K_EMPTY, B_S_FULL = L::B_S_FULL,
+                B_S_EMPTY = L::B_S_EMPTY, B_P_FULL = L::B_P_FULL, B_P_EMPTY = L::B_P_EMPTY,
+                B_O_DONE = L::B_O_DONE, B_O_FINAL = L::B_O_FINAL, B_M_READY = L::B_M_READY, B_FIN = L::B_FIN;
   const DecodeArgs& a = prm.a;
   const mla_plan& p = a.plan;
-  extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
-  auto bar = [&](int i) -> uint32_t { return sb + kBarOff + 8u * (uint32_t)i; };
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kMiscOff + 4);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kMiscOff);
+  auto bar = [&](int i) -> uint32_t { return sb + L::kBarOff + 8u * (uint32_t)i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hv = blockIdx.x & 1;  // output-column half of this CTA
@@ -148,17 +166,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fp8_partial_kernel(const __gri
   const int n_tiles = (key1 - key0 + kTileKeys - 1) / kTileKeys;
   const int tile0 = key0 / kTileKeys;
   const int32_t* table = a.block_tables + (int64_t)b * a.max_pages_per_seq;
-  const bool two_term = n < kTwoTermKeys;
+  constexpr bool two_term = kTwo;
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
     mbar_init(bar(B_Q_ROPE), 1);
     mbar_init(bar(B_Q_TMEM), kSoftmaxWarps);
     mbar_init(bar(B_Q_MAIN), 1);
-    for (int i = 0; i < kNS; ++i) {
-      mbar_init(bar(B_K_FULL + i), 1);
-      mbar_init(bar(B_K_EMPTY + i), 2);   // released by both the QK and the P.V issuer
+    for (int i = 0; i < NV; ++i) {
+      mbar_init(bar(B_FULL + i), 1);
+      mbar_init(bar(B_V_EMPTY + i), 1);   // released by the P.V issuer
     }
+    for (int i = 0; i < NK; ++i) mbar_init(bar(B_K_EMPTY + i), 1);  // released by the QK issuer
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(B_S_FULL + i), 1);
       mbar_init(bar(B_S_EMPTY + i), 4);   // one softmax group (4 warps) per tile parity
@@ -174,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fp8_partial_kernel(const __gri
   }
   if (M < 128) {
     // Q rope rows the TMA box does not cover are zero (rows are independent).
-    uint4* rb = reinterpret_cast<uint4*>(smem + kQRope + M * 64);
+    uint4* rb = reinterpret_cast<uint4*>(smem + L::kQRope + M * 64);
     for (int i = threadIdx.x; i < (128 - M) * 4; i += blockDim.x) rb[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
   }
@@ -199,25 +218,30 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fp8_partial_kernel(const __gri
       mbar_arrive_expect_tx(bar(B_Q_MAIN), 4u * 128u * (uint32_t)M);
 #pragma unroll
       for (int ci = 0; ci < 4; ++ci)
-        tma_load_2d((ci < 2 ? sb + kQStage01 : sb + kQStage23) + (ci & 1) * 16384, &prm.tm_q_main, 128 * ci,
+        tma_load_2d(sb + L::kQStage + ci * 16384, &prm.tm_q_main, 128 * ci,
                     (int)row0, bar(B_Q_MAIN), pol_q);
       mbar_arrive_expect_tx(bar(B_Q_ROPE), 64u * (uint32_t)M);
-      tma_load_2d(sb + kQRope, &prm.tm_q_rope, 512, (int)row0, bar(B_Q_ROPE), pol_q);
+      tma_load_2d(sb + L::kQRope, &prm.tm_q_rope, 512, (int)row0, bar(B_Q_ROPE), pol_q);
       for (int j = 0; j < n_tiles; ++j) {
-        const int st = j % kNS;
-        // the last stage holds staged Q until it has been copied into TMEM
-        if (j == kNS - 1 && !bounded_wait(bar(B_Q_TMEM), 0, abort_flag, a.status)) break;
-        if (!bounded_wait(bar(B_K_EMPTY + st), ((j / kNS) & 1) ^ 1, abort_flag, a.status)) break;
+        const int sk = j % NK, sv = j % NV;
+        // V slots NV-4 .. NV-1 hold staged Q until it has been copied into TMEM
+        if (j == NV - 4 && !bounded_wait(bar(B_Q_TMEM), 0, abort_flag, a.status)) break;
+        if (!bounded_wait(bar(B_K_EMPTY + sk), ((j / NK) & 1) ^ 1, abort_flag, a.status)) break;
+        if (!bounded_wait(bar(B_V_EMPTY + sv), ((j / NV) & 1) ^ 1, abort_flag, a.status)) break;
         int page = table[tile0 + j];
         if (page < 0 || (int64_t)page >= a.num_pages) page = 0;  // masked by the softmax warps
-        const uint32_t stage = sb + kStage0 + st * kStageBytes;
-        mbar_arrive_expect_tx(bar(B_K_FULL + st), kStageBytes);
+        const uint32_t vs = sb + L::kVOff + sv * L::kVSlot;
+        const uint32_t ks = sb + L::kKOff + sk * L::kKSlot;
+        const uint32_t full = bar(B_FULL + sv);
+        mbar_arrive_expect_tx(full, L::kVSlot + L::kKSlot);
 #pragma unroll
-        for (int ci = 0; ci < 4; ++ci)
-          tma_load_2d(stage + ci * 8192, &prm.tm_kv_main, 128 * ci, page * kTileKeys, bar(B_K_FULL + st), pol_kv);
-        tma_load_2d(stage + kStageMain, &prm.tm_kv_rope, 512, page * kTileKeys, bar(B_K_FULL + st), pol_kv);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_2d(vs + c * 8192, &prm.tm_kv_main, 128 * (2 * hv + c), page * kTileKeys, full, pol_kv);
+          tma_load_2d(ks + c * 8192, &prm.tm_kv_main, 128 * (2 - 2 * hv + c), page * kTileKeys, full, pol_kv);
+        }
+        tma_load_2d(ks + 16384, &prm.tm_kv_rope, 512, page * kTileKeys, full, pol_kv);
       }
-      drain_loads(bar(B_K_FULL), kNS, n_tiles);
+      drain_loads(bar(B_FULL), NV, n_tiles);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ QK issuer
@@ -228,26 +252,29 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fp8_partial_kernel(const __gri
       constexpr uint32_t idq = instr_desc(0, 0, 0, 128, 64);   // E4M3 x E4M3, K-major B
       bool ok = warp_wait(bar(B_Q_ROPE), 0, abort_flag, a.status) &&
                 warp_wait(bar(B_Q_TMEM), 0, abort_flag, a.status);
-      const uint64_t dq_rope = smem_desc(sb + kQRope, 16, 512, kSw64);
+      const uint64_t dq_rope = smem_desc(sb + L::kQRope, 16, 512, kSw64);
       for (int j = 0; ok && j < n_tiles; ++j) {
-        const int st = j % kNS, buf = j & 1;
-        if (!(ok = warp_wait(bar(B_K_FULL + st), (j / kNS) & 1, abort_flag, a.status))) break;
+        const int sk = j % NK, sv = j % NV, buf = j & 1;
+        if (!(ok = warp_wait(bar(B_FULL + sv), (j / NV) & 1, abort_flag, a.status))) break;
         if (!(ok = warp_wait(bar(B_S_EMPTY + buf), ((j >> 1) & 1) ^ 1, abort_flag, a.status))) break;
         tc_fence_after();
         const uint32_t d = tmem + kSCol + 64u * buf;
-        const uint32_t stage = sb + kStage0 + st * kStageBytes;
-        const uint64_t dk = smem_desc(stage, 16, 1024, kSw128);
-        const uint64_t dr = smem_desc(stage + kStageMain, 16, 512, kSw64);
+        const uint32_t vs = sb + L::kVOff + sv * L::kVSlot;
+        const uint32_t ks = sb + L::kKOff + sk * L::kKSlot;
+        const uint64_t dr = smem_desc(ks + 16384, 16, 512, kSw64);
 #pragma unroll
-        for (int ci = 0; ci < 4; ++ci)
+        for (int ci = 0; ci < 4; ++ci) {
+          // latent chunk ci (dims 128ci ..) sits in the V slot for this CTA's half
+          const uint64_t dk = smem_desc(((ci >> 1) == hv ? vs : ks) + (ci & 1) * 8192, 16, 1024, kSw128);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_f8_ts_e(d, tmem + kQCol + (uint32_t)(8 * (4 * ci + kk)), dk + (uint64_t)((ci * 8192 + kk * 32) >> 4),
-                        idq, (ci | kk) ? 1u : 0u);
+            mma_f8_ts_e(d, tmem + kQCol + (uint32_t)(8 * (4 * ci + kk)), dk + (uint64_t)((kk * 32) >> 4), idq,
+                        (ci | kk) ? 1u : 0u);
+        }
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk) mma_f8_ss_e(d, dq_rope + (uint64_t)(kk * 2), dr + (uint64_t)(kk * 2), idq, 1u);
         mma_commit_e(bar(B_S_FULL + buf));
-        mma_commit_e(bar(B_K_EMPTY + st));
+        mma_commit_e(bar(B_K_EMPTY + sk));
       }
     }
   } else if (warp == kPvWarp) {
@@ -255,24 +282,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fp8_partial_kernel(const __gri
     constexpr uint32_t idp = instr_desc(0, 0, 1, 128, 256);  // V is MN-major
     bool ok = true;
     for (int j = 0; ok && j < n_tiles; ++j) {
-      const int buf = j & 1, st = j % kNS;
+      const int buf = j & 1, sv = j % NV;
       if (!(ok = warp_wait(bar(B_P_FULL + buf), (j >> 1) & 1, abort_flag, a.status))) break;
       tc_fence_after();
-      const uint64_t dv = smem_desc(sb + kStage0 + st * kStageBytes + (uint32_t)(2 * hv) * 8192, 8192, 1024, kSw128);
-      const uint64_t dp = smem_desc(sb + kPOff + buf * kPBuf, 16, 512, kSw64);
+      const uint64_t dv = smem_desc(sb + L::kVOff + sv * L::kVSlot, 8192, 1024, kSw128);
+      const uint64_t dp = smem_desc(sb + L::kPOff + buf * L::kPBuf, 16, 512, kSw64);
 #pragma unroll
       for (int kk = 0; kk < 2; ++kk)
         mma_f8_ss_e(tmem + kOCol, dp + (uint64_t)(kk * 2), dv + (uint64_t)(kk * 256), idp, (j > 0 || kk > 0) ? 1u : 0u);
       if (two_term) {
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk)
-          mma_f8_ss_e(tmem + kOCol, dp + (uint64_t)((kPPlane + kk * 32) >> 4), dv + (uint64_t)(kk * 256), idp, 1u);
+          mma_f8_ss_e(tmem + kOCol, dp + (uint64_t)((L::kPPlane + kk * 32) >> 4), dv + (uint64_t)(kk * 256), idp, 1u);
       }
       // O_DONE first: a softmax group that has seen P_EMPTY of tile j-2 may
       // rely on O_DONE having completed that tile's phase too.
       mma_commit_e(bar(B_O_DONE));
       mma_commit_e(bar(B_P_EMPTY + buf));
-      mma_commit_e(bar(B_K_EMPTY + st));
+      mma_commit_e(bar(B_V_EMPTY + sv));
       if (j == n_tiles - 1) mma_commit_e(bar(B_O_FINAL));
     }
   } else if (warp >= 2 && warp < 2 + kSoftmaxWarps) {
@@ -287,8 +314,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fp8_partial_kernel(const __gri
     const int r = 32 * q + lane;  // this thread's row (= TMEM lane)
     const uint32_t tl = (uint32_t)(32 * q) << 16;
     const int limit = (r < M) ? n - T + g * p.fold + r / H : n - 1;
-    float* mref = reinterpret_cast<float*>(smem + kMOff);   // [tile parity][row]
-    float* fin = reinterpret_cast<float*>(smem + kFinOff);  // [l | m][group][row]
+    float* mref = reinterpret_cast<float*>(smem + L::kMOff);   // [tile parity][row]
+    float* fin = reinterpret_cast<float*>(smem + L::kFinOff);  // [l | m][group][row]
     bool ok = true;
 
     // Q latent dims 0..511 of row r: staged by TMA (SW128 chunks of 128 bytes =
@@ -299,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fp8_partial_kernel(const __gri
 #pragma unroll 1
       for (int c2 = 0; c2 < 2; ++c2) {
         const int cc = 2 * grp + c2;
-        const uint8_t* chunk = smem + (cc < 2 ? kQStage01 : kQStage23) + (cc & 1) * 16384 + r * 128;
+        const uint8_t* chunk = smem + L::kQStage + cc * 16384 + r * 128;
         uint32_t w[32];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -383,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fp8_partial_kernel(const __gri
       // exact fp32 sum normalises O and gives the LSE (E4M3 rounding is
       // unbiased and averages out; short rows use the two-term split).
       float se[4] = {0.f, 0.f, 0.f, 0.f};
-      uint8_t* prow = smem + kPOff + buf * kPBuf + r * 64;
+      uint8_t* prow = smem + L::kPOff + buf * L::kPBuf + r * 64;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         uint32_t hi[4], lo[4];
@@ -404,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fp8_partial_kernel(const __gri
         }
         const int phys = u ^ ((r >> 1) & 3);
         *reinterpret_cast<uint4*>(prow + phys * 16) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        if (two_term) *reinterpret_cast<uint4*>(prow + kPPlane + phys * 16) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        if (two_term) *reinterpret_cast<uint4*>(prow + L::kPPlane + phys * 16) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
       const float sum = (se[0] + se[1]) + (se[2] + se[3]);
       l_grp = (m_grp == m_j) ? l_grp + sum : fmaf(l_grp, ex2_approx(m_grp - m_j), sum);
@@ -485,6 +512,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fp8_partial_kernel(const __gri
   }
 }
 
+static_assert(Fp8Layout<true>::kSmemBytes == Fp8Layout<false>::kSmemBytes, "both variants share one launch");
+
+__global__ void __launch_bounds__(kThreads, 1) tc_fp8_partial_kernel(const __grid_constant__ Fp8Params prm) {
+  extern __shared__ uint8_t smem_raw[];
+  const mla_plan& p = prm.a.plan;
+  const int b = (blockIdx.x >> 1) / (p.q_groups * p.split_kv);
+  // Entries shorter than kTwoTermKeys send P as two E4M3 terms (the choice
+  // is per entry, so it is uniform over the CTA).
+  if (effective_seq_len(prm.a, b, false) < kTwoTermKeys)
+    fp8_cta<true>(prm, smem_raw);
+  else
+    fp8_cta<false>(prm, smem_raw);
+}
+
 }  // namespace
 
 cudaError_t launch_tc_fp8_partial(const DecodeArgs& a, cudaStream_t stream) {
@@ -502,12 +543,12 @@ cudaError_t launch_tc_fp8_partial(const DecodeArgs& a, cudaStream_t stream) {
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(tc_fp8_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(tc_fp8_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Fp8Layout<false>::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  tc_fp8_partial_kernel<<<(unsigned)(2 * pairs), kThreads, kSmemBytes, stream>>>(prm);
+  tc_fp8_partial_kernel<<<(unsigned)(2 * pairs), kThreads, Fp8Layout<false>::kSmemBytes, stream>>>(prm);
   return cudaGetLastError();
 }
 
