@@ -43,7 +43,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="fp8_long_b16")
-    ap.add_argument("--kernel", default="auto", choices=["auto", "tcgen05", "simt"])
+    ap.add_argument("--kernel", default="auto", choices=["auto", "tcgen05", "simt", "tcgen05_solo"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--clock-window-s", type=float, default=1.5,
@@ -227,6 +227,8 @@ def run_ours(args):
         dist.barrier()
     wall1 = time.perf_counter()
     clocks = sampler.stop()
+    if dec.status() != 0:
+        raise RuntimeError("device status word set during the timed steps")
     step_ms = [e0.elapsed_time(e2) for e0, _, e2 in evs]
     part_ms = [e0.elapsed_time(e1) for e0, e1, _ in evs]
     total_ms = sum(step_ms)
@@ -282,7 +284,13 @@ def run_ours(args):
     peak, peak_kind = measured_peak()
     part_avg_s = statistics.mean(part_ms) / 1e3
     achieved = alg_bytes_partial / part_avg_s / 1e9
-    kname = "mla_tc_partial" if plan.kernel == 1 else "mla_simt_partial"
+    # the partial kernel's function name, as ncu lists it
+    if plan.kernel == 2:
+        kname = "simt_partial_kernel"
+    elif g.dtype == "fp8":
+        kname = "tc_fp8_pair_kernel" if plan.kernel == 1 else "tc_fp8_partial_kernel"
+    else:
+        kname = "tc_partial_kernel"
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "peak_source": peak_kind,
                 "traffic": traffic_from_profile(args.workload, kname), "kernel": kname,

@@ -24,7 +24,10 @@
  *     argument errors are detected before anything is enqueued.
  *   - Device pointers are raw CUDA device addresses owned by the caller (in
  *     practice allocated by PyTorch). The library allocates no device memory
- *     and never synchronises the stream in mla_decode.
+ *     and never synchronises the stream in mla_decode. A pointer the current
+ *     device cannot address (pageable host memory, another device's memory)
+ *     is refused with MLA_ERR_INVALID_ARG before anything is enqueued;
+ *     mapped pinned host memory and managed memory are accepted.
  *   - `stream` is a cudaStream_t passed as void*; NULL means the legacy
  *     default stream. All device work is enqueued on it, asynchronously.
  *   - Problems only the device can see (a block-table entry outside
@@ -68,9 +71,12 @@ typedef enum {
 #define MLA_DEV_TIMEOUT 0x4      /* a bounded pipeline wait gave up; outputs unspecified */
 
 typedef enum {
-  MLA_KERNEL_AUTO = 0,    /* the tcgen05 CTA-pair kernel */
-  MLA_KERNEL_TCGEN05 = 1, /* sm_100a tensor-core split-KV kernel (TMA + tcgen05 + TMEM) */
-  MLA_KERNEL_SIMT = 2     /* plain CUDA-core kernel: a slow, simple cross-check */
+  MLA_KERNEL_AUTO = 0,         /* MLA_KERNEL_TCGEN05 */
+  MLA_KERNEL_TCGEN05 = 1,      /* sm_100a tensor-core split-KV kernel (TMA + tcgen05 + TMEM); for FP8 the
+                                  CTA-pair form whose MMAs span both CTAs (cta_group::2) */
+  MLA_KERNEL_SIMT = 2,         /* plain CUDA-core kernel: a slow, simple cross-check */
+  MLA_KERNEL_TCGEN05_SOLO = 3  /* FP8 only: tensor-core kernel whose two CTAs per unit each compute all
+                                  scores and keep half of the output columns (no cross-CTA MMA) */
 } mla_kernel;
 
 /*
@@ -215,6 +221,14 @@ const char* mla_status_string(int code);
 
 /* Library version string, e.g. "0.1.0". */
 const char* mla_version(void);
+
+/*
+ * The CUDA runtime error behind this thread's most recent MLA_ERR_CUDA
+ * (cudaError_t value; 0 if none yet). If `name` is not NULL it receives the
+ * error's name (static storage, e.g. "cudaErrorInvalidValue"). Host only; no
+ * CUDA call is made.
+ */
+int mla_last_cuda_error(const char** name);
 
 #ifdef __cplusplus
 }

@@ -18,14 +18,15 @@ LIB_PATH = os.path.join(_HERE, "libmla_decode.so")
 
 MLA_BF16, MLA_FP16, MLA_FP8_E4M3 = 0, 1, 2
 DTYPES = {"bf16": MLA_BF16, "fp16": MLA_FP16, "fp8": MLA_FP8_E4M3}
-MLA_KERNEL_AUTO, MLA_KERNEL_TCGEN05, MLA_KERNEL_SIMT = 0, 1, 2
-KERNELS = {"auto": MLA_KERNEL_AUTO, "tcgen05": MLA_KERNEL_TCGEN05, "simt": MLA_KERNEL_SIMT}
+MLA_KERNEL_AUTO, MLA_KERNEL_TCGEN05, MLA_KERNEL_SIMT, MLA_KERNEL_TCGEN05_SOLO = 0, 1, 2, 3
+KERNELS = {"auto": MLA_KERNEL_AUTO, "tcgen05": MLA_KERNEL_TCGEN05, "simt": MLA_KERNEL_SIMT,
+           "tcgen05_solo": MLA_KERNEL_TCGEN05_SOLO}
 
 MLA_DEV_BAD_PAGE, MLA_DEV_SEQ_TOO_LONG, MLA_DEV_TIMEOUT = 0x1, 0x2, 0x4
 
 EXPORTED = ["mla_decode_plan", "mla_decode_plan_custom", "mla_decode", "mla_decode_partial",
             "mla_decode_combine", "mla_decode_status", "mla_status_string", "mla_version",
-            "mla_decode_no_alloc"]
+            "mla_decode_no_alloc", "mla_last_cuda_error"]
 MLA_NO_ALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -46,7 +47,12 @@ class MlaPlan(ctypes.Structure):
 
 class MlaError(RuntimeError):
     def __init__(self, code: int, what: str):
-        super().__init__(f"{what} failed: {status_string(code)} ({code})")
+        msg = f"{what} failed: {status_string(code)} ({code})"
+        self.cuda_error = None
+        if code == -5:  # MLA_ERR_CUDA: name the CUDA runtime error behind it
+            self.cuda_error = last_cuda_error()
+            msg += f" [{self.cuda_error[1]} ({self.cuda_error[0]})]"
+        super().__init__(msg)
         self.code = code
 
 
@@ -73,6 +79,8 @@ def _load():
     lib.mla_status_string.restype = ctypes.c_char_p
     lib.mla_version.argtypes = []
     lib.mla_version.restype = ctypes.c_char_p
+    lib.mla_last_cuda_error.argtypes = [ctypes.POINTER(ctypes.c_char_p)]
+    lib.mla_last_cuda_error.restype = i32
     return lib
 
 
@@ -85,6 +93,13 @@ def lib():
 
 def status_string(code: int) -> str:
     return _lib.mla_status_string(int(code)).decode()
+
+
+def last_cuda_error():
+    """(code, name) of the CUDA runtime error behind this thread's last MLA_ERR_CUDA."""
+    name = ctypes.c_char_p()
+    code = _lib.mla_last_cuda_error(ctypes.byref(name))
+    return int(code), (name.value.decode() if name.value else "")
 
 
 def mla_version() -> str:
@@ -126,8 +141,28 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _check_tensors(q, **named):
+    """Every tensor argument is a contiguous CUDA tensor on q's device."""
+    if not (isinstance(q, torch.Tensor) and q.is_cuda):
+        raise ValueError("q must be a CUDA tensor")
+    for k, t in named.items():
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.device != q.device:
+            raise ValueError(f"{k} must be a CUDA tensor on {q.device} (got "
+                             f"{t.device if isinstance(t, torch.Tensor) else type(t).__name__})")
+        if not t.is_contiguous():
+            raise ValueError(f"{k} must be contiguous")
+    for k in ("block_tables", "seq_lens"):
+        t = named.get(k)
+        if t is not None and t.dtype != torch.int32:
+            raise ValueError(f"{k} must be int32")
+
+
 def _call(name, plan, q, kv_cache, block_tables, seq_lens, softmax_scale, out, lse, workspace,
           q_scale, kv_scale, stream):
+    _check_tensors(q, kv_cache=kv_cache, block_tables=block_tables, seq_lens=seq_lens, out=out,
+                   lse=lse, workspace=workspace)
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream if q.is_cuda else 0
     elif isinstance(stream, torch.cuda.Stream):

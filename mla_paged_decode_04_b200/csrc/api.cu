@@ -5,6 +5,16 @@
 #include "internal.h"
 
 namespace mla {
+
+namespace {
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+}  // namespace
+
+int cuda_failure(cudaError_t e) {
+  g_last_cuda_error = e;
+  return MLA_ERR_CUDA;
+}
+
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -14,7 +24,7 @@ int check_device_arch() {
   static int cached[64];
   static bool init = false;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_failure(e);
   if (dev < 0 || dev >= 64) return MLA_ERR_ARCH;
   std::lock_guard<std::mutex> lk(mu);
   if (!init) {
@@ -23,15 +33,32 @@ int check_device_arch() {
   }
   if (cached[dev] == 1) {
     int major = 0, minor = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-      return MLA_ERR_CUDA;
+    if (cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev); e != cudaSuccess)
+      return cuda_failure(e);
+    if (cudaError_t e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev); e != cudaSuccess)
+      return cuda_failure(e);
     cached[dev] = (major == 10 && minor == 0) ? MLA_OK : MLA_ERR_ARCH;
   }
   return cached[dev];
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// The current device can address `ptr`: its own device or managed memory, or
+// host memory mapped into the device address space. A pageable host pointer
+// (or another device's memory) would fault inside a kernel, so it is refused
+// here. A host-side query; nothing is enqueued.
+bool device_addressable(const void* ptr, int dev) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, ptr) != cudaSuccess) {
+    (void)cudaGetLastError();  // not the caller's error to see later
+    return false;
+  }
+  if (at.type == cudaMemoryTypeDevice) return at.device == dev;
+  if (at.type == cudaMemoryTypeManaged) return true;
+  if (at.type == cudaMemoryTypeHost) return at.devicePointer == ptr;
+  return false;
+}
 
 // The plan must be one the planner could have produced for its own fields.
 int check_plan(const mla_plan* p) {
@@ -46,7 +73,9 @@ int check_plan(const mla_plan* p) {
   if (p->split_kv < 1 || p->keys_per_split < kTileKeys || p->keys_per_split % kTileKeys != 0)
     return MLA_ERR_PLAN_MISMATCH;
   if ((int64_t)p->split_kv * p->keys_per_split < (int64_t)p->max_seq_len) return MLA_ERR_PLAN_MISMATCH;
-  if (p->kernel != MLA_KERNEL_TCGEN05 && p->kernel != MLA_KERNEL_SIMT) return MLA_ERR_PLAN_MISMATCH;
+  if (p->kernel != MLA_KERNEL_TCGEN05 && p->kernel != MLA_KERNEL_SIMT && p->kernel != MLA_KERNEL_TCGEN05_SOLO)
+    return MLA_ERR_PLAN_MISMATCH;
+  if (p->kernel == MLA_KERNEL_TCGEN05_SOLO && p->dtype != MLA_FP8_E4M3) return MLA_ERR_PLAN_MISMATCH;
   const uint64_t rows = (uint64_t)p->batch * p->q_len * p->num_heads;
   if (p->split_kv > 1) {
     if (p->partial_offset < (uint64_t)kHeaderBytes || p->partial_offset % 256 != 0 ||
@@ -87,6 +116,13 @@ int prepare(const mla_plan* plan, const void* q, const void* kv_cache, int64_t n
       return MLA_ERR_INVALID_ARG;
     if (num_pages < 1 || max_pages_per_seq < 1) return MLA_ERR_INVALID_ARG;
     if (num_pages > (int64_t(1) << 31) / MLA_PAGE_SIZE) return MLA_ERR_UNSUPPORTED_SHAPE;
+    int dev = 0;
+    if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_failure(e);
+    if (!device_addressable(q, dev) || !device_addressable(kv_cache, dev) ||
+        !device_addressable(block_tables, dev) || !device_addressable(seq_lens, dev) ||
+        !device_addressable(out, dev) || (lse && !device_addressable(lse, dev)) ||
+        !device_addressable(workspace, dev))
+      return MLA_ERR_INVALID_ARG;
   }
   rc = check_device_arch();
   if (rc != MLA_OK) return rc;
@@ -113,21 +149,24 @@ int prepare(const mla_plan* plan, const void* q, const void* kv_cache, int64_t n
 }
 
 int run_partial(const DecodeArgs& a, cudaStream_t st) {
-  if (cudaMemsetAsync(a.status, 0, sizeof(int32_t), st) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaError_t e = cudaMemsetAsync(a.status, 0, sizeof(int32_t), st); e != cudaSuccess) return cuda_failure(e);
   if (a.plan.batch == 0) return MLA_OK;
   cudaError_t e;
   if (a.plan.kernel == MLA_KERNEL_SIMT)
     e = launch_simt_partial(a, st);
-  else if (a.plan.dtype == MLA_FP8_E4M3)
+  else if (a.plan.kernel == MLA_KERNEL_TCGEN05_SOLO)
     e = launch_tc_fp8_partial(a, st);
+  else if (a.plan.dtype == MLA_FP8_E4M3)
+    e = launch_tc_fp8_pair_partial(a, st);
   else
     e = launch_tc_partial(a, st);
-  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return e == cudaSuccess ? MLA_OK : cuda_failure(e);
 }
 
 int run_combine(const DecodeArgs& a, cudaStream_t st) {
   if (a.plan.batch == 0 || a.plan.split_kv == 1) return MLA_OK;
-  return launch_combine(a, st) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  const cudaError_t e = launch_combine(a, st);
+  return e == cudaSuccess ? MLA_OK : cuda_failure(e);
 }
 
 }  // namespace
@@ -171,10 +210,13 @@ extern "C" int mla_decode_combine(MLA_ARGS_DECL) {
 extern "C" int mla_decode_status(void* workspace, void* stream, int clear, int32_t* device_status) {
   if (!workspace || !device_status) return MLA_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaError_t e = cudaStreamSynchronize(st); e != cudaSuccess) return cuda_failure(e);
   int32_t v = 0;
-  if (cudaMemcpy(&v, workspace, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return MLA_ERR_CUDA;
-  if (clear && cudaMemset(workspace, 0, sizeof v) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaError_t e = cudaMemcpy(&v, workspace, sizeof v, cudaMemcpyDeviceToHost); e != cudaSuccess)
+    return cuda_failure(e);
+  if (clear) {
+    if (cudaError_t e = cudaMemset(workspace, 0, sizeof v); e != cudaSuccess) return cuda_failure(e);
+  }
   *device_status = v;
   return MLA_OK;
 }
@@ -193,3 +235,8 @@ extern "C" const char* mla_status_string(int code) {
 }
 
 extern "C" const char* mla_version(void) { return "0.1.0"; }
+
+extern "C" int mla_last_cuda_error(const char** name) {
+  if (name) *name = cudaGetErrorName(g_last_cuda_error);
+  return (int)g_last_cuda_error;
+}

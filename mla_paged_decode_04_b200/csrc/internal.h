@@ -31,12 +31,17 @@ struct DecodeArgs {
   float* lse_part;         // fp32 [B*T*H, S]       (split_kv > 1)
 };
 
+// Records `e` as this thread's last CUDA error (read by mla_last_cuda_error)
+// and returns MLA_ERR_CUDA.
+int cuda_failure(cudaError_t e);
+
 int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, int split_kv,
               int fold, int kernel, mla_plan* plan);
 
 cudaError_t launch_simt_partial(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_tc_partial(const DecodeArgs& a, cudaStream_t stream);      // 16-bit inputs
-cudaError_t launch_tc_fp8_partial(const DecodeArgs& a, cudaStream_t stream);  // FP8 E4M3 inputs
+cudaError_t launch_tc_fp8_partial(const DecodeArgs& a, cudaStream_t stream);  // FP8, per-CTA MMAs
+cudaError_t launch_tc_fp8_pair_partial(const DecodeArgs& a, cudaStream_t stream);  // FP8, CTA-pair MMAs
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t stream);
 
 }  // namespace mla

@@ -29,12 +29,13 @@ void* g_scratch_ptr[kMaxDevices] = {nullptr};
 // Device address of the scratch array on the current device (looked up once).
 int scratch_address(void** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return mla::cuda_failure(e);
   if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_no_alloc_scratch) != cudaSuccess || p == nullptr) return MLA_ERR_CUDA;
+    if (cudaError_t e = cudaGetSymbolAddress(&p, g_no_alloc_scratch); e != cudaSuccess) return mla::cuda_failure(e);
+    if (p == nullptr) return mla::cuda_failure(cudaErrorInvalidSymbol);
     g_scratch_ptr[dev] = p;
   }
   *out = g_scratch_ptr[dev];

@@ -71,8 +71,10 @@ int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, i
   if (batch < 0 || q_len < 1 || num_heads < 1 || max_seq_len < 0 || split_kv < 0 || fold < 0)
     return MLA_ERR_INVALID_ARG;
   if (dtype != MLA_BF16 && dtype != MLA_FP16 && dtype != MLA_FP8_E4M3) return MLA_ERR_INVALID_ARG;
-  if (kernel != MLA_KERNEL_AUTO && kernel != MLA_KERNEL_TCGEN05 && kernel != MLA_KERNEL_SIMT)
+  if (kernel != MLA_KERNEL_AUTO && kernel != MLA_KERNEL_TCGEN05 && kernel != MLA_KERNEL_SIMT &&
+      kernel != MLA_KERNEL_TCGEN05_SOLO)
     return MLA_ERR_INVALID_ARG;
+  if (kernel == MLA_KERNEL_TCGEN05_SOLO && dtype != MLA_FP8_E4M3) return MLA_ERR_INVALID_ARG;
   if (num_heads > MLA_MAX_ROWS) return MLA_ERR_UNSUPPORTED_SHAPE;
   if (max_seq_len > (1 << 30)) return MLA_ERR_UNSUPPORTED_SHAPE;
 

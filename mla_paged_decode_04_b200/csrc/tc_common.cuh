@@ -57,6 +57,14 @@ __device__ __forceinline__ void drain_loads(uint32_t full_bar0, int stages, int 
   }
 }
 
+// Wait (bounded, whatever the abort flag says) for the phase of `bar` with
+// the given parity to complete.
+__device__ __forceinline__ void drain_phase(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = ptx::globaltimer();
+  while (!ptx::mbar_try_wait(bar, parity) && ptx::globaltimer() - t0 < kWaitLimitNs) {
+  }
+}
+
 // Write 32 output columns [col, col + 32) of flat row `rg`: BF16 to `out`
 // when there is one split, else fp32 to the split's partial. inv = 0 means the
 // row saw no key (written as exact zeros).

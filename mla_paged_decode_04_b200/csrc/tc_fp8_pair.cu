@@ -1,0 +1,619 @@
+// Split-KV partial kernel for FP8 E4M3 inputs with CTA-pair tensor-core MMAs.
+//
+// The first of the two decode kernels (TokenSpeed MLA article
+// 最快MLA内核背后的秘密, section 二) with query-token folding (section 三), using
+// the 2-CTA MMA of section 四: the two CTAs of a cluster pair execute every
+// tcgen05.mma together (cta_group::2, M = 128), each holding half of the
+// operands and half of the result.
+//
+// Work split. A pair owns one (entry, query group, split) and walks it in
+// pair tiles of 128 keys = two cache pages; page 2j of the split goes to CTA
+// 0 and page 2j+1 to CTA 1.
+//  * S = Q.K^T (N = 128 keys): CTA c supplies query rows [64c, 64c+64) as
+//    the A operand (tensor memory) and its own page as B (shared memory);
+//    it receives S for its 64 rows and all 128 keys. Every score is computed
+//    once: no row, page or softmax work is duplicated in the pair.
+//  * Softmax: CTA c finishes its own 64 rows. S row r of a CTA lies in TMEM
+//    lane r (keys 0..63, the leader's page) and lane 64+r (keys 64..127), so
+//    two threads of different warps share a row and swap their maxima
+//    through shared memory.
+//  * O += P.V (N = 256 output columns per MMA, two MMAs per K step): CTA c
+//    supplies its P rows as A and V columns [256h + 128c, 256h + 128c + 128)
+//    of all 128 keys as B; its O rows stay in its own TMEM (both column
+//    halves h, 256 TMEM columns).
+// Because B of the P.V is laid out by output column and B of Q.K^T by key,
+// each CTA loads, besides its own page (K ring, freed once S is computed),
+// its 256 V columns of both pages into a V ring. Those loads are issued once
+// the scores of the tile exist, so they are served by L2 (the pages were
+// just read for S) while the softmax runs, and a V slot is held only for
+// about the softmax: the split of K and V loads of section 四.
+//
+// P = 2^(x - m + SIGMA) with x the log2-scaled score and m a lazily updated
+// row maximum (moved only when exceeded by more than TAU), as E4M3; for
+// entries shorter than kTwoTermKeys it is sent as two E4M3 terms (hi, lo)
+// so that short rows keep about 8 significant bits. O is normalised by the
+// exact fp32 sum of P, which also gives the LSE.
+//
+// Roles (384 threads per CTA): warp 0 lane 0 loads Q and the K ring; warp 1
+// owns TMEM (both CTAs) and, in the leader (cluster rank 0), issues the
+// S MMAs; warp 2 issues the P.V MMAs (leader); warp 3 lane 0 loads the V
+// ring; warps 4-11 are two softmax groups of four warps taking alternate
+// pair tiles (one thread per (row, key half), 64 keys each), which also do
+// the O rescales and the epilogue. Barriers the MMA issuer waits on live in
+// the leader; the follower's loads and arrivals reach them through cluster
+// addresses. MMA completions are multicast to both CTAs.
+//
+// Every wait is bounded; on expiry the CTA sets MLA_DEV_TIMEOUT, leaves the
+// pipeline, waits for its peer at the final cluster barrier, frees TMEM and
+// returns. No TMA load uses multicast.
+#include <cuda.h>
+
+#include "device_common.cuh"
+#include "sm100_ptx.cuh"
+#include "tc_common.cuh"
+
+namespace mla {
+namespace {
+
+using namespace ptx;
+
+constexpr int kTwoTermKeys = 16384;  // entries shorter than this use two-term P
+constexpr float kTau = 2.f;          // lazy-rescale threshold (log2 units)
+constexpr float kSigma = 6.f;        // P <= 2^(kTau + kSigma) = 256 <= 448
+constexpr int kPairKeys = 128;       // keys per pair tile (one page per CTA)
+
+template <bool kTwo>
+struct PairLayout {
+  static constexpr int NK = 3;                                  // K-ring slots: own page
+  static constexpr int NV = 2;                                  // V-ring slots: 256 V columns of both pages
+  static constexpr uint32_t kQRope = 0;                         // 64 rows x 64 B (SW64)
+  static constexpr uint32_t kPPlane = 64 * 128;                 // 64 rows x 128 keys E4M3 (SW128)
+  static constexpr uint32_t kPBuf = (kTwo ? 2 : 1) * kPPlane;   // hi (and lo) plane
+  static constexpr uint32_t kPOff = 4096;                       // P[2 buffers]
+  static constexpr uint32_t kKSlot = 4 * 8192 + 64 * 64;        // 4 latent chunks (SW128) + rope (SW64)
+  static constexpr uint32_t kKOff = kPOff + 2 * kPBuf;
+  static constexpr uint32_t kVSlot = 4 * 8192;                  // [column half h][page] chunks (SW128)
+  static constexpr uint32_t kVOff = kKOff + NK * kKSlot;
+  // Q latent dims (64 rows x 512 B) are staged in the last V slot, which is
+  // first filled after the S MMA of tile NV-1 (and so after Q reached TMEM).
+  static constexpr uint32_t kQStage = kVOff + (NV - 1) * kVSlot;
+  static constexpr uint32_t kMOff = kVOff + NV * kVSlot;        // row reference maxima [tile parity][64]
+  static constexpr uint32_t kXOff = kMOff + 512;                // half-row maxima [group][phase][half][64]
+  static constexpr uint32_t kFinOff = kXOff + 2048;             // final (l, m) [l|m][group][half][64]
+  static constexpr uint32_t kBarOff = kFinOff + 2048;
+  // barriers ("leader": only the leader's copy is used)
+  static constexpr int B_Q_MAIN = 0;                 // local: staged Q latent landed
+  static constexpr int B_Q_ROPE = 1;                 // leader: both CTAs' Q rope landed
+  static constexpr int B_Q_TMEM = 2;                 // leader: both CTAs copied Q into TMEM
+  static constexpr int B_K_FULL = 3;                 // leader, + K slot: both pages landed
+  static constexpr int B_K_EMPTY = B_K_FULL + NK;    // both, + K slot
+  static constexpr int B_V_FULL = B_K_EMPTY + NK;    // leader, + V slot
+  static constexpr int B_V_EMPTY = B_V_FULL + NV;    // both, + V slot
+  static constexpr int B_S_FULL = B_V_EMPTY + NV;    // both, + buffer
+  static constexpr int B_S_EMPTY = B_S_FULL + 2;     // leader, + buffer
+  static constexpr int B_P_FULL = B_S_EMPTY + 2;     // leader, + buffer
+  static constexpr int B_P_EMPTY = B_P_FULL + 2;     // both, + buffer
+  static constexpr int B_O_DONE = B_P_EMPTY + 2;     // both
+  static constexpr int B_O_FINAL = B_O_DONE + 1;     // both: completes once, after the last P.V
+  static constexpr int B_M_READY = B_O_FINAL + 1;    // local, + tile parity
+  static constexpr int B_X = B_M_READY + 2;          // local, + group: half-row maxima exchanged
+  static constexpr int B_FIN = B_X + 2;              // local: both groups published (l, m)
+  static constexpr int kNBars = B_FIN + 1;
+  static_assert(8 * kNBars <= 512, "barrier area");
+  static constexpr uint32_t kMiscOff = kBarOff + 512;
+  static constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;
+  static_assert(kPOff % 1024 == 0 && kKOff % 1024 == 0 && kKSlot % 1024 == 0 && kVOff % 1024 == 0, "alignment");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+constexpr uint32_t kPairSmemBytes =
+    PairLayout<true>::kSmemBytes > PairLayout<false>::kSmemBytes ? PairLayout<true>::kSmemBytes
+                                                                 : PairLayout<false>::kSmemBytes;
+
+constexpr int kSoftmaxWarp0 = 4;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kThreads = 32 * (kSoftmaxWarp0 + kSoftmaxWarps);
+
+// tensor memory columns (per CTA)
+constexpr uint32_t kOCol = 0;    // O: column half h at [128h, 128h + 128)
+constexpr uint32_t kQCol = 256;  // Q latent dims, 4 E4M3 per column, rows duplicated over lane halves
+constexpr uint32_t kSCol = 384;  // two S buffers of 64 columns
+
+struct PairParams {
+  CUtensorMap tm_q_main, tm_q_rope, tm_kv_main, tm_kv_rope;
+  DecodeArgs a;
+};
+
+template <bool kTwo>
+__device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_raw) {
+  using L = PairLayout<kTwo>;
+  constexpr int NK = L::NK, NV = L::NV;
+  const DecodeArgs& a = prm.a;
+  const mla_plan& p = a.plan;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sb + L::kBarOff + 8u * (uint32_t)i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0 = leader
+  const int pair = blockIdx.x >> 1;
+  const int G = p.q_groups, S = p.split_kv, T = p.q_len, H = p.num_heads, M = p.rows_per_unit;
+  const int g = pair % G;
+  const int s = (pair / G) % S;
+  const int b = pair / (G * S);
+  const int n = effective_seq_len(a, b, rank == 0 && s == 0 && g == 0 && threadIdx.x == 0);
+  const int key0 = s * p.keys_per_split;
+  const int64_t row0 = (int64_t)b * T * H + (int64_t)g * M;
+  const int box_q = M < 64 ? M : 64;  // query rows per TMA box (the tensor maps' box height)
+
+  if (key0 >= n) {  // same decision in both CTAs of the pair
+    if (S == 1) {
+      for (int r = threadIdx.x; r < 64; r += blockDim.x) {
+        const int rr = 64 * (int)rank + r;
+        if (rr >= M) continue;
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + (row0 + rr) * MLA_D_V);
+        for (int i = 0; i < 64; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+        if (a.lse) a.lse[row0 + rr] = -INFINITY;
+      }
+    }
+    return;
+  }
+  const int key1 = min(n, key0 + p.keys_per_split);
+  const int n_tiles = (key1 - key0 + kTileKeys - 1) / kTileKeys;  // 64-key pages
+  const int n_pt = (n_tiles + 1) / 2;                              // pair tiles
+  const int tile0 = key0 / kTileKeys;
+  const int32_t* table = a.block_tables + (int64_t)b * a.max_pages_per_seq;
+  // page of 64-key tile t of the split (t < n_tiles), 0 when absent or invalid
+  auto page_of = [&](int t) -> int {
+    if (t >= n_tiles) return 0;
+    const int pg = table[tile0 + t];
+    return (pg < 0 || (int64_t)pg >= a.num_pages) ? 0 : pg;
+  };
+  // the leader's copy of barrier i, as a cluster address
+  auto lead = [&](int i) -> uint32_t { return mapa(bar(i), 0); };
+
+  // ---------------------------------------------------------------- setup
+  if (threadIdx.x == 0) {
+    mbar_init(bar(L::B_Q_MAIN), 1);
+    mbar_init(bar(L::B_Q_ROPE), 1);
+    mbar_init(bar(L::B_Q_TMEM), 2 * kSoftmaxWarps);
+    for (int i = 0; i < NK; ++i) {
+      mbar_init(bar(L::B_K_FULL + i), 1);
+      mbar_init(bar(L::B_K_EMPTY + i), 1);
+    }
+    for (int i = 0; i < NV; ++i) {
+      mbar_init(bar(L::B_V_FULL + i), 1);
+      mbar_init(bar(L::B_V_EMPTY + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(L::B_S_FULL + i), 1);
+      mbar_init(bar(L::B_S_EMPTY + i), 2 * 4 + 2);  // one group in each CTA + both V loaders
+      mbar_init(bar(L::B_P_FULL + i), 2 * 4);
+      mbar_init(bar(L::B_P_EMPTY + i), 1);
+      mbar_init(bar(L::B_M_READY + i), 4);
+      mbar_init(bar(L::B_X + i), 4);
+    }
+    mbar_init(bar(L::B_O_DONE), 1);
+    mbar_init(bar(L::B_O_FINAL), 1);
+    mbar_init(bar(L::B_FIN), kSoftmaxWarps);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (box_q < 64) {
+    // Q rope rows the TMA box does not cover are zero (rows are independent).
+    uint4* rb = reinterpret_cast<uint4*>(smem + L::kQRope + box_q * 64);
+    for (int i = threadIdx.x; i < (64 - box_q) * 4; i += blockDim.x) rb[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers and TMEM exist before any cross-CTA use
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ Q and K-ring loads
+    if (lane == 0) {
+      prefetch_tmap(&prm.tm_q_main);
+      prefetch_tmap(&prm.tm_q_rope);
+      prefetch_tmap(&prm.tm_kv_main);
+      prefetch_tmap(&prm.tm_kv_rope);
+      const uint64_t pol_q = policy_evict_first();
+      const uint64_t pol_kv = policy_evict_last();  // read again right away for V
+      const int qrow = (int)row0 + 64 * (int)rank;  // rows past the unit are read but never stored
+      mbar_arrive_expect_tx(bar(L::B_Q_MAIN), 4u * 128u * (uint32_t)box_q);
+#pragma unroll
+      for (int ci = 0; ci < 4; ++ci)
+        tma_load_2d(sb + L::kQStage + ci * 8192, &prm.tm_q_main, 128 * ci, qrow, bar(L::B_Q_MAIN), pol_q);
+      if (rank == 0) mbar_arrive_expect_tx(bar(L::B_Q_ROPE), 2u * 64u * (uint32_t)box_q);
+      tma_load_2d_pair(sb + L::kQRope, &prm.tm_q_rope, 512, qrow, lead(L::B_Q_ROPE), pol_q);
+      for (int j = 0; j < n_pt; ++j) {
+        const int sk = j % NK;
+        if (!bounded_wait(bar(L::B_K_EMPTY + sk), ((j / NK) & 1) ^ 1, abort_flag, a.status)) break;
+        const int page = page_of(2 * j + (int)rank);
+        const uint32_t ks = sb + L::kKOff + sk * L::kKSlot;
+        const uint32_t full = lead(L::B_K_FULL + sk);
+        if (rank == 0) mbar_arrive_expect_tx(bar(L::B_K_FULL + sk), 2u * L::kKSlot);
+#pragma unroll
+        for (int ci = 0; ci < 4; ++ci)
+          tma_load_2d_pair(ks + ci * 8192, &prm.tm_kv_main, 128 * ci, page * kTileKeys, full, pol_kv);
+        tma_load_2d_pair(ks + 4 * 8192, &prm.tm_kv_rope, 512, page * kTileKeys, full, pol_kv);
+      }
+      // The leader's K_FULL phases count both CTAs' bytes: the leader waits for
+      // the last ones before the pair may leave (the follower waits at the
+      // final cluster barrier).
+      if (rank == 0) drain_loads(bar(L::B_K_FULL), NK, n_pt);
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ V-ring loads
+    if (lane == 0) {
+      const uint64_t pol_v = policy_evict_first();  // last use of these bytes
+      for (int j = 0; j < n_pt; ++j) {
+        const int sv = j % NV, buf = j & 1;
+        // the scores of tile j exist: its pages are in L2 now
+        if (!bounded_wait(bar(L::B_S_FULL + buf), (j >> 1) & 1, abort_flag, a.status)) break;
+        mbar_arrive_remote(lead(L::B_S_EMPTY + buf));
+        if (!bounded_wait(bar(L::B_V_EMPTY + sv), ((j / NV) & 1) ^ 1, abort_flag, a.status)) break;
+        const int pg0 = page_of(2 * j), pg1 = page_of(2 * j + 1);
+        const uint32_t vs = sb + L::kVOff + sv * L::kVSlot;
+        const uint32_t full = lead(L::B_V_FULL + sv);
+        if (rank == 0) mbar_arrive_expect_tx(bar(L::B_V_FULL + sv), 2u * L::kVSlot);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int x = 128 * (2 * h + (int)rank);  // this CTA's 128 of the 256 columns of half h
+          tma_load_2d_pair(vs + h * 16384, &prm.tm_kv_main, x, pg0 * kTileKeys, full, pol_v);
+          tma_load_2d_pair(vs + h * 16384 + 8192, &prm.tm_kv_main, x, pg1 * kTileKeys, full, pol_v);
+        }
+      }
+      if (rank == 0) drain_loads(bar(L::B_V_FULL), NV, n_pt);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ S = Q.K^T issuer (leader)
+    if (rank == 0) {
+      constexpr uint32_t idq = instr_desc(0, 0, 0, 128, kPairKeys);  // E4M3 x E4M3, K-major B
+      bool ok = warp_wait(bar(L::B_Q_ROPE), 0, abort_flag, a.status) &&
+                warp_wait(bar(L::B_Q_TMEM), 0, abort_flag, a.status);
+      const uint64_t dq_rope = smem_desc(sb + L::kQRope, 16, 512, kSw64);
+      for (int j = 0; ok && j < n_pt; ++j) {
+        const int sk = j % NK, buf = j & 1;
+        if (!(ok = warp_wait(bar(L::B_K_FULL + sk), (j / NK) & 1, abort_flag, a.status))) break;
+        if (!(ok = warp_wait(bar(L::B_S_EMPTY + buf), ((j >> 1) & 1) ^ 1, abort_flag, a.status))) break;
+        tc_fence_after();
+        const uint32_t d = tmem + kSCol + 64u * buf;
+        const uint32_t ks = sb + L::kKOff + sk * L::kKSlot;
+#pragma unroll
+        for (int ci = 0; ci < 4; ++ci) {
+          const uint64_t dk = smem_desc(ks + ci * 8192, 16, 1024, kSw128);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f8_ts_pair_e(d, tmem + kQCol + (uint32_t)(8 * (4 * ci + kk)), dk + (uint64_t)((kk * 32) >> 4), idq,
+                             (ci | kk) ? 1u : 0u);
+        }
+        const uint64_t dr = smem_desc(ks + 4 * 8192, 16, 512, kSw64);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+          mma_f8_ss_pair_e(d, dq_rope + (uint64_t)(kk * 2), dr + (uint64_t)(kk * 2), idq, 1u);
+        mma_commit_pair_mc_e(bar(L::B_S_FULL + buf), 3);
+        mma_commit_pair_mc_e(bar(L::B_K_EMPTY + sk), 3);
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ O += P.V issuer (leader)
+    if (rank == 0) {
+      constexpr uint32_t idp = instr_desc(0, 0, 1, 128, 256);  // V is MN-major
+      bool ok = true;
+      for (int j = 0; ok && j < n_pt; ++j) {
+        const int buf = j & 1, sv = j % NV;
+        if (!(ok = warp_wait(bar(L::B_V_FULL + sv), (j / NV) & 1, abort_flag, a.status))) break;
+        if (!(ok = warp_wait(bar(L::B_P_FULL + buf), (j >> 1) & 1, abort_flag, a.status))) break;
+        tc_fence_after();
+        const uint32_t vs = sb + L::kVOff + sv * L::kVSlot;
+        const uint64_t dp = smem_desc(sb + L::kPOff + buf * L::kPBuf, 16, 1024, kSw128);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {  // 32 keys per MMA: page k4/2, rows (k4%2)*32
+            const uint64_t dv =
+                smem_desc(vs + h * 16384 + (k4 >> 1) * 8192 + (k4 & 1) * 4096, 8192, 1024, kSw128);
+            mma_f8_ss_pair_e(tmem + kOCol + 128u * h, dp + (uint64_t)((k4 * 32) >> 4), dv, idp,
+                             (j > 0 || k4 > 0) ? 1u : 0u);
+            if (kTwo)
+              mma_f8_ss_pair_e(tmem + kOCol + 128u * h, dp + (uint64_t)((L::kPPlane + k4 * 32) >> 4), dv, idp, 1u);
+          }
+        }
+        // O_DONE first: a softmax group that has seen P_EMPTY of tile j-2 may
+        // rely on O_DONE having completed that tile's phase too.
+        mma_commit_pair_mc_e(bar(L::B_O_DONE), 3);
+        mma_commit_pair_mc_e(bar(L::B_P_EMPTY + buf), 3);
+        mma_commit_pair_mc_e(bar(L::B_V_EMPTY + sv), 3);
+        if (j == n_pt - 1) mma_commit_pair_mc_e(bar(L::B_O_FINAL), 3);
+      }
+    }
+  } else if (warp >= kSoftmaxWarp0) {
+    // ------------------------------------------------------------ softmax warps
+    // Group grp takes pair tiles grp, grp+2, ...; warp w serves TMEM lane
+    // quarter q = w%4: local rows 32(q%2) .. +31, key half hf = q/2.
+    const int q = warp & 3;
+    const int grp = (warp - kSoftmaxWarp0) >> 2;
+    const int hf = q >> 1;
+    const int rl = 32 * (q & 1) + lane;  // local row (0..63)
+    const int r = 64 * (int)rank + rl;   // row within the unit
+    const uint32_t tl = (uint32_t)(32 * q) << 16;
+    const int limit = min((r < M) ? n - T + g * p.fold + r / H : n - 1, key1 - 1);
+    float* mref = reinterpret_cast<float*>(smem + L::kMOff);  // [tile parity][64]
+    float* xm = reinterpret_cast<float*>(smem + L::kXOff);    // [group][phase][half][64]
+    float* fin = reinterpret_cast<float*>(smem + L::kFinOff); // [l|m][group][half][64]
+    bool ok = true;
+
+    // Q latent dims of local row rl into TMEM (A operand of S = Q.K^T): lane
+    // quarters q and q^2 both hold rows 32(q%2)..; group g copies chunks 2g, 2g+1.
+    ok = warp_wait(bar(L::B_Q_MAIN), 0, abort_flag, a.status);
+    if (ok) {
+#pragma unroll 1
+      for (int c2 = 0; c2 < 2; ++c2) {
+        const int cc = 2 * grp + c2;
+        const uint8_t* chunk = smem + L::kQStage + cc * 8192 + rl * 128;
+        uint32_t w[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 v = *reinterpret_cast<const uint4*>(chunk + ((u ^ (rl & 7)) * 16));
+          w[4 * u] = v.x;
+          w[4 * u + 1] = v.y;
+          w[4 * u + 2] = v.z;
+          w[4 * u + 3] = v.w;
+        }
+        if (r >= M) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w[i] = 0;
+        }
+        tmem_st32(tmem + tl + kQCol + 32u * cc, w);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(lead(L::B_Q_TMEM));
+    }
+
+    const float sl2 = a.score_scale_log2;
+    float m_grp = -INFINITY, l_grp = 0.f;  // this group's reference and partial sum (this half row)
+    for (int j = grp; ok && j < n_pt; j += 2) {
+      const int buf = j & 1;  // == grp
+      const int ph = (j >> 1) & 1;
+      if (!(ok = warp_wait(bar(L::B_S_FULL + buf), ph, abort_flag, a.status))) break;
+      tc_fence_after();
+      uint32_t sv[64];
+      {
+        uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
+        uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
+        tmem_ld32(tmem + tl + kSCol + 64u * buf, s0);
+        tmem_ld32(tmem + tl + kSCol + 64u * buf + 32u, s1);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(lead(L::B_S_EMPTY + buf));
+
+      const int t = 2 * j + hf;  // 64-key tile of this half
+      bool page_ok = t < n_tiles;
+      if (page_ok) {
+        const int pg = table[tile0 + t];
+        if (pg < 0 || (int64_t)pg >= a.num_pages) {
+          page_ok = false;
+          if (lane == 0 && (q & 1) == 0) atomicOr(a.status, MLA_DEV_BAD_PAGE);
+        }
+      }
+      const int kb = key0 + kPairKeys * j + 64 * hf;
+      // raw scores; masked keys become -inf (sl2 > 0, so max commutes with the scale)
+      if (!(page_ok && kb + 63 <= limit)) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (!(page_ok && kb + i <= limit)) sv[i] = __float_as_uint(-INFINITY);
+      }
+      float mt;
+      {
+        float m8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float v = __uint_as_float(sv[8 * i]);
+#pragma unroll
+          for (int k = 1; k < 8; ++k) v = fmaxf(v, __uint_as_float(sv[8 * i + k]));
+          m8[i] = v;
+        }
+        mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sl2;
+      }
+      // the other half of the row lives in the warp of quarter q^2
+      xm[((grp * 2 + ph) * 2 + hf) * 64 + rl] = mt;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::B_X + grp));
+      if (!(ok = warp_wait(bar(L::B_X + grp), ph, abort_flag, a.status))) break;
+      mt = fmaxf(mt, xm[((grp * 2 + ph) * 2 + (hf ^ 1)) * 64 + rl]);
+      // reference maximum after tile j-1 (from the other group), lazily updated
+      float m_prev = -INFINITY;
+      if (j > 0) {
+        if (!(ok = warp_wait(bar(L::B_M_READY + (buf ^ 1)), ((j - 1) >> 1) & 1, abort_flag, a.status))) break;
+        m_prev = mref[(buf ^ 1) * 64 + rl];
+      }
+      const float m_j = (mt > m_prev + kTau) ? mt : m_prev;
+      mref[buf * 64 + rl] = m_j;  // both halves write the same value
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::B_M_READY + buf));
+      const float alpha = (m_j == m_prev) ? 1.f : ex2_approx(m_prev - m_j);  // O rescale for tile j
+      const float m_use = (m_j == -INFINITY) ? 0.f : m_j - kSigma;
+
+      // P buffer is free once the P.V two tiles back has finished
+      if (j >= 2 && !(ok = warp_wait(bar(L::B_P_EMPTY + buf), ph ^ 1, abort_flag, a.status))) break;
+
+      // P = 2^(s * sl2 - m_use), 16 keys (one 16-byte chunk) at a time; this
+      // half's 64 keys are bytes [64hf, 64hf + 64) of the 128-byte P row.
+      float se[4] = {0.f, 0.f, 0.f, 0.f};
+      uint8_t* prow = smem + L::kPOff + buf * L::kPBuf + rl * 128;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int e = 16 * u + 2 * i;
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -m_use));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -m_use));
+          se[i & 3] += p0 + p1;
+          const uint32_t qh = cvt_e4m3x2(p0, p1);
+          if (i & 1) hi[i >> 1] |= qh << 16; else hi[i >> 1] = qh;
+          if (kTwo) {
+            const uint32_t rl16 = hsub2(cvt_f16x2(p0, p1), cvt_e4m3x2_to_f16x2(qh));
+            const uint32_t ql = cvt_f16x2_to_e4m3x2(rl16);
+            if (i & 1) lo[i >> 1] |= ql << 16; else lo[i >> 1] = ql;
+          }
+        }
+        const int phys = (4 * hf + u) ^ (rl & 7);
+        *reinterpret_cast<uint4*>(prow + phys * 16) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        if (kTwo) *reinterpret_cast<uint4*>(prow + L::kPPlane + phys * 16) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      const float sum = (se[0] + se[1]) + (se[2] + se[3]);
+      l_grp = (m_grp == m_j) ? l_grp + sum : fmaf(l_grp, ex2_approx(m_grp - m_j), sum);
+      m_grp = m_j;
+
+      // rescale this thread's 256 O columns if the reference maximum moved
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (!(ok = warp_wait(bar(L::B_O_DONE), (j - 1) & 1, abort_flag, a.status))) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tmem + tl + kOCol + 32u * cc, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tmem + tl + kOCol + 32u * cc, o);
+        }
+        tmem_wait_st();
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(lead(L::B_P_FULL + buf));
+    }
+
+    // ------------------------------------------------------------ epilogue
+    // Row sum over both groups and both key halves, relative to the final
+    // reference maximum.
+    ok = __all_sync(0xffffffffu, ok);
+    fin[((0 * 2 + grp) * 2 + hf) * 64 + rl] = l_grp;
+    fin[((1 * 2 + grp) * 2 + hf) * 64 + rl] = m_grp;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(L::B_FIN));
+    if (ok) ok = warp_wait(bar(L::B_FIN), 0, abort_flag, a.status);
+    float le = 0.f, m_fin = -INFINITY;
+    if (ok) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) m_fin = fmaxf(m_fin, fin[(4 + i) * 64 + rl]);
+      if (m_fin != -INFINITY) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float mi = fin[(4 + i) * 64 + rl];
+          if (mi != -INFINITY) le += fin[i * 64 + rl] * ex2_approx(mi - m_fin);
+        }
+      }
+    }
+    if (ok) ok = warp_wait(bar(L::B_O_FINAL), 0, abort_flag, a.status);
+    if (ok) {
+      tc_fence_after();
+      const float inv = (le > 0.f) ? a.v_scale / le : 0.f;
+      const bool live = r < M;
+      const int64_t rg = row0 + r;
+      // group grp stores column half h = grp: output dims 256h + 128hf + [0, 128)
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tmem + tl + kOCol + 128u * grp + 32u * cc, o);
+        tmem_wait_ld();
+        if (!live) continue;
+        store_out_chunk(a, rg, s, 256 * grp + 128 * hf + 32 * cc, o, inv);
+      }
+      if (live && grp == 0 && hf == 0) {
+        const float lse_val = (le > 0.f) ? (m_fin - kSigma + log2f(le)) * kLn2 : -INFINITY;
+        if (S == 1) {
+          if (a.lse) a.lse[rg] = lse_val;
+        } else {
+          a.lse_part[rg * S + s] = lse_val;
+        }
+      }
+    }
+    tc_fence_before();
+  }
+
+  // ---------------------------------------------------------------- teardown
+  // MMA completions are multicast to both CTAs, and only some of them are
+  // consumed: before the pair may leave, each CTA waits for the last phase of
+  // every barrier the leader's commits arrive on, so that no arrival lands in
+  // shared memory after the CTA has exited. It runs once every role is done
+  // (the epilogue saw O_FINAL, so every commit has been triggered and each
+  // barrier is at most its last arrival short of its final phase). Bounded;
+  // skipped after an abort, when the phases may never complete.
+  __syncthreads();
+  if (warp == 2 && lane == 0 && !*abort_flag) {
+    for (int j = n_pt - 1; j >= 0 && j >= n_pt - NK; --j) drain_phase(bar(L::B_K_EMPTY + j % NK), (j / NK) & 1);
+    for (int j = n_pt - 1; j >= 0 && j >= n_pt - NV; --j) drain_phase(bar(L::B_V_EMPTY + j % NV), (j / NV) & 1);
+    for (int j = n_pt - 1; j >= 0 && j >= n_pt - 2; --j) {
+      drain_phase(bar(L::B_P_EMPTY + (j & 1)), (j >> 1) & 1);
+      drain_phase(bar(L::B_S_FULL + (j & 1)), (j >> 1) & 1);
+    }
+    if (n_pt > 0) {
+      drain_phase(bar(L::B_O_DONE), (n_pt - 1) & 1);
+      drain_phase(bar(L::B_O_FINAL), 0);
+    }
+  }
+  __syncthreads();
+  tc_fence_before();
+  cluster_sync();  // the peer no longer touches this CTA's shared or tensor memory
+  if (warp == 1) {
+    tc_fence_after();
+    if (*abort_flag) spin_ns(1000000ull);  // let any MMA still in flight finish
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    tc_fp8_pair_kernel(const __grid_constant__ PairParams prm) {
+  extern __shared__ uint8_t smem_raw[];
+  const mla_plan& p = prm.a.plan;
+  const int b = (blockIdx.x >> 1) / (p.q_groups * p.split_kv);
+  // Short entries send P as two E4M3 terms; the choice is per entry, so both
+  // CTAs of the pair take the same variant and layout.
+  if (effective_seq_len(prm.a, b, false) < kTwoTermKeys)
+    pair_cta<true>(prm, smem_raw);
+  else
+    pair_cta<false>(prm, smem_raw);
+}
+
+}  // namespace
+
+cudaError_t launch_tc_fp8_pair_partial(const DecodeArgs& a, cudaStream_t stream) {
+  const mla_plan& p = a.plan;
+  const uint64_t pairs = (uint64_t)p.batch * p.q_groups * p.split_kv;
+  if (pairs == 0) return cudaSuccess;
+  PairParams prm;
+  prm.a = a;
+  const uint64_t q_rows = (uint64_t)p.batch * p.q_len * p.num_heads;
+  const uint64_t kv_rows = (uint64_t)a.num_pages * kTileKeys;
+  const uint32_t box_q = p.rows_per_unit < 64 ? (uint32_t)p.rows_per_unit : 64u;
+  if (!encode_rows_576(&prm.tm_q_main, a.q, 1, q_rows, 128, box_q, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_rows_576(&prm.tm_q_rope, a.q, 1, q_rows, 64, box_q, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !encode_rows_576(&prm.tm_kv_main, a.kv_cache, 1, kv_rows, 128, kTileKeys, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_rows_576(&prm.tm_kv_rope, a.kv_cache, 1, kv_rows, 64, kTileKeys, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e =
+        cudaFuncSetAttribute(tc_fp8_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  tc_fp8_pair_kernel<<<(unsigned)(2 * pairs), kThreads, kPairSmemBytes, stream>>>(prm);
+  return cudaGetLastError();
+}
+
+}  // namespace mla

@@ -96,11 +96,21 @@ def test_decode_rejects_bad_arguments_before_any_launch():
     assert _call(p, scale=float("inf")) == -1
 
 
-def test_workspace_error_from_python_wrapper():
+def test_python_wrapper_refuses_host_tensors():
+    """The binding names the first argument that is not a CUDA tensor before calling the library."""
     torch = pytest.importorskip("torch")
     p = mla.mla_decode_plan(1, 1, 16, 256, "bf16")
     t = torch.empty(0)
-    with pytest.raises(mla.MlaError) as e:
+    with pytest.raises(ValueError, match="q must be a CUDA tensor"):
         mla.mla_decode(p, t, torch.empty(1, 32, 576), torch.empty(1, 4, dtype=torch.int32), t,
                        0.04, t, None, torch.empty(0, dtype=torch.uint8))
-    assert e.value.code in (-1, -2)
+
+
+def test_last_cuda_error_starts_clean():
+    """No CUDA failure has been recorded on a fresh thread: code 0, name cudaSuccess."""
+    import threading
+    res = {}
+    t = threading.Thread(target=lambda: res.setdefault("v", mla.last_cuda_error()))
+    t.start()
+    t.join()
+    assert res["v"] == (0, "cudaSuccess")

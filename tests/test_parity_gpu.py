@@ -16,10 +16,14 @@ from helpers import compare, oracle_rows, sample_rows
 
 pytestmark = pytest.mark.gpu
 
-KERNELS = ["tcgen05", "simt"]
+# tcgen05: the default tensor-core kernel (for FP8 the CTA-pair form);
+# tcgen05_solo: the FP8 variant without cross-CTA MMAs; simt: the cross-check.
+KERNELS = ["tcgen05", "simt", "tcgen05_solo"]
 
 
 def run(inp, kernel="auto", split_kv=0, fold=0, want_lse=True):
+    if kernel == "tcgen05_solo" and inp.dtype != "fp8":
+        pytest.skip("the solo variant is FP8 only")
     dev = torch.device("cuda", 0)
     g = inp.to(dev)
     dec = mla.MlaDecoder(g.batch, g.q_len, g.heads, max(g.max_seq_len, 0), g.dtype, dev,
@@ -42,6 +46,9 @@ SMALL = [
     (1, 3, 40, "fp8", [200], 1.0, 1.0, 1.0),
     (4, 1, 8, "bf16", [1, 2, 63, 64], 1.0, 1.0, 1.0),
     (3, 4, 32, "fp16", [2, 0, 5], 1.0, 1.0, 1.0),   # seq_len < q_len and empty entries
+    (3, 1, 16, "fp8", [64, 130, 1], 2.0, 1.0, 1.0),  # 16 rows; odd page counts; one key
+    (4, 4, 32, "fp8", [2, 0, 191, 4097], 1.5, 1.0, 1.0),  # seq_len < q_len, empty entry, ragged tails
+    (2, 2, 48, "fp8", [300, 64], 1.0, 1.0, 1.0),    # 96 rows: the second CTA holds 32 live rows
 ]
 
 
@@ -115,14 +122,18 @@ def test_lse_optional(kernel):
     assert torch.equal(out1, out2)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
 @pytest.mark.parametrize("kernel", KERNELS)
-def test_cuda_graph_replay_matches_eager(kernel):
+def test_cuda_graph_replay_matches_eager(kernel, dtype):
+    if kernel == "tcgen05_solo" and dtype != "fp8":
+        pytest.skip("the solo variant is FP8 only")
     dev = torch.device("cuda", 0)
-    inp = make_inputs_custom(2, 4, 32, "bf16", [900, 2100], seed=12, pool=2.0).to(dev)
-    dec = mla.MlaDecoder(2, 4, 32, 2100, "bf16", dev, kernel=kernel)
+    inp = make_inputs_custom(2, 4, 32, dtype, [900, 2100], seed=12, pool=2.0).to(dev)
+    dec = mla.MlaDecoder(2, 4, 32, 2100, dtype, dev, kernel=kernel)
     out = torch.empty(2, 4, 32, 512, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(2, 4, 32, dtype=torch.float32, device=dev)
-    dec(inp.q, inp.kv_cache, inp.block_tables, inp.seq_lens, inp.softmax_scale, out=out, lse=lse)
+    sc = (inp.q_scale, inp.kv_scale)
+    dec(inp.q, inp.kv_cache, inp.block_tables, inp.seq_lens, inp.softmax_scale, *sc, out=out, lse=lse)
     torch.cuda.synchronize()
     eager_o, eager_l = out.clone(), lse.clone()
     out.zero_()
@@ -130,7 +141,7 @@ def test_cuda_graph_replay_matches_eager(kernel):
     s.wait_stream(torch.cuda.current_stream())
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
-        dec(inp.q, inp.kv_cache, inp.block_tables, inp.seq_lens, inp.softmax_scale, out=out, lse=lse)
+        dec(inp.q, inp.kv_cache, inp.block_tables, inp.seq_lens, inp.softmax_scale, *sc, out=out, lse=lse)
     for _ in range(3):
         out.zero_()
         g.replay()
@@ -139,23 +150,26 @@ def test_cuda_graph_replay_matches_eager(kernel):
     del g
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
 @pytest.mark.parametrize("kernel", KERNELS)
-def test_status_word_flags_bad_pages_and_long_sequences(kernel):
-    inp = make_inputs_custom(2, 1, 16, "bf16", [200, 100], seed=13, pool=1.0)
+def test_status_word_flags_bad_pages_and_long_sequences(kernel, dtype):
+    if kernel == "tcgen05_solo" and dtype != "fp8":
+        pytest.skip("the solo variant is FP8 only")
+    inp = make_inputs_custom(2, 1, 16, dtype, [200, 100], seed=13, pool=1.0)
     inp.block_tables[1, 0] = inp.num_pages + 5          # outside the pool
     _, _, status, _ = run(inp, kernel)
     assert status & mla.MLA_DEV_BAD_PAGE
-    inp2 = make_inputs_custom(1, 1, 16, "bf16", [200], seed=14, pool=1.0)
+    inp2 = make_inputs_custom(1, 1, 16, dtype, [200], seed=14, pool=1.0)
     dev = torch.device("cuda", 0)
     g = inp2.to(dev)
-    dec = mla.MlaDecoder(1, 1, 16, 100, "bf16", dev, kernel=kernel)   # planned for 100 keys
-    out, lse = dec(g.q, g.kv_cache, g.block_tables, g.seq_lens, g.softmax_scale)
+    dec = mla.MlaDecoder(1, 1, 16, 100, dtype, dev, kernel=kernel)   # planned for 100 keys
+    out, lse = dec(g.q, g.kv_cache, g.block_tables, g.seq_lens, g.softmax_scale, g.q_scale, g.kv_scale)
     torch.cuda.synchronize()
     assert dec.status() & mla.MLA_DEV_SEQ_TOO_LONG
     assert torch.isfinite(out.float()).all()
     # a clean call clears the word again
     g.seq_lens.fill_(90)
-    dec(g.q, g.kv_cache, g.block_tables, g.seq_lens, g.softmax_scale)
+    dec(g.q, g.kv_cache, g.block_tables, g.seq_lens, g.softmax_scale, g.q_scale, g.kv_scale)
     assert dec.status() == 0
 
 
@@ -188,3 +202,28 @@ def test_full_size_workloads(name):
     compare(out, lse, ref_o, ref_l, inp.dtype, rows=rows, what=name)
     # properties that hold at any size: finite outputs, LSE bounded by the closed form
     assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+
+
+def test_host_pointers_are_refused_before_launch():
+    """A pageable host pointer reaching the C ABI (here the block table) is refused with
+    MLA_ERR_INVALID_ARG and nothing is enqueued; the context stays usable."""
+    import ctypes
+    from mla_paged_decode_04_b200 import _lib
+    dev = torch.device("cuda", 0)
+    inp = make_inputs_custom(1, 1, 16, "bf16", [256], seed=15, pool="exact")
+    g = inp.to(dev)
+    dec = mla.MlaDecoder(1, 1, 16, 256, "bf16", dev)
+    out = torch.empty(1, 1, 16, 512, dtype=torch.bfloat16, device=dev)
+    host_bt = inp.block_tables.contiguous()          # CPU tensor
+    assert not host_bt.is_cuda
+    vp = ctypes.c_void_p
+    rc = _lib.lib().mla_decode(ctypes.byref(dec.plan), vp(g.q.data_ptr()), vp(g.kv_cache.data_ptr()),
+                               g.kv_cache.shape[0], 64, vp(host_bt.data_ptr()), host_bt.shape[1],
+                               vp(g.seq_lens.data_ptr()), g.softmax_scale, 1.0, 1.0, vp(out.data_ptr()),
+                               None, vp(dec.workspace.data_ptr()), dec.workspace.numel(),
+                               vp(torch.cuda.current_stream().cuda_stream))
+    assert rc == -1
+    torch.cuda.synchronize()
+    o, l = dec(g.q, g.kv_cache, g.block_tables, g.seq_lens, g.softmax_scale)
+    torch.cuda.synchronize()
+    assert dec.status() == 0 and torch.isfinite(o.float()).all()
