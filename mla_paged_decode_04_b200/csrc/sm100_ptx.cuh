@@ -429,3 +429,28 @@ __device__ __forceinline__ void tma_prefetch_2d(const void* tmap, int32_t x, int
 }
 }  // namespace ptx
 }  // namespace mla
+
+namespace mla {
+namespace ptx {
+// Arrive on an mbarrier of another CTA of the cluster without ordering this
+// thread's earlier memory accesses (for signals that publish no data, e.g.
+// "I have read my tensor-memory slice", after tcgen05.wait::ld).
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+}  // namespace ptx
+}  // namespace mla
+
+namespace mla {
+namespace ptx {
+// Arrive on an mbarrier of another CTA of the cluster after this thread's
+// writes to its own shared memory (ordered by a release fence restricted to
+// shared::cta accesses, so outstanding global loads are not waited for).
+__device__ __forceinline__ void mbar_arrive_remote_publish_smem(uint32_t cluster_bar) {
+  asm volatile(
+      "fence.release.sync_restrict::shared::cta.cluster;\n\t"
+      "mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+      : "memory");
+}
+}  // namespace ptx
+}  // namespace mla

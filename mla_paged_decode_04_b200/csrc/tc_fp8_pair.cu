@@ -172,6 +172,18 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
   };
   // the leader's copy of barrier i, as a cluster address
   auto lead = [&](int i) -> uint32_t { return mapa(bar(i), 0); };
+  // Arrive on the leader's barrier i: a plain local arrive in the leader; in
+  // the follower a cluster arrive, after a release fence over this CTA's
+  // shared memory when it publishes data the leader's MMA will read (tensor
+  // memory writes are ordered by tcgen05.fence::before_thread_sync), relaxed
+  // otherwise. A full cluster-scope release would also wait for this
+  // thread's outstanding global loads (the block-table prefetch).
+  auto arrive_lead = [&](int i) {
+    if (rank == 0) mbar_arrive(bar(i)); else mbar_arrive_remote_publish_smem(lead(i));
+  };
+  auto arrive_lead_relaxed = [&](int i) {
+    if (rank == 0) mbar_arrive(bar(i)); else mbar_arrive_remote_relaxed(lead(i));
+  };
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
@@ -256,7 +268,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
         const int sv = j % NV, buf = j & 1;
         // the scores of tile j exist: its pages are in L2 now
         if (!bounded_wait(bar(L::B_S_FULL + buf), (j >> 1) & 1, abort_flag, a.status)) break;
-        mbar_arrive_remote(lead(L::B_S_EMPTY + buf));
+        arrive_lead_relaxed(L::B_S_EMPTY + buf);
         if (!bounded_wait(bar(L::B_V_EMPTY + sv), ((j / NV) & 1) ^ 1, abort_flag, a.status)) break;
         const int pg0 = page_of(2 * j), pg1 = page_of(2 * j + 1);
         const uint32_t vs = sb + L::kVOff + sv * L::kVSlot;
@@ -375,12 +387,18 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(lead(L::B_Q_TMEM));
+      if (lane == 0) arrive_lead(L::B_Q_TMEM);
     }
 
     const float sl2 = a.score_scale_log2;
     float m_grp = -INFINITY, l_grp = 0.f;  // this group's reference and partial sum (this half row)
+    // block-table entry of this half's page for the group's next tile, read
+    // one tile ahead so that the dependent load is off the critical path
+    auto table_entry = [&](int jj) -> int { const int t = 2 * jj + hf; return t < n_tiles ? table[tile0 + t] : 0; };
+    int pg_next = (grp < n_pt) ? table_entry(grp) : 0;
     for (int j = grp; ok && j < n_pt; j += 2) {
+      const int pg_cur = pg_next;
+      if (j + 2 < n_pt) pg_next = table_entry(j + 2);
       const int buf = j & 1;  // == grp
       const int ph = (j >> 1) & 1;
       if (!(ok = warp_wait(bar(L::B_S_FULL + buf), ph, abort_flag, a.status))) break;
@@ -395,12 +413,12 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(lead(L::B_S_EMPTY + buf));
+      if (lane == 0) arrive_lead_relaxed(L::B_S_EMPTY + buf);  // the slice was read (wait::ld above)
 
       const int t = 2 * j + hf;  // 64-key tile of this half
       bool page_ok = t < n_tiles;
       if (page_ok) {
-        const int pg = table[tile0 + t];
+        const int pg = pg_cur;
         if (pg < 0 || (int64_t)pg >= a.num_pages) {
           page_ok = false;
           if (lane == 0 && (q & 1) == 0) atomicOr(a.status, MLA_DEV_BAD_PAGE);
@@ -494,7 +512,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(lead(L::B_P_FULL + buf));
+      if (lane == 0) arrive_lead(L::B_P_FULL + buf);
     }
 
     // ------------------------------------------------------------ epilogue
