@@ -98,7 +98,14 @@ struct PairLayout {
   static constexpr int B_M_READY = B_O_FINAL + 1;    // local, + tile parity
   static constexpr int B_X = B_M_READY + 2;          // local, + group: half-row maxima exchanged
   static constexpr int B_FIN = B_X + 2;              // local: both groups published (l, m)
-  static constexpr int kNBars = B_FIN + 1;
+  // both, + tile % NQ: the scores of the tile exist (the V loads may go).
+  // NQ = 6 rules out phase aliasing: S = Q.K^T of tile j+6 needs the scores
+  // of tile j+4 read, which needs P of tile j+2 written, which needs the
+  // P.V of tile j done, which needs the V loads of tile j issued.
+  static constexpr int NQ = 6;
+  static constexpr int B_QK_DONE = B_FIN + 1;
+  static constexpr int B_EPI = B_QK_DONE + NQ;       // local: the output tile is staged
+  static constexpr int kNBars = B_EPI + 1;
   static_assert(8 * kNBars <= 512, "barrier area");
   static constexpr uint32_t kMiscOff = kBarOff + 512;
   static constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;
@@ -200,7 +207,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(L::B_S_FULL + i), 1);
-      mbar_init(bar(L::B_S_EMPTY + i), 2 * 4 + 2);  // one group in each CTA + both V loaders
+      mbar_init(bar(L::B_S_EMPTY + i), 2 * 4);  // the tile's softmax group in each CTA
       mbar_init(bar(L::B_P_FULL + i), 2 * 4);
       mbar_init(bar(L::B_P_EMPTY + i), 1);
       mbar_init(bar(L::B_M_READY + i), 4);
@@ -209,6 +216,8 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
     mbar_init(bar(L::B_O_DONE), 1);
     mbar_init(bar(L::B_O_FINAL), 1);
     mbar_init(bar(L::B_FIN), kSoftmaxWarps);
+    for (int i = 0; i < L::NQ; ++i) mbar_init(bar(L::B_QK_DONE + i), 1);
+    mbar_init(bar(L::B_EPI), kSoftmaxWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -243,10 +252,13 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
         tma_load_2d(sb + L::kQStage + ci * 8192, &prm.tm_q_main, 128 * ci, qrow, bar(L::B_Q_MAIN), pol_q);
       if (rank == 0) mbar_arrive_expect_tx(bar(L::B_Q_ROPE), 2u * 64u * (uint32_t)box_q);
       tma_load_2d_pair(sb + L::kQRope, &prm.tm_q_rope, 512, qrow, lead(L::B_Q_ROPE), pol_q);
+      // block-table entries are read one tile ahead, off the critical path
+      int page_nx = n_pt > 0 ? page_of((int)rank) : 0;
       for (int j = 0; j < n_pt; ++j) {
         const int sk = j % NK;
+        const int page = page_nx;
+        if (j + 1 < n_pt) page_nx = page_of(2 * (j + 1) + (int)rank);
         if (!bounded_wait(bar(L::B_K_EMPTY + sk), ((j / NK) & 1) ^ 1, abort_flag, a.status)) break;
-        const int page = page_of(2 * j + (int)rank);
         const uint32_t ks = sb + L::kKOff + sk * L::kKSlot;
         const uint32_t full = lead(L::B_K_FULL + sk);
         if (rank == 0) mbar_arrive_expect_tx(bar(L::B_K_FULL + sk), 2u * L::kKSlot);
@@ -264,13 +276,17 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
     // ------------------------------------------------------------ V-ring loads
     if (lane == 0) {
       const uint64_t pol_v = policy_evict_first();  // last use of these bytes
+      int pg0_nx = n_pt > 0 ? page_of(0) : 0, pg1_nx = n_pt > 0 ? page_of(1) : 0;
       for (int j = 0; j < n_pt; ++j) {
-        const int sv = j % NV, buf = j & 1;
+        const int sv = j % NV;
+        const int pg0 = pg0_nx, pg1 = pg1_nx;
+        if (j + 1 < n_pt) {
+          pg0_nx = page_of(2 * (j + 1));
+          pg1_nx = page_of(2 * (j + 1) + 1);
+        }
         // the scores of tile j exist: its pages are in L2 now
-        if (!bounded_wait(bar(L::B_S_FULL + buf), (j >> 1) & 1, abort_flag, a.status)) break;
-        arrive_lead_relaxed(L::B_S_EMPTY + buf);
+        if (!bounded_wait(bar(L::B_QK_DONE + j % L::NQ), (j / L::NQ) & 1, abort_flag, a.status)) break;
         if (!bounded_wait(bar(L::B_V_EMPTY + sv), ((j / NV) & 1) ^ 1, abort_flag, a.status)) break;
-        const int pg0 = page_of(2 * j), pg1 = page_of(2 * j + 1);
         const uint32_t vs = sb + L::kVOff + sv * L::kVSlot;
         const uint32_t full = lead(L::B_V_FULL + sv);
         if (rank == 0) mbar_arrive_expect_tx(bar(L::B_V_FULL + sv), 2u * L::kVSlot);
@@ -311,6 +327,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
           mma_f8_ss_pair_e(d, dq_rope + (uint64_t)(kk * 2), dr + (uint64_t)(kk * 2), idq, 1u);
         mma_commit_pair_mc_e(bar(L::B_S_FULL + buf), 3);
         mma_commit_pair_mc_e(bar(L::B_K_EMPTY + sk), 3);
+        mma_commit_pair_mc_e(bar(L::B_QK_DONE + j % L::NQ), 3);
       }
     }
   } else if (warp == 2) {
@@ -498,14 +515,21 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         if (!(ok = warp_wait(bar(L::B_O_DONE), (j - 1) & 1, abort_flag, a.status))) break;
         tc_fence_after();
+        // two 32-column chunks per tensor-memory round trip (the score
+        // registers are free by now)
 #pragma unroll 1
-        for (int cc = 0; cc < 8; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(tmem + tl + kOCol + 32u * cc, o);
+        for (int cc = 0; cc < 8; cc += 2) {
+          uint32_t o0[32], o1[32];
+          tmem_ld32(tmem + tl + kOCol + 32u * cc, o0);
+          tmem_ld32(tmem + tl + kOCol + 32u * (cc + 1), o1);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tmem + tl + kOCol + 32u * cc, o);
+          for (int i = 0; i < 32; ++i) {
+            o0[i] = __float_as_uint(__uint_as_float(o0[i]) * alpha);
+            o1[i] = __float_as_uint(__uint_as_float(o1[i]) * alpha);
+          }
+          tmem_st32(tmem + tl + kOCol + 32u * cc, o0);
+          tmem_st32(tmem + tl + kOCol + 32u * (cc + 1), o1);
         }
         tmem_wait_st();
       }
@@ -537,26 +561,85 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
       }
     }
     if (ok) ok = warp_wait(bar(L::B_O_FINAL), 0, abort_flag, a.status);
+    // The output tile is staged in shared memory (the K and V rings are idle
+    // once every MMA has completed) and written back by whole rows: a warp
+    // then stores 512 contiguous bytes per instruction instead of 32 rows'
+    // scattered 16-byte pieces. Staging row r keeps its 16-byte chunk c at
+    // position c ^ (r & 7), so that neither the per-row writes nor the
+    // per-row reads conflict on shared-memory banks.
+    float* stage = reinterpret_cast<float*>(smem + L::kKOff);  // [64 rows][512] fp32
+    float* rowinv = mref;                                        // free once the loop is done
     if (ok) {
       tc_fence_after();
       const float inv = (le > 0.f) ? a.v_scale / le : 0.f;
-      const bool live = r < M;
-      const int64_t rg = row0 + r;
-      // group grp stores column half h = grp: output dims 256h + 128hf + [0, 128)
+      if (grp == 0 && hf == 0) rowinv[rl] = inv;
+      // group grp holds column half h = grp: output dims 256h + 128hf + [0, 128)
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t o[32];
         tmem_ld32(tmem + tl + kOCol + 128u * grp + 32u * cc, o);
         tmem_wait_ld();
-        if (!live) continue;
-        store_out_chunk(a, rg, s, 256 * grp + 128 * hf + 32 * cc, o, inv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int c = 64 * grp + 32 * hf + 8 * cc + i;  // 16-byte chunk of the 2 KB row
+          *reinterpret_cast<uint4*>(stage + rl * MLA_D_V + ((c ^ (rl & 7)) * 4)) =
+              make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        }
       }
-      if (live && grp == 0 && hf == 0) {
+      if (r < M && grp == 0 && hf == 0) {
+        const int64_t rg = row0 + r;
         const float lse_val = (le > 0.f) ? (m_fin - kSigma + log2f(le)) * kLn2 : -INFINITY;
         if (S == 1) {
           if (a.lse) a.lse[rg] = lse_val;
         } else {
           a.lse_part[rg * S + s] = lse_val;
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(L::B_EPI));
+    if (ok) ok = warp_wait(bar(L::B_EPI), 0, abort_flag, a.status);
+    if (ok) {
+      // softmax warp w writes local rows 8w .. 8w+7
+      const int w8 = warp - kSoftmaxWarp0;
+#pragma unroll 1
+      for (int i = 0; i < 8; ++i) {
+        const int rr = 8 * w8 + i;
+        if (64 * (int)rank + rr >= M) break;  // rows past the unit belong to no output
+        const float inv2 = rowinv[rr];
+        const int64_t rg2 = row0 + 64 * (int)rank + rr;
+        const float* srow = stage + rr * MLA_D_V;
+        if (S == 1) {
+          // BF16: lane writes 8 consecutive values (16 bytes) per step
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int c0 = 2 * lane + 64 * k;
+            const float4 x0 = *reinterpret_cast<const float4*>(srow + ((c0 ^ (rr & 7)) * 4));
+            const float4 x1 = *reinterpret_cast<const float4*>(srow + (((c0 + 1) ^ (rr & 7)) * 4));
+            const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(inv2 > 0.f ? v[2 * e] * inv2 : 0.f,
+                                                        inv2 > 0.f ? v[2 * e + 1] * inv2 : 0.f);
+              pk[e] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+            *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + rg2 * MLA_D_V + 4 * c0) =
+                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        } else {
+          float* dst = a.o_part + (rg2 * S + s) * MLA_D_V;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int c = lane + 32 * k;
+            float4 x = *reinterpret_cast<const float4*>(srow + ((c ^ (rr & 7)) * 4));
+            if (inv2 > 0.f) {
+              x.x *= inv2; x.y *= inv2; x.z *= inv2; x.w *= inv2;
+            } else {
+              x = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            *reinterpret_cast<float4*>(dst + 4 * c) = x;
+          }
         }
       }
     }
@@ -575,6 +658,8 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
   if (warp == 2 && lane == 0 && !*abort_flag) {
     for (int j = n_pt - 1; j >= 0 && j >= n_pt - NK; --j) drain_phase(bar(L::B_K_EMPTY + j % NK), (j / NK) & 1);
     for (int j = n_pt - 1; j >= 0 && j >= n_pt - NV; --j) drain_phase(bar(L::B_V_EMPTY + j % NV), (j / NV) & 1);
+    for (int j = n_pt - 1; j >= 0 && j >= n_pt - L::NQ; --j)
+      drain_phase(bar(L::B_QK_DONE + j % L::NQ), (j / L::NQ) & 1);
     for (int j = n_pt - 1; j >= 0 && j >= n_pt - 2; --j) {
       drain_phase(bar(L::B_P_EMPTY + (j & 1)), (j >> 1) & 1);
       drain_phase(bar(L::B_S_FULL + (j & 1)), (j >> 1) & 1);
