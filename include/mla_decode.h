@@ -51,7 +51,7 @@ extern "C" {
 #define MLA_D_V 512         /* V = first 512 dims of the cached row */
 #define MLA_PAGE_SIZE 64    /* tokens per cache page (the only page size supported) */
 #define MLA_MAX_ROWS 128    /* rows (heads x folded tokens) one CTA pair processes */
-#define MLA_NO_ALLOC_SCRATCH_BYTES (32u << 20) /* scratch of mla_decode_no_alloc, per device */
+#define MLA_NO_ALLOC_SCRATCH_BYTES (48u << 20) /* scratch of mla_decode_no_alloc, per device */
 
 typedef enum { MLA_BF16 = 0, MLA_FP16 = 1, MLA_FP8_E4M3 = 2 } mla_dtype;
 
@@ -64,6 +64,10 @@ typedef enum {
   MLA_ERR_CUDA = -5,              /* a CUDA runtime call failed */
   MLA_ERR_PLAN_MISMATCH = -6      /* plan fields inconsistent or not from mla_decode_plan */
 } mla_status;
+
+/* Work schedules of a plan (mla_plan.schedule). */
+#define MLA_SCHEDULE_SPLITS 0u
+#define MLA_SCHEDULE_BALANCED 1u
 
 /* Bits of the device status word (workspace header). */
 #define MLA_DEV_BAD_PAGE 0x1     /* block-table entry outside [0, num_pages): keys masked */
@@ -81,6 +85,16 @@ typedef enum {
 
 /*
  * Plan of one decode shape. Filled by mla_decode_plan; treat as read-only.
+ * Two work schedules exist (field `schedule`):
+ *   MLA_SCHEDULE_SPLITS: every unit is cut into split_kv chunks of
+ *     keys_per_split keys, one CTA (pair) each; partials [B*q_len*H, S, 512].
+ *   MLA_SCHEDULE_BALANCED (FP8 CTA-pair kernel): split_kv = P CTA pairs stay
+ *     resident; the units' 128-key tiles, counted from the device seq_lens,
+ *     are dealt out as equal contiguous ranges. A unit a pair covers whole
+ *     is written to out/lse directly; a unit cut between pairs leaves
+ *     partials in slots [2P, M, 512] (pair p: slot 2p for its first unit,
+ *     2p+1 for its last) that the combine merges. keys_per_split then only
+ *     bounds seq_len (>= max_seq_len).
  *   fold            F: query tokens folded into the row dimension
  *   q_groups        G = q_len / F; each (batch entry, group) is one unit
  *   rows_per_unit   M = H * F <= 128 query rows that share each K tile
@@ -99,8 +113,8 @@ typedef struct {
   int32_t split_kv, keys_per_split;
   int32_t kernel, num_ctas;
   uint64_t workspace_bytes, partial_offset, lse_offset;
-  uint32_t magic; /* set by the planner; checked by mla_decode */
-  uint32_t reserved;
+  uint32_t magic;    /* set by the planner; checked by mla_decode */
+  uint32_t schedule; /* MLA_SCHEDULE_* below */
 } mla_plan;
 
 /*

@@ -27,7 +27,7 @@ MLA_DEV_BAD_PAGE, MLA_DEV_SEQ_TOO_LONG, MLA_DEV_TIMEOUT = 0x1, 0x2, 0x4
 EXPORTED = ["mla_decode_plan", "mla_decode_plan_custom", "mla_decode", "mla_decode_partial",
             "mla_decode_combine", "mla_decode_status", "mla_status_string", "mla_version",
             "mla_decode_no_alloc", "mla_last_cuda_error"]
-MLA_NO_ALLOC_SCRATCH_BYTES = 32 << 20
+MLA_NO_ALLOC_SCRATCH_BYTES = 48 << 20
 
 
 class MlaPlan(ctypes.Structure):
@@ -38,7 +38,7 @@ class MlaPlan(ctypes.Structure):
         ("split_kv", ctypes.c_int32), ("keys_per_split", ctypes.c_int32),
         ("kernel", ctypes.c_int32), ("num_ctas", ctypes.c_int32),
         ("workspace_bytes", ctypes.c_uint64), ("partial_offset", ctypes.c_uint64),
-        ("lse_offset", ctypes.c_uint64), ("magic", ctypes.c_uint32), ("reserved", ctypes.c_uint32),
+        ("lse_offset", ctypes.c_uint64), ("magic", ctypes.c_uint32), ("schedule", ctypes.c_uint32),
     ]
 
     def as_dict(self):

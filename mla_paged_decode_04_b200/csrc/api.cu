@@ -76,6 +76,20 @@ int check_plan(const mla_plan* p) {
   if (p->kernel != MLA_KERNEL_TCGEN05 && p->kernel != MLA_KERNEL_SIMT && p->kernel != MLA_KERNEL_TCGEN05_SOLO)
     return MLA_ERR_PLAN_MISMATCH;
   if (p->kernel == MLA_KERNEL_TCGEN05_SOLO && p->dtype != MLA_FP8_E4M3) return MLA_ERR_PLAN_MISMATCH;
+  if (p->schedule != MLA_SCHEDULE_SPLITS && p->schedule != MLA_SCHEDULE_BALANCED) return MLA_ERR_PLAN_MISMATCH;
+  if (p->schedule == MLA_SCHEDULE_BALANCED) {
+    // FP8 CTA-pair kernel only; slots [2P, M, 512] fp32 + [2P, M] + unit table
+    if (p->kernel != MLA_KERNEL_TCGEN05 || p->dtype != MLA_FP8_E4M3 || p->split_kv > kNumSMs / 2)
+      return MLA_ERR_PLAN_MISMATCH;
+    const int64_t units = (int64_t)p->batch * p->q_groups;
+    if (units > kMaxBalancedUnits) return MLA_ERR_PLAN_MISMATCH;
+    const uint64_t slot_rows = 2ull * p->split_kv * p->rows_per_unit;
+    if (p->partial_offset < (uint64_t)kHeaderBytes || p->partial_offset % 256 != 0 ||
+        p->lse_offset < p->partial_offset + slot_rows * MLA_D_V * 4 || p->lse_offset % 256 != 0 ||
+        p->workspace_bytes < p->lse_offset + slot_rows * 4 + balanced_table_bytes(units))
+      return MLA_ERR_PLAN_MISMATCH;
+    return MLA_OK;
+  }
   const uint64_t rows = (uint64_t)p->batch * p->q_len * p->num_heads;
   if (p->split_kv > 1) {
     if (p->partial_offset < (uint64_t)kHeaderBytes || p->partial_offset % 256 != 0 ||
@@ -143,8 +157,13 @@ int prepare(const mla_plan* plan, const void* q, const void* kv_cache, int64_t n
   a->lse = lse;
   a->status = reinterpret_cast<int32_t*>(workspace);
   char* ws = reinterpret_cast<char*>(workspace);
-  a->o_part = p.split_kv > 1 ? reinterpret_cast<float*>(ws + p.partial_offset) : nullptr;
-  a->lse_part = p.split_kv > 1 ? reinterpret_cast<float*>(ws + p.lse_offset) : nullptr;
+  const bool partials = p.split_kv > 1 || p.schedule == MLA_SCHEDULE_BALANCED;
+  a->o_part = partials ? reinterpret_cast<float*>(ws + p.partial_offset) : nullptr;
+  a->lse_part = partials ? reinterpret_cast<float*>(ws + p.lse_offset) : nullptr;
+  a->sched = p.schedule == MLA_SCHEDULE_BALANCED
+                 ? reinterpret_cast<int32_t*>(ws + p.workspace_bytes -
+                                              balanced_table_bytes((int64_t)p.batch * p.q_groups))
+                 : nullptr;
   return MLA_OK;
 }
 
@@ -164,7 +183,12 @@ int run_partial(const DecodeArgs& a, cudaStream_t st) {
 }
 
 int run_combine(const DecodeArgs& a, cudaStream_t st) {
-  if (a.plan.batch == 0 || a.plan.split_kv == 1) return MLA_OK;
+  if (a.plan.batch == 0) return MLA_OK;
+  if (a.plan.schedule == MLA_SCHEDULE_BALANCED) {
+    const cudaError_t e = launch_combine_balanced(a, st);
+    return e == cudaSuccess ? MLA_OK : cuda_failure(e);
+  }
+  if (a.plan.split_kv == 1) return MLA_OK;
   const cudaError_t e = launch_combine(a, st);
   return e == cudaSuccess ? MLA_OK : cuda_failure(e);
 }

@@ -12,6 +12,16 @@ constexpr uint32_t kPlanMagic = 0x4d4c4131u;  // "MLA1"
 constexpr int kNumSMs = 148;                    // B200
 constexpr int kHeaderBytes = 256;               // workspace header (status word at offset 0)
 constexpr int kTileKeys = 64;                   // keys per tile = one cache page
+constexpr int kPairTileKeys = 128;              // keys per CTA-pair tile (one page per CTA)
+constexpr int kMaxBalancedUnits = 2048;         // units (entry x query group) the balanced schedule takes
+
+// Balanced schedule table at the end of the workspace: int32 start tile of
+// every unit (U + 1 entries, the last = W, the total pair tiles), then the
+// number of pairs that have work. Written by the partial kernel, read by the
+// combine.
+inline uint64_t balanced_table_bytes(int64_t units) {
+  return ((uint64_t)(units + 2) * 4 + 255) & ~uint64_t(255);
+}
 
 // Everything a launch needs, validated by the ABI layer.
 struct DecodeArgs {
@@ -29,7 +39,15 @@ struct DecodeArgs {
   int32_t* status;         // device status word
   float* o_part;           // fp32 [B*T*H, S, 512] (split_kv > 1)
   float* lse_part;         // fp32 [B*T*H, S]       (split_kv > 1)
+  int32_t* sched;          // balanced schedule table (MLA_SCHEDULE_BALANCED), else null
 };
+
+// Pair of the balanced schedule whose range holds pair tile x (0 <= x < W):
+// pair p covers [floor(W p / np), floor(W (p + 1) / np)).
+__host__ __device__ inline int balanced_pair_of(int64_t x, int64_t W, int np) {
+  return (int)(((x + 1) * np + W - 1) / W) - 1;
+}
+__host__ __device__ inline int64_t balanced_lo(int p, int64_t W, int np) { return W * p / np; }
 
 // Records `e` as this thread's last CUDA error (read by mla_last_cuda_error)
 // and returns MLA_ERR_CUDA.
@@ -43,5 +61,6 @@ cudaError_t launch_tc_partial(const DecodeArgs& a, cudaStream_t stream);      //
 cudaError_t launch_tc_fp8_partial(const DecodeArgs& a, cudaStream_t stream);  // FP8, per-CTA MMAs
 cudaError_t launch_tc_fp8_pair_partial(const DecodeArgs& a, cudaStream_t stream);  // FP8, CTA-pair MMAs
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_combine_balanced(const DecodeArgs& a, cudaStream_t stream);
 
 }  // namespace mla

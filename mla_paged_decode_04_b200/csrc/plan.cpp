@@ -12,6 +12,10 @@
 //   waves * (tiles per split + fixed CTA cost) + combine cost,
 // with one CTA pair per two SMs (74 pairs per wave on 148 SMs), and take the
 // cheapest. The result is memoised per shape.
+//
+// The FP8 CTA-pair kernel instead keeps all 74 pairs resident and balances
+// the work on the device (MLA_SCHEDULE_BALANCED): the plan only fixes the
+// number of pairs and sizes the partial slots and the schedule table.
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -101,7 +105,7 @@ int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, i
   }
   const int G = q_len / F;
   const int M = num_heads * F;
-  const int kern = kernel == MLA_KERNEL_AUTO ? MLA_KERNEL_TCGEN05 : kernel;
+  int kern = kernel == MLA_KERNEL_AUTO ? MLA_KERNEL_TCGEN05 : kernel;
   const int64_t units = (int64_t)batch * G;
   const int64_t tiles = ceil_div(max_seq_len, kTileKeys);
   // The tcgen05 kernel runs one CTA pair per two SMs; the SIMT kernel uses
@@ -119,23 +123,46 @@ int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, i
   p.fold = F;
   p.q_groups = G;
   p.rows_per_unit = M;
-  p.split_kv = S;
-  p.keys_per_split = chunk_tiles * kTileKeys;
-  p.kernel = kern;
-  p.num_ctas = (int32_t)(units * S * (kern == MLA_KERNEL_TCGEN05 ? 2 : 1));
   const uint64_t rows = (uint64_t)batch * q_len * num_heads;
-  uint64_t off = kHeaderBytes;
-  p.partial_offset = off;
-  p.lse_offset = off;
-  if (S > 1) {
+  // The balanced schedule keeps a per-pair piece list in shared memory; far
+  // more units than pairs can hold fall back to fixed splits (solo kernel).
+  if (kern == MLA_KERNEL_TCGEN05 && dtype == MLA_FP8_E4M3 && units > kMaxBalancedUnits)
+    kern = MLA_KERNEL_TCGEN05_SOLO;
+  p.kernel = kern;
+  if (kern == MLA_KERNEL_TCGEN05 && dtype == MLA_FP8_E4M3) {
+    const int P = split_kv > 0 ? (split_kv < kNumSMs / 2 ? split_kv : kNumSMs / 2) : kNumSMs / 2;
+    p.schedule = MLA_SCHEDULE_BALANCED;
+    p.split_kv = P;
+    p.keys_per_split = (int32_t)(ceil_div(max_seq_len > 0 ? max_seq_len : 1, kTileKeys) * kTileKeys);
+    p.num_ctas = 2 * P;
+    const uint64_t slots = 2 * (uint64_t)P;
+    uint64_t off = kHeaderBytes;
     p.partial_offset = off;
-    off += rows * (uint64_t)S * MLA_D_V * sizeof(float);
+    off += slots * (uint64_t)M * MLA_D_V * sizeof(float);
     off = (off + 255) & ~uint64_t(255);
     p.lse_offset = off;
-    off += rows * (uint64_t)S * sizeof(float);
+    off += slots * (uint64_t)M * sizeof(float);
     off = (off + 255) & ~uint64_t(255);
+    off += balanced_table_bytes(units);  // unit start table, at the end of the workspace
+    p.workspace_bytes = off;
+  } else {
+    p.schedule = MLA_SCHEDULE_SPLITS;
+    p.split_kv = S;
+    p.keys_per_split = chunk_tiles * kTileKeys;
+    p.num_ctas = (int32_t)(units * S * (kern == MLA_KERNEL_TCGEN05 || kern == MLA_KERNEL_TCGEN05_SOLO ? 2 : 1));
+    uint64_t off = kHeaderBytes;
+    p.partial_offset = off;
+    p.lse_offset = off;
+    if (S > 1) {
+      p.partial_offset = off;
+      off += rows * (uint64_t)S * MLA_D_V * sizeof(float);
+      off = (off + 255) & ~uint64_t(255);
+      p.lse_offset = off;
+      off += rows * (uint64_t)S * sizeof(float);
+      off = (off + 255) & ~uint64_t(255);
+    }
+    p.workspace_bytes = off;
   }
-  p.workspace_bytes = off;
   p.magic = kPlanMagic;
   {
     std::lock_guard<std::mutex> lk(g_mu);

@@ -1,4 +1,5 @@
-// Split-KV partial kernel for FP8 E4M3 inputs with CTA-pair tensor-core MMAs.
+// Split-KV partial kernel for FP8 E4M3 inputs with CTA-pair tensor-core MMAs
+// and a balanced, persistent schedule.
 //
 // The first of the two decode kernels (TokenSpeed MLA article
 // 最快MLA内核背后的秘密, section 二) with query-token folding (section 三), using
@@ -6,13 +7,22 @@
 // tcgen05.mma together (cta_group::2, M = 128), each holding half of the
 // operands and half of the result.
 //
-// Work split. A pair owns one (entry, query group, split) and walks it in
-// pair tiles of 128 keys = two cache pages; page 2j of the split goes to CTA
-// 0 and page 2j+1 to CTA 1.
+// Schedule. The pairs stay resident (one per two SMs). A unit (batch entry,
+// query group) of n keys is ceil(n / 128) pair tiles of two cache pages; the
+// units' tiles, counted from the device seq_lens, form one sequence that is
+// dealt out as equal contiguous ranges, one per pair. A pair walks its range
+// as pieces (the part of one unit inside the range): a piece that is a whole
+// unit writes out / lse directly; a unit cut between pairs leaves partial O
+// and LSE in the pair's slot (2p for its first piece, 2p + 1 for its last),
+// merged by the combine kernel. Every pair therefore does the same amount of
+// work whatever the length mix, and the pipeline runs on across pieces. This
+// is the article's split_kv auto-sizing (section 二) made exact on the device.
+//
+// Inside a pair tile, page 2j of the piece goes to CTA 0 and page 2j+1 to CTA 1.
 //  * S = Q.K^T (N = 128 keys): CTA c supplies query rows [64c, 64c+64) as
 //    the A operand (tensor memory) and its own page as B (shared memory);
-//    it receives S for its 64 rows and all 128 keys. Every score is computed
-//    once: no row, page or softmax work is duplicated in the pair.
+//    it receives S for its 64 rows and all 128 keys. No score, page or
+//    softmax work is duplicated in the pair.
 //  * Softmax: CTA c finishes its own 64 rows. S row r of a CTA lies in TMEM
 //    lane r (keys 0..63, the leader's page) and lane 64+r (keys 64..127), so
 //    two threads of different warps share a row and swap their maxima
@@ -39,9 +49,12 @@
 // S MMAs; warp 2 issues the P.V MMAs (leader); warp 3 lane 0 loads the V
 // ring; warps 4-11 are two softmax groups of four warps taking alternate
 // pair tiles (one thread per (row, key half), 64 keys each), which also do
-// the O rescales and the epilogue. Barriers the MMA issuer waits on live in
-// the leader; the follower's loads and arrivals reach them through cluster
-// addresses. MMA completions are multicast to both CTAs.
+// the O rescales and the epilogue of every piece. Ring slots and their
+// barrier phases follow a tile counter that runs across the pieces; the
+// per-piece barriers (Q, O_FINAL, FIN, EPI, O_FREE) advance once per piece.
+// Barriers the MMA issuer waits on live in the leader; the follower's loads
+// and arrivals reach them through cluster addresses. MMA completions are
+// multicast to both CTAs.
 //
 // Every wait is bounded; on expiry the CTA sets MLA_DEV_TIMEOUT, leaves the
 // pipeline, waits for its peer at the final cluster barrier, frees TMEM and
@@ -60,31 +73,46 @@ using namespace ptx;
 constexpr int kTwoTermKeys = 16384;  // entries shorter than this use two-term P
 constexpr float kTau = 2.f;          // lazy-rescale threshold (log2 units)
 constexpr float kSigma = 6.f;        // P <= 2^(kTau + kSigma) = 256 <= 448
-constexpr int kPairKeys = 128;       // keys per pair tile (one page per CTA)
+constexpr int kMaxPieces = 64;       // pieces per pair (units its range touches)
+constexpr int kMinPairTiles = 2;     // fewer tiles than this per pair: use fewer pairs
+
+// One piece: pair tiles [t0, t1) of unit u.
+struct Piece {
+  int u, t0, t1;
+};
+struct SchedInfo {
+  int npc;  // pieces of this pair
+  int two;  // some piece needs two-term P
+};
+// Schedule area at the start of shared memory (the same place in both layouts).
+constexpr uint32_t kSchedBytes = 1024;
+static_assert(kMaxPieces * sizeof(Piece) + sizeof(SchedInfo) <= kSchedBytes, "schedule area");
 
 template <bool kTwo>
 struct PairLayout {
   static constexpr int NK = 3;                                  // K-ring slots: own page
   static constexpr int NV = 2;                                  // V-ring slots: 256 V columns of both pages
-  static constexpr uint32_t kQRope = 0;                         // 64 rows x 64 B (SW64)
+  static constexpr uint32_t kQRope = kSchedBytes;               // 64 rows x 64 B (SW64)
   static constexpr uint32_t kPPlane = 64 * 128;                 // 64 rows x 128 keys E4M3 (SW128)
   static constexpr uint32_t kPBuf = (kTwo ? 2 : 1) * kPPlane;   // hi (and lo) plane
-  static constexpr uint32_t kPOff = 4096;                       // P[2 buffers]
+  static constexpr uint32_t kPOff = kQRope + 5120;              // P[2 buffers] (1024-aligned)
   static constexpr uint32_t kKSlot = 4 * 8192 + 64 * 64;        // 4 latent chunks (SW128) + rope (SW64)
   static constexpr uint32_t kKOff = kPOff + 2 * kPBuf;
   static constexpr uint32_t kVSlot = 4 * 8192;                  // [column half h][page] chunks (SW128)
   static constexpr uint32_t kVOff = kKOff + NK * kKSlot;
-  // Q latent dims (64 rows x 512 B) are staged in the last V slot, which is
-  // first filled after the S MMA of tile NV-1 (and so after Q reached TMEM).
+  // Q latent dims (64 rows x 512 B) are staged in the last V slot: the K
+  // loader fills it once the previous piece's MMAs are all done, and the V
+  // loader refills it only after the piece's first S MMAs (so after Q
+  // reached TMEM).
   static constexpr uint32_t kQStage = kVOff + (NV - 1) * kVSlot;
   static constexpr uint32_t kMOff = kVOff + NV * kVSlot;        // row reference maxima [tile parity][64]
   static constexpr uint32_t kXOff = kMOff + 512;                // half-row maxima [group][phase][half][64]
   static constexpr uint32_t kFinOff = kXOff + 2048;             // final (l, m) [l|m][group][half][64]
   static constexpr uint32_t kBarOff = kFinOff + 2048;
   // barriers ("leader": only the leader's copy is used)
-  static constexpr int B_Q_MAIN = 0;                 // local: staged Q latent landed
-  static constexpr int B_Q_ROPE = 1;                 // leader: both CTAs' Q rope landed
-  static constexpr int B_Q_TMEM = 2;                 // leader: both CTAs copied Q into TMEM
+  static constexpr int B_Q_MAIN = 0;                 // local, per piece: staged Q latent landed
+  static constexpr int B_Q_ROPE = 1;                 // leader, per piece: both CTAs' Q rope landed
+  static constexpr int B_Q_TMEM = 2;                 // leader, per piece: both CTAs copied Q into TMEM
   static constexpr int B_K_FULL = 3;                 // leader, + K slot: both pages landed
   static constexpr int B_K_EMPTY = B_K_FULL + NK;    // both, + K slot
   static constexpr int B_V_FULL = B_K_EMPTY + NK;    // leader, + V slot
@@ -94,23 +122,27 @@ struct PairLayout {
   static constexpr int B_P_FULL = B_S_EMPTY + 2;     // leader, + buffer
   static constexpr int B_P_EMPTY = B_P_FULL + 2;     // both, + buffer
   static constexpr int B_O_DONE = B_P_EMPTY + 2;     // both
-  static constexpr int B_O_FINAL = B_O_DONE + 1;     // both: completes once, after the last P.V
+  static constexpr int B_O_FINAL = B_O_DONE + 1;     // both, per piece: after the piece's last P.V
   static constexpr int B_M_READY = B_O_FINAL + 1;    // local, + tile parity
   static constexpr int B_X = B_M_READY + 2;          // local, + group: half-row maxima exchanged
-  static constexpr int B_FIN = B_X + 2;              // local: both groups published (l, m)
+  static constexpr int B_FIN = B_X + 2;              // local, per piece: both groups published (l, m)
   // both, + tile % NQ: the scores of the tile exist (the V loads may go).
   // NQ = 6 rules out phase aliasing: S = Q.K^T of tile j+6 needs the scores
   // of tile j+4 read, which needs P of tile j+2 written, which needs the
   // P.V of tile j done, which needs the V loads of tile j issued.
   static constexpr int NQ = 6;
   static constexpr int B_QK_DONE = B_FIN + 1;
-  static constexpr int B_EPI = B_QK_DONE + NQ;       // local: the output tile is staged
-  static constexpr int kNBars = B_EPI + 1;
+  static constexpr int B_EPI = B_QK_DONE + NQ;       // local, per piece: the output tile is staged
+  static constexpr int B_O_FREE = B_EPI + 1;         // leader, per piece: both CTAs read O
+  static constexpr int kNBars = B_O_FREE + 1;
   static_assert(8 * kNBars <= 512, "barrier area");
   static constexpr uint32_t kMiscOff = kBarOff + 512;
   static constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;
   static_assert(kPOff % 1024 == 0 && kKOff % 1024 == 0 && kKSlot % 1024 == 0 && kVOff % 1024 == 0, "alignment");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
+  // the last piece's epilogue stages the 64 x 512 fp32 output tile in the
+  // (then idle) K and V rings
+  static_assert(NK * kKSlot + NV * kVSlot >= 64 * MLA_D_V * 4, "staging area");
 };
 constexpr uint32_t kPairSmemBytes =
     PairLayout<true>::kSmemBytes > PairLayout<false>::kSmemBytes ? PairLayout<true>::kSmemBytes
@@ -130,13 +162,129 @@ struct PairParams {
   DecodeArgs a;
 };
 
+// Pair tiles of unit u (= b * G + g): every group of entry b sees its keys.
+__device__ __forceinline__ int unit_tiles(const DecodeArgs& a, int u, bool flag) {
+  const int n = effective_seq_len(a, u / a.plan.q_groups, flag);
+  return (n + kPairTileKeys - 1) / kPairTileKeys;
+}
+
+// One warp: the balanced schedule of this pair. Every lane takes a run of
+// consecutive units and a warp scan gives each run's first tile; the pieces
+// of the pair's range [lo, hi) go to `pcs` in unit order. CTA 0 of pair 0
+// also writes the unit start table the combine reads.
+__device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, Piece* pcs, SchedInfo* info) {
+  const mla_plan& p = a.plan;
+  const int lane = threadIdx.x & 31;
+  const int U = p.batch * p.q_groups;
+  const int per = (U + 31) / 32;
+  const int u_beg = min(U, lane * per), u_end = min(U, u_beg + per);
+  const bool writer = pair == 0 && rank == 0;
+  int run = 0;
+  for (int u = u_beg; u < u_end; ++u) run += unit_tiles(a, u, writer && u % p.q_groups == 0);
+  int excl = run;  // inclusive prefix, then exclusive
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, excl, d);
+    if (lane >= d) excl += y;
+  }
+  const int W = __shfl_sync(0xffffffffu, excl, 31);
+  excl -= run;
+  const int np = max(1, min(p.split_kv, (W + kMinPairTiles - 1) / kMinPairTiles));
+  const int64_t lo = pair < np ? balanced_lo(pair, W, np) : W;
+  const int64_t hi = pair < np ? balanced_lo(pair + 1, W, np) : W;
+  if (writer) {
+    int start = excl;
+    for (int u = u_beg; u < u_end; ++u) {
+      a.sched[u] = start;
+      start += unit_tiles(a, u, false);
+    }
+    if (lane == 31) {
+      a.sched[U] = W;
+      a.sched[U + 1] = np;
+    }
+  }
+  // pieces: units of this lane's run that meet [lo, hi)
+  int cnt = 0;
+  {
+    int start = excl;
+    for (int u = u_beg; u < u_end; ++u) {
+      const int t = unit_tiles(a, u, false);
+      if (t > 0 && start < hi && start + t > lo) ++cnt;
+      start += t;
+    }
+  }
+  int base = cnt;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, base, d);
+    if (lane >= d) base += y;
+  }
+  const int npc = __shfl_sync(0xffffffffu, base, 31);
+  base -= cnt;
+  int two = 0;
+  {
+    int start = excl, k = base;
+    for (int u = u_beg; u < u_end; ++u) {
+      const int t = unit_tiles(a, u, false);
+      if (t > 0 && start < hi && start + t > lo) {
+        if (k < kMaxPieces) {
+          pcs[k].u = u;
+          pcs[k].t0 = lo > start ? (int)(lo - start) : 0;
+          pcs[k].t1 = hi - start < t ? (int)(hi - start) : t;
+          if (effective_seq_len(a, u / p.q_groups, false) < kTwoTermKeys) two = 1;
+        }
+        ++k;
+      }
+      start += t;
+    }
+  }
+  two = __any_sync(0xffffffffu, two);
+  if (lane == 0) {
+    info->npc = npc;
+    info->two = two;
+  }
+}
+
+// Per-piece constants every role derives the same way.
+struct PieceCtx {
+  int b, g, n, key0, key1, n_pt, n_tiles, tile0;
+  int64_t row0;
+  const int32_t* table;
+  bool whole;  // the piece is the whole unit: final output, not a partial
+  bool two;    // two-term P
+};
+
+__device__ __forceinline__ PieceCtx piece_ctx(const DecodeArgs& a, const Piece& pc, bool kTwo) {
+  const mla_plan& p = a.plan;
+  PieceCtx c;
+  c.b = pc.u / p.q_groups;
+  c.g = pc.u % p.q_groups;
+  c.n = effective_seq_len(a, c.b, false);
+  c.key0 = pc.t0 * kPairTileKeys;
+  c.key1 = min(c.n, pc.t1 * kPairTileKeys);
+  c.n_pt = pc.t1 - pc.t0;
+  c.n_tiles = (c.key1 - c.key0 + kTileKeys - 1) / kTileKeys;
+  c.tile0 = c.key0 / kTileKeys;
+  c.row0 = (int64_t)c.b * p.q_len * p.num_heads + (int64_t)c.g * p.rows_per_unit;
+  c.table = a.block_tables + (int64_t)c.b * a.max_pages_per_seq;
+  c.whole = pc.t0 == 0 && c.key1 >= c.n;
+  c.two = kTwo && c.n < kTwoTermKeys;
+  return c;
+}
+
+// page of 64-key tile t of the piece (t < n_tiles), 0 when absent or invalid
+__device__ __forceinline__ int piece_page(const DecodeArgs& a, const PieceCtx& c, int t) {
+  if (t >= c.n_tiles) return 0;
+  const int pg = c.table[c.tile0 + t];
+  return (pg < 0 || (int64_t)pg >= a.num_pages) ? 0 : pg;
+}
+
 template <bool kTwo>
-__device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_raw) {
+__device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, const Piece* pcs, int npc) {
   using L = PairLayout<kTwo>;
-  constexpr int NK = L::NK, NV = L::NV;
+  constexpr int NK = L::NK, NV = L::NV, NQ = L::NQ;
   const DecodeArgs& a = prm.a;
   const mla_plan& p = a.plan;
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   auto bar = [&](int i) -> uint32_t { return sb + L::kBarOff + 8u * (uint32_t)i; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
@@ -145,38 +293,11 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();  // 0 = leader
   const int pair = blockIdx.x >> 1;
-  const int G = p.q_groups, S = p.split_kv, T = p.q_len, H = p.num_heads, M = p.rows_per_unit;
-  const int g = pair % G;
-  const int s = (pair / G) % S;
-  const int b = pair / (G * S);
-  const int n = effective_seq_len(a, b, rank == 0 && s == 0 && g == 0 && threadIdx.x == 0);
-  const int key0 = s * p.keys_per_split;
-  const int64_t row0 = (int64_t)b * T * H + (int64_t)g * M;
+  const int T = p.q_len, H = p.num_heads, M = p.rows_per_unit;
   const int box_q = M < 64 ? M : 64;  // query rows per TMA box (the tensor maps' box height)
+  // slot of piece k: 2p for the pair's first piece, 2p + 1 for its last
+  auto slot_of = [&](int k) -> int64_t { return 2 * (int64_t)pair + (k == 0 ? 0 : 1); };
 
-  if (key0 >= n) {  // same decision in both CTAs of the pair
-    if (S == 1) {
-      for (int r = threadIdx.x; r < 64; r += blockDim.x) {
-        const int rr = 64 * (int)rank + r;
-        if (rr >= M) continue;
-        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + (row0 + rr) * MLA_D_V);
-        for (int i = 0; i < 64; ++i) dst[i] = make_uint4(0, 0, 0, 0);
-        if (a.lse) a.lse[row0 + rr] = -INFINITY;
-      }
-    }
-    return;
-  }
-  const int key1 = min(n, key0 + p.keys_per_split);
-  const int n_tiles = (key1 - key0 + kTileKeys - 1) / kTileKeys;  // 64-key pages
-  const int n_pt = (n_tiles + 1) / 2;                              // pair tiles
-  const int tile0 = key0 / kTileKeys;
-  const int32_t* table = a.block_tables + (int64_t)b * a.max_pages_per_seq;
-  // page of 64-key tile t of the split (t < n_tiles), 0 when absent or invalid
-  auto page_of = [&](int t) -> int {
-    if (t >= n_tiles) return 0;
-    const int pg = table[tile0 + t];
-    return (pg < 0 || (int64_t)pg >= a.num_pages) ? 0 : pg;
-  };
   // the leader's copy of barrier i, as a cluster address
   auto lead = [&](int i) -> uint32_t { return mapa(bar(i), 0); };
   // Arrive on the leader's barrier i: a plain local arrive in the leader; in
@@ -216,8 +337,9 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
     mbar_init(bar(L::B_O_DONE), 1);
     mbar_init(bar(L::B_O_FINAL), 1);
     mbar_init(bar(L::B_FIN), kSoftmaxWarps);
-    for (int i = 0; i < L::NQ; ++i) mbar_init(bar(L::B_QK_DONE + i), 1);
+    for (int i = 0; i < NQ; ++i) mbar_init(bar(L::B_QK_DONE + i), 1);
     mbar_init(bar(L::B_EPI), kSoftmaxWarps);
+    mbar_init(bar(L::B_O_FREE), 2 * kSoftmaxWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -235,6 +357,8 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
   cluster_sync();  // both CTAs' barriers and TMEM exist before any cross-CTA use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  int n_all = 0;  // pair tiles over all pieces
+  for (int k = 0; k < npc; ++k) n_all += pcs[k].t1 - pcs[k].t0;
 
   if (warp == 0) {
     // ------------------------------------------------------------ Q and K-ring loads
@@ -245,143 +369,185 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
       prefetch_tmap(&prm.tm_kv_rope);
       const uint64_t pol_q = policy_evict_first();
       const uint64_t pol_kv = policy_evict_last();  // read again right away for V
-      const int qrow = (int)row0 + 64 * (int)rank;  // rows past the unit are read but never stored
-      mbar_arrive_expect_tx(bar(L::B_Q_MAIN), 4u * 128u * (uint32_t)box_q);
-#pragma unroll
-      for (int ci = 0; ci < 4; ++ci)
-        tma_load_2d(sb + L::kQStage + ci * 8192, &prm.tm_q_main, 128 * ci, qrow, bar(L::B_Q_MAIN), pol_q);
-      if (rank == 0) mbar_arrive_expect_tx(bar(L::B_Q_ROPE), 2u * 64u * (uint32_t)box_q);
-      tma_load_2d_pair(sb + L::kQRope, &prm.tm_q_rope, 512, qrow, lead(L::B_Q_ROPE), pol_q);
-      // block-table entries are read one tile ahead, off the critical path
-      int page_nx = n_pt > 0 ? page_of((int)rank) : 0;
-      for (int j = 0; j < n_pt; ++j) {
-        const int sk = j % NK;
-        const int page = page_nx;
-        if (j + 1 < n_pt) page_nx = page_of(2 * (j + 1) + (int)rank);
-        if (!bounded_wait(bar(L::B_K_EMPTY + sk), ((j / NK) & 1) ^ 1, abort_flag, a.status)) break;
-        const uint32_t ks = sb + L::kKOff + sk * L::kKSlot;
-        const uint32_t full = lead(L::B_K_FULL + sk);
-        if (rank == 0) mbar_arrive_expect_tx(bar(L::B_K_FULL + sk), 2u * L::kKSlot);
+      int jt = 0;     // tile counter across pieces
+      bool ok = true;
+      for (int k = 0; ok && k < npc; ++k) {
+        const PieceCtx c = piece_ctx(a, pcs[k], kTwo);
+        if (k > 0) {
+          // Q rope, Q in TMEM and the staging slot are free once every MMA of
+          // the previous piece is done: its O_FINAL phase. (The V ring's own
+          // barriers could be two phases behind here, since S runs ahead of
+          // P.V; O_FINAL cannot, as its next phase needs this very load.)
+          if (!(ok = bounded_wait(bar(L::B_O_FINAL), (k - 1) & 1, abort_flag, a.status))) break;
+        }
+        const int qrow = (int)c.row0 + 64 * (int)rank;  // rows past the unit are read but never stored
+        mbar_arrive_expect_tx(bar(L::B_Q_MAIN), 4u * 128u * (uint32_t)box_q);
 #pragma unroll
         for (int ci = 0; ci < 4; ++ci)
-          tma_load_2d_pair(ks + ci * 8192, &prm.tm_kv_main, 128 * ci, page * kTileKeys, full, pol_kv);
-        tma_load_2d_pair(ks + 4 * 8192, &prm.tm_kv_rope, 512, page * kTileKeys, full, pol_kv);
+          tma_load_2d(sb + L::kQStage + ci * 8192, &prm.tm_q_main, 128 * ci, qrow, bar(L::B_Q_MAIN), pol_q);
+        if (rank == 0) mbar_arrive_expect_tx(bar(L::B_Q_ROPE), 2u * 64u * (uint32_t)box_q);
+        tma_load_2d_pair(sb + L::kQRope, &prm.tm_q_rope, 512, qrow, lead(L::B_Q_ROPE), pol_q);
+        // block-table entries are read one tile ahead, off the critical path
+        int page_nx = piece_page(a, c, (int)rank);
+        for (int j = 0; j < c.n_pt; ++j, ++jt) {
+          const int sk = jt % NK;
+          const int page = page_nx;
+          if (j + 1 < c.n_pt) page_nx = piece_page(a, c, 2 * (j + 1) + (int)rank);
+          if (!(ok = bounded_wait(bar(L::B_K_EMPTY + sk), ((jt / NK) & 1) ^ 1, abort_flag, a.status))) break;
+          const uint32_t ks = sb + L::kKOff + sk * L::kKSlot;
+          const uint32_t full = lead(L::B_K_FULL + sk);
+          if (rank == 0) mbar_arrive_expect_tx(bar(L::B_K_FULL + sk), 2u * L::kKSlot);
+#pragma unroll
+          for (int ci = 0; ci < 4; ++ci)
+            tma_load_2d_pair(ks + ci * 8192, &prm.tm_kv_main, 128 * ci, page * kTileKeys, full, pol_kv);
+          tma_load_2d_pair(ks + 4 * 8192, &prm.tm_kv_rope, 512, page * kTileKeys, full, pol_kv);
+        }
       }
       // The leader's K_FULL phases count both CTAs' bytes: the leader waits for
       // the last ones before the pair may leave (the follower waits at the
       // final cluster barrier).
-      if (rank == 0) drain_loads(bar(L::B_K_FULL), NK, n_pt);
+      if (rank == 0) drain_loads(bar(L::B_K_FULL), NK, n_all);
     }
   } else if (warp == 3) {
     // ------------------------------------------------------------ V-ring loads
     if (lane == 0) {
       const uint64_t pol_v = policy_evict_first();  // last use of these bytes
-      int pg0_nx = n_pt > 0 ? page_of(0) : 0, pg1_nx = n_pt > 0 ? page_of(1) : 0;
-      for (int j = 0; j < n_pt; ++j) {
-        const int sv = j % NV;
-        const int pg0 = pg0_nx, pg1 = pg1_nx;
-        if (j + 1 < n_pt) {
-          pg0_nx = page_of(2 * (j + 1));
-          pg1_nx = page_of(2 * (j + 1) + 1);
-        }
-        // the scores of tile j exist: its pages are in L2 now
-        if (!bounded_wait(bar(L::B_QK_DONE + j % L::NQ), (j / L::NQ) & 1, abort_flag, a.status)) break;
-        if (!bounded_wait(bar(L::B_V_EMPTY + sv), ((j / NV) & 1) ^ 1, abort_flag, a.status)) break;
-        const uint32_t vs = sb + L::kVOff + sv * L::kVSlot;
-        const uint32_t full = lead(L::B_V_FULL + sv);
-        if (rank == 0) mbar_arrive_expect_tx(bar(L::B_V_FULL + sv), 2u * L::kVSlot);
+      int jt = 0;
+      bool ok = true;
+      for (int k = 0; ok && k < npc; ++k) {
+        const PieceCtx c = piece_ctx(a, pcs[k], kTwo);
+        int pg0_nx = piece_page(a, c, 0), pg1_nx = piece_page(a, c, 1);
+        for (int j = 0; j < c.n_pt; ++j, ++jt) {
+          const int sv = jt % NV;
+          const int pg0 = pg0_nx, pg1 = pg1_nx;
+          if (j + 1 < c.n_pt) {
+            pg0_nx = piece_page(a, c, 2 * (j + 1));
+            pg1_nx = piece_page(a, c, 2 * (j + 1) + 1);
+          }
+          // the scores of the tile exist: its pages are in L2 now
+          if (!(ok = bounded_wait(bar(L::B_QK_DONE + jt % NQ), (jt / NQ) & 1, abort_flag, a.status))) break;
+          if (!(ok = bounded_wait(bar(L::B_V_EMPTY + sv), ((jt / NV) & 1) ^ 1, abort_flag, a.status))) break;
+          const uint32_t vs = sb + L::kVOff + sv * L::kVSlot;
+          const uint32_t full = lead(L::B_V_FULL + sv);
+          if (rank == 0) mbar_arrive_expect_tx(bar(L::B_V_FULL + sv), 2u * L::kVSlot);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int x = 128 * (2 * h + (int)rank);  // this CTA's 128 of the 256 columns of half h
-          tma_load_2d_pair(vs + h * 16384, &prm.tm_kv_main, x, pg0 * kTileKeys, full, pol_v);
-          tma_load_2d_pair(vs + h * 16384 + 8192, &prm.tm_kv_main, x, pg1 * kTileKeys, full, pol_v);
+          for (int h = 0; h < 2; ++h) {
+            const int x = 128 * (2 * h + (int)rank);  // this CTA's 128 of the 256 columns of half h
+            tma_load_2d_pair(vs + h * 16384, &prm.tm_kv_main, x, pg0 * kTileKeys, full, pol_v);
+            tma_load_2d_pair(vs + h * 16384 + 8192, &prm.tm_kv_main, x, pg1 * kTileKeys, full, pol_v);
+          }
         }
       }
-      if (rank == 0) drain_loads(bar(L::B_V_FULL), NV, n_pt);
+      if (rank == 0) drain_loads(bar(L::B_V_FULL), NV, n_all);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ S = Q.K^T issuer (leader)
     if (rank == 0) {
-      constexpr uint32_t idq = instr_desc(0, 0, 0, 128, kPairKeys);  // E4M3 x E4M3, K-major B
-      bool ok = warp_wait(bar(L::B_Q_ROPE), 0, abort_flag, a.status) &&
-                warp_wait(bar(L::B_Q_TMEM), 0, abort_flag, a.status);
+      constexpr uint32_t idq = instr_desc(0, 0, 0, 128, kPairTileKeys);  // E4M3 x E4M3, K-major B
       const uint64_t dq_rope = smem_desc(sb + L::kQRope, 16, 512, kSw64);
-      for (int j = 0; ok && j < n_pt; ++j) {
-        const int sk = j % NK, buf = j & 1;
-        if (!(ok = warp_wait(bar(L::B_K_FULL + sk), (j / NK) & 1, abort_flag, a.status))) break;
-        if (!(ok = warp_wait(bar(L::B_S_EMPTY + buf), ((j >> 1) & 1) ^ 1, abort_flag, a.status))) break;
-        tc_fence_after();
-        const uint32_t d = tmem + kSCol + 64u * buf;
-        const uint32_t ks = sb + L::kKOff + sk * L::kKSlot;
+      int jt = 0;
+      bool ok = true;
+      for (int k = 0; ok && k < npc; ++k) {
+        const int n_pt = pcs[k].t1 - pcs[k].t0;
+        if (!(ok = warp_wait(bar(L::B_Q_ROPE), k & 1, abort_flag, a.status) &&
+                   warp_wait(bar(L::B_Q_TMEM), k & 1, abort_flag, a.status)))
+          break;
+        for (int j = 0; j < n_pt; ++j, ++jt) {
+          const int sk = jt % NK, buf = jt & 1;
+          if (!(ok = warp_wait(bar(L::B_K_FULL + sk), (jt / NK) & 1, abort_flag, a.status))) break;
+          if (!(ok = warp_wait(bar(L::B_S_EMPTY + buf), ((jt >> 1) & 1) ^ 1, abort_flag, a.status))) break;
+          tc_fence_after();
+          const uint32_t d = tmem + kSCol + 64u * buf;
+          const uint32_t ks = sb + L::kKOff + sk * L::kKSlot;
 #pragma unroll
-        for (int ci = 0; ci < 4; ++ci) {
-          const uint64_t dk = smem_desc(ks + ci * 8192, 16, 1024, kSw128);
+          for (int ci = 0; ci < 4; ++ci) {
+            const uint64_t dk = smem_desc(ks + ci * 8192, 16, 1024, kSw128);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f8_ts_pair_e(d, tmem + kQCol + (uint32_t)(8 * (4 * ci + kk)), dk + (uint64_t)((kk * 32) >> 4), idq,
-                             (ci | kk) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f8_ts_pair_e(d, tmem + kQCol + (uint32_t)(8 * (4 * ci + kk)), dk + (uint64_t)((kk * 32) >> 4),
+                               idq, (ci | kk) ? 1u : 0u);
+          }
+          const uint64_t dr = smem_desc(ks + 4 * 8192, 16, 512, kSw64);
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk)
+            mma_f8_ss_pair_e(d, dq_rope + (uint64_t)(kk * 2), dr + (uint64_t)(kk * 2), idq, 1u);
+          mma_commit_pair_mc_e(bar(L::B_S_FULL + buf), 3);
+          mma_commit_pair_mc_e(bar(L::B_K_EMPTY + sk), 3);
+          mma_commit_pair_mc_e(bar(L::B_QK_DONE + jt % NQ), 3);
         }
-        const uint64_t dr = smem_desc(ks + 4 * 8192, 16, 512, kSw64);
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk)
-          mma_f8_ss_pair_e(d, dq_rope + (uint64_t)(kk * 2), dr + (uint64_t)(kk * 2), idq, 1u);
-        mma_commit_pair_mc_e(bar(L::B_S_FULL + buf), 3);
-        mma_commit_pair_mc_e(bar(L::B_K_EMPTY + sk), 3);
-        mma_commit_pair_mc_e(bar(L::B_QK_DONE + j % L::NQ), 3);
       }
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ O += P.V issuer (leader)
     if (rank == 0) {
       constexpr uint32_t idp = instr_desc(0, 0, 1, 128, 256);  // V is MN-major
+      int jt = 0;
       bool ok = true;
-      for (int j = 0; ok && j < n_pt; ++j) {
-        const int buf = j & 1, sv = j % NV;
-        if (!(ok = warp_wait(bar(L::B_V_FULL + sv), (j / NV) & 1, abort_flag, a.status))) break;
-        if (!(ok = warp_wait(bar(L::B_P_FULL + buf), (j >> 1) & 1, abort_flag, a.status))) break;
-        tc_fence_after();
-        const uint32_t vs = sb + L::kVOff + sv * L::kVSlot;
-        const uint64_t dp = smem_desc(sb + L::kPOff + buf * L::kPBuf, 16, 1024, kSw128);
+      for (int k = 0; ok && k < npc; ++k) {
+        const PieceCtx c = piece_ctx(a, pcs[k], kTwo);
+        // the piece's first P.V overwrites O: the previous piece's epilogue
+        // must have read it
+        if (k > 0 && !(ok = warp_wait(bar(L::B_O_FREE), (k - 1) & 1, abort_flag, a.status))) break;
+        for (int j = 0; j < c.n_pt; ++j, ++jt) {
+          const int buf = jt & 1, sv = jt % NV;
+          if (!(ok = warp_wait(bar(L::B_V_FULL + sv), (jt / NV) & 1, abort_flag, a.status))) break;
+          if (!(ok = warp_wait(bar(L::B_P_FULL + buf), (jt >> 1) & 1, abort_flag, a.status))) break;
+          tc_fence_after();
+          const uint32_t vs = sb + L::kVOff + sv * L::kVSlot;
+          const uint64_t dp = smem_desc(sb + L::kPOff + buf * L::kPBuf, 16, 1024, kSw128);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+          for (int h = 0; h < 2; ++h) {
 #pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) {  // 32 keys per MMA: page k4/2, rows (k4%2)*32
-            const uint64_t dv =
-                smem_desc(vs + h * 16384 + (k4 >> 1) * 8192 + (k4 & 1) * 4096, 8192, 1024, kSw128);
-            mma_f8_ss_pair_e(tmem + kOCol + 128u * h, dp + (uint64_t)((k4 * 32) >> 4), dv, idp,
-                             (j > 0 || k4 > 0) ? 1u : 0u);
-            if (kTwo)
-              mma_f8_ss_pair_e(tmem + kOCol + 128u * h, dp + (uint64_t)((L::kPPlane + k4 * 32) >> 4), dv, idp, 1u);
+            for (int k4 = 0; k4 < 4; ++k4) {  // 32 keys per MMA: page k4/2, rows (k4%2)*32
+              const uint64_t dv =
+                  smem_desc(vs + h * 16384 + (k4 >> 1) * 8192 + (k4 & 1) * 4096, 8192, 1024, kSw128);
+              mma_f8_ss_pair_e(tmem + kOCol + 128u * h, dp + (uint64_t)((k4 * 32) >> 4), dv, idp,
+                               (j > 0 || k4 > 0) ? 1u : 0u);
+              if (c.two)
+                mma_f8_ss_pair_e(tmem + kOCol + 128u * h, dp + (uint64_t)((L::kPPlane + k4 * 32) >> 4), dv, idp,
+                                 1u);
+            }
           }
+          // O_DONE first: a softmax group that has seen P_EMPTY of tile j-2 may
+          // rely on O_DONE having completed that tile's phase too.
+          mma_commit_pair_mc_e(bar(L::B_O_DONE), 3);
+          mma_commit_pair_mc_e(bar(L::B_P_EMPTY + buf), 3);
+          mma_commit_pair_mc_e(bar(L::B_V_EMPTY + sv), 3);
+          if (j == c.n_pt - 1) mma_commit_pair_mc_e(bar(L::B_O_FINAL), 3);
         }
-        // O_DONE first: a softmax group that has seen P_EMPTY of tile j-2 may
-        // rely on O_DONE having completed that tile's phase too.
-        mma_commit_pair_mc_e(bar(L::B_O_DONE), 3);
-        mma_commit_pair_mc_e(bar(L::B_P_EMPTY + buf), 3);
-        mma_commit_pair_mc_e(bar(L::B_V_EMPTY + sv), 3);
-        if (j == n_pt - 1) mma_commit_pair_mc_e(bar(L::B_O_FINAL), 3);
       }
     }
   } else if (warp >= kSoftmaxWarp0) {
     // ------------------------------------------------------------ softmax warps
-    // Group grp takes pair tiles grp, grp+2, ...; warp w serves TMEM lane
-    // quarter q = w%4: local rows 32(q%2) .. +31, key half hf = q/2.
+    // Group grp takes the tiles whose running index has parity grp; warp w
+    // serves TMEM lane quarter q = w%4: local rows 32(q%2) .. +31, key half
+    // hf = q/2.
     const int q = warp & 3;
     const int grp = (warp - kSoftmaxWarp0) >> 2;
     const int hf = q >> 1;
     const int rl = 32 * (q & 1) + lane;  // local row (0..63)
     const int r = 64 * (int)rank + rl;   // row within the unit
     const uint32_t tl = (uint32_t)(32 * q) << 16;
-    const int limit = min((r < M) ? n - T + g * p.fold + r / H : n - 1, key1 - 1);
     float* mref = reinterpret_cast<float*>(smem + L::kMOff);  // [tile parity][64]
     float* xm = reinterpret_cast<float*>(smem + L::kXOff);    // [group][phase][half][64]
     float* fin = reinterpret_cast<float*>(smem + L::kFinOff); // [l|m][group][half][64]
+    const float sl2 = a.score_scale_log2;
     bool ok = true;
+    int jt = 0;  // running index of the piece's first tile
 
-    // Q latent dims of local row rl into TMEM (A operand of S = Q.K^T): lane
-    // quarters q and q^2 both hold rows 32(q%2)..; group g copies chunks 2g, 2g+1.
-    ok = warp_wait(bar(L::B_Q_MAIN), 0, abort_flag, a.status);
-    if (ok) {
+    for (int k = 0; ok && k < npc; ++k) {
+      const PieceCtx c = piece_ctx(a, pcs[k], kTwo);
+      const bool last_piece = k == npc - 1;
+      const int limit = min((r < M) ? c.n - T + c.g * p.fold + r / H : c.n - 1, c.key1 - 1);
+
+      // Q latent dims of local row rl into TMEM (A operand of S = Q.K^T): lane
+      // quarters q and q^2 both hold rows 32(q%2)..; group g copies chunks
+      // 2g, 2g+1. The previous piece's S MMAs read Q until its last tile.
+      if (k > 0) {
+        const int jl = jt - 1;
+        if (!(ok = warp_wait(bar(L::B_S_FULL + (jl & 1)), (jl >> 1) & 1, abort_flag, a.status))) break;
+      }
+      if (!(ok = warp_wait(bar(L::B_Q_MAIN), k & 1, abort_flag, a.status))) break;
 #pragma unroll 1
       for (int c2 = 0; c2 < 2; ++c2) {
         const int cc = 2 * grp + c2;
@@ -405,243 +571,288 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
       tc_fence_before();
       __syncwarp();
       if (lane == 0) arrive_lead(L::B_Q_TMEM);
-    }
 
-    const float sl2 = a.score_scale_log2;
-    float m_grp = -INFINITY, l_grp = 0.f;  // this group's reference and partial sum (this half row)
-    // block-table entry of this half's page for the group's next tile, read
-    // one tile ahead so that the dependent load is off the critical path
-    auto table_entry = [&](int jj) -> int { const int t = 2 * jj + hf; return t < n_tiles ? table[tile0 + t] : 0; };
-    int pg_next = (grp < n_pt) ? table_entry(grp) : 0;
-    for (int j = grp; ok && j < n_pt; j += 2) {
-      const int pg_cur = pg_next;
-      if (j + 2 < n_pt) pg_next = table_entry(j + 2);
-      const int buf = j & 1;  // == grp
-      const int ph = (j >> 1) & 1;
-      if (!(ok = warp_wait(bar(L::B_S_FULL + buf), ph, abort_flag, a.status))) break;
-      tc_fence_after();
-      uint32_t sv[64];
-      {
-        uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
-        uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
-        tmem_ld32(tmem + tl + kSCol + 64u * buf, s0);
-        tmem_ld32(tmem + tl + kSCol + 64u * buf + 32u, s1);
-        tmem_wait_ld();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) arrive_lead_relaxed(L::B_S_EMPTY + buf);  // the slice was read (wait::ld above)
+      float m_grp = -INFINITY, l_grp = 0.f;  // this group's reference and partial sum (this half row)
+      // block-table entry of this half's page for the group's next tile, read
+      // one tile ahead so that the dependent load is off the critical path
+      auto table_entry = [&](int jj) -> int {
+        const int t = 2 * jj + hf;
+        return t < c.n_tiles ? c.table[c.tile0 + t] : 0;
+      };
+      const int j_first = (jt & 1) == grp ? 0 : 1;
+      int pg_next = j_first < c.n_pt ? table_entry(j_first) : 0;
+      for (int j = j_first; ok && j < c.n_pt; j += 2) {
+        const int jg = jt + j;   // running tile index
+        const int buf = jg & 1;  // == grp
+        const int ph = (jg >> 1) & 1;
+        const int pg_cur = pg_next;
+        if (j + 2 < c.n_pt) pg_next = table_entry(j + 2);
+        if (!(ok = warp_wait(bar(L::B_S_FULL + buf), ph, abort_flag, a.status))) break;
+        tc_fence_after();
+        uint32_t sv[64];
+        {
+          uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
+          uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
+          tmem_ld32(tmem + tl + kSCol + 64u * buf, s0);
+          tmem_ld32(tmem + tl + kSCol + 64u * buf + 32u, s1);
+          tmem_wait_ld();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_lead_relaxed(L::B_S_EMPTY + buf);  // the slice was read (wait::ld above)
 
-      const int t = 2 * j + hf;  // 64-key tile of this half
-      bool page_ok = t < n_tiles;
-      if (page_ok) {
-        const int pg = pg_cur;
-        if (pg < 0 || (int64_t)pg >= a.num_pages) {
+        const int t = 2 * j + hf;  // 64-key tile of this half
+        bool page_ok = t < c.n_tiles;
+        if (page_ok && (pg_cur < 0 || (int64_t)pg_cur >= a.num_pages)) {
           page_ok = false;
           if (lane == 0 && (q & 1) == 0) atomicOr(a.status, MLA_DEV_BAD_PAGE);
         }
-      }
-      const int kb = key0 + kPairKeys * j + 64 * hf;
-      // raw scores; masked keys become -inf (sl2 > 0, so max commutes with the scale)
-      if (!(page_ok && kb + 63 <= limit)) {
+        const int kb = c.key0 + kPairTileKeys * j + 64 * hf;
+        // raw scores; masked keys become -inf (sl2 > 0, so max commutes with the scale)
+        if (!(page_ok && kb + 63 <= limit)) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (!(page_ok && kb + i <= limit)) sv[i] = __float_as_uint(-INFINITY);
-      }
-      float mt;
-      {
-        float m8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float v = __uint_as_float(sv[8 * i]);
-#pragma unroll
-          for (int k = 1; k < 8; ++k) v = fmaxf(v, __uint_as_float(sv[8 * i + k]));
-          m8[i] = v;
+          for (int i = 0; i < 64; ++i)
+            if (!(page_ok && kb + i <= limit)) sv[i] = __float_as_uint(-INFINITY);
         }
-        mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sl2;
-      }
-      // the other half of the row lives in the warp of quarter q^2
-      xm[((grp * 2 + ph) * 2 + hf) * 64 + rl] = mt;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(L::B_X + grp));
-      if (!(ok = warp_wait(bar(L::B_X + grp), ph, abort_flag, a.status))) break;
-      mt = fmaxf(mt, xm[((grp * 2 + ph) * 2 + (hf ^ 1)) * 64 + rl]);
-      // reference maximum after tile j-1 (from the other group), lazily updated
-      float m_prev = -INFINITY;
-      if (j > 0) {
-        if (!(ok = warp_wait(bar(L::B_M_READY + (buf ^ 1)), ((j - 1) >> 1) & 1, abort_flag, a.status))) break;
-        m_prev = mref[(buf ^ 1) * 64 + rl];
-      }
-      const float m_j = (mt > m_prev + kTau) ? mt : m_prev;
-      mref[buf * 64 + rl] = m_j;  // both halves write the same value
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(L::B_M_READY + buf));
-      const float alpha = (m_j == m_prev) ? 1.f : ex2_approx(m_prev - m_j);  // O rescale for tile j
-      const float m_use = (m_j == -INFINITY) ? 0.f : m_j - kSigma;
-
-      // P buffer is free once the P.V two tiles back has finished
-      if (j >= 2 && !(ok = warp_wait(bar(L::B_P_EMPTY + buf), ph ^ 1, abort_flag, a.status))) break;
-
-      // P = 2^(s * sl2 - m_use), 16 keys (one 16-byte chunk) at a time; this
-      // half's 64 keys are bytes [64hf, 64hf + 64) of the 128-byte P row.
-      float se[4] = {0.f, 0.f, 0.f, 0.f};
-      uint8_t* prow = smem + L::kPOff + buf * L::kPBuf + rl * 128;
+        float mt;
+        {
+          float m8[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        uint32_t hi[4], lo[4];
+          for (int i = 0; i < 8; ++i) {
+            float v = __uint_as_float(sv[8 * i]);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int e = 16 * u + 2 * i;
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -m_use));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -m_use));
-          se[i & 3] += p0 + p1;
-          const uint32_t qh = cvt_e4m3x2(p0, p1);
-          if (i & 1) hi[i >> 1] |= qh << 16; else hi[i >> 1] = qh;
-          if (kTwo) {
-            const uint32_t rl16 = hsub2(cvt_f16x2(p0, p1), cvt_e4m3x2_to_f16x2(qh));
-            const uint32_t ql = cvt_f16x2_to_e4m3x2(rl16);
-            if (i & 1) lo[i >> 1] |= ql << 16; else lo[i >> 1] = ql;
+            for (int e = 1; e < 8; ++e) v = fmaxf(v, __uint_as_float(sv[8 * i + e]));
+            m8[i] = v;
           }
+          mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) *
+               sl2;
         }
-        const int phys = (4 * hf + u) ^ (rl & 7);
-        *reinterpret_cast<uint4*>(prow + phys * 16) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        if (kTwo) *reinterpret_cast<uint4*>(prow + L::kPPlane + phys * 16) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      }
-      const float sum = (se[0] + se[1]) + (se[2] + se[3]);
-      l_grp = (m_grp == m_j) ? l_grp + sum : fmaf(l_grp, ex2_approx(m_grp - m_j), sum);
-      m_grp = m_j;
+        // the other half of the row lives in the warp of quarter q^2
+        xm[((grp * 2 + ph) * 2 + hf) * 64 + rl] = mt;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_X + grp));
+        if (!(ok = warp_wait(bar(L::B_X + grp), ph, abort_flag, a.status))) break;
+        mt = fmaxf(mt, xm[((grp * 2 + ph) * 2 + (hf ^ 1)) * 64 + rl]);
+        // reference maximum after the previous tile (from the other group; a
+        // new piece starts afresh but still takes the hand-off, which keeps
+        // the reference array's reuse ordered), lazily updated
+        float m_prev = -INFINITY;
+        if (jg > 0) {
+          if (!(ok = warp_wait(bar(L::B_M_READY + (buf ^ 1)), ((jg - 1) >> 1) & 1, abort_flag, a.status))) break;
+          if (j > 0) m_prev = mref[(buf ^ 1) * 64 + rl];
+        }
+        const float m_j = (mt > m_prev + kTau) ? mt : m_prev;
+        mref[buf * 64 + rl] = m_j;  // both halves write the same value
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_M_READY + buf));
+        const float alpha = (m_j == m_prev) ? 1.f : ex2_approx(m_prev - m_j);  // O rescale for tile j
+        const float m_use = (m_j == -INFINITY) ? 0.f : m_j - kSigma;
 
-      // rescale this thread's 256 O columns if the reference maximum moved
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        if (!(ok = warp_wait(bar(L::B_O_DONE), (j - 1) & 1, abort_flag, a.status))) break;
-        tc_fence_after();
-        // two 32-column chunks per tensor-memory round trip (the score
-        // registers are free by now)
+        // P buffer is free once the P.V two tiles back has finished
+        if (jg >= 2 && !(ok = warp_wait(bar(L::B_P_EMPTY + buf), ph ^ 1, abort_flag, a.status))) break;
+
+        // P = 2^(s * sl2 - m_use), 16 keys (one 16-byte chunk) at a time; this
+        // half's 64 keys are bytes [64hf, 64hf + 64) of the 128-byte P row.
+        float se[4] = {0.f, 0.f, 0.f, 0.f};
+        uint8_t* prow = smem + L::kPOff + buf * L::kPBuf + rl * 128;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int e = 16 * u + 2 * i;
+            const float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -m_use));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -m_use));
+            se[i & 3] += p0 + p1;
+            const uint32_t qh = cvt_e4m3x2(p0, p1);
+            if (i & 1) hi[i >> 1] |= qh << 16; else hi[i >> 1] = qh;
+            if (kTwo) {
+              const uint32_t rl16 = hsub2(cvt_f16x2(p0, p1), cvt_e4m3x2_to_f16x2(qh));
+              const uint32_t ql = cvt_f16x2_to_e4m3x2(rl16);
+              if (i & 1) lo[i >> 1] |= ql << 16; else lo[i >> 1] = ql;
+            }
+          }
+          const int phys = (4 * hf + u) ^ (rl & 7);
+          *reinterpret_cast<uint4*>(prow + phys * 16) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          if (kTwo && c.two)
+            *reinterpret_cast<uint4*>(prow + L::kPPlane + phys * 16) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+        const float sum = (se[0] + se[1]) + (se[2] + se[3]);
+        l_grp = (m_grp == m_j) ? l_grp + sum : fmaf(l_grp, ex2_approx(m_grp - m_j), sum);
+        m_grp = m_j;
+
+        // rescale this thread's 256 O columns if the reference maximum moved
+        // (not on a piece's first tile: O is reset by its first P.V)
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          if (!(ok = warp_wait(bar(L::B_O_DONE), (jg - 1) & 1, abort_flag, a.status))) break;
+          tc_fence_after();
+          // two 32-column chunks per tensor-memory round trip (the score
+          // registers are free by now)
 #pragma unroll 1
-        for (int cc = 0; cc < 8; cc += 2) {
-          uint32_t o0[32], o1[32];
-          tmem_ld32(tmem + tl + kOCol + 32u * cc, o0);
-          tmem_ld32(tmem + tl + kOCol + 32u * (cc + 1), o1);
-          tmem_wait_ld();
+          for (int cc = 0; cc < 8; cc += 2) {
+            uint32_t o0[32], o1[32];
+            tmem_ld32(tmem + tl + kOCol + 32u * cc, o0);
+            tmem_ld32(tmem + tl + kOCol + 32u * (cc + 1), o1);
+            tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            o0[i] = __float_as_uint(__uint_as_float(o0[i]) * alpha);
-            o1[i] = __float_as_uint(__uint_as_float(o1[i]) * alpha);
+            for (int i = 0; i < 32; ++i) {
+              o0[i] = __float_as_uint(__uint_as_float(o0[i]) * alpha);
+              o1[i] = __float_as_uint(__uint_as_float(o1[i]) * alpha);
+            }
+            tmem_st32(tmem + tl + kOCol + 32u * cc, o0);
+            tmem_st32(tmem + tl + kOCol + 32u * (cc + 1), o1);
           }
-          tmem_st32(tmem + tl + kOCol + 32u * cc, o0);
-          tmem_st32(tmem + tl + kOCol + 32u * (cc + 1), o1);
+          tmem_wait_st();
         }
-        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_lead(L::B_P_FULL + buf);
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) arrive_lead(L::B_P_FULL + buf);
-    }
 
-    // ------------------------------------------------------------ epilogue
-    // Row sum over both groups and both key halves, relative to the final
-    // reference maximum.
-    ok = __all_sync(0xffffffffu, ok);
-    fin[((0 * 2 + grp) * 2 + hf) * 64 + rl] = l_grp;
-    fin[((1 * 2 + grp) * 2 + hf) * 64 + rl] = m_grp;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar(L::B_FIN));
-    if (ok) ok = warp_wait(bar(L::B_FIN), 0, abort_flag, a.status);
-    float le = 0.f, m_fin = -INFINITY;
-    if (ok) {
+      // ---------------------------------------------------------- epilogue of the piece
+      // Row sum over both groups and both key halves, relative to the final
+      // reference maximum.
+      ok = __all_sync(0xffffffffu, ok);
+      fin[((0 * 2 + grp) * 2 + hf) * 64 + rl] = l_grp;
+      fin[((1 * 2 + grp) * 2 + hf) * 64 + rl] = m_grp;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::B_FIN));
+      if (ok) ok = warp_wait(bar(L::B_FIN), k & 1, abort_flag, a.status);
+      float le = 0.f, m_fin = -INFINITY;
+      if (ok) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) m_fin = fmaxf(m_fin, fin[(4 + i) * 64 + rl]);
-      if (m_fin != -INFINITY) {
+        for (int i = 0; i < 4; ++i) m_fin = fmaxf(m_fin, fin[(4 + i) * 64 + rl]);
+        if (m_fin != -INFINITY) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float mi = fin[(4 + i) * 64 + rl];
-          if (mi != -INFINITY) le += fin[i * 64 + rl] * ex2_approx(mi - m_fin);
+          for (int i = 0; i < 4; ++i) {
+            const float mi = fin[(4 + i) * 64 + rl];
+            if (mi != -INFINITY) le += fin[i * 64 + rl] * ex2_approx(mi - m_fin);
+          }
         }
       }
-    }
-    if (ok) ok = warp_wait(bar(L::B_O_FINAL), 0, abort_flag, a.status);
-    // The output tile is staged in shared memory (the K and V rings are idle
-    // once every MMA has completed) and written back by whole rows: a warp
-    // then stores 512 contiguous bytes per instruction instead of 32 rows'
-    // scattered 16-byte pieces. Staging row r keeps its 16-byte chunk c at
-    // position c ^ (r & 7), so that neither the per-row writes nor the
-    // per-row reads conflict on shared-memory banks.
-    float* stage = reinterpret_cast<float*>(smem + L::kKOff);  // [64 rows][512] fp32
-    float* rowinv = mref;                                        // free once the loop is done
-    if (ok) {
+      if (ok) ok = warp_wait(bar(L::B_O_FINAL), k & 1, abort_flag, a.status);
+      if (!ok) break;
       tc_fence_after();
       const float inv = (le > 0.f) ? a.v_scale / le : 0.f;
-      if (grp == 0 && hf == 0) rowinv[rl] = inv;
-      // group grp holds column half h = grp: output dims 256h + 128hf + [0, 128)
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t o[32];
-        tmem_ld32(tmem + tl + kOCol + 128u * grp + 32u * cc, o);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int c = 64 * grp + 32 * hf + 8 * cc + i;  // 16-byte chunk of the 2 KB row
-          *reinterpret_cast<uint4*>(stage + rl * MLA_D_V + ((c ^ (rl & 7)) * 4)) =
-              make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-        }
-      }
+      const int64_t slot = slot_of(k);
       if (r < M && grp == 0 && hf == 0) {
-        const int64_t rg = row0 + r;
         const float lse_val = (le > 0.f) ? (m_fin - kSigma + log2f(le)) * kLn2 : -INFINITY;
-        if (S == 1) {
-          if (a.lse) a.lse[rg] = lse_val;
+        if (c.whole) {
+          if (a.lse) a.lse[c.row0 + r] = lse_val;
         } else {
-          a.lse_part[rg * S + s] = lse_val;
+          a.lse_part[slot * M + r] = lse_val;
         }
       }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar(L::B_EPI));
-    if (ok) ok = warp_wait(bar(L::B_EPI), 0, abort_flag, a.status);
-    if (ok) {
-      // softmax warp w writes local rows 8w .. 8w+7
-      const int w8 = warp - kSoftmaxWarp0;
+      if (!last_piece) {
+        // O is needed again right away: store straight from registers.
 #pragma unroll 1
-      for (int i = 0; i < 8; ++i) {
-        const int rr = 8 * w8 + i;
-        if (64 * (int)rank + rr >= M) break;  // rows past the unit belong to no output
-        const float inv2 = rowinv[rr];
-        const int64_t rg2 = row0 + 64 * (int)rank + rr;
-        const float* srow = stage + rr * MLA_D_V;
-        if (S == 1) {
-          // BF16: lane writes 8 consecutive values (16 bytes) per step
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tmem + tl + kOCol + 128u * grp + 32u * cc, o);
+          tmem_wait_ld();
+          if (r >= M) continue;
+          const int col = 256 * grp + 128 * hf + 32 * cc;
+          if (c.whole) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + (c.row0 + r) * MLA_D_V + col);
 #pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int c0 = 2 * lane + 64 * k;
-            const float4 x0 = *reinterpret_cast<const float4*>(srow + ((c0 ^ (rr & 7)) * 4));
-            const float4 x1 = *reinterpret_cast<const float4*>(srow + (((c0 + 1) ^ (rr & 7)) * 4));
-            const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-            uint32_t pk[4];
+            for (int u = 0; u < 4; ++u) {
+              uint32_t pk[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(inv2 > 0.f ? v[2 * e] * inv2 : 0.f,
-                                                        inv2 > 0.f ? v[2 * e + 1] * inv2 : 0.f);
-              pk[e] = *reinterpret_cast<uint32_t*>(&h2);
+              for (int e = 0; e < 4; ++e) {
+                const float f0 = inv > 0.f ? __uint_as_float(o[8 * u + 2 * e]) * inv : 0.f;
+                const float f1 = inv > 0.f ? __uint_as_float(o[8 * u + 2 * e + 1]) * inv : 0.f;
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(f0, f1);
+                pk[e] = *reinterpret_cast<uint32_t*>(&h2);
+              }
+              dst[u] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
-            *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + rg2 * MLA_D_V + 4 * c0) =
-                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          } else {
+            float4* dst = reinterpret_cast<float4*>(a.o_part + (slot * M + r) * MLA_D_V + col);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              float4 f;
+              f.x = inv > 0.f ? __uint_as_float(o[4 * u + 0]) * inv : 0.f;
+              f.y = inv > 0.f ? __uint_as_float(o[4 * u + 1]) * inv : 0.f;
+              f.z = inv > 0.f ? __uint_as_float(o[4 * u + 2]) * inv : 0.f;
+              f.w = inv > 0.f ? __uint_as_float(o[4 * u + 3]) * inv : 0.f;
+              dst[u] = f;
+            }
           }
-        } else {
-          float* dst = a.o_part + (rg2 * S + s) * MLA_D_V;
+        }
+        // O may be reset by the next piece's first P.V
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_lead(L::B_O_FREE);
+      } else {
+        // The pair's last piece: the K and V rings are idle, so the output
+        // tile is staged there and written back by whole rows: a warp then
+        // stores 512 contiguous bytes per instruction instead of 32 rows'
+        // scattered pieces. Staging row r keeps its 16-byte chunk c at
+        // position c ^ (r & 7), so that neither the per-row writes nor the
+        // per-row reads conflict on shared-memory banks.
+        float* stage = reinterpret_cast<float*>(smem + L::kKOff);  // [64 rows][512] fp32
+        float* rowinv = mref;                                        // free once the loop is done
+        if (grp == 0 && hf == 0) rowinv[rl] = inv;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tmem + tl + kOCol + 128u * grp + 32u * cc, o);
+          tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int c = lane + 32 * k;
-            float4 x = *reinterpret_cast<const float4*>(srow + ((c ^ (rr & 7)) * 4));
-            if (inv2 > 0.f) {
-              x.x *= inv2; x.y *= inv2; x.z *= inv2; x.w *= inv2;
-            } else {
-              x = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int i = 0; i < 8; ++i) {
+            const int ch = 64 * grp + 32 * hf + 8 * cc + i;  // 16-byte chunk of the 2 KB row
+            *reinterpret_cast<uint4*>(stage + rl * MLA_D_V + ((ch ^ (rl & 7)) * 4)) =
+                make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_EPI));
+        if (!(ok = warp_wait(bar(L::B_EPI), 0, abort_flag, a.status))) break;
+        // softmax warp w writes local rows 8w .. 8w+7
+        const int w8 = warp - kSoftmaxWarp0;
+#pragma unroll 1
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 8 * w8 + i;
+          if (64 * (int)rank + rr >= M) break;  // rows past the unit belong to no output
+          const float inv2 = rowinv[rr];
+          const int rr_u = 64 * (int)rank + rr;  // row within the unit
+          const float* srow = stage + rr * MLA_D_V;
+          if (c.whole) {
+            // BF16: a lane writes 8 consecutive values (16 bytes) per step
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+              const int c0 = 2 * lane + 64 * kk;
+              const float4 x0 = *reinterpret_cast<const float4*>(srow + ((c0 ^ (rr & 7)) * 4));
+              const float4 x1 = *reinterpret_cast<const float4*>(srow + (((c0 + 1) ^ (rr & 7)) * 4));
+              const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+              uint32_t pk[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(inv2 > 0.f ? v[2 * e] * inv2 : 0.f,
+                                                          inv2 > 0.f ? v[2 * e + 1] * inv2 : 0.f);
+                pk[e] = *reinterpret_cast<uint32_t*>(&h2);
+              }
+              *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + (c.row0 + rr_u) * MLA_D_V + 4 * c0) =
+                  make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
-            *reinterpret_cast<float4*>(dst + 4 * c) = x;
+          } else {
+            float* dst = a.o_part + (slot * M + rr_u) * MLA_D_V;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const int ch = lane + 32 * kk;
+              float4 x = *reinterpret_cast<const float4*>(srow + ((ch ^ (rr & 7)) * 4));
+              if (inv2 > 0.f) {
+                x.x *= inv2; x.y *= inv2; x.z *= inv2; x.w *= inv2;
+              } else {
+                x = make_float4(0.f, 0.f, 0.f, 0.f);
+              }
+              *reinterpret_cast<float4*>(dst + 4 * ch) = x;
+            }
           }
         }
       }
+      jt += c.n_pt;
     }
     tc_fence_before();
   }
@@ -651,23 +862,20 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
   // consumed: before the pair may leave, each CTA waits for the last phase of
   // every barrier the leader's commits arrive on, so that no arrival lands in
   // shared memory after the CTA has exited. It runs once every role is done
-  // (the epilogue saw O_FINAL, so every commit has been triggered and each
-  // barrier is at most its last arrival short of its final phase). Bounded;
-  // skipped after an abort, when the phases may never complete.
+  // (the epilogue saw the last O_FINAL, so every commit has been triggered
+  // and each barrier is at most its last arrival short of its final phase).
+  // Bounded; skipped after an abort, when the phases may never complete.
   __syncthreads();
-  if (warp == 2 && lane == 0 && !*abort_flag) {
-    for (int j = n_pt - 1; j >= 0 && j >= n_pt - NK; --j) drain_phase(bar(L::B_K_EMPTY + j % NK), (j / NK) & 1);
-    for (int j = n_pt - 1; j >= 0 && j >= n_pt - NV; --j) drain_phase(bar(L::B_V_EMPTY + j % NV), (j / NV) & 1);
-    for (int j = n_pt - 1; j >= 0 && j >= n_pt - L::NQ; --j)
-      drain_phase(bar(L::B_QK_DONE + j % L::NQ), (j / L::NQ) & 1);
-    for (int j = n_pt - 1; j >= 0 && j >= n_pt - 2; --j) {
+  if (warp == 2 && lane == 0 && !*abort_flag && n_all > 0) {
+    for (int j = n_all - 1; j >= 0 && j >= n_all - NK; --j) drain_phase(bar(L::B_K_EMPTY + j % NK), (j / NK) & 1);
+    for (int j = n_all - 1; j >= 0 && j >= n_all - NV; --j) drain_phase(bar(L::B_V_EMPTY + j % NV), (j / NV) & 1);
+    for (int j = n_all - 1; j >= 0 && j >= n_all - NQ; --j) drain_phase(bar(L::B_QK_DONE + j % NQ), (j / NQ) & 1);
+    for (int j = n_all - 1; j >= 0 && j >= n_all - 2; --j) {
       drain_phase(bar(L::B_P_EMPTY + (j & 1)), (j >> 1) & 1);
       drain_phase(bar(L::B_S_FULL + (j & 1)), (j >> 1) & 1);
     }
-    if (n_pt > 0) {
-      drain_phase(bar(L::B_O_DONE), (n_pt - 1) & 1);
-      drain_phase(bar(L::B_O_FINAL), 0);
-    }
+    drain_phase(bar(L::B_O_DONE), (n_all - 1) & 1);
+    drain_phase(bar(L::B_O_FINAL), (npc - 1) & 1);
   }
   __syncthreads();
   tc_fence_before();
@@ -682,22 +890,30 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem_ra
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_fp8_pair_kernel(const __grid_constant__ PairParams prm) {
   extern __shared__ uint8_t smem_raw[];
-  const mla_plan& p = prm.a.plan;
-  const int b = (blockIdx.x >> 1) / (p.q_groups * p.split_kv);
-  // Short entries send P as two E4M3 terms; the choice is per entry, so both
-  // CTAs of the pair take the same variant and layout.
-  if (effective_seq_len(prm.a, b, false) < kTwoTermKeys)
-    pair_cta<true>(prm, smem_raw);
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Piece* pcs = reinterpret_cast<Piece*>(smem);
+  SchedInfo* info = reinterpret_cast<SchedInfo*>(smem + kMaxPieces * sizeof(Piece));
+  if (threadIdx.x < 32) build_schedule(prm.a, blockIdx.x >> 1, cluster_ctarank(), pcs, info);
+  __syncthreads();
+  const int npc = info->npc;
+  if (npc == 0) return;  // no work for this pair (the same in both CTAs)
+  if (npc > kMaxPieces) {  // cannot happen within the planner's unit limit
+    if (threadIdx.x == 0) atomicOr(prm.a.status, MLA_DEV_TIMEOUT);
+    return;
+  }
+  // Short entries send P as two E4M3 terms; a pair with any such piece takes
+  // the layout with room for both planes (the choice is the same in both CTAs).
+  if (info->two)
+    pair_cta<true>(prm, smem, pcs, npc);
   else
-    pair_cta<false>(prm, smem_raw);
+    pair_cta<false>(prm, smem, pcs, npc);
 }
 
 }  // namespace
 
 cudaError_t launch_tc_fp8_pair_partial(const DecodeArgs& a, cudaStream_t stream) {
   const mla_plan& p = a.plan;
-  const uint64_t pairs = (uint64_t)p.batch * p.q_groups * p.split_kv;
-  if (pairs == 0) return cudaSuccess;
+  if (p.batch == 0 || p.split_kv < 1) return cudaSuccess;
   PairParams prm;
   prm.a = a;
   const uint64_t q_rows = (uint64_t)p.batch * p.q_len * p.num_heads;
@@ -715,7 +931,7 @@ cudaError_t launch_tc_fp8_pair_partial(const DecodeArgs& a, cudaStream_t stream)
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  tc_fp8_pair_kernel<<<(unsigned)(2 * pairs), kThreads, kPairSmemBytes, stream>>>(prm);
+  tc_fp8_pair_kernel<<<(unsigned)(2 * p.split_kv), kThreads, kPairSmemBytes, stream>>>(prm);
   return cudaGetLastError();
 }
 

@@ -227,3 +227,26 @@ def test_host_pointers_are_refused_before_launch():
     o, l = dec(g.q, g.kv_cache, g.block_tables, g.seq_lens, g.softmax_scale)
     torch.cuda.synchronize()
     assert dec.status() == 0 and torch.isfinite(o.float()).all()
+
+
+@pytest.mark.parametrize("pairs", [1, 2, 3, 7, 74])
+def test_balanced_schedule_forced_pairs(pairs):
+    """FP8 CTA-pair kernel with its balanced schedule forced onto few pairs: units are cut
+    between pairs and pairs cover several units (empty, one-key, ragged, single-term entries)."""
+    inp = make_inputs_custom(6, 2, 32, "fp8", [0, 1, 130, 700, 4097, 20000], seed=31, pool=1.5)
+    out, lse, status, dec = run(inp, "tcgen05", split_kv=pairs)
+    assert dec.plan.schedule == 1 and status == 0
+    ref_o, ref_l = oracle_rows(inp)
+    compare(out, lse, ref_o, ref_l, "fp8", what=f"{pairs} pairs")
+
+
+def test_balanced_schedule_many_ragged_units():
+    g = torch.Generator().manual_seed(33)
+    sl = torch.randint(0, 3000, (40,), generator=g).tolist()
+    sl[3] = 0
+    sl[7] = 1
+    inp = make_inputs_custom(40, 1, 16, "fp8", sl, seed=34, pool=1.3)
+    out, lse, status, dec = run(inp, "tcgen05")
+    assert dec.plan.schedule == 1 and status == 0
+    ref_o, ref_l = oracle_rows(inp)
+    compare(out, lse, ref_o, ref_l, "fp8", what="40 ragged units")

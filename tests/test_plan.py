@@ -46,19 +46,99 @@ def test_split_covers_all_keys(batch, q_len, heads, n):
 
 def test_workspace_holds_the_partials():
     for (b, t, h, n) in [(4, 4, 32, 81920), (16, 4, 32, 81920), (1, 1, 16, 256)]:
-        p = mla.mla_decode_plan(b, t, h, n, "fp8")
+        # fixed splits: [rows, S, 512] partials
+        p = mla.mla_decode_plan_custom(b, t, h, n, "fp8", kernel="tcgen05_solo")
+        assert p.schedule == 0
         rows = b * t * h
         if p.split_kv > 1:
             assert p.partial_offset >= 256 and p.partial_offset % 256 == 0
             assert p.lse_offset >= p.partial_offset + rows * p.split_kv * 512 * 4
             assert p.workspace_bytes >= p.lse_offset + rows * p.split_kv * 4
         assert p.workspace_bytes >= 256 and p.workspace_bytes % 256 == 0
+        # balanced CTA-pair schedule: 2P slots of M rows, then the unit table
+        p = mla.mla_decode_plan(b, t, h, n, "fp8")
+        assert p.schedule == 1 and p.kernel == 1 and p.num_ctas == 2 * p.split_kv
+        slot_rows = 2 * p.split_kv * p.rows_per_unit
+        units = b * p.q_groups
+        assert p.partial_offset >= 256 and p.partial_offset % 256 == 0
+        assert p.lse_offset >= p.partial_offset + slot_rows * 512 * 4 and p.lse_offset % 256 == 0
+        assert p.workspace_bytes >= p.lse_offset + slot_rows * 4 + (units + 2) * 4
+        assert p.split_kv * p.keys_per_split >= n
+
+
+def test_balanced_plan_uses_every_sm_and_caps_units():
+    p = mla.mla_decode_plan(16, 4, 32, 81920, "fp8")
+    assert (p.schedule, p.split_kv, p.num_ctas) == (1, 74, 148)
+    assert mla.mla_decode_plan_custom(16, 4, 32, 81920, "fp8", split_kv=5).split_kv == 5
+    assert mla.mla_decode_plan_custom(16, 4, 32, 81920, "fp8", split_kv=1000).split_kv == 74
+    # more units than the per-pair piece list can hold: fixed splits, solo kernel
+    big = mla.mla_decode_plan(4096, 1, 16, 1024, "fp8")
+    assert big.schedule == 0 and big.kernel == 3
+    # 16-bit inputs keep fixed splits
+    assert mla.mla_decode_plan(16, 4, 32, 81920, "bf16").schedule == 0
+
+
+def _balanced_schedule(tiles, P, min_tiles=2):
+    """Host model of the device schedule: unit starts, pairs with work, each pair's pieces."""
+    starts = [0]
+    for t in tiles:
+        starts.append(starts[-1] + t)
+    W = starts[-1]
+    np_ = max(1, min(P, -(-W // min_tiles)))
+    pieces = []
+    for p in range(P):
+        lo, hi = (W * p // np_, W * (p + 1) // np_) if p < np_ else (W, W)
+        pp = []
+        for u, t in enumerate(tiles):
+            if t > 0 and starts[u] < hi and starts[u] + t > lo:
+                pp.append((u, max(lo - starts[u], 0), min(hi - starts[u], t)))
+        pieces.append(pp)
+    return starts, W, np_, pieces
+
+
+def _pair_of(x, W, np_):
+    return ((x + 1) * np_ + W - 1) // W - 1
+
+
+@pytest.mark.parametrize("tiles", [[640] * 16, [1, 0, 3, 2], [2] * 2048, [190, 3, 0, 640, 1, 1, 77] * 9,
+                                   [5], [0, 0, 4]])
+def test_balanced_schedule_covers_each_tile_once(tiles):
+    """Every tile of every unit lies in exactly one piece; a pair leaves at most two partial
+    pieces (its first and last), in slots 2p and 2p + 1; the combine's rule (unit u is pair q's
+    first unit iff q's range starts at or after u) finds the same slots; pieces fit the list."""
+    P = 74
+    starts, W, np_, pieces = _balanced_schedule(tiles, P)
+    seen = {}
+    slot_of_piece = {}
+    for p, pp in enumerate(pieces):
+        assert len(pp) <= 64
+        for k, (u, t0, t1) in enumerate(pp):
+            for t in range(t0, t1):
+                assert (u, t) not in seen
+                seen[(u, t)] = p
+            whole = t0 == 0 and t1 == tiles[u]
+            if not whole:
+                assert k == 0 or k == len(pp) - 1
+                slot = 2 * p + (0 if k == 0 else 1)
+                assert slot not in slot_of_piece.values()
+                slot_of_piece[(u, p)] = slot
+    assert len(seen) == sum(tiles)
+    for u, t in enumerate(tiles):
+        if t == 0:
+            continue
+        p0, p1 = _pair_of(starts[u], W, np_), _pair_of(starts[u] + t - 1, W, np_)
+        if p0 == p1:
+            assert (u, p0) not in slot_of_piece  # whole: written directly
+            continue
+        for q in range(p0, p1 + 1):
+            slot = 2 * q if W * q // np_ >= starts[u] else 2 * q + 1
+            assert slot_of_piece[(u, q)] == slot
 
 
 def test_split_fills_the_gpu_for_the_long_fp8_case():
-    p4 = mla.mla_decode_plan(4, 4, 32, 81920, "fp8")
+    p4 = mla.mla_decode_plan_custom(4, 4, 32, 81920, "fp8", kernel="tcgen05_solo")
     assert p4.split_kv * 4 <= 74 and p4.split_kv * 4 >= 60  # one wave of CTA pairs
-    p16 = mla.mla_decode_plan(16, 4, 32, 81920, "fp8")
+    p16 = mla.mla_decode_plan_custom(16, 4, 32, 81920, "fp8", kernel="tcgen05_solo")
     waves = math.ceil(p16.split_kv * 16 / 74)
     assert p16.split_kv * 16 / (waves * 74) > 0.85  # little wave quantisation
 
