@@ -92,8 +92,10 @@ typedef enum {
  *     resident; the units' 128-key tiles, counted from the device seq_lens,
  *     are dealt out as equal contiguous ranges. A unit a pair covers whole
  *     is written to out/lse directly; a unit cut between pairs leaves
- *     partials in slots [2P, M, 512] (pair p: slot 2p for its first unit,
- *     2p+1 for its last) that the combine merges. keys_per_split then only
+ *     partials in slots (pair p: slot 2p for its first unit, 2p+1 for its
+ *     last) that the combine merges: fp32 O as [2P][128 chunks of 4
+ *     columns][M rows][4] at partial_offset, fp32 LSE as [2P][M] at
+ *     lse_offset. keys_per_split then only
  *     bounds seq_len (>= max_seq_len).
  *   fold            F: query tokens folded into the row dimension
  *   q_groups        G = q_len / F; each (batch entry, group) is one unit

@@ -85,86 +85,91 @@ namespace {
 // Combine for the balanced CTA-pair schedule. Units a single pair covered
 // whole were finished by the partial kernel and are left alone; units with
 // no key get out = 0, lse = -inf; a unit cut between pairs p0 .. p1 merges
-// the pieces in their slots (pair p: slot 2p if the unit is its first, else
-// 2p + 1), as above. One warp per output row.
+// the pieces in their slots (pair q: slot 2q if the unit is its first, else
+// 2q + 1) as above. Slots are laid out [slot][16-byte column chunk][row]:
+// thread (row i, chunk pair c) of a block of 32 rows x 16 chunk pairs sums
+// 8 output columns of row i over the pieces, and the 32 threads of a warp
+// read 32 consecutive rows (512 contiguous bytes) per load. The grid holds
+// units x row blocks x 8 column blocks, so that even a few long units that
+// were cut into many pieces spread over the whole GPU.
+constexpr int kCombineColBlocks = 8;  // 512 columns = 8 blocks x 16 chunk pairs x 4 columns x 2
 __global__ void __launch_bounds__(256) combine_balanced_kernel(const DecodeArgs a) {
   const mla_plan& p = a.plan;
-  const int64_t rows = (int64_t)p.batch * p.q_len * p.num_heads;
-  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  const int TH = p.q_len * p.num_heads;
-  const int b = (int)(row / TH);
-  const int t = (int)(row % TH) / p.num_heads;
-  const int h = (int)(row % TH) % p.num_heads;
-  const int g = t / p.fold;
-  const int r = (t - g * p.fold) * p.num_heads + h;  // row within the unit
+  const int M = p.rows_per_unit;
+  const int nb = (M + 31) / 32;
+  const int cb = blockIdx.x % kCombineColBlocks;
+  const int blk = blockIdx.x / kCombineColBlocks;
+  const int u = blk / nb;
+  const int r = (blk % nb) * 32 + (threadIdx.x & 31);       // row within the unit
+  const int c4_0 = cb * 16 + (threadIdx.x >> 5) * 2;         // first of this thread's two 16-byte chunks
+  if (r >= M) return;
   const int U = p.batch * p.q_groups;
-  const int u = b * p.q_groups + g;
+  const int b = u / p.q_groups, g = u % p.q_groups;
+  const int64_t row = (int64_t)b * p.q_len * p.num_heads + (int64_t)g * M + r;
   const int32_t* tbl = a.sched;
   const int64_t start = tbl[u], end = tbl[u + 1], W = tbl[U];
   const int np = tbl[U + 1];
-  uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + row * MLA_D_V + lane * 16);
+  uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + row * MLA_D_V + c4_0 * 4);
+  const bool lse_writer = a.lse && cb == 0 && (threadIdx.x >> 5) == 0;
   if (end == start) {  // no key at all
-    dst[0] = make_uint4(0, 0, 0, 0);
-    dst[1] = make_uint4(0, 0, 0, 0);
-    if (a.lse && lane == 0) a.lse[row] = -INFINITY;
+    *dst = make_uint4(0, 0, 0, 0);
+    if (lse_writer) a.lse[row] = -INFINITY;
     return;
   }
   const int p0 = balanced_pair_of(start, W, np), p1 = balanced_pair_of(end - 1, W, np);
   if (p0 == p1) return;  // written by its pair
-  const int M = p.rows_per_unit;
-  auto slot_of = [&](int q) { return balanced_lo(q, W, np) >= start ? 2 * q : 2 * q + 1; };
-  const int npc = p1 - p0 + 1;
+  // The unit is pair p0's first unit only if p0's range starts exactly at
+  // it; every later pair's range starts inside the unit (slot 2q).
+  const int64_t first_slot = balanced_lo(p0, W, np) == start ? 2 * (int64_t)p0 : 2 * (int64_t)p0 + 1;
 
-  float m = -INFINITY;
-  for (int k = lane; k < npc; k += 32) m = fmaxf(m, a.lse_part[(int64_t)slot_of(p0 + k) * M + r]);
-  m = warp_max(m);
-  float L = -INFINITY;
-  if (m != -INFINITY) {
-    float sum = 0.f;
-    for (int k = lane; k < npc; k += 32) sum += expf(a.lse_part[(int64_t)slot_of(p0 + k) * M + r] - m);
-    sum = warp_sum(sum);
-    L = m + logf(sum);
-  }
-  float acc[16];
+  // One pass over the pieces with a running maximum (online LSE merge).
+  float m = -INFINITY, sum = 0.f;
+  float acc[8];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  if (L != -INFINITY) {
-    for (int k = 0; k < npc; ++k) {
-      const int64_t sl = slot_of(p0 + k);
-      const float ls = a.lse_part[sl * M + r];
-      if (ls == -INFINITY) continue;
-      const float w = expf(ls - L);
-      const float4* src = reinterpret_cast<const float4*>(a.o_part + (sl * M + r) * MLA_D_V + lane * 16);
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const float4 x = src[v];
-        acc[4 * v + 0] = fmaf(w, x.x, acc[4 * v + 0]);
-        acc[4 * v + 1] = fmaf(w, x.y, acc[4 * v + 1]);
-        acc[4 * v + 2] = fmaf(w, x.z, acc[4 * v + 2]);
-        acc[4 * v + 3] = fmaf(w, x.w, acc[4 * v + 3]);
-      }
-    }
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll 4
+  for (int q = p0; q <= p1; ++q) {
+    const int64_t sl = q == p0 ? first_slot : 2 * (int64_t)q;
+    const float ls = a.lse_part[sl * M + r];
+    const float* src = a.o_part + ((sl * (MLA_D_V / 4) + c4_0) * M + r) * 4;
+    const float4 x0 = *reinterpret_cast<const float4*>(src);
+    const float4 x1 = *reinterpret_cast<const float4*>(src + (int64_t)M * 4);
+    if (ls == -INFINITY) continue;  // an empty piece may hold anything
+    const float m_new = fmaxf(m, ls);
+    const float keep = expf(m - m_new);  // 0 on the first piece
+    const float w = expf(ls - m_new);
+    sum = fmaf(sum, keep, w);
+    acc[0] = fmaf(acc[0], keep, w * x0.x);
+    acc[1] = fmaf(acc[1], keep, w * x0.y);
+    acc[2] = fmaf(acc[2], keep, w * x0.z);
+    acc[3] = fmaf(acc[3], keep, w * x0.w);
+    acc[4] = fmaf(acc[4], keep, w * x1.x);
+    acc[5] = fmaf(acc[5], keep, w * x1.y);
+    acc[6] = fmaf(acc[6], keep, w * x1.z);
+    acc[7] = fmaf(acc[7], keep, w * x1.w);
+    m = m_new;
   }
-  uint4 packed[2];
-  uint32_t* pw = reinterpret_cast<uint32_t*>(packed);
+  const float L = m == -INFINITY ? -INFINITY : m + logf(sum);
+  const float inv = m == -INFINITY ? 0.f : 1.f / sum;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-    pw[i] = *reinterpret_cast<uint32_t*>(&h2);
+  for (int i = 0; i < 8; ++i) acc[i] *= inv;
+  uint32_t pk[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
+    pk[e] = *reinterpret_cast<uint32_t*>(&h2);
   }
-  dst[0] = packed[0];
-  dst[1] = packed[1];
-  if (a.lse && lane == 0) a.lse[row] = L;
+  *dst = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  if (lse_writer) a.lse[row] = L;
 }
 
 }  // namespace
 
 cudaError_t launch_combine_balanced(const DecodeArgs& a, cudaStream_t stream) {
-  const int64_t rows = (int64_t)a.plan.batch * a.plan.q_len * a.plan.num_heads;
-  if (rows == 0) return cudaSuccess;
-  combine_balanced_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(a);
+  const int64_t units = (int64_t)a.plan.batch * a.plan.q_groups;
+  if (units == 0) return cudaSuccess;
+  const int nb = (a.plan.rows_per_unit + 31) / 32;
+  combine_balanced_kernel<<<(unsigned)(units * nb * kCombineColBlocks), 256, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -744,8 +744,11 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
           a.lse_part[slot * M + r] = lse_val;
         }
       }
-      if (!last_piece) {
-        // O is needed again right away: store straight from registers.
+      if (!(c.whole && last_piece)) {
+        // Straight from registers. Partial slots use the layout
+        // [slot][16-byte column chunk][row]: the 32 consecutive rows of a warp
+        // then store 512 contiguous bytes per instruction. A whole unit that
+        // is not the pair's last piece is stored as BF16 rows.
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t o[32];
@@ -768,27 +771,29 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
               dst[u] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
           } else {
-            float4* dst = reinterpret_cast<float4*>(a.o_part + (slot * M + r) * MLA_D_V + col);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
+              const int64_t c4 = col / 4 + u;  // 16-byte column chunk
               float4 f;
               f.x = inv > 0.f ? __uint_as_float(o[4 * u + 0]) * inv : 0.f;
               f.y = inv > 0.f ? __uint_as_float(o[4 * u + 1]) * inv : 0.f;
               f.z = inv > 0.f ? __uint_as_float(o[4 * u + 2]) * inv : 0.f;
               f.w = inv > 0.f ? __uint_as_float(o[4 * u + 3]) * inv : 0.f;
-              dst[u] = f;
+              *reinterpret_cast<float4*>(a.o_part + ((slot * (MLA_D_V / 4) + c4) * M + r) * 4) = f;
             }
           }
         }
-        // O may be reset by the next piece's first P.V
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) arrive_lead(L::B_O_FREE);
+        if (!last_piece) {
+          // O may be reset by the next piece's first P.V
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) arrive_lead(L::B_O_FREE);
+        }
       } else {
-        // The pair's last piece: the K and V rings are idle, so the output
-        // tile is staged there and written back by whole rows: a warp then
-        // stores 512 contiguous bytes per instruction instead of 32 rows'
-        // scattered pieces. Staging row r keeps its 16-byte chunk c at
+        // A whole unit as the pair's last piece: the K and V rings are idle,
+        // so the output tile is staged there and written back by whole rows:
+        // a warp then stores 512 contiguous bytes per instruction instead of
+        // 32 rows' scattered pieces. Staging row r keeps its 16-byte chunk c at
         // position c ^ (r & 7), so that neither the per-row writes nor the
         // per-row reads conflict on shared-memory banks.
         float* stage = reinterpret_cast<float*>(smem + L::kKOff);  // [64 rows][512] fp32
@@ -818,7 +823,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
           const float inv2 = rowinv[rr];
           const int rr_u = 64 * (int)rank + rr;  // row within the unit
           const float* srow = stage + rr * MLA_D_V;
-          if (c.whole) {
+          {
             // BF16: a lane writes 8 consecutive values (16 bytes) per step
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk) {
@@ -835,19 +840,6 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
               }
               *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + (c.row0 + rr_u) * MLA_D_V + 4 * c0) =
                   make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            }
-          } else {
-            float* dst = a.o_part + (slot * M + rr_u) * MLA_D_V;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const int ch = lane + 32 * kk;
-              float4 x = *reinterpret_cast<const float4*>(srow + ((ch ^ (rr & 7)) * 4));
-              if (inv2 > 0.f) {
-                x.x *= inv2; x.y *= inv2; x.z *= inv2; x.w *= inv2;
-              } else {
-                x = make_float4(0.f, 0.f, 0.f, 0.f);
-              }
-              *reinterpret_cast<float4*>(dst + 4 * ch) = x;
             }
           }
         }
