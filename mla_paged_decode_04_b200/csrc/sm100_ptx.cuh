@@ -12,6 +12,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// A read-only global load kept in program order with the other volatile asm
+// (mbarrier waits, TMA issues): an index read one step ahead is then issued
+// before the wait it is meant to overlap, and the compiler cannot sink it
+// behind that wait.
+__device__ __forceinline__ int ld_nc_ordered(const int* p) {
+  int v;
+  asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

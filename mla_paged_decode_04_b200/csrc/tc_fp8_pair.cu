@@ -71,8 +71,8 @@ namespace {
 using namespace ptx;
 
 constexpr int kTwoTermKeys = 16384;  // entries shorter than this use two-term P
-constexpr float kTau = 2.f;          // lazy-rescale threshold (log2 units)
-constexpr float kSigma = 6.f;        // P <= 2^(kTau + kSigma) = 256 <= 448
+constexpr float kTau = 4.f;          // lazy-rescale threshold (log2 units)
+constexpr float kSigma = 4.f;        // P <= 2^(kTau + kSigma) = 256 <= 448
 constexpr int kMaxPieces = 64;       // pieces per pair (units its range touches)
 constexpr int kMinPairTiles = 2;     // fewer tiles than this per pair: use fewer pairs
 
@@ -272,10 +272,14 @@ __device__ __forceinline__ PieceCtx piece_ctx(const DecodeArgs& a, const Piece& 
   return c;
 }
 
-// page of 64-key tile t of the piece (t < n_tiles), 0 when absent or invalid
-__device__ __forceinline__ int piece_page(const DecodeArgs& a, const PieceCtx& c, int t) {
-  if (t >= c.n_tiles) return 0;
-  const int pg = c.table[c.tile0 + t];
+// Block-table entry of 64-key tile t of the piece (0 past its end), read one
+// tile ahead of its use: the load is issued before the next barrier wait and
+// checked after it, so its latency stays off the ring's critical path.
+__device__ __forceinline__ int piece_entry(const PieceCtx& c, int t) {
+  return t < c.n_tiles ? ld_nc_ordered(c.table + c.tile0 + t) : 0;
+}
+// an entry outside the cache reads page 0 (its keys are masked by the softmax)
+__device__ __forceinline__ int valid_page(const DecodeArgs& a, int pg) {
   return (pg < 0 || (int64_t)pg >= a.num_pages) ? 0 : pg;
 }
 
@@ -387,12 +391,11 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
           tma_load_2d(sb + L::kQStage + ci * 8192, &prm.tm_q_main, 128 * ci, qrow, bar(L::B_Q_MAIN), pol_q);
         if (rank == 0) mbar_arrive_expect_tx(bar(L::B_Q_ROPE), 2u * 64u * (uint32_t)box_q);
         tma_load_2d_pair(sb + L::kQRope, &prm.tm_q_rope, 512, qrow, lead(L::B_Q_ROPE), pol_q);
-        // block-table entries are read one tile ahead, off the critical path
-        int page_nx = piece_page(a, c, (int)rank);
+        int entry_nx = piece_entry(c, (int)rank);
         for (int j = 0; j < c.n_pt; ++j, ++jt) {
           const int sk = jt % NK;
-          const int page = page_nx;
-          if (j + 1 < c.n_pt) page_nx = piece_page(a, c, 2 * (j + 1) + (int)rank);
+          const int page = valid_page(a, entry_nx);
+          if (j + 1 < c.n_pt) entry_nx = piece_entry(c, 2 * (j + 1) + (int)rank);
           if (!(ok = bounded_wait(bar(L::B_K_EMPTY + sk), ((jt / NK) & 1) ^ 1, abort_flag, a.status))) break;
           const uint32_t ks = sb + L::kKOff + sk * L::kKSlot;
           const uint32_t full = lead(L::B_K_FULL + sk);
@@ -416,13 +419,13 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
       bool ok = true;
       for (int k = 0; ok && k < npc; ++k) {
         const PieceCtx c = piece_ctx(a, pcs[k], kTwo);
-        int pg0_nx = piece_page(a, c, 0), pg1_nx = piece_page(a, c, 1);
+        int e0_nx = piece_entry(c, 0), e1_nx = piece_entry(c, 1);
         for (int j = 0; j < c.n_pt; ++j, ++jt) {
           const int sv = jt % NV;
-          const int pg0 = pg0_nx, pg1 = pg1_nx;
+          const int pg0 = valid_page(a, e0_nx), pg1 = valid_page(a, e1_nx);
           if (j + 1 < c.n_pt) {
-            pg0_nx = piece_page(a, c, 2 * (j + 1));
-            pg1_nx = piece_page(a, c, 2 * (j + 1) + 1);
+            e0_nx = piece_entry(c, 2 * (j + 1));
+            e1_nx = piece_entry(c, 2 * (j + 1) + 1);
           }
           // the scores of the tile exist: its pages are in L2 now
           if (!(ok = bounded_wait(bar(L::B_QK_DONE + jt % NQ), (jt / NQ) & 1, abort_flag, a.status))) break;
@@ -577,7 +580,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
       // one tile ahead so that the dependent load is off the critical path
       auto table_entry = [&](int jj) -> int {
         const int t = 2 * jj + hf;
-        return t < c.n_tiles ? c.table[c.tile0 + t] : 0;
+        return piece_entry(c, t);
       };
       const int j_first = (jt & 1) == grp ? 0 : 1;
       int pg_next = j_first < c.n_pt ? table_entry(j_first) : 0;
