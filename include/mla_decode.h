@@ -95,7 +95,12 @@ typedef enum {
  *     partials in slots (pair p: slot 2p for its first unit, 2p+1 for its
  *     last) that the combine merges: fp32 O as [2P][128 chunks of 4
  *     columns][M rows][4] at partial_offset, fp32 LSE as [2P][M] at
- *     lse_offset. keys_per_split then only
+ *     lse_offset. Between the 256-byte status header and partial_offset
+ *     lie B*G + 1 int32 counters (finished pieces per unit, then a flag for
+ *     the unit table at the end of the workspace), cleared with the status
+ *     word before every launch: the combine kernel is launched as the
+ *     partial kernel's programmatic dependent and merges each unit as soon
+ *     as its counter is complete. keys_per_split then only
  *     bounds seq_len (>= max_seq_len).
  *   fold            F: query tokens folded into the row dimension
  *   q_groups        G = q_len / F; each (batch entry, group) is one unit

@@ -84,7 +84,7 @@ int check_plan(const mla_plan* p) {
     const int64_t units = (int64_t)p->batch * p->q_groups;
     if (units > kMaxBalancedUnits) return MLA_ERR_PLAN_MISMATCH;
     const uint64_t slot_rows = 2ull * p->split_kv * p->rows_per_unit;
-    if (p->partial_offset < (uint64_t)kHeaderBytes || p->partial_offset % 256 != 0 ||
+    if (p->partial_offset < (uint64_t)kHeaderBytes + balanced_counter_bytes(units) || p->partial_offset % 256 != 0 ||
         p->lse_offset < p->partial_offset + slot_rows * MLA_D_V * 4 || p->lse_offset % 256 != 0 ||
         p->workspace_bytes < p->lse_offset + slot_rows * 4 + balanced_table_bytes(units))
       return MLA_ERR_PLAN_MISMATCH;
@@ -164,11 +164,15 @@ int prepare(const mla_plan* plan, const void* q, const void* kv_cache, int64_t n
                  ? reinterpret_cast<int32_t*>(ws + p.workspace_bytes -
                                               balanced_table_bytes((int64_t)p.batch * p.q_groups))
                  : nullptr;
+  a->unit_done = p.schedule == MLA_SCHEDULE_BALANCED ? reinterpret_cast<int32_t*>(ws + kHeaderBytes) : nullptr;
   return MLA_OK;
 }
 
 int run_partial(const DecodeArgs& a, cudaStream_t st) {
-  if (cudaError_t e = cudaMemsetAsync(a.status, 0, sizeof(int32_t), st); e != cudaSuccess) return cuda_failure(e);
+  // the status word, and for the balanced schedule the unit counters after it
+  const size_t clear = a.unit_done ? kHeaderBytes + balanced_counter_bytes((int64_t)a.plan.batch * a.plan.q_groups)
+                                   : sizeof(int32_t);
+  if (cudaError_t e = cudaMemsetAsync(a.status, 0, clear, st); e != cudaSuccess) return cuda_failure(e);
   if (a.plan.batch == 0) return MLA_OK;
   cudaError_t e;
   if (a.plan.kernel == MLA_KERNEL_SIMT)

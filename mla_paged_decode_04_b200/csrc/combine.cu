@@ -10,6 +10,7 @@
 // never written and are skipped; a split whose lse is -inf (no visible key)
 // has weight 0; a row with no visible key at all gets out = 0, lse = -inf.
 #include "device_common.cuh"
+#include "sm100_ptx.cuh"
 
 namespace mla {
 namespace {
@@ -93,22 +94,57 @@ namespace {
 // units x row blocks x 8 column blocks, so that even a few long units that
 // were cut into many pieces spread over the whole GPU.
 constexpr int kCombineColBlocks = 8;  // 512 columns = 8 blocks x 16 chunk pairs x 4 columns x 2
+constexpr uint64_t kUnitWaitNs = 500ull * 1000 * 1000;  // per wait: 0.5 s
+
+// Bounded wait (one thread) for a counter written by the partial kernel;
+// sets MLA_DEV_TIMEOUT and returns false when the limit passes.
+__device__ bool wait_count(const int32_t* ctr, int target, int32_t* status) {
+  const uint64_t t0 = ptx::globaltimer();
+  while (ptx::ld_acquire_gpu(ctr) < target) {
+    if (ptx::globaltimer() - t0 > kUnitWaitNs) {
+      atomicOr(status, MLA_DEV_TIMEOUT);
+      return false;
+    }
+    __nanosleep(256);
+  }
+  return true;
+}
+
 __global__ void __launch_bounds__(256) combine_balanced_kernel(const DecodeArgs a) {
   const mla_plan& p = a.plan;
   const int M = p.rows_per_unit;
+  const int U = p.batch * p.q_groups;
+  // Launched as the partial kernel's programmatic dependent, this block may
+  // start while pairs still run: it waits for the unit table, then for
+  // every piece of its unit (kPieceArrivals arrivals each). Each thread then
+  // acquires the counter itself before reading what it guards.
+  __shared__ int s_ok;
+  if (threadIdx.x == 0) s_ok = wait_count(a.unit_done + U, 1, a.status);
+  __syncthreads();
+  if (!s_ok) return;
+  (void)ptx::ld_acquire_gpu(a.unit_done + U);
   const int nb = (M + 31) / 32;
   const int cb = blockIdx.x % kCombineColBlocks;
   const int blk = blockIdx.x / kCombineColBlocks;
-  const int u = blk / nb;
-  const int r = (blk % nb) * 32 + (threadIdx.x & 31);       // row within the unit
-  const int c4_0 = cb * 16 + (threadIdx.x >> 5) * 2;         // first of this thread's two 16-byte chunks
-  if (r >= M) return;
-  const int U = p.batch * p.q_groups;
-  const int b = u / p.q_groups, g = u % p.q_groups;
-  const int64_t row = (int64_t)b * p.q_len * p.num_heads + (int64_t)g * M + r;
+  const int u = blk / nb;  // the same for the whole block
   const int32_t* tbl = a.sched;
   const int64_t start = tbl[u], end = tbl[u + 1], W = tbl[U];
   const int np = tbl[U + 1];
+  const int p0 = end > start ? balanced_pair_of(start, W, np) : 0;
+  const int p1 = end > start ? balanced_pair_of(end - 1, W, np) : 0;
+  if (end > start && p0 == p1) return;  // a whole unit: written by its pair
+  if (end > start) {
+    __syncthreads();  // every thread has read s_ok
+    if (threadIdx.x == 0) s_ok = wait_count(a.unit_done + u, kPieceArrivals * (p1 - p0 + 1), a.status);
+    __syncthreads();
+    if (!s_ok) return;
+    (void)ptx::ld_acquire_gpu(a.unit_done + u);
+  }
+  const int r = (blk % nb) * 32 + (threadIdx.x & 31);       // row within the unit
+  const int c4_0 = cb * 16 + (threadIdx.x >> 5) * 2;         // first of this thread's two 16-byte chunks
+  if (r >= M) return;
+  const int b = u / p.q_groups, g = u % p.q_groups;
+  const int64_t row = (int64_t)b * p.q_len * p.num_heads + (int64_t)g * M + r;
   uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + row * MLA_D_V + c4_0 * 4);
   const bool lse_writer = a.lse && cb == 0 && (threadIdx.x >> 5) == 0;
   if (end == start) {  // no key at all
@@ -116,38 +152,55 @@ __global__ void __launch_bounds__(256) combine_balanced_kernel(const DecodeArgs 
     if (lse_writer) a.lse[row] = -INFINITY;
     return;
   }
-  const int p0 = balanced_pair_of(start, W, np), p1 = balanced_pair_of(end - 1, W, np);
-  if (p0 == p1) return;  // written by its pair
   // The unit is pair p0's first unit only if p0's range starts exactly at
   // it; every later pair's range starts inside the unit (slot 2q).
   const int64_t first_slot = balanced_lo(p0, W, np) == start ? 2 * (int64_t)p0 : 2 * (int64_t)p0 + 1;
 
-  // One pass over the pieces with a running maximum (online LSE merge).
-  float m = -INFINITY, sum = 0.f;
+  auto slot = [&](int q) -> int64_t { return q == p0 ? first_slot : 2 * (int64_t)q; };
+
+  // The maximum piece LSE first, then the weighted sum. Pieces go in batches
+  // of kBatch whose loads are all issued before any of them is used (no
+  // branch depends on a loaded value), so their latencies overlap.
+  constexpr int kBatch = 8;
+  float m = -INFINITY;
+  for (int q0 = p0; q0 <= p1; q0 += kBatch) {
+    float ls[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) ls[i] = q0 + i <= p1 ? a.lse_part[slot(q0 + i) * M + r] : -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) m = fmaxf(m, ls[i]);
+  }
+  float sum = 0.f;
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-#pragma unroll 4
-  for (int q = p0; q <= p1; ++q) {
-    const int64_t sl = q == p0 ? first_slot : 2 * (int64_t)q;
-    const float ls = a.lse_part[sl * M + r];
-    const float* src = a.o_part + ((sl * (MLA_D_V / 4) + c4_0) * M + r) * 4;
-    const float4 x0 = *reinterpret_cast<const float4*>(src);
-    const float4 x1 = *reinterpret_cast<const float4*>(src + (int64_t)M * 4);
-    if (ls == -INFINITY) continue;  // an empty piece may hold anything
-    const float m_new = fmaxf(m, ls);
-    const float keep = expf(m - m_new);  // 0 on the first piece
-    const float w = expf(ls - m_new);
-    sum = fmaf(sum, keep, w);
-    acc[0] = fmaf(acc[0], keep, w * x0.x);
-    acc[1] = fmaf(acc[1], keep, w * x0.y);
-    acc[2] = fmaf(acc[2], keep, w * x0.z);
-    acc[3] = fmaf(acc[3], keep, w * x0.w);
-    acc[4] = fmaf(acc[4], keep, w * x1.x);
-    acc[5] = fmaf(acc[5], keep, w * x1.y);
-    acc[6] = fmaf(acc[6], keep, w * x1.z);
-    acc[7] = fmaf(acc[7], keep, w * x1.w);
-    m = m_new;
+  for (int q0 = p0; m != -INFINITY && q0 <= p1; q0 += kBatch) {
+    float ls[kBatch];
+    float4 x0[kBatch], x1[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const bool in = q0 + i <= p1;
+      const int64_t sl = slot(in ? q0 + i : p0);
+      const float* src = a.o_part + ((sl * (MLA_D_V / 4) + c4_0) * M + r) * 4;
+      ls[i] = in ? a.lse_part[sl * M + r] : -INFINITY;
+      x0[i] = in ? *reinterpret_cast<const float4*>(src) : make_float4(0.f, 0.f, 0.f, 0.f);
+      x1[i] = in ? *reinterpret_cast<const float4*>(src + (int64_t)M * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      // an empty piece (lse -inf) has weight 0 and may hold anything
+      const bool live = ls[i] != -INFINITY;
+      const float w = live ? expf(ls[i] - m) : 0.f;
+      sum += w;
+      acc[0] = fmaf(w, live ? x0[i].x : 0.f, acc[0]);
+      acc[1] = fmaf(w, live ? x0[i].y : 0.f, acc[1]);
+      acc[2] = fmaf(w, live ? x0[i].z : 0.f, acc[2]);
+      acc[3] = fmaf(w, live ? x0[i].w : 0.f, acc[3]);
+      acc[4] = fmaf(w, live ? x1[i].x : 0.f, acc[4]);
+      acc[5] = fmaf(w, live ? x1[i].y : 0.f, acc[5]);
+      acc[6] = fmaf(w, live ? x1[i].z : 0.f, acc[6]);
+      acc[7] = fmaf(w, live ? x1[i].w : 0.f, acc[7]);
+    }
   }
   const float L = m == -INFINITY ? -INFINITY : m + logf(sum);
   const float inv = m == -INFINITY ? 0.f : 1.f / sum;
@@ -169,8 +222,20 @@ cudaError_t launch_combine_balanced(const DecodeArgs& a, cudaStream_t stream) {
   const int64_t units = (int64_t)a.plan.batch * a.plan.q_groups;
   if (units == 0) return cudaSuccess;
   const int nb = (a.plan.rows_per_unit + 31) / 32;
-  combine_balanced_kernel<<<(unsigned)(units * nb * kCombineColBlocks), 256, 0, stream>>>(a);
-  return cudaGetLastError();
+  // programmatic dependent of the partial kernel: blocks take the SMs of
+  // pairs that are done and wait for their own unit (the partial kernel
+  // never waits for this grid)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(units * nb * kCombineColBlocks));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_balanced_kernel, a);
 }
 
 }  // namespace mla

@@ -19,6 +19,13 @@ constexpr int kMaxBalancedUnits = 2048;         // units (entry x query group) t
 // every unit (U + 1 entries, the last = W, the total pair tiles), then the
 // number of pairs that have work. Written by the partial kernel, read by the
 // combine.
+// Balanced schedule: per-unit counts of finished partial pieces, then the
+// unit table's ready flag; right after the status header, and cleared with it
+// before every launch of the partial kernel.
+constexpr int kPieceArrivals = 16;  // softmax warps of a CTA pair: counter arrivals per partial piece
+inline uint64_t balanced_counter_bytes(int64_t units) {
+  return ((uint64_t)(units + 1) * 4 + 255) & ~uint64_t(255);
+}
 inline uint64_t balanced_table_bytes(int64_t units) {
   return ((uint64_t)(units + 2) * 4 + 255) & ~uint64_t(255);
 }
@@ -40,6 +47,7 @@ struct DecodeArgs {
   float* o_part;           // fp32 [B*T*H, S, 512] (split_kv > 1)
   float* lse_part;         // fp32 [B*T*H, S]       (split_kv > 1)
   int32_t* sched;          // balanced schedule table (MLA_SCHEDULE_BALANCED), else null
+  int32_t* unit_done;      // balanced: [U] finished-piece counts, [U] table-ready flag; else null
 };
 
 // Pair of the balanced schedule whose range holds pair tile x (0 <= x < W):

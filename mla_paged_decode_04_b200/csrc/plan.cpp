@@ -136,7 +136,7 @@ int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, i
     p.keys_per_split = (int32_t)(ceil_div(max_seq_len > 0 ? max_seq_len : 1, kTileKeys) * kTileKeys);
     p.num_ctas = 2 * P;
     const uint64_t slots = 2 * (uint64_t)P;
-    uint64_t off = kHeaderBytes;
+    uint64_t off = kHeaderBytes + balanced_counter_bytes(units);  // status, then the unit counters
     p.partial_offset = off;
     off += slots * (uint64_t)M * MLA_D_V * sizeof(float);
     off = (off + 255) & ~uint64_t(255);

@@ -16,6 +16,18 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 // (mbarrier waits, TMA issues): an index read one step ahead is then issued
 // before the wait it is meant to overlap, and the compiler cannot sink it
 // behind that wait.
+// GPU-scope release store and acquire load of a flag or counter.
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Lets the grid launched after this one as its programmatic dependent be
+// scheduled once every CTA of this grid has executed it (or exited).
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ int ld_nc_ordered(const int* p) {
   int v;
   asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(p));

@@ -150,6 +150,7 @@ constexpr uint32_t kPairSmemBytes =
 
 constexpr int kSoftmaxWarp0 = 4;
 constexpr int kSoftmaxWarps = 8;
+static_assert(2 * kSoftmaxWarps == kPieceArrivals, "unit counter arrivals per piece");
 constexpr int kThreads = 32 * (kSoftmaxWarp0 + kSoftmaxWarps);
 
 // tensor memory columns (per CTA)
@@ -201,6 +202,13 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, Pie
     if (lane == 31) {
       a.sched[U] = W;
       a.sched[U + 1] = np;
+    }
+    // the table is complete: the combine (which may already run) reads it
+    // once this flag is set
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence();
+      st_release_gpu(a.unit_done + U, 1);
     }
   }
   // pieces: units of this lane's run that meet [lo, hi)
@@ -786,6 +794,15 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
             }
           }
         }
+        if (!c.whole) {
+          // this warp's share of the unit's partial O and LSE is stored: one
+          // of the kPieceArrivals arrivals the combine waits for per piece
+          __syncwarp();
+          if (lane == 0) {
+            __threadfence();
+            atomicAdd(a.unit_done + pcs[k].u, 1);
+          }
+        }
         if (!last_piece) {
           // O may be reset by the next piece's first P.V
           tc_fence_before();
@@ -884,6 +901,9 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_fp8_pair_kernel(const __grid_constant__ PairParams prm) {
+  // the combine grid may take the SMs of pairs that finish early: it waits
+  // for each unit's pieces itself
+  launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Piece* pcs = reinterpret_cast<Piece*>(smem);

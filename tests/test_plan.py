@@ -55,12 +55,14 @@ def test_workspace_holds_the_partials():
             assert p.lse_offset >= p.partial_offset + rows * p.split_kv * 512 * 4
             assert p.workspace_bytes >= p.lse_offset + rows * p.split_kv * 4
         assert p.workspace_bytes >= 256 and p.workspace_bytes % 256 == 0
-        # balanced CTA-pair schedule: 2P slots of M rows, then the unit table
+        # balanced CTA-pair schedule: the status header and the unit
+        # completion counters (units + 1 int32, cleared before each launch),
+        # 2P slots of M rows, then the unit table
         p = mla.mla_decode_plan(b, t, h, n, "fp8")
         assert p.schedule == 1 and p.kernel == 1 and p.num_ctas == 2 * p.split_kv
         slot_rows = 2 * p.split_kv * p.rows_per_unit
         units = b * p.q_groups
-        assert p.partial_offset >= 256 and p.partial_offset % 256 == 0
+        assert p.partial_offset >= 256 + (units + 1) * 4 and p.partial_offset % 256 == 0
         assert p.lse_offset >= p.partial_offset + slot_rows * 512 * 4 and p.lse_offset % 256 == 0
         assert p.workspace_bytes >= p.lse_offset + slot_rows * 4 + (units + 2) * 4
         assert p.split_kv * p.keys_per_split >= n
