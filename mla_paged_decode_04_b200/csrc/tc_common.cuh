@@ -31,6 +31,29 @@ __device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, vola
   }
 }
 
+// The same with a CTA-scope acquire (see mbar_try_wait_cta).
+__device__ __forceinline__ bool bounded_wait_cta(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                 int32_t* status) {
+  if (ptx::mbar_try_wait_cta(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (ptx::mbar_try_wait_cta(bar, parity)) return true;
+    if ((it & 127) == 0) {
+      if (*abort_flag) return false;
+      if (ptx::globaltimer() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        atomicOr(status, MLA_DEV_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ bool warp_wait_cta(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                              int32_t* status) {
+  const bool ok = bounded_wait_cta(bar, parity, abort_flag, status);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // Warp-uniform bounded wait: every lane waits (and so acquires); the warp
 // goes on only if all lanes saw the phase complete.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,

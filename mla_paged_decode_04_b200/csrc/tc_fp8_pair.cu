@@ -390,7 +390,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
           // the previous piece is done: its O_FINAL phase. (The V ring's own
           // barriers could be two phases behind here, since S runs ahead of
           // P.V; O_FINAL cannot, as its next phase needs this very load.)
-          if (!(ok = bounded_wait(bar(L::B_O_FINAL), (k - 1) & 1, abort_flag, a.status))) break;
+          if (!(ok = bounded_wait_cta(bar(L::B_O_FINAL), (k - 1) & 1, abort_flag, a.status))) break;
         }
         const int qrow = (int)c.row0 + 64 * (int)rank;  // rows past the unit are read but never stored
         mbar_arrive_expect_tx(bar(L::B_Q_MAIN), 4u * 128u * (uint32_t)box_q);
@@ -404,7 +404,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
           const int sk = jt % NK;
           const int page = valid_page(a, entry_nx);
           if (j + 1 < c.n_pt) entry_nx = piece_entry(c, 2 * (j + 1) + (int)rank);
-          if (!(ok = bounded_wait(bar(L::B_K_EMPTY + sk), ((jt / NK) & 1) ^ 1, abort_flag, a.status))) break;
+          if (!(ok = bounded_wait_cta(bar(L::B_K_EMPTY + sk), ((jt / NK) & 1) ^ 1, abort_flag, a.status))) break;
           const uint32_t ks = sb + L::kKOff + sk * L::kKSlot;
           const uint32_t full = lead(L::B_K_FULL + sk);
           if (rank == 0) mbar_arrive_expect_tx(bar(L::B_K_FULL + sk), 2u * L::kKSlot);
@@ -436,8 +436,8 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
             e1_nx = piece_entry(c, 2 * (j + 1) + 1);
           }
           // the scores of the tile exist: its pages are in L2 now
-          if (!(ok = bounded_wait(bar(L::B_QK_DONE + jt % NQ), (jt / NQ) & 1, abort_flag, a.status))) break;
-          if (!(ok = bounded_wait(bar(L::B_V_EMPTY + sv), ((jt / NV) & 1) ^ 1, abort_flag, a.status))) break;
+          if (!(ok = bounded_wait_cta(bar(L::B_QK_DONE + jt % NQ), (jt / NQ) & 1, abort_flag, a.status))) break;
+          if (!(ok = bounded_wait_cta(bar(L::B_V_EMPTY + sv), ((jt / NV) & 1) ^ 1, abort_flag, a.status))) break;
           const uint32_t vs = sb + L::kVOff + sv * L::kVSlot;
           const uint32_t full = lead(L::B_V_FULL + sv);
           if (rank == 0) mbar_arrive_expect_tx(bar(L::B_V_FULL + sv), 2u * L::kVSlot);
@@ -556,9 +556,9 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
       // 2g, 2g+1. The previous piece's S MMAs read Q until its last tile.
       if (k > 0) {
         const int jl = jt - 1;
-        if (!(ok = warp_wait(bar(L::B_S_FULL + (jl & 1)), (jl >> 1) & 1, abort_flag, a.status))) break;
+        if (!(ok = warp_wait_cta(bar(L::B_S_FULL + (jl & 1)), (jl >> 1) & 1, abort_flag, a.status))) break;
       }
-      if (!(ok = warp_wait(bar(L::B_Q_MAIN), k & 1, abort_flag, a.status))) break;
+      if (!(ok = warp_wait_cta(bar(L::B_Q_MAIN), k & 1, abort_flag, a.status))) break;
 #pragma unroll 1
       for (int c2 = 0; c2 < 2; ++c2) {
         const int cc = 2 * grp + c2;
@@ -598,7 +598,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
         const int ph = (jg >> 1) & 1;
         const int pg_cur = pg_next;
         if (j + 2 < c.n_pt) pg_next = table_entry(j + 2);
-        if (!(ok = warp_wait(bar(L::B_S_FULL + buf), ph, abort_flag, a.status))) break;
+        if (!(ok = warp_wait_cta(bar(L::B_S_FULL + buf), ph, abort_flag, a.status))) break;
         tc_fence_after();
         uint32_t sv[64];
         {
@@ -642,14 +642,14 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
         xm[((grp * 2 + ph) * 2 + hf) * 64 + rl] = mt;
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(L::B_X + grp));
-        if (!(ok = warp_wait(bar(L::B_X + grp), ph, abort_flag, a.status))) break;
+        if (!(ok = warp_wait_cta(bar(L::B_X + grp), ph, abort_flag, a.status))) break;
         mt = fmaxf(mt, xm[((grp * 2 + ph) * 2 + (hf ^ 1)) * 64 + rl]);
         // reference maximum after the previous tile (from the other group; a
         // new piece starts afresh but still takes the hand-off, which keeps
         // the reference array's reuse ordered), lazily updated
         float m_prev = -INFINITY;
         if (jg > 0) {
-          if (!(ok = warp_wait(bar(L::B_M_READY + (buf ^ 1)), ((jg - 1) >> 1) & 1, abort_flag, a.status))) break;
+          if (!(ok = warp_wait_cta(bar(L::B_M_READY + (buf ^ 1)), ((jg - 1) >> 1) & 1, abort_flag, a.status))) break;
           if (j > 0) m_prev = mref[(buf ^ 1) * 64 + rl];
         }
         const float m_j = (mt > m_prev + kTau) ? mt : m_prev;
@@ -660,7 +660,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
         const float m_use = (m_j == -INFINITY) ? 0.f : m_j - kSigma;
 
         // P buffer is free once the P.V two tiles back has finished
-        if (jg >= 2 && !(ok = warp_wait(bar(L::B_P_EMPTY + buf), ph ^ 1, abort_flag, a.status))) break;
+        if (jg >= 2 && !(ok = warp_wait_cta(bar(L::B_P_EMPTY + buf), ph ^ 1, abort_flag, a.status))) break;
 
         // P = 2^(s * sl2 - m_use), 16 keys (one 16-byte chunk) at a time; this
         // half's 64 keys are bytes [64hf, 64hf + 64) of the 128-byte P row.
@@ -695,7 +695,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
         // rescale this thread's 256 O columns if the reference maximum moved
         // (not on a piece's first tile: O is reset by its first P.V)
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-          if (!(ok = warp_wait(bar(L::B_O_DONE), (jg - 1) & 1, abort_flag, a.status))) break;
+          if (!(ok = warp_wait_cta(bar(L::B_O_DONE), (jg - 1) & 1, abort_flag, a.status))) break;
           tc_fence_after();
           // two 32-column chunks per tensor-memory round trip (the score
           // registers are free by now)
@@ -729,7 +729,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
       fin[((1 * 2 + grp) * 2 + hf) * 64 + rl] = m_grp;
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(L::B_FIN));
-      if (ok) ok = warp_wait(bar(L::B_FIN), k & 1, abort_flag, a.status);
+      if (ok) ok = warp_wait_cta(bar(L::B_FIN), k & 1, abort_flag, a.status);
       float le = 0.f, m_fin = -INFINITY;
       if (ok) {
 #pragma unroll
@@ -742,7 +742,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
           }
         }
       }
-      if (ok) ok = warp_wait(bar(L::B_O_FINAL), k & 1, abort_flag, a.status);
+      if (ok) ok = warp_wait_cta(bar(L::B_O_FINAL), k & 1, abort_flag, a.status);
       if (!ok) break;
       tc_fence_after();
       const float inv = (le > 0.f) ? a.v_scale / le : 0.f;
@@ -833,7 +833,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(L::B_EPI));
-        if (!(ok = warp_wait(bar(L::B_EPI), 0, abort_flag, a.status))) break;
+        if (!(ok = warp_wait_cta(bar(L::B_EPI), 0, abort_flag, a.status))) break;
         // softmax warp w writes local rows 8w .. 8w+7
         const int w8 = warp - kSoftmaxWarp0;
 #pragma unroll 1
