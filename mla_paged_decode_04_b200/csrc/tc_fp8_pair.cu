@@ -627,16 +627,17 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
         }
         float mt;
         {
-          float m8[8];
+          // four independent chains of three-input maxima over 16 keys each
+          float m4[4];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float v = __uint_as_float(sv[8 * i]);
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const uint32_t* x = sv + 16 * c4;
+            float v = max3f(__uint_as_float(x[0]), __uint_as_float(x[1]), __uint_as_float(x[2]));
 #pragma unroll
-            for (int e = 1; e < 8; ++e) v = fmaxf(v, __uint_as_float(sv[8 * i + e]));
-            m8[i] = v;
+            for (int e = 3; e < 15; e += 2) v = max3f(v, __uint_as_float(x[e]), __uint_as_float(x[e + 1]));
+            m4[c4] = fmaxf(v, __uint_as_float(x[15]));
           }
-          mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) *
-               sl2;
+          mt = fmaxf(max3f(m4[0], m4[1], m4[2]), m4[3]) * sl2;
         }
         // the other half of the row lives in the warp of quarter q^2
         xm[((grp * 2 + ph) * 2 + hf) * 64 + rl] = mt;
@@ -664,7 +665,9 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
 
         // P = 2^(s * sl2 - m_use), 16 keys (one 16-byte chunk) at a time; this
         // half's 64 keys are bytes [64hf, 64hf + 64) of the 128-byte P row.
-        float se[4] = {0.f, 0.f, 0.f, 0.f};
+        // packed pairs: one FMA and one add for two keys
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), nmx2 = f2_pack(-m_use, -m_use);
+        uint64_t se2[2] = {0ull, 0ull};  // two (even key, odd key) partial sums
         uint8_t* prow = smem + L::kPOff + buf * L::kPBuf + rl * 128;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -672,9 +675,11 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int e = 16 * u + 2 * i;
-            const float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -m_use));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -m_use));
-            se[i & 3] += p0 + p1;
+            float a0, a1;
+            f2_unpack(fma_f32x2(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nmx2), a0, a1);
+            const float p0 = ex2_approx(a0);
+            const float p1 = ex2_approx(a1);
+            se2[i & 1] = add_f32x2(se2[i & 1], f2_pack(p0, p1));
             const uint32_t qh = cvt_e4m3x2(p0, p1);
             if (i & 1) hi[i >> 1] |= qh << 16; else hi[i >> 1] = qh;
             if (kTwo) {
@@ -688,7 +693,10 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
           if (kTwo && c.two)
             *reinterpret_cast<uint4*>(prow + L::kPPlane + phys * 16) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
-        const float sum = (se[0] + se[1]) + (se[2] + se[3]);
+        float s0, s1, s2, s3;
+        f2_unpack(se2[0], s0, s1);
+        f2_unpack(se2[1], s2, s3);
+        const float sum = (s0 + s1) + (s2 + s3);
         l_grp = (m_grp == m_j) ? l_grp + sum : fmaf(l_grp, ex2_approx(m_grp - m_j), sum);
         m_grp = m_j;
 
