@@ -300,7 +300,7 @@ def run_ours(args):
     elif g.dtype == "fp8":
         kname = "tc_fp8_pair_kernel" if plan.kernel == 1 else "tc_fp8_partial_kernel"
     else:
-        kname = "tc_partial_kernel"
+        kname = "tc16_pair_kernel" if plan.schedule == 1 else "tc_partial_kernel"
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "peak_source": peak_kind,
                 "traffic": traffic_from_profile(args.workload, kname), "kernel": kname,

@@ -79,7 +79,7 @@ int check_plan(const mla_plan* p) {
   if (p->schedule != MLA_SCHEDULE_SPLITS && p->schedule != MLA_SCHEDULE_BALANCED) return MLA_ERR_PLAN_MISMATCH;
   if (p->schedule == MLA_SCHEDULE_BALANCED) {
     // FP8 CTA-pair kernel only; slots [2P, M, 512] fp32 + [2P, M] + unit table
-    if (p->kernel != MLA_KERNEL_TCGEN05 || p->dtype != MLA_FP8_E4M3 || p->split_kv > kNumSMs / 2)
+    if (p->kernel != MLA_KERNEL_TCGEN05 || p->split_kv > kNumSMs / 2)
       return MLA_ERR_PLAN_MISMATCH;
     const int64_t units = (int64_t)p->batch * p->q_groups;
     if (units > kMaxBalancedUnits) return MLA_ERR_PLAN_MISMATCH;
@@ -179,8 +179,8 @@ int run_partial(const DecodeArgs& a, cudaStream_t st) {
     e = launch_simt_partial(a, st);
   else if (a.plan.kernel == MLA_KERNEL_TCGEN05_SOLO)
     e = launch_tc_fp8_partial(a, st);
-  else if (a.plan.dtype == MLA_FP8_E4M3)
-    e = launch_tc_fp8_pair_partial(a, st);
+  else if (a.plan.schedule == MLA_SCHEDULE_BALANCED)
+    e = a.plan.dtype == MLA_FP8_E4M3 ? launch_tc_fp8_pair_partial(a, st) : launch_tc16_pair_partial(a, st);
   else
     e = launch_tc_partial(a, st);
   return e == cudaSuccess ? MLA_OK : cuda_failure(e);

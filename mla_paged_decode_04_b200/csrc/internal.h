@@ -69,6 +69,7 @@ cudaError_t launch_tc_partial(const DecodeArgs& a, cudaStream_t stream);      //
 cudaError_t launch_tc_fp8_partial(const DecodeArgs& a, cudaStream_t stream);  // FP8, per-CTA MMAs
 cudaError_t launch_tc_fp8_pair_partial(const DecodeArgs& a, cudaStream_t stream);  // FP8, CTA-pair MMAs
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_tc16_pair_partial(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_combine_balanced(const DecodeArgs& a, cudaStream_t stream);
 
 }  // namespace mla

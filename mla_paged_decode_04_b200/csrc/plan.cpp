@@ -124,12 +124,13 @@ int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, i
   p.q_groups = G;
   p.rows_per_unit = M;
   const uint64_t rows = (uint64_t)batch * q_len * num_heads;
-  // The balanced schedule keeps a per-pair piece list in shared memory; far
-  // more units than pairs can hold fall back to fixed splits (solo kernel).
+  // The balanced schedule (CTA-pair kernels) keeps a per-pair piece list in
+  // shared memory; far more units than pairs can hold fall back to fixed
+  // splits (FP8: the solo kernel; 16-bit: the exchange kernel).
   if (kern == MLA_KERNEL_TCGEN05 && dtype == MLA_FP8_E4M3 && units > kMaxBalancedUnits)
     kern = MLA_KERNEL_TCGEN05_SOLO;
   p.kernel = kern;
-  if (kern == MLA_KERNEL_TCGEN05 && dtype == MLA_FP8_E4M3) {
+  if (kern == MLA_KERNEL_TCGEN05 && units <= kMaxBalancedUnits) {
     const int P = split_kv > 0 ? (split_kv < kNumSMs / 2 ? split_kv : kNumSMs / 2) : kNumSMs / 2;
     p.schedule = MLA_SCHEDULE_BALANCED;
     p.split_kv = P;

@@ -1,0 +1,887 @@
+// Split-KV partial kernel for BF16 / FP16 inputs with CTA-pair tensor-core
+// MMAs and the balanced, persistent schedule.
+//
+// The first of the two decode kernels (TokenSpeed MLA article
+// 最快MLA内核背后的秘密, section 二) with query-token folding (section 三) and
+// the 2-CTA MMA of section 四: the two CTAs of a cluster execute every
+// tcgen05.mma together (cta_group::2, M = 128, kind::f16), each holding half
+// of the operands and half of the result. The structure follows the FP8
+// pair kernel; what differs is sized for 2-byte elements:
+//
+// * A pair tile is one 64-key page: CTA c loads keys [32c, 32c + 32) of it
+//   (36 KB: 512 latent dims in eight SW128 chunks plus the rope chunk), so a
+//   K slot has the size it has in FP8.
+// * Q's 576 dims per row take 1152 bytes, too many for tensor memory next to
+//   O. Dims 0..255 and the rope (64 dims) go to tensor memory (160 columns,
+//   A operand read by the MMA itself); dims 256..511 stay in shared memory
+//   (32 KB per CTA, A operand from shared memory). S = Q.K^T of a tile is
+//   16 + 16 + 4 MMAs of K = 16 into one accumulator.
+// * S is M = 128 by N = 64: CTA c receives its 64 rows, keys 0..31 in TMEM
+//   lanes 0..63 and keys 32..63 in lanes 64..127 (32 columns per buffer).
+//   One softmax thread takes one (row, key half): 32 keys per tile.
+// * P is the inputs' 16-bit type (64 keys x 2 bytes = one 128-byte row per
+//   query row); O += P.V is two MMAs of N = 256 per 16-key step, CTA c
+//   supplying V columns [256h + 128c, 256h + 128c + 128) as B from its V
+//   ring (the page's 64 keys, re-read from L2 once S exists).
+//
+// Roles (384 threads per CTA), barriers, the piece walk, the epilogue and
+// the bounded waits are those of the FP8 pair kernel (warp 0 Q and K loads,
+// warp 1 TMEM and S MMAs, warp 2 P.V MMAs, warp 3 V loads, warps 4-11 two
+// softmax groups on alternate tiles). No TMA load uses multicast.
+#include <cuda.h>
+
+#include "device_common.cuh"
+#include "sm100_ptx.cuh"
+#include "tc_common.cuh"
+
+namespace mla {
+namespace {
+
+using namespace ptx;
+
+constexpr float kTau = 4.f;          // lazy-rescale threshold (log2 units)
+constexpr float kSigma = 8.f;        // P <= 2^(kTau + kSigma) = 4096, inside FP16's range
+constexpr int kMaxPieces = 64;       // pieces per pair (units its range touches)
+constexpr int kMinPairTiles = 2;     // fewer tiles than this per pair: use fewer pairs
+constexpr int kHalfKeys = 32;        // keys per CTA per pair tile
+constexpr int kTile16 = 64;          // keys per pair tile (one page)
+
+struct Piece {
+  int u, t0, t1;  // pair tiles [t0, t1) of unit u
+};
+struct SchedInfo {
+  int npc;  // pieces of this pair
+  int pad;
+};
+constexpr uint32_t kSchedBytes = 1024;
+static_assert(kMaxPieces * sizeof(Piece) + sizeof(SchedInfo) <= kSchedBytes, "schedule area");
+
+struct Layout16 {
+  static constexpr int NK = 3;                                  // K-ring slots: this CTA's half page
+  static constexpr int NV = 2;                                  // V-ring slots: 256 V columns of the page
+  static constexpr uint32_t kQRes = kSchedBytes;                // Q dims 256..511: 4 chunks of 64 rows x 128 B
+  static constexpr uint32_t kPOff = kQRes + 4 * 8192;           // P[2 buffers]: 64 rows x 64 keys x 2 B
+  static constexpr uint32_t kPBuf = 64 * 128;
+  static constexpr uint32_t kKSlot = 9 * 4096;                  // 8 latent chunks + rope, 32 rows x 128 B each
+  static constexpr uint32_t kKOff = kPOff + 2 * kPBuf;
+  static constexpr uint32_t kVSlot = 4 * 8192;                  // [h][2 chunks][64 keys][128 B]
+  static constexpr uint32_t kVOff = kKOff + NK * kKSlot;
+  // At a piece's start the V ring is idle: Q dims 0..255 are staged in the
+  // last V slot and the Q rope in the first, until the softmax warps have
+  // copied them into tensor memory.
+  static constexpr uint32_t kQStage = kVOff + (NV - 1) * kVSlot;
+  static constexpr uint32_t kQRopeStage = kVOff;
+  static constexpr uint32_t kMOff = kVOff + NV * kVSlot;        // row reference maxima [tile parity][64]
+  static constexpr uint32_t kXOff = kMOff + 512;                // half-row maxima [group][phase][half][64]
+  static constexpr uint32_t kFinOff = kXOff + 2048;             // final (l, m) [l|m][group][half][64]
+  static constexpr uint32_t kBarOff = kFinOff + 2048;
+  static constexpr int B_Q_MAIN = 0;                 // local, per piece: Q landed (all three parts)
+  static constexpr int B_Q_TMEM = 1;                 // leader, per piece: both CTAs copied Q into TMEM
+  static constexpr int B_K_FULL = 2;                 // leader, + K slot: both halves landed
+  static constexpr int B_K_EMPTY = B_K_FULL + NK;    // both, + K slot
+  static constexpr int B_V_FULL = B_K_EMPTY + NK;    // leader, + V slot
+  static constexpr int B_V_EMPTY = B_V_FULL + NV;    // both, + V slot
+  static constexpr int B_S_FULL = B_V_EMPTY + NV;    // both, + buffer
+  static constexpr int B_S_EMPTY = B_S_FULL + 2;     // leader, + buffer
+  static constexpr int B_P_FULL = B_S_EMPTY + 2;     // leader, + buffer
+  static constexpr int B_P_EMPTY = B_P_FULL + 2;     // both, + buffer
+  static constexpr int B_O_DONE = B_P_EMPTY + 2;     // both
+  static constexpr int B_O_FINAL = B_O_DONE + 1;     // both, per piece: after the piece's last P.V
+  static constexpr int B_M_READY = B_O_FINAL + 1;    // local, + tile parity
+  static constexpr int B_X = B_M_READY + 2;          // local, + group: half-row maxima exchanged
+  static constexpr int B_FIN = B_X + 2;              // local, per piece: both groups published (l, m)
+  // both, + tile % NQ: the scores of the tile exist (the V loads may go).
+  // NQ = 6 rules out phase aliasing as in the FP8 kernel.
+  static constexpr int NQ = 6;
+  static constexpr int B_QK_DONE = B_FIN + 1;
+  static constexpr int B_EPI = B_QK_DONE + NQ;       // local, per piece: the output tile is staged
+  static constexpr int B_O_FREE = B_EPI + 1;         // leader, per piece: both CTAs read O
+  static constexpr int kNBars = B_O_FREE + 1;
+  static_assert(8 * kNBars <= 512, "barrier area");
+  static constexpr uint32_t kMiscOff = kBarOff + 512;
+  // The dynamic shared memory base is 1024-aligned (checked at run time;
+  // the kernel refuses to run otherwise), so no alignment slack is added.
+  static constexpr uint32_t kSmemBytes = kMiscOff + 16;
+  static_assert(kQRes % 1024 == 0 && kPOff % 1024 == 0 && kKOff % 1024 == 0 && kVOff % 1024 == 0, "alignment");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  // the last piece's epilogue stages the 64 x 512 fp32 output tile in the
+  // (then idle) K and V rings
+  static_assert(NK * kKSlot + NV * kVSlot >= 64 * MLA_D_V * 4, "staging area");
+};
+
+constexpr int kSoftmaxWarp0 = 4;
+constexpr int kSoftmaxWarps = 8;
+static_assert(2 * kSoftmaxWarps == kPieceArrivals, "unit counter arrivals per piece");
+constexpr int kThreads = 32 * (kSoftmaxWarp0 + kSoftmaxWarps);
+
+// tensor memory columns (per CTA)
+constexpr uint32_t kOCol = 0;       // O: column half h at [128h, 128h + 128)
+constexpr uint32_t kQCol = 256;     // Q dims 0..255, two per column, rows duplicated over lane halves
+constexpr uint32_t kQRopeCol = 384; // Q rope dims, two per column
+constexpr uint32_t kSCol = 448;     // two S buffers of 32 columns
+
+struct Pair16Params {
+  CUtensorMap tm_q, tm_k8, tm_kv, tm_v[2];
+  DecodeArgs a;
+};
+
+// Pair tiles of unit u (= b * G + g): one per 64-key page of entry b.
+__device__ __forceinline__ int unit_tiles16(const DecodeArgs& a, int u, bool flag) {
+  const int n = effective_seq_len(a, u / a.plan.q_groups, flag);
+  return (n + kTile16 - 1) / kTile16;
+}
+
+// One warp: the balanced schedule of this pair (the FP8 kernel's, with
+// 64-key pair tiles). CTA 0 of pair 0 also writes the unit start table the
+// combine reads, then its ready flag.
+__device__ void build_schedule16(const DecodeArgs& a, int pair, uint32_t rank, Piece* pcs, SchedInfo* info) {
+  const mla_plan& p = a.plan;
+  const int lane = threadIdx.x & 31;
+  const int U = p.batch * p.q_groups;
+  const int per = (U + 31) / 32;
+  const int u_beg = min(U, lane * per), u_end = min(U, u_beg + per);
+  const bool writer = pair == 0 && rank == 0;
+  int run = 0;
+  for (int u = u_beg; u < u_end; ++u) run += unit_tiles16(a, u, writer && u % p.q_groups == 0);
+  int excl = run;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, excl, d);
+    if (lane >= d) excl += y;
+  }
+  const int W = __shfl_sync(0xffffffffu, excl, 31);
+  excl -= run;
+  const int np = max(1, min(p.split_kv, (W + kMinPairTiles - 1) / kMinPairTiles));
+  const int64_t lo = pair < np ? balanced_lo(pair, W, np) : W;
+  const int64_t hi = pair < np ? balanced_lo(pair + 1, W, np) : W;
+  if (writer) {
+    int start = excl;
+    for (int u = u_beg; u < u_end; ++u) {
+      a.sched[u] = start;
+      start += unit_tiles16(a, u, false);
+    }
+    if (lane == 31) {
+      a.sched[U] = W;
+      a.sched[U + 1] = np;
+    }
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence();
+      st_release_gpu(a.unit_done + U, 1);
+    }
+  }
+  int cnt = 0;
+  {
+    int start = excl;
+    for (int u = u_beg; u < u_end; ++u) {
+      const int t = unit_tiles16(a, u, false);
+      if (t > 0 && start < hi && start + t > lo) ++cnt;
+      start += t;
+    }
+  }
+  int base = cnt;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, base, d);
+    if (lane >= d) base += y;
+  }
+  const int npc = __shfl_sync(0xffffffffu, base, 31);
+  base -= cnt;
+  {
+    int start = excl, k = base;
+    for (int u = u_beg; u < u_end; ++u) {
+      const int t = unit_tiles16(a, u, false);
+      if (t > 0 && start < hi && start + t > lo) {
+        if (k < kMaxPieces) {
+          pcs[k].u = u;
+          pcs[k].t0 = lo > start ? (int)(lo - start) : 0;
+          pcs[k].t1 = hi - start < t ? (int)(hi - start) : t;
+        }
+        ++k;
+      }
+      start += t;
+    }
+  }
+  if (lane == 0) info->npc = npc;
+}
+
+// Per-piece constants every role derives the same way.
+struct PieceCtx16 {
+  int b, g, n, key0, key1, n_pt, page0;
+  int64_t row0;
+  const int32_t* table;
+  bool whole;  // the piece is the whole unit: final output, not a partial
+};
+
+__device__ __forceinline__ PieceCtx16 piece_ctx16(const DecodeArgs& a, const Piece& pc) {
+  const mla_plan& p = a.plan;
+  PieceCtx16 c;
+  c.b = pc.u / p.q_groups;
+  c.g = pc.u % p.q_groups;
+  c.n = effective_seq_len(a, c.b, false);
+  c.key0 = pc.t0 * kTile16;
+  c.key1 = min(c.n, pc.t1 * kTile16);
+  c.n_pt = pc.t1 - pc.t0;
+  c.page0 = pc.t0;  // block-table index of the piece's first page
+  c.row0 = (int64_t)c.b * p.q_len * p.num_heads + (int64_t)c.g * p.rows_per_unit;
+  c.table = a.block_tables + (int64_t)c.b * a.max_pages_per_seq;
+  c.whole = pc.t0 == 0 && c.key1 >= c.n;
+  return c;
+}
+
+// Block-table entry of pair tile j of the piece, read one tile ahead of its
+// use with a load kept ahead of the next barrier wait.
+__device__ __forceinline__ int piece_entry16(const PieceCtx16& c, int j) {
+  return j < c.n_pt ? ld_nc_ordered(c.table + c.page0 + j) : 0;
+}
+// an entry outside the cache reads page 0 (its keys are masked by the softmax)
+__device__ __forceinline__ int valid_page16(const DecodeArgs& a, int pg) {
+  return (pg < 0 || (int64_t)pg >= a.num_pages) ? 0 : pg;
+}
+
+template <bool kBf16>
+__device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* smem, const Piece* pcs, int npc) {
+  using L = Layout16;
+  constexpr int NK = L::NK, NV = L::NV, NQ = L::NQ;
+  const DecodeArgs& a = prm.a;
+  const mla_plan& p = a.plan;
+  const uint32_t sb = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sb + L::kBarOff + 8u * (uint32_t)i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0 = leader
+  const int pair = blockIdx.x >> 1;
+  const int T = p.q_len, H = p.num_heads, M = p.rows_per_unit;
+  const int box_q = M < 64 ? M : 64;  // query rows per TMA box
+  auto slot_of = [&](int k) -> int64_t { return 2 * (int64_t)pair + (k == 0 ? 0 : 1); };
+  auto lead = [&](int i) -> uint32_t { return mapa(bar(i), 0); };
+  auto arrive_lead = [&](int i) {
+    if (rank == 0) mbar_arrive(bar(i)); else mbar_arrive_remote_publish_smem(lead(i));
+  };
+  auto arrive_lead_relaxed = [&](int i) {
+    if (rank == 0) mbar_arrive(bar(i)); else mbar_arrive_remote_relaxed(lead(i));
+  };
+
+  // ---------------------------------------------------------------- setup
+  if (threadIdx.x == 0) {
+    mbar_init(bar(L::B_Q_MAIN), 1);
+    mbar_init(bar(L::B_Q_TMEM), 2 * kSoftmaxWarps);
+    for (int i = 0; i < NK; ++i) {
+      mbar_init(bar(L::B_K_FULL + i), 1);
+      mbar_init(bar(L::B_K_EMPTY + i), 1);
+    }
+    for (int i = 0; i < NV; ++i) {
+      mbar_init(bar(L::B_V_FULL + i), 1);
+      mbar_init(bar(L::B_V_EMPTY + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(L::B_S_FULL + i), 1);
+      mbar_init(bar(L::B_S_EMPTY + i), 2 * 4);  // the tile's softmax group in each CTA
+      mbar_init(bar(L::B_P_FULL + i), 2 * 4);
+      mbar_init(bar(L::B_P_EMPTY + i), 1);
+      mbar_init(bar(L::B_M_READY + i), 4);
+      mbar_init(bar(L::B_X + i), 4);
+    }
+    mbar_init(bar(L::B_O_DONE), 1);
+    mbar_init(bar(L::B_O_FINAL), 1);
+    mbar_init(bar(L::B_FIN), kSoftmaxWarps);
+    for (int i = 0; i < NQ; ++i) mbar_init(bar(L::B_QK_DONE + i), 1);
+    mbar_init(bar(L::B_EPI), kSoftmaxWarps);
+    mbar_init(bar(L::B_O_FREE), 2 * kSoftmaxWarps);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (box_q < 64) {
+    // Rows the Q boxes do not cover are zero in the resident Q part (its
+    // rows are independent A rows of S; zero keeps them finite).
+    for (int i = threadIdx.x; i < 4 * (64 - box_q) * 8; i += blockDim.x) {
+      const int ci = i / ((64 - box_q) * 8), rem = i % ((64 - box_q) * 8);
+      reinterpret_cast<uint4*>(smem + L::kQRes + ci * 8192 + box_q * 128)[rem] = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers and TMEM exist before any cross-CTA use
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  int n_all = 0;  // pair tiles over all pieces
+  for (int k = 0; k < npc; ++k) n_all += pcs[k].t1 - pcs[k].t0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ Q and K-ring loads
+    if (lane == 0) {
+      prefetch_tmap(&prm.tm_q);
+      prefetch_tmap(&prm.tm_k8);
+      prefetch_tmap(&prm.tm_kv);
+      const uint64_t pol_q = policy_evict_first();
+      const uint64_t pol_kv = policy_evict_last();  // read again right away for V
+      int jt = 0;
+      bool ok = true;
+      for (int k = 0; ok && k < npc; ++k) {
+        const PieceCtx16 c = piece_ctx16(a, pcs[k]);
+        if (k > 0) {
+          // the Q areas and the staging slots are free once every MMA of the
+          // previous piece is done: its O_FINAL phase
+          if (!(ok = bounded_wait_cta(bar(L::B_O_FINAL), (k - 1) & 1, abort_flag, a.status))) break;
+        }
+        const int qrow = (int)c.row0 + 64 * (int)rank;  // rows past the unit are read but never stored
+        mbar_arrive_expect_tx(bar(L::B_Q_MAIN), 9u * 128u * (uint32_t)box_q);
+#pragma unroll
+        for (int ci = 0; ci < 4; ++ci) {
+          tma_load_2d(sb + L::kQStage + ci * 8192, &prm.tm_q, 64 * ci, qrow, bar(L::B_Q_MAIN), pol_q);
+          tma_load_2d(sb + L::kQRes + ci * 8192, &prm.tm_q, 256 + 64 * ci, qrow, bar(L::B_Q_MAIN), pol_q);
+        }
+        tma_load_2d(sb + L::kQRopeStage, &prm.tm_q, 512, qrow, bar(L::B_Q_MAIN), pol_q);
+        int entry_nx = piece_entry16(c, 0);
+        for (int j = 0; j < c.n_pt; ++j, ++jt) {
+          const int sk = jt % NK;
+          const int page = valid_page16(a, entry_nx);
+          if (j + 1 < c.n_pt) entry_nx = piece_entry16(c, j + 1);
+          if (!(ok = bounded_wait_cta(bar(L::B_K_EMPTY + sk), ((jt / NK) & 1) ^ 1, abort_flag, a.status))) break;
+          const uint32_t ks = sb + L::kKOff + sk * L::kKSlot;
+          const uint32_t full = lead(L::B_K_FULL + sk);
+          const int row = page * kTile16 + kHalfKeys * (int)rank;  // this CTA's 32 keys of the page
+          if (rank == 0) mbar_arrive_expect_tx(bar(L::B_K_FULL + sk), 2u * L::kKSlot);
+          tma_load_3d_pair(ks, &prm.tm_k8, 0, row, 0, full, pol_kv);            // 8 latent chunks
+          tma_load_2d_pair(ks + 8 * 4096, &prm.tm_kv, 512, row, full, pol_kv);   // rope
+        }
+      }
+      // The leader's K_FULL phases count both CTAs' bytes: the leader waits for
+      // the last ones before the pair may leave.
+      if (rank == 0) drain_loads(bar(L::B_K_FULL), NK, n_all);
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ V-ring loads
+    if (lane == 0) {
+      prefetch_tmap(&prm.tm_v[rank]);
+      const uint64_t pol_v = policy_evict_first();  // last use of these bytes
+      int jt = 0;
+      bool ok = true;
+      for (int k = 0; ok && k < npc; ++k) {
+        const PieceCtx16 c = piece_ctx16(a, pcs[k]);
+        int e_nx = piece_entry16(c, 0);
+        for (int j = 0; j < c.n_pt; ++j, ++jt) {
+          const int sv = jt % NV;
+          const int pg = valid_page16(a, e_nx);
+          if (j + 1 < c.n_pt) e_nx = piece_entry16(c, j + 1);
+          // the scores of the tile exist: its page is in L2 now
+          if (!(ok = bounded_wait_cta(bar(L::B_QK_DONE + jt % NQ), (jt / NQ) & 1, abort_flag, a.status))) break;
+          if (!(ok = bounded_wait_cta(bar(L::B_V_EMPTY + sv), ((jt / NV) & 1) ^ 1, abort_flag, a.status))) break;
+          const uint32_t vs = sb + L::kVOff + sv * L::kVSlot;
+          const uint32_t full = lead(L::B_V_FULL + sv);
+          if (rank == 0) mbar_arrive_expect_tx(bar(L::B_V_FULL + sv), 2u * L::kVSlot);
+          // half h: this CTA's V columns [256h + 128 rank, +128), two chunks
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            tma_load_3d_pair(vs + h * 16384, &prm.tm_v[rank], 0, pg * kTile16, 4 * h, full, pol_v);
+        }
+      }
+      if (rank == 0) drain_loads(bar(L::B_V_FULL), NV, n_all);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ S = Q.K^T issuer (leader)
+    if (rank == 0) {
+      constexpr uint32_t fmt = kBf16 ? 1u : 0u;
+      constexpr uint32_t idq = instr_desc(fmt, fmt, 0, 128, kTile16);  // K-major B
+      int jt = 0;
+      bool ok = true;
+      for (int k = 0; ok && k < npc; ++k) {
+        const int n_pt = pcs[k].t1 - pcs[k].t0;
+        if (!(ok = warp_wait(bar(L::B_Q_TMEM), k & 1, abort_flag, a.status))) break;
+        for (int j = 0; j < n_pt; ++j, ++jt) {
+          const int sk = jt % NK, buf = jt & 1;
+          if (!(ok = warp_wait(bar(L::B_K_FULL + sk), (jt / NK) & 1, abort_flag, a.status))) break;
+          if (!(ok = warp_wait(bar(L::B_S_EMPTY + buf), ((jt >> 1) & 1) ^ 1, abort_flag, a.status))) break;
+          tc_fence_after();
+          const uint32_t d = tmem + kSCol + 32u * buf;
+          const uint32_t ks = sb + L::kKOff + sk * L::kKSlot;
+          // dims 0..255: A from tensor memory, 16 dims (8 columns) per MMA
+#pragma unroll
+          for (int ci = 0; ci < 4; ++ci) {
+            const uint64_t dk = smem_desc(ks + ci * 4096, 16, 1024, kSw128);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16_ts_pair_e(d, tmem + kQCol + (uint32_t)(8 * (4 * ci + kk)), dk + (uint64_t)(kk * 2), idq,
+                                (ci | kk) ? 1u : 0u);
+          }
+          // dims 256..511: A from the resident shared-memory part
+#pragma unroll
+          for (int ci = 0; ci < 4; ++ci) {
+            const uint64_t dk = smem_desc(ks + (4 + ci) * 4096, 16, 1024, kSw128);
+            const uint64_t dq = smem_desc(sb + L::kQRes + ci * 8192, 16, 1024, kSw128);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16_ss_pair_e(d, dq + (uint64_t)(kk * 2), dk + (uint64_t)(kk * 2), idq, 1u);
+          }
+          // rope: A from tensor memory
+          {
+            const uint64_t dk = smem_desc(ks + 8 * 4096, 16, 1024, kSw128);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16_ts_pair_e(d, tmem + kQRopeCol + (uint32_t)(8 * kk), dk + (uint64_t)(kk * 2), idq, 1u);
+          }
+          mma_commit_pair_mc_e(bar(L::B_S_FULL + buf), 3);
+          mma_commit_pair_mc_e(bar(L::B_K_EMPTY + sk), 3);
+          mma_commit_pair_mc_e(bar(L::B_QK_DONE + jt % NQ), 3);
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ O += P.V issuer (leader)
+    if (rank == 0) {
+      constexpr uint32_t fmt = kBf16 ? 1u : 0u;
+      constexpr uint32_t idp = instr_desc(fmt, fmt, 1, 128, 256);  // V is MN-major
+      int jt = 0;
+      bool ok = true;
+      for (int k = 0; ok && k < npc; ++k) {
+        const int n_pt = pcs[k].t1 - pcs[k].t0;
+        if (k > 0 && !(ok = warp_wait(bar(L::B_O_FREE), (k - 1) & 1, abort_flag, a.status))) break;
+        for (int j = 0; j < n_pt; ++j, ++jt) {
+          const int buf = jt & 1, sv = jt % NV;
+          if (!(ok = warp_wait(bar(L::B_V_FULL + sv), (jt / NV) & 1, abort_flag, a.status))) break;
+          if (!(ok = warp_wait(bar(L::B_P_FULL + buf), (jt >> 1) & 1, abort_flag, a.status))) break;
+          tc_fence_after();
+          const uint32_t vs = sb + L::kVOff + sv * L::kVSlot;
+          const uint64_t dp = smem_desc(sb + L::kPOff + buf * L::kPBuf, 16, 1024, kSw128);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int ks4 = 0; ks4 < 4; ++ks4) {  // 16 keys per MMA
+              const uint64_t dv = smem_desc(vs + h * 16384 + ks4 * 2048, 8192, 1024, kSw128);
+              mma_f16_ss_pair_e(tmem + kOCol + 128u * h, dp + (uint64_t)(ks4 * 2), dv, idp,
+                                (j > 0 || ks4 > 0) ? 1u : 0u);
+            }
+          }
+          mma_commit_pair_mc_e(bar(L::B_O_DONE), 3);
+          mma_commit_pair_mc_e(bar(L::B_P_EMPTY + buf), 3);
+          mma_commit_pair_mc_e(bar(L::B_V_EMPTY + sv), 3);
+          if (j == n_pt - 1) mma_commit_pair_mc_e(bar(L::B_O_FINAL), 3);
+        }
+      }
+    }
+  } else if (warp >= kSoftmaxWarp0) {
+    // ------------------------------------------------------------ softmax warps
+    // Group grp takes the tiles whose running index has parity grp; warp w
+    // serves TMEM lane quarter q = w%4: local rows 32(q%2) .. +31, key half
+    // hf = q/2 (keys [32hf, 32hf + 32) of the page).
+    const int q = warp & 3;
+    const int grp = (warp - kSoftmaxWarp0) >> 2;
+    const int hf = q >> 1;
+    const int rl = 32 * (q & 1) + lane;  // local row (0..63)
+    const int r = 64 * (int)rank + rl;   // row within the unit
+    const uint32_t tl = (uint32_t)(32 * q) << 16;
+    float* mref = reinterpret_cast<float*>(smem + L::kMOff);  // [tile parity][64]
+    float* xm = reinterpret_cast<float*>(smem + L::kXOff);    // [group][phase][half][64]
+    float* fin = reinterpret_cast<float*>(smem + L::kFinOff); // [l|m][group][half][64]
+    const float sl2 = a.score_scale_log2;
+    bool ok = true;
+    int jt = 0;  // running index of the piece's first tile
+
+    for (int k = 0; ok && k < npc; ++k) {
+      const PieceCtx16 c = piece_ctx16(a, pcs[k]);
+      const bool last_piece = k == npc - 1;
+      const int limit = min((r < M) ? c.n - T + c.g * p.fold + r / H : c.n - 1, c.key1 - 1);
+
+      // Q dims 0..255 (and, group 0, the rope) of local row rl into TMEM:
+      // lane quarters q and q^2 both hold rows 32(q%2)..; group g copies
+      // chunks 2g, 2g+1. The previous piece's S MMAs read Q until its last tile.
+      if (k > 0) {
+        const int jl = jt - 1;
+        if (!(ok = warp_wait_cta(bar(L::B_S_FULL + (jl & 1)), (jl >> 1) & 1, abort_flag, a.status))) break;
+      }
+      if (!(ok = warp_wait_cta(bar(L::B_Q_MAIN), k & 1, abort_flag, a.status))) break;
+#pragma unroll 1
+      for (int c2 = 0; c2 < (grp == 0 ? 3 : 2); ++c2) {
+        const bool rope = c2 == 2;
+        const int cc = 2 * grp + c2;
+        const uint8_t* chunk = smem + (rope ? L::kQRopeStage : L::kQStage + cc * 8192) + rl * 128;
+        uint32_t w[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 v = *reinterpret_cast<const uint4*>(chunk + ((u ^ (rl & 7)) * 16));
+          w[4 * u] = v.x;
+          w[4 * u + 1] = v.y;
+          w[4 * u + 2] = v.z;
+          w[4 * u + 3] = v.w;
+        }
+        if (r >= M) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w[i] = 0;
+        }
+        tmem_st32(tmem + tl + (rope ? kQRopeCol : kQCol + 32u * cc), w);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) arrive_lead(L::B_Q_TMEM);
+
+      float m_grp = -INFINITY, l_grp = 0.f;  // this group's reference and partial sum (this half row)
+      const int j_first = (jt & 1) == grp ? 0 : 1;
+      int pg_next = j_first < c.n_pt ? piece_entry16(c, j_first) : 0;
+      for (int j = j_first; ok && j < c.n_pt; j += 2) {
+        const int jg = jt + j;   // running tile index
+        const int buf = jg & 1;  // == grp
+        const int ph = (jg >> 1) & 1;
+        const int pg_cur = pg_next;
+        if (j + 2 < c.n_pt) pg_next = piece_entry16(c, j + 2);
+        if (!(ok = warp_wait_cta(bar(L::B_S_FULL + buf), ph, abort_flag, a.status))) break;
+        tc_fence_after();
+        uint32_t sv[32];
+        tmem_ld32(tmem + tl + kSCol + 32u * buf, sv);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_lead_relaxed(L::B_S_EMPTY + buf);  // the slice was read (wait::ld above)
+
+        bool page_ok = true;
+        if (pg_cur < 0 || (int64_t)pg_cur >= a.num_pages) {
+          page_ok = false;
+          if (lane == 0 && (q & 1) == 0) atomicOr(a.status, MLA_DEV_BAD_PAGE);
+        }
+        const int kb = c.key0 + kTile16 * j + kHalfKeys * hf;
+        // raw scores; masked keys become -inf (sl2 > 0, so max commutes with the scale)
+        if (!(page_ok && kb + 31 <= limit)) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (!(page_ok && kb + i <= limit)) sv[i] = __float_as_uint(-INFINITY);
+        }
+        float mt;
+        {
+          float m2[2];
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const uint32_t* x = sv + 16 * h2;
+            float v = max3f(__uint_as_float(x[0]), __uint_as_float(x[1]), __uint_as_float(x[2]));
+#pragma unroll
+            for (int e = 3; e < 15; e += 2) v = max3f(v, __uint_as_float(x[e]), __uint_as_float(x[e + 1]));
+            m2[h2] = fmaxf(v, __uint_as_float(x[15]));
+          }
+          mt = fmaxf(m2[0], m2[1]) * sl2;
+        }
+        // the other half of the row lives in the warp of quarter q^2
+        xm[((grp * 2 + ph) * 2 + hf) * 64 + rl] = mt;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_X + grp));
+        if (!(ok = warp_wait_cta(bar(L::B_X + grp), ph, abort_flag, a.status))) break;
+        mt = fmaxf(mt, xm[((grp * 2 + ph) * 2 + (hf ^ 1)) * 64 + rl]);
+        // reference maximum after the previous tile (from the other group),
+        // lazily updated; a new piece starts afresh but takes the hand-off
+        float m_prev = -INFINITY;
+        if (jg > 0) {
+          if (!(ok = warp_wait_cta(bar(L::B_M_READY + (buf ^ 1)), ((jg - 1) >> 1) & 1, abort_flag, a.status)))
+            break;
+          if (j > 0) m_prev = mref[(buf ^ 1) * 64 + rl];
+        }
+        const float m_j = (mt > m_prev + kTau) ? mt : m_prev;
+        mref[buf * 64 + rl] = m_j;  // both halves write the same value
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_M_READY + buf));
+        const float alpha = (m_j == m_prev) ? 1.f : ex2_approx(m_prev - m_j);  // O rescale for tile j
+        const float m_use = (m_j == -INFINITY) ? 0.f : m_j - kSigma;
+
+        // P buffer is free once the P.V two tiles back has finished
+        if (jg >= 2 && !(ok = warp_wait_cta(bar(L::B_P_EMPTY + buf), ph ^ 1, abort_flag, a.status))) break;
+
+        // P = 2^(s * sl2 - m_use) in the inputs' 16-bit type, 8 keys (one
+        // 16-byte chunk) at a time; this half's 32 keys are bytes
+        // [64hf, 64hf + 64) of the 128-byte P row.
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), nmx2 = f2_pack(-m_use, -m_use);
+        uint64_t se2[2] = {0ull, 0ull};
+        uint8_t* prow = smem + L::kPOff + buf * L::kPBuf + rl * 128;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int e = 8 * u + 2 * i;
+            float a0, a1;
+            f2_unpack(fma_f32x2(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nmx2), a0, a1);
+            const float p0 = ex2_approx(a0);
+            const float p1 = ex2_approx(a1);
+            se2[i & 1] = add_f32x2(se2[i & 1], f2_pack(p0, p1));
+            if (kBf16) {
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+              pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+            } else {
+              __half2 h2 = __floats2half2_rn(p0, p1);
+              pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+          }
+          const int phys = (4 * hf + u) ^ (rl & 7);
+          *reinterpret_cast<uint4*>(prow + phys * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+        float s0, s1, s2, s3;
+        f2_unpack(se2[0], s0, s1);
+        f2_unpack(se2[1], s2, s3);
+        const float sum = (s0 + s1) + (s2 + s3);
+        l_grp = (m_grp == m_j) ? l_grp + sum : fmaf(l_grp, ex2_approx(m_grp - m_j), sum);
+        m_grp = m_j;
+
+        // rescale this thread's 256 O columns if the reference maximum moved
+        // (not on a piece's first tile: O is reset by its first P.V)
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          if (!(ok = warp_wait_cta(bar(L::B_O_DONE), (jg - 1) & 1, abort_flag, a.status))) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int cc = 0; cc < 8; cc += 2) {
+            uint32_t o0[32], o1[32];
+            tmem_ld32(tmem + tl + kOCol + 32u * cc, o0);
+            tmem_ld32(tmem + tl + kOCol + 32u * (cc + 1), o1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              o0[i] = __float_as_uint(__uint_as_float(o0[i]) * alpha);
+              o1[i] = __float_as_uint(__uint_as_float(o1[i]) * alpha);
+            }
+            tmem_st32(tmem + tl + kOCol + 32u * cc, o0);
+            tmem_st32(tmem + tl + kOCol + 32u * (cc + 1), o1);
+          }
+          tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_lead(L::B_P_FULL + buf);
+      }
+      // ---------------------------------------------------------- epilogue of the piece
+      // Row sum over both groups and both key halves, relative to the final
+      // reference maximum.
+      ok = __all_sync(0xffffffffu, ok);
+      fin[((0 * 2 + grp) * 2 + hf) * 64 + rl] = l_grp;
+      fin[((1 * 2 + grp) * 2 + hf) * 64 + rl] = m_grp;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::B_FIN));
+      if (ok) ok = warp_wait_cta(bar(L::B_FIN), k & 1, abort_flag, a.status);
+      float le = 0.f, m_fin = -INFINITY;
+      if (ok) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m_fin = fmaxf(m_fin, fin[(4 + i) * 64 + rl]);
+        if (m_fin != -INFINITY) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float mi = fin[(4 + i) * 64 + rl];
+            if (mi != -INFINITY) le += fin[i * 64 + rl] * ex2_approx(mi - m_fin);
+          }
+        }
+      }
+      if (ok) ok = warp_wait_cta(bar(L::B_O_FINAL), k & 1, abort_flag, a.status);
+      if (!ok) break;
+      tc_fence_after();
+      const float inv = (le > 0.f) ? a.v_scale / le : 0.f;
+      const int64_t slot = slot_of(k);
+      if (r < M && grp == 0 && hf == 0) {
+        const float lse_val = (le > 0.f) ? (m_fin - kSigma + log2f(le)) * kLn2 : -INFINITY;
+        if (c.whole) {
+          if (a.lse) a.lse[c.row0 + r] = lse_val;
+        } else {
+          a.lse_part[slot * M + r] = lse_val;
+        }
+      }
+      if (!(c.whole && last_piece)) {
+        // Straight from registers. Partial slots use the layout
+        // [slot][16-byte column chunk][row]: the 32 consecutive rows of a warp
+        // then store 512 contiguous bytes per instruction. A whole unit that
+        // is not the pair's last piece is stored as BF16 rows.
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tmem + tl + kOCol + 128u * grp + 32u * cc, o);
+          tmem_wait_ld();
+          if (r >= M) continue;
+          const int col = 256 * grp + 128 * hf + 32 * cc;
+          if (c.whole) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + (c.row0 + r) * MLA_D_V + col);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              uint32_t pk[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float f0 = inv > 0.f ? __uint_as_float(o[8 * u + 2 * e]) * inv : 0.f;
+                const float f1 = inv > 0.f ? __uint_as_float(o[8 * u + 2 * e + 1]) * inv : 0.f;
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(f0, f1);
+                pk[e] = *reinterpret_cast<uint32_t*>(&h2);
+              }
+              dst[u] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          } else {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int64_t c4 = col / 4 + u;  // 16-byte column chunk
+              float4 f;
+              f.x = inv > 0.f ? __uint_as_float(o[4 * u + 0]) * inv : 0.f;
+              f.y = inv > 0.f ? __uint_as_float(o[4 * u + 1]) * inv : 0.f;
+              f.z = inv > 0.f ? __uint_as_float(o[4 * u + 2]) * inv : 0.f;
+              f.w = inv > 0.f ? __uint_as_float(o[4 * u + 3]) * inv : 0.f;
+              *reinterpret_cast<float4*>(a.o_part + ((slot * (MLA_D_V / 4) + c4) * M + r) * 4) = f;
+            }
+          }
+        }
+        if (!c.whole) {
+          // this warp's share of the unit's partial O and LSE is stored: one
+          // of the kPieceArrivals arrivals the combine waits for per piece
+          __syncwarp();
+          if (lane == 0) {
+            __threadfence();
+            atomicAdd(a.unit_done + pcs[k].u, 1);
+          }
+        }
+        if (!last_piece) {
+          // O may be reset by the next piece's first P.V
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) arrive_lead(L::B_O_FREE);
+        }
+      } else {
+        // A whole unit as the pair's last piece: the K and V rings are idle,
+        // so the output tile is staged there and written back by whole rows:
+        // a warp then stores 512 contiguous bytes per instruction instead of
+        // 32 rows' scattered pieces. Staging row r keeps its 16-byte chunk c at
+        // position c ^ (r & 7), so that neither the per-row writes nor the
+        // per-row reads conflict on shared-memory banks.
+        float* stage = reinterpret_cast<float*>(smem + L::kKOff);  // [64 rows][512] fp32
+        float* rowinv = mref;                                        // free once the loop is done
+        if (grp == 0 && hf == 0) rowinv[rl] = inv;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tmem + tl + kOCol + 128u * grp + 32u * cc, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int ch = 64 * grp + 32 * hf + 8 * cc + i;  // 16-byte chunk of the 2 KB row
+            *reinterpret_cast<uint4*>(stage + rl * MLA_D_V + ((ch ^ (rl & 7)) * 4)) =
+                make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_EPI));
+        if (!(ok = warp_wait_cta(bar(L::B_EPI), 0, abort_flag, a.status))) break;
+        // softmax warp w writes local rows 8w .. 8w+7
+        const int w8 = warp - kSoftmaxWarp0;
+#pragma unroll 1
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 8 * w8 + i;
+          if (64 * (int)rank + rr >= M) break;  // rows past the unit belong to no output
+          const float inv2 = rowinv[rr];
+          const int rr_u = 64 * (int)rank + rr;  // row within the unit
+          const float* srow = stage + rr * MLA_D_V;
+          {
+            // BF16: a lane writes 8 consecutive values (16 bytes) per step
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+              const int c0 = 2 * lane + 64 * kk;
+              const float4 x0 = *reinterpret_cast<const float4*>(srow + ((c0 ^ (rr & 7)) * 4));
+              const float4 x1 = *reinterpret_cast<const float4*>(srow + (((c0 + 1) ^ (rr & 7)) * 4));
+              const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+              uint32_t pk[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(inv2 > 0.f ? v[2 * e] * inv2 : 0.f,
+                                                          inv2 > 0.f ? v[2 * e + 1] * inv2 : 0.f);
+                pk[e] = *reinterpret_cast<uint32_t*>(&h2);
+              }
+              *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + (c.row0 + rr_u) * MLA_D_V + 4 * c0) =
+                  make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          }
+        }
+      }
+      jt += c.n_pt;
+    }
+    tc_fence_before();
+  }
+
+  // ---------------------------------------------------------------- teardown
+  // MMA completions are multicast to both CTAs, and only some of them are
+  // consumed: before the pair may leave, each CTA waits for the last phase of
+  // every barrier the leader's commits arrive on, so that no arrival lands in
+  // shared memory after the CTA has exited. It runs once every role is done
+  // (the epilogue saw the last O_FINAL, so every commit has been triggered
+  // and each barrier is at most its last arrival short of its final phase).
+  // Bounded; skipped after an abort, when the phases may never complete.
+  __syncthreads();
+  if (warp == 2 && lane == 0 && !*abort_flag && n_all > 0) {
+    for (int j = n_all - 1; j >= 0 && j >= n_all - NK; --j) drain_phase(bar(L::B_K_EMPTY + j % NK), (j / NK) & 1);
+    for (int j = n_all - 1; j >= 0 && j >= n_all - NV; --j) drain_phase(bar(L::B_V_EMPTY + j % NV), (j / NV) & 1);
+    for (int j = n_all - 1; j >= 0 && j >= n_all - NQ; --j) drain_phase(bar(L::B_QK_DONE + j % NQ), (j / NQ) & 1);
+    for (int j = n_all - 1; j >= 0 && j >= n_all - 2; --j) {
+      drain_phase(bar(L::B_P_EMPTY + (j & 1)), (j >> 1) & 1);
+      drain_phase(bar(L::B_S_FULL + (j & 1)), (j >> 1) & 1);
+    }
+    drain_phase(bar(L::B_O_DONE), (n_all - 1) & 1);
+    drain_phase(bar(L::B_O_FINAL), (npc - 1) & 1);
+  }
+  __syncthreads();
+  tc_fence_before();
+  cluster_sync();  // the peer no longer touches this CTA's shared or tensor memory
+  if (warp == 1) {
+    tc_fence_after();
+    if (*abort_flag) spin_ns(1000000ull);  // let any MMA still in flight finish
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    tc16_pair_kernel(const __grid_constant__ Pair16Params prm) {
+  // the combine grid may take the SMs of pairs that finish early: it waits
+  // for each unit's pieces itself
+  launch_dependents();
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // The layout has no alignment slack: a base off 1024 bytes (never seen)
+  // stops both CTAs of every pair before any shared memory is used.
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(prm.a.status, MLA_DEV_TIMEOUT);
+    return;
+  }
+  uint8_t* smem = smem_raw;
+  Piece* pcs = reinterpret_cast<Piece*>(smem);
+  SchedInfo* info = reinterpret_cast<SchedInfo*>(smem + kMaxPieces * sizeof(Piece));
+  if (threadIdx.x < 32) build_schedule16(prm.a, blockIdx.x >> 1, cluster_ctarank(), pcs, info);
+  __syncthreads();
+  const int npc = info->npc;
+  if (npc == 0) return;  // no work for this pair (the same in both CTAs)
+  if (npc > kMaxPieces) {  // cannot happen within the planner's unit limit
+    if (threadIdx.x == 0) atomicOr(prm.a.status, MLA_DEV_TIMEOUT);
+    return;
+  }
+  if (prm.a.plan.dtype == MLA_BF16)
+    pair_cta16<true>(prm, smem, pcs, npc);
+  else
+    pair_cta16<false>(prm, smem, pcs, npc);
+}
+
+}  // namespace
+
+cudaError_t launch_tc16_pair_partial(const DecodeArgs& a, cudaStream_t stream) {
+  const mla_plan& p = a.plan;
+  if (p.batch == 0 || p.split_kv < 1) return cudaSuccess;
+  Pair16Params prm;
+  prm.a = a;
+  const uint64_t q_rows = (uint64_t)p.batch * p.q_len * p.num_heads;
+  const uint64_t kv_rows = (uint64_t)a.num_pages * kTileKeys;
+  const uint32_t box_q = p.rows_per_unit < 64 ? (uint32_t)p.rows_per_unit : 64u;
+  const uint8_t* kv = static_cast<const uint8_t*>(a.kv_cache);
+  if (!encode_rows_576(&prm.tm_q, a.q, 2, q_rows, 64, box_q, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_rows_576(&prm.tm_kv, a.kv_cache, 2, kv_rows, 64, kHalfKeys, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_rows_576_chunks(&prm.tm_k8, a.kv_cache, 2, kv_rows, 8, 128, kHalfKeys, 8) ||
+      !encode_rows_576_chunks(&prm.tm_v[0], kv, 2, kv_rows, 6, 128, kTile16, 2) ||
+      !encode_rows_576_chunks(&prm.tm_v[1], kv + 256, 2, kv_rows, 6, 128, kTile16, 2))
+    return cudaErrorInvalidValue;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(tc16_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Layout16::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  tc16_pair_kernel<<<(unsigned)(2 * p.split_kv), kThreads, Layout16::kSmemBytes, stream>>>(prm);
+  return cudaGetLastError();
+}
+
+}  // namespace mla

@@ -124,6 +124,8 @@ __device__ __forceinline__ void store_out_chunk(const DecodeArgs& a, int64_t rg,
 
 // 2-D tensor map over a row-major [rows, 576] array of 1- or 2-byte elements
 // (q or the cache viewed as [num_pages * 64, 576]); box = box_x x box_y.
+bool encode_rows_576_chunks(CUtensorMap* m, const void* base, int esize, uint64_t rows, uint32_t nchunks,
+                            uint64_t chunk_stride, uint32_t box_rows, uint32_t box_chunks);
 bool encode_rows_576(CUtensorMap* m, const void* base, int esize, uint64_t rows, uint32_t box_x, uint32_t box_y,
                      CUtensorMapSwizzle sw);
 

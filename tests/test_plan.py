@@ -35,7 +35,8 @@ def test_fold_examples_from_the_article():
                                                   (16, 4, 32, 81920), (32, 4, 64, 65536),
                                                   (128, 2, 128, 81920), (3, 1, 8, 1), (2, 2, 2, 0)])
 def test_split_covers_all_keys(batch, q_len, heads, n):
-    p = mla.mla_decode_plan(batch, q_len, heads, n, "bf16")
+    # the fixed-split rule (the SIMT kernel and plans past the balanced unit limit use it)
+    p = mla.mla_decode_plan_custom(batch, q_len, heads, n, "bf16", kernel="simt")
     tiles = math.ceil(n / 64)
     assert p.keys_per_split % 64 == 0 and p.keys_per_split >= 64
     assert p.split_kv * p.keys_per_split >= n
@@ -76,8 +77,12 @@ def test_balanced_plan_uses_every_sm_and_caps_units():
     # more units than the per-pair piece list can hold: fixed splits, solo kernel
     big = mla.mla_decode_plan(4096, 1, 16, 1024, "fp8")
     assert big.schedule == 0 and big.kernel == 3
-    # 16-bit inputs keep fixed splits
-    assert mla.mla_decode_plan(16, 4, 32, 81920, "bf16").schedule == 0
+    # 16-bit inputs take the balanced schedule too (16-bit CTA-pair kernel),
+    # and past the unit limit fixed splits on the exchange kernel
+    assert mla.mla_decode_plan(16, 4, 32, 81920, "bf16").schedule == 1
+    assert mla.mla_decode_plan(128, 2, 128, 81920, "bf16").schedule == 1
+    big16 = mla.mla_decode_plan(4096, 1, 16, 1024, "fp16")
+    assert big16.schedule == 0 and big16.kernel == 1
 
 
 def _balanced_schedule(tiles, P, min_tiles=2):
@@ -149,10 +154,13 @@ def test_plan_is_deterministic_and_forced_values_apply():
     a = mla.mla_decode_plan(4, 4, 32, 8192, "bf16").as_dict()
     b = mla.mla_decode_plan(4, 4, 32, 8192, "bf16").as_dict()
     assert a == b
-    p = mla.mla_decode_plan_custom(4, 4, 32, 8192, "bf16", split_kv=3)
+    p = mla.mla_decode_plan_custom(4, 4, 32, 8192, "bf16", split_kv=3, kernel="simt")
     assert p.split_kv == 3 and p.keys_per_split == 64 * math.ceil(128 / 3)
-    p = mla.mla_decode_plan_custom(4, 4, 32, 8192, "bf16", split_kv=10 ** 6)
+    p = mla.mla_decode_plan_custom(4, 4, 32, 8192, "bf16", split_kv=10 ** 6, kernel="simt")
     assert p.split_kv == 128 and p.keys_per_split == 64
+    # the balanced schedule takes a forced split as the number of CTA pairs
+    p = mla.mla_decode_plan_custom(4, 4, 32, 8192, "bf16", split_kv=3)
+    assert (p.schedule, p.split_kv, p.num_ctas) == (1, 3, 6)
     p = mla.mla_decode_plan_custom(4, 4, 32, 8192, "bf16", fold=2)
     assert (p.fold, p.q_groups, p.rows_per_unit) == (2, 2, 64)
     p = mla.mla_decode_plan_custom(4, 4, 32, 8192, "bf16", kernel="simt")

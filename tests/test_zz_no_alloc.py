@@ -69,7 +69,8 @@ def test_no_alloc_refuses_plans_larger_than_its_scratch():
     dev = torch.device("cuda", 0)
     fn = _entry()
     g = make_inputs_custom(1, 1, 16, "bf16", [100], seed=23).to(dev)
-    plan = mla.mla_decode_plan(128, 2, 128, 81920, "bf16")
+    # fixed splits over 32768 rows: partials far above the scratch
+    plan = mla.mla_decode_plan_custom(128, 2, 128, 81920, "bf16", kernel="simt")
     assert plan.workspace_bytes > _lib.MLA_NO_ALLOC_SCRATCH_BYTES
     out = torch.empty(1, 1, 16, 512, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(1, 1, 16, device=dev)
