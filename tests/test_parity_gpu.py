@@ -229,24 +229,38 @@ def test_host_pointers_are_refused_before_launch():
     assert dec.status() == 0 and torch.isfinite(o.float()).all()
 
 
+@pytest.mark.parametrize("dtype", ["fp8", "bf16", "fp16"])
 @pytest.mark.parametrize("pairs", [1, 2, 3, 7, 74])
-def test_balanced_schedule_forced_pairs(pairs):
-    """FP8 CTA-pair kernel with its balanced schedule forced onto few pairs: units are cut
+def test_balanced_schedule_forced_pairs(pairs, dtype):
+    """CTA-pair kernels with the balanced schedule forced onto few pairs: units are cut
     between pairs and pairs cover several units (empty, one-key, ragged, single-term entries)."""
-    inp = make_inputs_custom(6, 2, 32, "fp8", [0, 1, 130, 700, 4097, 20000], seed=31, pool=1.5)
+    inp = make_inputs_custom(6, 2, 32, dtype, [0, 1, 130, 700, 4097, 20000], seed=31, pool=1.5)
     out, lse, status, dec = run(inp, "tcgen05", split_kv=pairs)
     assert dec.plan.schedule == 1 and status == 0
     ref_o, ref_l = oracle_rows(inp)
-    compare(out, lse, ref_o, ref_l, "fp8", what=f"{pairs} pairs")
+    compare(out, lse, ref_o, ref_l, dtype, what=f"{pairs} pairs")
 
 
-def test_balanced_schedule_many_ragged_units():
+@pytest.mark.parametrize("dtype", ["fp8", "bf16", "fp16"])
+def test_balanced_schedule_many_ragged_units(dtype):
     g = torch.Generator().manual_seed(33)
     sl = torch.randint(0, 3000, (40,), generator=g).tolist()
     sl[3] = 0
     sl[7] = 1
-    inp = make_inputs_custom(40, 1, 16, "fp8", sl, seed=34, pool=1.3)
+    inp = make_inputs_custom(40, 1, 16, dtype, sl, seed=34, pool=1.3)
     out, lse, status, dec = run(inp, "tcgen05")
     assert dec.plan.schedule == 1 and status == 0
     ref_o, ref_l = oracle_rows(inp)
-    compare(out, lse, ref_o, ref_l, "fp8", what="40 ragged units")
+    compare(out, lse, ref_o, ref_l, dtype, what="40 ragged units")
+
+
+def test_past_the_balanced_unit_limit_16bit_takes_fixed_splits():
+    """More units than the balanced schedule's piece list: 16-bit inputs go to the
+    fixed-split exchange kernel, still exact against the oracle (sampled rows)."""
+    g = torch.Generator().manual_seed(35)
+    sl = torch.randint(1, 200, (2100,), generator=g).tolist()
+    inp = make_inputs_custom(2100, 1, 16, "bf16", sl, seed=36, pool=1.2)
+    out, lse, status, dec = run(inp, "tcgen05")
+    assert dec.plan.schedule == 0 and dec.plan.kernel == 1 and status == 0
+    ref_o, ref_l = oracle_rows(inp)
+    compare(out, lse, ref_o, ref_l, "bf16", what="2100 units, fixed splits")
