@@ -43,6 +43,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="fp8_long_b16")
+    ap.add_argument("--op", default="decode", choices=["decode", "kv_pack"],
+                    help="decode (the headline) or the fused K/V pack + FP8 quantise kernel")
     ap.add_argument("--kernel", default="auto", choices=["auto", "tcgen05", "simt", "tcgen05_solo"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -431,8 +433,68 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_kv_pack(args):
+    """Fused K/V pack + FP8 quantise on a prefill-sized write: 16 x 81,920 BF16 tokens into an
+    FP8 cache of twice the pages (permuted slots). One JSON line; HBM roofline."""
+    import torch
+    import mla_paged_decode_04_b200 as mla
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    n = 16 * 81920
+    num_pages = 2 * n // 64
+    g = torch.Generator(device=dev).manual_seed(4242)
+    latent = torch.randn(n, 512, generator=g, device=dev).to(torch.bfloat16)
+    rope = torch.randn(n, 64, generator=g, device=dev).to(torch.bfloat16)
+    slots = torch.randperm(num_pages * 64, generator=g, device=dev)[:n].to(torch.int64)
+    cache = torch.empty(num_pages, 64, 576, dtype=torch.float8_e4m3fn, device=dev)
+    scale = float(mla.kv_amax(latent, rope).item()) / 448.0
+    alg = n * (512 + 64) * 2 + n * 576 + n * 8  # inputs, FP8 rows, slots
+    for _ in range(max(args.warmup, 3)):
+        mla.kv_pack(latent, rope, slots, cache, kv_scale=scale)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    t_end = time.perf_counter() + args.clock_window_s
+    while time.perf_counter() < t_end:
+        for _ in range(20):
+            mla.kv_pack(latent, rope, slots, cache, kv_scale=scale)
+        torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for k in range(args.steps):
+        evs[k][0].record()
+        mla.kv_pack(latent, rope, slots, cache, kv_scale=scale)
+        evs[k][1].record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    mean_s = statistics.mean(ms) / 1e3
+    peak, peak_kind = measured_peak()
+    achieved = alg / mean_s / 1e9
+    if rank != 0:
+        return
+    line = {
+        "metric": "fused K/V pack + FP8 quantise GB/s (inputs + FP8 rows + slots per call)",
+        "value": round(achieved, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(statistics.mean(ms), 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16->fp8_e4m3", "data": "synthetic (seeded, generated on device)",
+        "config": {"workload": "kv_pack_bf16_fp8", "tokens": n, "num_pages": num_pages,
+                   "l2": "inputs larger than L2 (1.5 GB read, 755 MB written per call), no flush"},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_source": peak_kind, "traffic": None,
+                     "kernel": "kv_pack_fp8_kernel", "alg_bytes_per_launch": int(alg)},
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
+    if args.op == "kv_pack":
+        run_kv_pack(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -251,6 +251,52 @@ const char* mla_version(void);
  */
 int mla_last_cuda_error(const char** name);
 
+/*
+ * mla_kv_pack: write new tokens into the paged latent cache, fused with the
+ * FP8 quantisation (tokenspeed-mla package card, "What it is and what it
+ * does": one kernel packs K/V and quantises to FP8 in place of separate cat
+ * and cast operations; TokenSpeed MLA article, section 一, kernel table
+ * entry mla_kv_pack_quantize_fp8, and section 六 for the 576-wide row).
+ *
+ *   latent        [n_tokens, 512] in_dtype, contiguous, 16-byte aligned: the
+ *                 latent (compressed K/V) part of each new token
+ *   rope          [n_tokens, 64] in_dtype, contiguous, 16-byte aligned: the
+ *                 rope key part
+ *   slot_mapping  [n_tokens] int64, device: cache row page * 64 + offset of
+ *                 token i; negative = skip the token; a slot at or past
+ *                 num_pages * 64 skips the token and sets MLA_DEV_BAD_PAGE
+ *                 in *device_status (when given)
+ *   kv_cache      [num_pages, 64, 576] cache_dtype: row s becomes
+ *                 [latent_i || rope_i]; other rows are untouched
+ *   in_dtype      MLA_BF16 or MLA_FP16
+ *   cache_dtype   MLA_FP8_E4M3: each element is E4M3FN(x / kv_scale), the
+ *                 quotient formed in fp32 (IEEE division, round to nearest)
+ *                 and rounded to nearest even, saturating to +-448, NaN
+ *                 kept; or in_dtype: the row is copied
+ *   kv_scale      finite, > 0 (the per-tensor dequantisation scale decode
+ *                 takes; ignored for a 16-bit cache)
+ *   device_status optional int32 device word (e.g. a decode workspace's
+ *                 status word); may be NULL
+ *
+ * All pointers are device-addressable from the current device and owned by
+ * the caller; nothing is allocated or synchronised. Argument errors return
+ * MLA_ERR_INVALID_ARG / MLA_ERR_UNSUPPORTED_SHAPE (page_size != 64) before
+ * any launch. n_tokens = 0 is a no-op.
+ */
+int mla_kv_pack(const void* latent, const void* rope, int64_t n_tokens, const int64_t* slot_mapping,
+                void* kv_cache, int64_t num_pages, int page_size, int in_dtype, int cache_dtype,
+                float kv_scale, int32_t* device_status, void* stream);
+
+/*
+ * mla_kv_amax: largest |x| over the non-NaN elements of latent [n_tokens,
+ * 512] and rope [n_tokens, 64] (in_dtype MLA_BF16 or MLA_FP16), written as
+ * one fp32 to the device pointer `amax` (zeroed first, on `stream`): the
+ * per-tensor scale amax / 448 of the FP8 cache recipe follows from it.
+ * Same pointer rules and errors as mla_kv_pack.
+ */
+int mla_kv_amax(const void* latent, const void* rope, int64_t n_tokens, int in_dtype, float* amax,
+                void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -23,10 +23,12 @@ KERNELS = {"auto": MLA_KERNEL_AUTO, "tcgen05": MLA_KERNEL_TCGEN05, "simt": MLA_K
            "tcgen05_solo": MLA_KERNEL_TCGEN05_SOLO}
 
 MLA_DEV_BAD_PAGE, MLA_DEV_SEQ_TOO_LONG, MLA_DEV_TIMEOUT = 0x1, 0x2, 0x4
+(MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED_SHAPE, MLA_ERR_WORKSPACE_TOO_SMALL, MLA_ERR_ARCH, MLA_ERR_CUDA,
+ MLA_ERR_PLAN_MISMATCH) = (-1, -2, -3, -4, -5, -6)
 
 EXPORTED = ["mla_decode_plan", "mla_decode_plan_custom", "mla_decode", "mla_decode_partial",
             "mla_decode_combine", "mla_decode_status", "mla_status_string", "mla_version",
-            "mla_decode_no_alloc", "mla_last_cuda_error"]
+            "mla_decode_no_alloc", "mla_last_cuda_error", "mla_kv_pack", "mla_kv_amax"]
 MLA_NO_ALLOC_SCRATCH_BYTES = 48 << 20
 
 
@@ -81,6 +83,10 @@ def _load():
     lib.mla_version.restype = ctypes.c_char_p
     lib.mla_last_cuda_error.argtypes = [ctypes.POINTER(ctypes.c_char_p)]
     lib.mla_last_cuda_error.restype = i32
+    lib.mla_kv_pack.argtypes = [vp, vp, i64, vp, vp, i64, i32, i32, i32, f32, vp, vp]
+    lib.mla_kv_pack.restype = i32
+    lib.mla_kv_amax.argtypes = [vp, vp, i64, i32, vp, vp]
+    lib.mla_kv_amax.restype = i32
     return lib
 
 
@@ -213,6 +219,45 @@ def mla_decode_status(workspace, clear=True, stream=None) -> int:
     if rc != 0:
         raise MlaError(rc, "mla_decode_status")
     return int(v.value)
+
+
+def _stream_of(t, stream):
+    if stream is None:
+        return torch.cuda.current_stream(t.device).cuda_stream
+    return stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else stream
+
+
+def kv_pack(latent, rope, slot_mapping, kv_cache, kv_scale=1.0, device_status=None, stream=None) -> None:
+    """Write tokens into the paged cache, fused with FP8 quantisation when kv_cache is FP8.
+
+    latent [n, 512] and rope [n, 64] (bf16 or fp16), slot_mapping [n] int64
+    (page * 64 + offset; negative = skip), kv_cache [num_pages, 64, 576] of
+    the inputs' dtype or float8_e4m3fn; see include/mla_decode.h.
+    """
+    _check_tensors(latent, rope=rope, slot_mapping=slot_mapping, kv_cache=kv_cache, device_status=device_status)
+    if slot_mapping.dtype != torch.int64:
+        raise ValueError("slot_mapping must be int64")
+    if latent.dtype != rope.dtype:
+        raise ValueError("latent and rope must have one dtype")
+    in_dtype = _dtype_code(latent.dtype)
+    cache_dtype = _dtype_code(kv_cache.dtype)
+    rc = _lib.mla_kv_pack(_ptr(latent), _ptr(rope), int(latent.shape[0]), _ptr(slot_mapping), _ptr(kv_cache),
+                          int(kv_cache.shape[0]), int(kv_cache.shape[1]), in_dtype, cache_dtype, float(kv_scale),
+                          _ptr(device_status), ctypes.c_void_p(_stream_of(latent, stream)))
+    if rc != 0:
+        raise MlaError(rc, "mla_kv_pack")
+
+
+def kv_amax(latent, rope, out=None, stream=None) -> torch.Tensor:
+    """Device fp32 [1]: the largest |x| over latent and rope (NaN ignored)."""
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=latent.device)
+    _check_tensors(latent, rope=rope, out=out)
+    rc = _lib.mla_kv_amax(_ptr(latent), _ptr(rope), int(latent.shape[0]), _dtype_code(latent.dtype), _ptr(out),
+                          ctypes.c_void_p(_stream_of(latent, stream)))
+    if rc != 0:
+        raise MlaError(rc, "mla_kv_amax")
+    return out
 
 
 def alloc_workspace(plan: MlaPlan, device) -> torch.Tensor:

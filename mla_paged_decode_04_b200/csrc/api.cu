@@ -268,3 +268,45 @@ extern "C" int mla_last_cuda_error(const char** name) {
   if (name) *name = cudaGetErrorName(g_last_cuda_error);
   return (int)g_last_cuda_error;
 }
+
+extern "C" int mla_kv_pack(const void* latent, const void* rope, int64_t n_tokens, const int64_t* slot_mapping,
+                           void* kv_cache, int64_t num_pages, int page_size, int in_dtype, int cache_dtype,
+                           float kv_scale, int32_t* device_status, void* stream) {
+  if (n_tokens < 0 || num_pages < 0) return MLA_ERR_INVALID_ARG;
+  if (page_size != MLA_PAGE_SIZE) return MLA_ERR_UNSUPPORTED_SHAPE;
+  if (in_dtype != MLA_BF16 && in_dtype != MLA_FP16) return MLA_ERR_INVALID_ARG;
+  if (cache_dtype != MLA_FP8_E4M3 && cache_dtype != in_dtype) return MLA_ERR_INVALID_ARG;
+  if (cache_dtype == MLA_FP8_E4M3 && (!std::isfinite(kv_scale) || kv_scale <= 0.f)) return MLA_ERR_INVALID_ARG;
+  if (n_tokens == 0) return MLA_OK;
+  if (!latent || !rope || !slot_mapping || !kv_cache) return MLA_ERR_INVALID_ARG;
+  if (!aligned(latent, 16) || !aligned(rope, 16) || !aligned(kv_cache, 16) || !aligned(slot_mapping, 8) ||
+      (device_status && !aligned(device_status, 4)))
+    return MLA_ERR_INVALID_ARG;
+  if (num_pages > (int64_t(1) << 40) / MLA_PAGE_SIZE) return MLA_ERR_UNSUPPORTED_SHAPE;
+  int dev = 0;
+  if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_failure(e);
+  if (!device_addressable(latent, dev) || !device_addressable(rope, dev) || !device_addressable(slot_mapping, dev) ||
+      !device_addressable(kv_cache, dev) || (device_status && !device_addressable(device_status, dev)))
+    return MLA_ERR_INVALID_ARG;
+  if (int rc = check_device_arch(); rc != MLA_OK) return rc;
+  const cudaError_t e = launch_kv_pack(latent, rope, n_tokens, slot_mapping, kv_cache, num_pages * MLA_PAGE_SIZE,
+                                       in_dtype, cache_dtype, kv_scale, device_status,
+                                       reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MLA_OK : cuda_failure(e);
+}
+
+extern "C" int mla_kv_amax(const void* latent, const void* rope, int64_t n_tokens, int in_dtype, float* amax,
+                           void* stream) {
+  if (n_tokens < 0 || !amax) return MLA_ERR_INVALID_ARG;
+  if (in_dtype != MLA_BF16 && in_dtype != MLA_FP16) return MLA_ERR_INVALID_ARG;
+  if (n_tokens > 0 && (!latent || !rope)) return MLA_ERR_INVALID_ARG;
+  if (!aligned(amax, 4) || (n_tokens > 0 && (!aligned(latent, 16) || !aligned(rope, 2)))) return MLA_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_failure(e);
+  if (!device_addressable(amax, dev) ||
+      (n_tokens > 0 && (!device_addressable(latent, dev) || !device_addressable(rope, dev))))
+    return MLA_ERR_INVALID_ARG;
+  if (int rc = check_device_arch(); rc != MLA_OK) return rc;
+  const cudaError_t e = launch_kv_amax(latent, rope, n_tokens, in_dtype, amax, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MLA_OK : cuda_failure(e);
+}

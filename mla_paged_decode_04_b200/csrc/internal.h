@@ -70,6 +70,11 @@ cudaError_t launch_tc_fp8_partial(const DecodeArgs& a, cudaStream_t stream);  //
 cudaError_t launch_tc_fp8_pair_partial(const DecodeArgs& a, cudaStream_t stream);  // FP8, CTA-pair MMAs
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_tc16_pair_partial(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_kv_pack(const void* latent, const void* rope, int64_t n, const int64_t* slots, void* cache,
+                           int64_t num_slots, int in_dtype, int cache_dtype, float kv_scale, int32_t* status,
+                           cudaStream_t stream);
+cudaError_t launch_kv_amax(const void* latent, const void* rope, int64_t n, int in_dtype, float* amax,
+                           cudaStream_t stream);
 cudaError_t launch_combine_balanced(const DecodeArgs& a, cudaStream_t stream);
 
 }  // namespace mla

@@ -72,6 +72,12 @@ def _load():
         lib.oracle_decode_buffer.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = i32
+        lib.oracle_encode_e4m3_buffer.argtypes = [vp, ctypes.c_size_t, vp]
+        lib.oracle_encode_e4m3_buffer.restype = None
+        lib.oracle_kv_pack.argtypes = [i32, i32, vp, vp, i64, vp, ctypes.c_float, vp, i64]
+        lib.oracle_kv_pack.restype = i32
+        lib.oracle_kv_amax.argtypes = [i32, vp, vp, i64]
+        lib.oracle_kv_amax.restype = f64
         _lib = lib
     return _lib
 
@@ -155,3 +161,41 @@ def lse_merge(o_parts, lse_parts):
     _load().oracle_lse_merge(n, Dv, o.ctypes.data, l.ctypes.data, out.ctypes.data,
                              lse.ctypes.data)
     return out, float(lse[0])
+
+
+def encode_e4m3(values) -> np.ndarray:
+    """OCP E4M3FN codes of fp32 values: round to nearest even, saturating to +-448, NaN -> 0x7f."""
+    v = np.ascontiguousarray(np.asarray(values, dtype=np.float32).reshape(-1))
+    out = np.empty(v.size, dtype=np.uint8)
+    _load().oracle_encode_e4m3_buffer(v.ctypes.data, v.size, out.ctypes.data)
+    return out
+
+
+def kv_pack(latent, rope, slot_mapping, cache_shape, *, in_dtype, cache_dtype, kv_scale=1.0, cache=None):
+    """Oracle fused K/V pack (+ FP8 quantise): cache row slot_mapping[i] = [latent_i || rope_i].
+
+    latent [n, 512] and rope [n, 64] are 16-bit tensors (raw bytes are read);
+    the cache (raw element bytes, shape [num_pages, page_size, 576]) starts as
+    `cache` (or zeros) and is returned as a uint8 array of those bytes.
+    """
+    lat = _raw_bytes(latent)
+    rp = _raw_bytes(rope)
+    n = lat.size // (512 * 2)
+    slots = np.ascontiguousarray(np.asarray(slot_mapping, dtype=np.int64).reshape(-1))
+    assert slots.size == n and rp.size == n * 64 * 2
+    esize = 1 if cache_dtype == "fp8" else 2
+    num_slots = int(np.prod(cache_shape[:-1]))
+    buf = np.zeros(num_slots * 576 * esize, dtype=np.uint8) if cache is None else _raw_bytes(cache).copy()
+    rc = _load().oracle_kv_pack(DTYPE_CODES[in_dtype], DTYPE_CODES[cache_dtype], lat.ctypes.data, rp.ctypes.data,
+                                n, slots.ctypes.data, float(kv_scale), buf.ctypes.data, num_slots)
+    if rc != 0:
+        raise ValueError(f"oracle kv_pack failed ({rc})")
+    return buf
+
+
+def kv_amax(latent, rope, *, in_dtype) -> float:
+    """Largest |x| over the non-NaN elements of the latent and rope tensors."""
+    lat = _raw_bytes(latent)
+    rp = _raw_bytes(rope)
+    n = lat.size // (512 * 2)
+    return float(_load().oracle_kv_amax(DTYPE_CODES[in_dtype], lat.ctypes.data, rp.ctypes.data, n))

@@ -304,3 +304,85 @@ int oracle_num_threads(void) {
   return 1;
 #endif
 }
+
+/*
+ * Fused K/V pack + FP8 quantise (the cache-writing step before decode).
+ * Sources: tokenspeed-mla package card, "What it is and what it does" (a
+ * fused kernel packs K/V and quantises to FP8 in place of separate cat and
+ * cast operations); TokenSpeed MLA article (最快MLA内核背后的秘密), section
+ * 一 (its kernel table: mla_kv_pack_quantize_fp8) and section 六 (the
+ * 576-wide cache row). Token i's cache row is [latent_i (512) || rope_i (64)]
+ * written at row slot_mapping[i] of [num_pages * page_size, 576] (slots < 0
+ * are skipped). With an FP8 cache each element is E4M3FN(x / kv_scale); the
+ * pages fix no precision for the quotient, so it is formed in fp32, the
+ * precision the CUDA kernel takes the same decision in, and rounded to
+ * E4M3 from that exact fp32 value.
+ */
+
+/* OCP OFP8 E4M3FN encoding: round to nearest, ties to even; finite values
+ * past the largest code and infinities saturate to +-448 (S.1111.110); NaN
+ * encodes as S.1111.111. */
+uint8_t oracle_encode_e4m3(float v) {
+  const int sign = signbit(v) ? 0x80 : 0;
+  double a = fabs((double)v);
+  if (isnan(v)) return (uint8_t)(sign | 0x7f);
+  if (a > 448.0) return (uint8_t)(sign | 0x7e);
+  if (a < ldexp(1.0, -6)) {
+    /* subnormal range: steps of 2^-9; rounding up to 8 steps gives the
+     * smallest normal code 0x08 */
+    const double q = nearbyint(a * 512.0);
+    return (uint8_t)(sign | (int)q);
+  }
+  int e = ilogb(a);                         /* 2^e <= a < 2^(e+1), e in [-6, 8] */
+  double q = nearbyint(ldexp(a, 3 - e));    /* 8 + 3 mantissa bits, in [8, 16] */
+  if (q == 16.0) {
+    q = 8.0;
+    e += 1;
+  }
+  if (e > 8) return (uint8_t)(sign | 0x7e); /* rounded past 448 */
+  return (uint8_t)(sign | ((e + 7) << 3) | ((int)q - 8));
+}
+
+void oracle_encode_e4m3_buffer(const float* src, size_t n, uint8_t* dst) {
+  for (size_t i = 0; i < n; ++i) dst[i] = oracle_encode_e4m3(src[i]);
+}
+
+/* Pack n tokens into the cache. in_dtype: ORACLE_BF16 or ORACLE_FP16;
+ * cache_dtype: ORACLE_FP8_E4M3 (quantise with kv_scale) or in_dtype (copy of
+ * the 16-bit bits). Returns ORACLE_EPAGE if a slot is >= num_slots. */
+int oracle_kv_pack(int in_dtype, int cache_dtype, const void* latent, const void* rope, int64_t n,
+                   const int64_t* slots, float kv_scale, void* cache, int64_t num_slots) {
+  if (in_dtype != ORACLE_BF16 && in_dtype != ORACLE_FP16) return ORACLE_EINVAL;
+  if (cache_dtype != ORACLE_FP8_E4M3 && cache_dtype != in_dtype) return ORACLE_EINVAL;
+  for (int64_t i = 0; i < n; ++i) {
+    const int64_t s = slots[i];
+    if (s < 0) continue;
+    if (s >= num_slots) return ORACLE_EPAGE;
+    for (int d = 0; d < 576; ++d) {
+      const uint16_t bits = d < 512 ? ((const uint16_t*)latent)[i * 512 + d]
+                                    : ((const uint16_t*)rope)[i * 64 + (d - 512)];
+      if (cache_dtype == ORACLE_FP8_E4M3) {
+        const float x = (float)decode_elem(in_dtype, &bits, 0); /* exact: 16-bit values fit fp32 */
+        const float quot = x / kv_scale;                         /* fp32 division, rounded to nearest */
+        ((uint8_t*)cache)[s * 576 + d] = oracle_encode_e4m3(quot);
+      } else {
+        ((uint16_t*)cache)[s * 576 + d] = bits;
+      }
+    }
+  }
+  return ORACLE_OK;
+}
+
+/* Largest |x| over the non-NaN elements of n tokens' latent and rope parts. */
+double oracle_kv_amax(int in_dtype, const void* latent, const void* rope, int64_t n) {
+  double m = 0.0;
+  for (int64_t i = 0; i < n * 512; ++i) {
+    const double x = fabs(decode_elem(in_dtype, latent, (size_t)i));
+    if (!isnan(x) && x > m) m = x;
+  }
+  for (int64_t i = 0; i < n * 64; ++i) {
+    const double x = fabs(decode_elem(in_dtype, rope, (size_t)i));
+    if (!isnan(x) && x > m) m = x;
+  }
+  return m;
+}
