@@ -66,6 +66,10 @@ def _load():
             i32, i32, i32, i32, i32, i32, vp, vp, i64, i32, vp, i32, vp,
             f64, f64, f64, i64, vp, i64, i64, i32, vp, vp]
         lib.oracle_mla_decode_range.restype = i32
+        lib.oracle_mla_decode_range_w.argtypes = [
+            i32, i32, i32, i32, i32, i32, vp, vp, i64, i32, vp, i32, vp,
+            f64, f64, f64, i64, vp, i64, i64, i64, i32, vp, vp]
+        lib.oracle_mla_decode_range_w.restype = i32
         lib.oracle_lse_merge.argtypes = [i32, i32, vp, vp, vp, vp]
         lib.oracle_lse_merge.restype = None
         lib.oracle_decode_buffer.argtypes = [i32, vp, ctypes.c_size_t, vp]
@@ -110,7 +114,7 @@ def decode_values(dtype: str, raw) -> np.ndarray:
 
 
 def mla_decode(q, kv_cache, block_tables, seq_lens, softmax_scale, *, dtype,
-               q_scale=1.0, kv_scale=1.0, rows=None, key_range=None,
+               q_scale=1.0, kv_scale=1.0, rows=None, key_range=None, window=0,
                mutation="none"):
     """Oracle MLA decode.
 
@@ -118,6 +122,7 @@ def mla_decode(q, kv_cache, block_tables, seq_lens, softmax_scale, *, dtype,
     fp16 / float8_e4m3fn, or their raw uint8/uint16 views); block_tables [B, P]
     int32, seq_lens [B] int32. rows: optional flat row indices (b*q_len+t)*H+h.
     key_range: optional (lo, hi) restriction of the keys (hi=-1: unbounded).
+    window: sliding window W > 0 (a row with n visible keys sees keys >= n - W); 0 = none.
     Returns (out [n_rows, Dv=512] float64, lse [n_rows] float64), natural log.
     """
     lib = _load()
@@ -141,10 +146,10 @@ def mla_decode(q, kv_cache, block_tables, seq_lens, softmax_scale, *, dtype,
     out = np.zeros((n_rows, Dv), dtype=np.float64)
     lse = np.zeros((n_rows,), dtype=np.float64)
     lo, hi = (0, -1) if key_range is None else key_range
-    rc = lib.oracle_mla_decode_range(
+    rc = lib.oracle_mla_decode_range_w(
         DTYPE_CODES[dtype], B, T, H, D, Dv, qb.ctypes.data, cb.ctypes.data, num_pages,
         page_size, bt.ctypes.data, bt.shape[1], sl.ctypes.data, float(softmax_scale),
-        float(q_scale), float(kv_scale), n_rows, rows_ptr, int(lo), int(hi),
+        float(q_scale), float(kv_scale), n_rows, rows_ptr, int(lo), int(hi), int(window),
         MUTATIONS[mutation], out.ctypes.data, lse.ctypes.data)
     if rc != 0:
         raise ValueError(f"oracle_mla_decode_range failed with code {rc}")

@@ -18,8 +18,11 @@ def _as_floats(t, scale=1.0):
 
 
 def mla_decode_brute(q, kv_cache, block_tables, seq_lens, softmax_scale,
-                     q_scale=1.0, kv_scale=1.0):
-    """q [B,T,H,D], kv_cache [P,page,D] torch tensors; returns (out rows, lse list)."""
+                     q_scale=1.0, kv_scale=1.0, window=0):
+    """q [B,T,H,D], kv_cache [P,page,D] torch tensors; returns (out rows, lse list).
+
+    window W > 0: a row with n visible keys attends to its last W keys only.
+    """
     B, T, H, D = (int(x) for x in q.shape)
     _, page, _ = (int(x) for x in kv_cache.shape)
     Dv = 512
@@ -37,14 +40,15 @@ def mla_decode_brute(q, kv_cache, block_tables, seq_lens, softmax_scale,
                     outs.append([0.0] * Dv)
                     lses.append(-math.inf)
                     continue
+                first = max(0, n - window) if window > 0 else 0
                 keys = []
-                for j in range(n):
+                for j in range(first, n):
                     p = bt[b][j // page]
                     keys.append(cache_rows[p * page + j % page])
                 s = [softmax_scale * math.fsum(qv[d] * k[d] for d in range(D)) for k in keys]
                 m = max(s)
                 lse = m + math.log(math.fsum(math.exp(x - m) for x in s))
                 w = [math.exp(x - lse) for x in s]
-                outs.append([math.fsum(w[j] * keys[j][d] for j in range(n)) for d in range(Dv)])
+                outs.append([math.fsum(w[j] * keys[j][d] for j in range(len(keys))) for d in range(Dv)])
                 lses.append(lse)
     return outs, lses

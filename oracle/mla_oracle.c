@@ -116,18 +116,21 @@ void oracle_decode_buffer(int dtype, const void* src, size_t n, double* dst) {
 /*
  * oracle_mla_decode_range: attention of the selected rows restricted to the
  * visible keys j with key_lo <= j < key_hi (key_hi < 0 means no upper bound).
- * With key_lo = 0, key_hi = -1 this is the full decode. Rows are flat indices
+ * With key_lo = 0, key_hi = -1 this is the full decode. A window W > 0
+ * (sliding-window decode, a decode option the TokenSpeed MLA article lists
+ * among its tests in section 六) further limits a row with n visible keys to
+ * its last W: keys j >= n - W. Rows are flat indices
  * r = (b * q_len + t) * H + h; rows == NULL means all B*q_len*H rows in order.
  * out is [n_rows, Dv] and lse [n_rows]; a row whose range holds no visible
  * key gets out = 0, lse = -inf.
  */
-int oracle_mla_decode_range(int dtype, int B, int q_len, int H, int D, int Dv,
-                            const void* q, const void* cache, int64_t num_pages,
-                            int page_size, const int32_t* block_tables,
-                            int max_pages_per_seq, const int32_t* seq_lens,
-                            double softmax_scale, double q_scale, double kv_scale,
-                            int64_t n_rows, const int64_t* rows, int64_t key_lo,
-                            int64_t key_hi, int mutation, double* out, double* lse) {
+int oracle_mla_decode_range_w(int dtype, int B, int q_len, int H, int D, int Dv,
+                              const void* q, const void* cache, int64_t num_pages,
+                              int page_size, const int32_t* block_tables,
+                              int max_pages_per_seq, const int32_t* seq_lens,
+                              double softmax_scale, double q_scale, double kv_scale,
+                              int64_t n_rows, const int64_t* rows, int64_t key_lo,
+                              int64_t key_hi, int64_t window, int mutation, double* out, double* lse) {
   if (B < 0 || q_len <= 0 || H <= 0 || D <= 0 || Dv <= 0 || Dv > D || page_size <= 0)
     return ORACLE_EINVAL;
   if (dtype != ORACLE_BF16 && dtype != ORACLE_FP16 && dtype != ORACLE_FP8_E4M3)
@@ -217,6 +220,7 @@ int oracle_mla_decode_range(int dtype, int B, int q_len, int H, int D, int Dv,
         int64_t n = (mutation == MUT_NO_CAUSAL) ? nb : nb - q_len + t + 1;
         if (n > nb) n = nb;
         int64_t lo = key_lo > 0 ? key_lo : 0;
+        if (window > 0 && n - window > lo) lo = n - window;
         int64_t hi = (key_hi >= 0 && key_hi < n) ? key_hi : n;
         if (hi <= lo) {
           lse[oi] = -INFINITY;
@@ -255,6 +259,18 @@ int oracle_mla_decode_range(int dtype, int B, int q_len, int H, int D, int Dv,
     if (alloc_fail) status = ORACLE_ENOMEM;
   }
   return status;
+}
+
+int oracle_mla_decode_range(int dtype, int B, int q_len, int H, int D, int Dv,
+                            const void* q, const void* cache, int64_t num_pages,
+                            int page_size, const int32_t* block_tables,
+                            int max_pages_per_seq, const int32_t* seq_lens,
+                            double softmax_scale, double q_scale, double kv_scale,
+                            int64_t n_rows, const int64_t* rows, int64_t key_lo,
+                            int64_t key_hi, int mutation, double* out, double* lse) {
+  return oracle_mla_decode_range_w(dtype, B, q_len, H, D, Dv, q, cache, num_pages, page_size, block_tables,
+                                   max_pages_per_seq, seq_lens, softmax_scale, q_scale, kv_scale, n_rows, rows,
+                                   key_lo, key_hi, 0, mutation, out, lse);
 }
 
 /* Full decode: all visible keys. */

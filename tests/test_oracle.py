@@ -311,3 +311,56 @@ def test_planted_mistakes_are_caught(mutation):
         if not (err <= tol):
             caught.append(name)
     assert caught, f"mutation {mutation} passed every pin"
+
+
+# ---------------------------------------------------------------- sliding window
+# A window W > 0 limits a row with n visible keys to keys n - W .. n - 1
+# (a decode option the TokenSpeed MLA article lists among its tests, section 六).
+
+@pytest.mark.parametrize("window", [1, 3, 64, 70])
+def test_window_matches_the_brute_force_decode(window):
+    worst = 0.0
+    cases = [(2, 3, 2, "bf16", [130, 5]), (1, 4, 3, "fp16", [199]), (2, 2, 4, "fp8", [70, 2])]
+    for i, (B, T, H, dt, sl) in enumerate(cases):
+        inp = make_inputs_custom(B, T, H, dt, sl, seed=40 + i, pool=1.5)
+        out, lse = _decode(inp, window=window)
+        bo, bl = mla_decode_brute(inp.q, inp.kv_cache, inp.block_tables, inp.seq_lens,
+                                  inp.softmax_scale, inp.q_scale, inp.kv_scale, window=window)
+        bo, bl = np.array(bo), np.array(bl)
+        fin = np.isfinite(bl)
+        assert np.array_equal(fin, np.isfinite(lse))
+        worst = max(worst, np.abs(out - bo).max(), np.abs(lse[fin] - bl[fin]).max(initial=0))
+    assert worst <= 1e-12
+
+
+def test_window_covering_the_sequence_changes_nothing():
+    inp = make_inputs_custom(2, 4, 3, "bf16", [300, 9], seed=44, pool=1.5)
+    o0, l0 = _decode(inp)
+    o1, l1 = _decode(inp, window=300)
+    assert np.array_equal(o0, o1) and np.array_equal(l0, l1)
+
+
+def test_window_of_one_returns_the_newest_visible_key():
+    inp = make_inputs_custom(2, 3, 2, "fp16", [90, 40], seed=45, pool=1.5)
+    out, lse = _decode(inp, window=1)
+    T, H = 3, 2
+    for b in range(2):
+        K = _keys(inp, b)
+        for t in range(T):
+            n = int(inp.seq_lens[b]) - T + t + 1
+            for h in range(H):
+                r = (b * T + t) * H + h
+                qv = _values(inp.q, inp.q_scale)[b, t, h]
+                assert np.array_equal(out[r], K[n - 1, :512])  # weight 1 on one key
+                assert abs(lse[r] - inp.softmax_scale * float(qv @ K[n - 1])) <= 1e-12
+
+
+def test_window_ignores_keys_before_its_start():
+    inp = make_inputs_custom(1, 2, 2, "bf16", [200], seed=46, pool=1.5)
+    o0, l0 = _decode(inp, window=50)
+    # overwrite every cache row the rows' windows do not reach (keys 0 .. 148)
+    bt = inp.block_tables[0]
+    for j in range(149):
+        inp.kv_cache[int(bt[j // 64]), j % 64] = 7.0
+    o1, l1 = _decode(inp, window=50)
+    assert np.array_equal(o0, o1) and np.array_equal(l0, l1)
