@@ -122,6 +122,8 @@ typedef struct {
   uint64_t workspace_bytes, partial_offset, lse_offset;
   uint32_t magic;    /* set by the planner; checked by mla_decode */
   uint32_t schedule; /* MLA_SCHEDULE_* below */
+  int32_t window;    /* sliding window in keys (0 = none); set with mla_decode_plan_window */
+  int32_t reserved;
 } mla_plan;
 
 /*
@@ -144,6 +146,18 @@ int mla_decode_plan(int batch, int q_len, int num_heads, int max_seq_len, int dt
  */
 int mla_decode_plan_custom(int batch, int q_len, int num_heads, int max_seq_len, int dtype,
                            int split_kv, int fold, int kernel, mla_plan* plan);
+
+/*
+ * mla_decode_plan_window: restrict every query row to its last `window`
+ * visible keys (sliding-window decode, a decode option the TokenSpeed MLA
+ * article lists among its tests, section 六): a row with n visible keys
+ * attends to keys [max(0, n - window), n). window = 0 restores full
+ * attention. Supported by the CTA-pair kernels (balanced schedule) and the
+ * SIMT kernel; other plans return MLA_ERR_UNSUPPORTED_SHAPE. The plan's
+ * workspace size does not change. Errors: MLA_ERR_INVALID_ARG (null plan,
+ * window < 0), MLA_ERR_PLAN_MISMATCH (plan not from mla_decode_plan*).
+ */
+int mla_decode_plan_window(mla_plan* plan, int window);
 
 /*
  * mla_decode: one decode step (tokenspeed-mla package card, "Quickstart":

@@ -6,5 +6,5 @@ seeded synthetic workloads.
 """
 from ._lib import (MLA_DEV_BAD_PAGE, MLA_DEV_SEQ_TOO_LONG, MLA_DEV_TIMEOUT, MlaDecoder,  # noqa: F401
                    MlaError, MlaPlan, alloc_workspace, last_cuda_error, mla_decode, mla_decode_plan,
-                   mla_decode_combine, mla_decode_partial, mla_decode_plan_custom,
+                   mla_decode_combine, mla_decode_partial, mla_decode_plan_custom, mla_decode_plan_window,
                    mla_decode_status, mla_version, status_string, kv_pack, kv_amax)

@@ -28,7 +28,8 @@ MLA_DEV_BAD_PAGE, MLA_DEV_SEQ_TOO_LONG, MLA_DEV_TIMEOUT = 0x1, 0x2, 0x4
 
 EXPORTED = ["mla_decode_plan", "mla_decode_plan_custom", "mla_decode", "mla_decode_partial",
             "mla_decode_combine", "mla_decode_status", "mla_status_string", "mla_version",
-            "mla_decode_no_alloc", "mla_last_cuda_error", "mla_kv_pack", "mla_kv_amax"]
+            "mla_decode_no_alloc", "mla_last_cuda_error", "mla_kv_pack", "mla_kv_amax",
+            "mla_decode_plan_window"]
 MLA_NO_ALLOC_SCRATCH_BYTES = 48 << 20
 
 
@@ -41,6 +42,7 @@ class MlaPlan(ctypes.Structure):
         ("kernel", ctypes.c_int32), ("num_ctas", ctypes.c_int32),
         ("workspace_bytes", ctypes.c_uint64), ("partial_offset", ctypes.c_uint64),
         ("lse_offset", ctypes.c_uint64), ("magic", ctypes.c_uint32), ("schedule", ctypes.c_uint32),
+        ("window", ctypes.c_int32), ("reserved", ctypes.c_int32),
     ]
 
     def as_dict(self):
@@ -83,6 +85,8 @@ def _load():
     lib.mla_version.restype = ctypes.c_char_p
     lib.mla_last_cuda_error.argtypes = [ctypes.POINTER(ctypes.c_char_p)]
     lib.mla_last_cuda_error.restype = i32
+    lib.mla_decode_plan_window.argtypes = [P, i32]
+    lib.mla_decode_plan_window.restype = i32
     lib.mla_kv_pack.argtypes = [vp, vp, i64, vp, vp, i64, i32, i32, i32, f32, vp, vp]
     lib.mla_kv_pack.restype = i32
     lib.mla_kv_amax.argtypes = [vp, vp, i64, i32, vp, vp]
@@ -141,6 +145,14 @@ def mla_decode_plan_custom(batch, q_len, num_heads, max_seq_len, dtype, split_kv
     if rc != 0:
         raise MlaError(rc, "mla_decode_plan_custom")
     return p
+
+
+def mla_decode_plan_window(plan: MlaPlan, window: int) -> MlaPlan:
+    """Set the plan's sliding window in place (0 = full attention) and return it."""
+    rc = _lib.mla_decode_plan_window(ctypes.byref(plan), int(window))
+    if rc != 0:
+        raise MlaError(rc, "mla_decode_plan_window")
+    return plan
 
 
 def _ptr(t):
@@ -269,9 +281,11 @@ class MlaDecoder:
     """Plan + workspace for one decode shape; call it once per decode step."""
 
     def __init__(self, batch, q_len, num_heads, max_seq_len, dtype, device, split_kv=0, fold=0,
-                 kernel="auto"):
+                 kernel="auto", window=0):
         self.plan = mla_decode_plan_custom(batch, q_len, num_heads, max_seq_len, dtype,
                                            split_kv, fold, kernel)
+        if window:
+            mla_decode_plan_window(self.plan, window)
         self.device = torch.device(device)
         self.workspace = alloc_workspace(self.plan, self.device)
         self.batch, self.q_len, self.num_heads = batch, q_len, num_heads

@@ -77,8 +77,12 @@ int check_plan(const mla_plan* p) {
     return MLA_ERR_PLAN_MISMATCH;
   if (p->kernel == MLA_KERNEL_TCGEN05_SOLO && p->dtype != MLA_FP8_E4M3) return MLA_ERR_PLAN_MISMATCH;
   if (p->schedule != MLA_SCHEDULE_SPLITS && p->schedule != MLA_SCHEDULE_BALANCED) return MLA_ERR_PLAN_MISMATCH;
+  if (p->window < 0) return MLA_ERR_PLAN_MISMATCH;
+  if (p->window > 0 && !(p->kernel == MLA_KERNEL_SIMT ||
+                         (p->kernel == MLA_KERNEL_TCGEN05 && p->schedule == MLA_SCHEDULE_BALANCED)))
+    return MLA_ERR_PLAN_MISMATCH;
   if (p->schedule == MLA_SCHEDULE_BALANCED) {
-    // FP8 CTA-pair kernel only; slots [2P, M, 512] fp32 + [2P, M] + unit table
+    // CTA-pair kernels only; slots [2P, M, 512] fp32 + [2P, M] + unit table
     if (p->kernel != MLA_KERNEL_TCGEN05 || p->split_kv > kNumSMs / 2)
       return MLA_ERR_PLAN_MISMATCH;
     const int64_t units = (int64_t)p->batch * p->q_groups;
@@ -309,4 +313,16 @@ extern "C" int mla_kv_amax(const void* latent, const void* rope, int64_t n_token
   if (int rc = check_device_arch(); rc != MLA_OK) return rc;
   const cudaError_t e = launch_kv_amax(latent, rope, n_tokens, in_dtype, amax, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MLA_OK : cuda_failure(e);
+}
+
+extern "C" int mla_decode_plan_window(mla_plan* plan, int window) {
+  if (!plan || window < 0) return MLA_ERR_INVALID_ARG;
+  mla_plan p = *plan;
+  p.window = 0;
+  if (int rc = check_plan(&p); rc != MLA_OK) return rc;
+  if (window > 0 && !(p.kernel == MLA_KERNEL_SIMT ||
+                      (p.kernel == MLA_KERNEL_TCGEN05 && p.schedule == MLA_SCHEDULE_BALANCED)))
+    return MLA_ERR_UNSUPPORTED_SHAPE;
+  plan->window = window;
+  return MLA_OK;
 }

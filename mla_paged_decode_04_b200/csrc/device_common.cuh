@@ -41,6 +41,18 @@ __device__ __forceinline__ int effective_seq_len(const DecodeArgs& a, int b, boo
   return n;
 }
 
+// Sliding window (plan.window = W > 0): query token t of an entry with n
+// keys sees keys [n - q_len + t + 1 - W, n - q_len + t]. First key of token t,
+// and of the first token of query group g (the lowest key its unit needs).
+__device__ __forceinline__ int window_row_lo(const mla_plan& p, int t, int n) {
+  if (p.window <= 0) return 0;
+  const int lo = n - p.q_len + t + 1 - p.window;
+  return lo > 0 ? lo : 0;
+}
+__device__ __forceinline__ int window_unit_lo(const mla_plan& p, int g, int n) {
+  return window_row_lo(p, g * p.fold, n);
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(256) simt_partial_kernel(const DecodeArgs a) {
     float o[MLA_D_V / 32];
 #pragma unroll
     for (int i = 0; i < MLA_D_V / 32; ++i) o[i] = 0.f;
-    for (int j = key0; j < jend; ++j) {
+    for (int j = max(key0, window_row_lo(p, t, n)); j < jend; ++j) {  // sliding window: the row's last keys
       const int page = table[j / kTileKeys];
       if (page < 0 || (int64_t)page >= a.num_pages) {
         if (lane == 0) atomicOr(a.status, MLA_DEV_BAD_PAGE);

@@ -125,10 +125,12 @@ struct Pair16Params {
   DecodeArgs a;
 };
 
-// Pair tiles of unit u (= b * G + g): one per 64-key page of entry b.
+// Pair tiles of unit u (= b * G + g): one per 64-key page of entry b, from
+// the page of the lowest key the group's rows see (its sliding window's start).
 __device__ __forceinline__ int unit_tiles16(const DecodeArgs& a, int u, bool flag) {
   const int n = effective_seq_len(a, u / a.plan.q_groups, flag);
-  return (n + kTile16 - 1) / kTile16;
+  const int tlo = window_unit_lo(a.plan, u % a.plan.q_groups, n) / kTile16;
+  return (n + kTile16 - 1) / kTile16 - tlo;
 }
 
 // One warp: the balanced schedule of this pair (the FP8 kernel's, with
@@ -219,10 +221,11 @@ __device__ __forceinline__ PieceCtx16 piece_ctx16(const DecodeArgs& a, const Pie
   c.b = pc.u / p.q_groups;
   c.g = pc.u % p.q_groups;
   c.n = effective_seq_len(a, c.b, false);
-  c.key0 = pc.t0 * kTile16;
-  c.key1 = min(c.n, pc.t1 * kTile16);
+  const int tlo = window_unit_lo(p, c.g, c.n) / kTile16;  // the unit's first page
+  c.key0 = (tlo + pc.t0) * kTile16;
+  c.key1 = min(c.n, (tlo + pc.t1) * kTile16);
   c.n_pt = pc.t1 - pc.t0;
-  c.page0 = pc.t0;  // block-table index of the piece's first page
+  c.page0 = tlo + pc.t0;  // block-table index of the piece's first page
   c.row0 = (int64_t)c.b * p.q_len * p.num_heads + (int64_t)c.g * p.rows_per_unit;
   c.table = a.block_tables + (int64_t)c.b * a.max_pages_per_seq;
   c.whole = pc.t0 == 0 && c.key1 >= c.n;
@@ -487,6 +490,7 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
       const PieceCtx16 c = piece_ctx16(a, pcs[k]);
       const bool last_piece = k == npc - 1;
       const int limit = min((r < M) ? c.n - T + c.g * p.fold + r / H : c.n - 1, c.key1 - 1);
+      const int lower = (r < M) ? window_row_lo(p, c.g * p.fold + r / H, c.n) : 0;  // sliding window
 
       // Q dims 0..255 (and, group 0, the rope) of local row rl into TMEM:
       // lane quarters q and q^2 both hold rows 32(q%2)..; group g copies
@@ -546,10 +550,10 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
         }
         const int kb = c.key0 + kTile16 * j + kHalfKeys * hf;
         // raw scores; masked keys become -inf (sl2 > 0, so max commutes with the scale)
-        if (!(page_ok && kb + 31 <= limit)) {
+        if (!(page_ok && kb >= lower && kb + 31 <= limit)) {
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (!(page_ok && kb + i <= limit)) sv[i] = __float_as_uint(-INFINITY);
+            if (!(page_ok && kb + i >= lower && kb + i <= limit)) sv[i] = __float_as_uint(-INFINITY);
         }
         float mt;
         {

@@ -163,10 +163,18 @@ struct PairParams {
   DecodeArgs a;
 };
 
-// Pair tiles of unit u (= b * G + g): every group of entry b sees its keys.
+// Most keys a row of an entry with n keys attends to (its window, if shorter):
+// the length the two-term P choice looks at.
+__device__ __forceinline__ int row_keys(const DecodeArgs& a, int n) {
+  return (a.plan.window > 0 && a.plan.window < n) ? a.plan.window : n;
+}
+
+// Pair tiles of unit u (= b * G + g): from the tile of the lowest key the
+// group's rows see (0, or its sliding window's start) to the entry's end.
 __device__ __forceinline__ int unit_tiles(const DecodeArgs& a, int u, bool flag) {
   const int n = effective_seq_len(a, u / a.plan.q_groups, flag);
-  return (n + kPairTileKeys - 1) / kPairTileKeys;
+  const int tlo = window_unit_lo(a.plan, u % a.plan.q_groups, n) / kPairTileKeys;
+  return (n + kPairTileKeys - 1) / kPairTileKeys - tlo;
 }
 
 // One warp: the balanced schedule of this pair. Every lane takes a run of
@@ -239,7 +247,7 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, Pie
           pcs[k].u = u;
           pcs[k].t0 = lo > start ? (int)(lo - start) : 0;
           pcs[k].t1 = hi - start < t ? (int)(hi - start) : t;
-          if (effective_seq_len(a, u / p.q_groups, false) < kTwoTermKeys) two = 1;
+          if (row_keys(a, effective_seq_len(a, u / p.q_groups, false)) < kTwoTermKeys) two = 1;
         }
         ++k;
       }
@@ -268,15 +276,16 @@ __device__ __forceinline__ PieceCtx piece_ctx(const DecodeArgs& a, const Piece& 
   c.b = pc.u / p.q_groups;
   c.g = pc.u % p.q_groups;
   c.n = effective_seq_len(a, c.b, false);
-  c.key0 = pc.t0 * kPairTileKeys;
-  c.key1 = min(c.n, pc.t1 * kPairTileKeys);
+  const int tlo = window_unit_lo(p, c.g, c.n) / kPairTileKeys;  // the unit's first pair tile
+  c.key0 = (tlo + pc.t0) * kPairTileKeys;
+  c.key1 = min(c.n, (tlo + pc.t1) * kPairTileKeys);
   c.n_pt = pc.t1 - pc.t0;
   c.n_tiles = (c.key1 - c.key0 + kTileKeys - 1) / kTileKeys;
   c.tile0 = c.key0 / kTileKeys;
   c.row0 = (int64_t)c.b * p.q_len * p.num_heads + (int64_t)c.g * p.rows_per_unit;
   c.table = a.block_tables + (int64_t)c.b * a.max_pages_per_seq;
   c.whole = pc.t0 == 0 && c.key1 >= c.n;
-  c.two = kTwo && c.n < kTwoTermKeys;
+  c.two = kTwo && row_keys(a, c.n) < kTwoTermKeys;
   return c;
 }
 
@@ -550,6 +559,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
       const PieceCtx c = piece_ctx(a, pcs[k], kTwo);
       const bool last_piece = k == npc - 1;
       const int limit = min((r < M) ? c.n - T + c.g * p.fold + r / H : c.n - 1, c.key1 - 1);
+      const int lower = (r < M) ? window_row_lo(p, c.g * p.fold + r / H, c.n) : 0;  // sliding window
 
       // Q latent dims of local row rl into TMEM (A operand of S = Q.K^T): lane
       // quarters q and q^2 both hold rows 32(q%2)..; group g copies chunks
@@ -620,10 +630,10 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
         }
         const int kb = c.key0 + kPairTileKeys * j + 64 * hf;
         // raw scores; masked keys become -inf (sl2 > 0, so max commutes with the scale)
-        if (!(page_ok && kb + 63 <= limit)) {
+        if (!(page_ok && kb >= lower && kb + 63 <= limit)) {
 #pragma unroll
           for (int i = 0; i < 64; ++i)
-            if (!(page_ok && kb + i <= limit)) sv[i] = __float_as_uint(-INFINITY);
+            if (!(page_ok && kb + i >= lower && kb + i <= limit)) sv[i] = __float_as_uint(-INFINITY);
         }
         float mt;
         {

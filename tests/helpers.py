@@ -19,8 +19,9 @@ ABS_TOL, REL_TOL, LSE_TOL = 1e-2, 2e-2, 1e-3
 REL_L2 = {"bf16": 1e-2, "fp16": 1e-2, "fp8": 3e-2}
 
 
-def oracle_rows(inp, rows=None):
-    """Oracle (out, lse) for flat rows (b*T+t)*H+h of `inp` (tensors on any device).
+def oracle_rows(inp, rows=None, window=0):
+    """Oracle (out, lse) for flat rows (b*T+t)*H+h of `inp` (tensors on any device),
+    with each row restricted to its last `window` visible keys when window > 0.
 
     Only the pages of the touched batch entries are copied to the host; the
     oracle sees exactly the bytes the GPU path reads.
@@ -46,7 +47,7 @@ def oracle_rows(inp, rows=None):
         local = rows[idx] - b * T * H
         o, l = oracle.mla_decode(inp.q[b:b + 1].cpu(), cache_b, bt_b, sl[b:b + 1],
                                  inp.softmax_scale, dtype=inp.dtype, q_scale=inp.q_scale,
-                                 kv_scale=inp.kv_scale, rows=local)
+                                 kv_scale=inp.kv_scale, rows=local, window=window)
         out[idx] = o
         lse[idx] = l
     return out, lse

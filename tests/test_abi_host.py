@@ -114,3 +114,15 @@ def test_last_cuda_error_starts_clean():
     t.start()
     t.join()
     assert res["v"] == (0, "cudaSuccess")
+
+
+def test_decode_rejects_a_window_the_plan_cannot_run():
+    """A window written into a plan by hand is checked like every other plan field."""
+    p = mla.mla_decode_plan(2, 4, 32, 256, "fp8")
+    bad = _lib.MlaPlan.from_buffer_copy(p)
+    bad.window = -4
+    assert _call(bad) == -6
+    solo = mla.mla_decode_plan_custom(2, 4, 32, 256, "fp8", kernel="tcgen05_solo")
+    bad = _lib.MlaPlan.from_buffer_copy(solo)
+    bad.window = 64
+    assert _call(bad) == -6

@@ -21,13 +21,13 @@ pytestmark = pytest.mark.gpu
 KERNELS = ["tcgen05", "simt", "tcgen05_solo"]
 
 
-def run(inp, kernel="auto", split_kv=0, fold=0, want_lse=True):
+def run(inp, kernel="auto", split_kv=0, fold=0, want_lse=True, window=0):
     if kernel == "tcgen05_solo" and inp.dtype != "fp8":
         pytest.skip("the solo variant is FP8 only")
     dev = torch.device("cuda", 0)
     g = inp.to(dev)
     dec = mla.MlaDecoder(g.batch, g.q_len, g.heads, max(g.max_seq_len, 0), g.dtype, dev,
-                         split_kv=split_kv, fold=fold, kernel=kernel)
+                         split_kv=split_kv, fold=fold, kernel=kernel, window=window)
     out, lse = dec(g.q, g.kv_cache, g.block_tables, g.seq_lens, g.softmax_scale,
                    g.q_scale, g.kv_scale, want_lse=want_lse)
     torch.cuda.synchronize()
@@ -264,3 +264,55 @@ def test_past_the_balanced_unit_limit_16bit_takes_fixed_splits():
     assert dec.plan.schedule == 0 and dec.plan.kernel == 1 and status == 0
     ref_o, ref_l = oracle_rows(inp)
     compare(out, lse, ref_o, ref_l, "bf16", what="2100 units, fixed splits")
+
+
+# ---------------------------------------------------------------- sliding window
+# A row with n visible keys attends to keys [max(0, n - W), n) (a decode option
+# the TokenSpeed MLA article lists among its tests, section 六). The CTA-pair
+# kernels skip the tiles below the unit's lowest window start and mask the
+# rest per row; the SIMT kernel starts each row's loop at its window start.
+
+WINDOW_LENS = [0, 1, 3, 130, 700, 4097]  # empty, single key, seq_len < q_len, ragged tails
+
+
+@pytest.mark.parametrize("dtype", ["fp8", "bf16", "fp16"])
+@pytest.mark.parametrize("kernel", ["tcgen05", "simt"])
+@pytest.mark.parametrize("window", [1, 2, 63, 64, 65, 200, 1000])
+def test_window_matches_the_oracle(window, kernel, dtype):
+    inp = make_inputs_custom(6, 4, 32, dtype, WINDOW_LENS, seed=41, pool=1.5)
+    out, lse, status, dec = run(inp, kernel, window=window)
+    assert dec.plan.window == window and status == 0
+    ref_o, ref_l = oracle_rows(inp, window=window)
+    compare(out, lse, ref_o, ref_l, dtype, what=f"{kernel} W={window}")
+
+
+@pytest.mark.parametrize("dtype", ["fp8", "bf16"])
+@pytest.mark.parametrize("pairs", [1, 3, 74])
+def test_window_with_units_cut_between_pairs(pairs, dtype):
+    """Few pairs, long entries: windowed units are still cut into pieces that the combine merges."""
+    inp = make_inputs_custom(3, 2, 64, dtype, [20000, 5000, 129], seed=42, pool=1.3)
+    out, lse, status, dec = run(inp, "tcgen05", split_kv=pairs, window=3000)
+    assert dec.plan.schedule == 1 and status == 0
+    ref_o, ref_l = oracle_rows(inp, window=3000)
+    compare(out, lse, ref_o, ref_l, dtype, what=f"W=3000, {pairs} pairs")
+
+
+@pytest.mark.parametrize("dtype", ["fp8", "bf16"])
+def test_window_past_every_length_is_bitwise_full_attention(dtype):
+    inp = make_inputs_custom(6, 4, 32, dtype, WINDOW_LENS, seed=43, pool=1.5)
+    o0, l0, s0, _ = run(inp, "tcgen05")
+    ow, lw, sw, _ = run(inp, "tcgen05", window=4097)
+    assert s0 == 0 and sw == 0
+    assert torch.equal(o0, ow) and torch.equal(l0, lw)
+
+
+@pytest.mark.parametrize("name", ["fp8_long_b16", "fold_fp16_h16"])
+def test_window_full_size_sampled_rows(name):
+    """Full-size workloads with an 8192-key window (for FP8 entries this also takes
+    the two-term P encoding, which the kernel picks for rows of fewer than 16384 keys)."""
+    inp = make_inputs(name, device=torch.device("cuda", 0))
+    out, lse, status, dec = run(inp, "auto", window=8192)
+    assert dec.plan.window == 8192 and status == 0
+    rows = sample_rows(inp.batch, inp.q_len, inp.heads, n=48, seed=45)
+    ref_o, ref_l = oracle_rows(inp, rows, window=8192)
+    compare(out, lse, ref_o, ref_l, inp.dtype, rows=rows, what=f"{name} W=8192")

@@ -183,3 +183,34 @@ def test_forced_fold_must_divide():
     assert e.value.code == -2
     with pytest.raises(mla.MlaError):
         mla.mla_decode_plan_custom(1, 4, 64, 10, "bf16", fold=4)  # 256 rows
+
+
+def test_window_is_set_only_on_plans_whose_kernels_support_it():
+    p = mla.mla_decode_plan(2, 4, 32, 4096, "fp8")
+    assert p.window == 0 and p.schedule == 1
+    ws = p.workspace_bytes
+    assert mla.mla_decode_plan_window(p, 300).window == 300
+    assert p.workspace_bytes == ws  # the window changes no buffer
+    assert mla.mla_decode_plan_window(p, 0).window == 0
+    p16 = mla.mla_decode_plan(2, 4, 32, 4096, "bf16")
+    assert mla.mla_decode_plan_window(p16, 64).window == 64
+    ps = mla.mla_decode_plan_custom(2, 4, 32, 4096, "fp16", kernel="simt")
+    assert mla.mla_decode_plan_window(ps, 1).window == 1
+    # fixed-split tensor-core plans (the FP8 solo kernel, the 16-bit exchange
+    # kernel past the balanced unit limit) do not take a window
+    solo = mla.mla_decode_plan_custom(2, 4, 32, 4096, "fp8", kernel="tcgen05_solo")
+    big16 = mla.mla_decode_plan_custom(2100, 1, 16, 256, "bf16")
+    assert big16.schedule == 0
+    for q in (solo, big16):
+        with pytest.raises(mla.MlaError) as e:
+            mla.mla_decode_plan_window(q, 128)
+        assert e.value.code == -2 and q.window == 0
+        assert mla.mla_decode_plan_window(q, 0).window == 0
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_decode_plan_window(p, -1)
+    assert e.value.code == -1
+    forged = mla.MlaPlan.from_buffer_copy(p)
+    forged.magic = 0
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_decode_plan_window(forged, 8)
+    assert e.value.code == -6
