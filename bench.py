@@ -44,7 +44,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="fp8_long_b16")
-    ap.add_argument("--op", default="decode", choices=["decode", "kv_pack"],
+    ap.add_argument("--op", default="decode", choices=["decode", "kv_pack", "prefill"],
                     help="decode (the headline) or the fused K/V pack + FP8 quantise kernel")
     ap.add_argument("--kernel", default="auto", choices=["auto", "tcgen05", "simt", "tcgen05_solo"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -530,10 +530,181 @@ def run_kv_pack(args):
     print(json.dumps(line), flush=True)
 
 
+def prefill_flops(cu, seq_lens, heads):
+    """Algorithmic flops of a ragged prefill step: 2 * (576 + 512) per (query row, visible key);
+    token t of an entry with qlen new tokens and n keys sees n - qlen + t + 1 keys."""
+    from mla_paged_decode_04_b200.inputs import D_QK, D_V
+    total = 0
+    for b in range(len(seq_lens)):
+        qlen, n = cu[b + 1] - cu[b], int(seq_lens[b])
+        # sum over t of max(0, n - qlen + t + 1)
+        for t in range(qlen):
+            total += max(0, n - qlen + t + 1)
+    return total * heads * 2 * (D_QK + D_V)
+
+
+def run_prefill(args):
+    """Ragged prefill over the paged cache (tokenspeed-mla package card: variable-length
+    sequences without padding): one mla_prefill call per step on a named workload. Compute-bound:
+    the roofline is the tensor peak of the input type, HBM beside it."""
+    import torch
+    import mla_paged_decode_04_b200 as mla
+    from mla_paged_decode_04_b200.inputs import PREFILL_WORKLOADS, make_prefill_workload
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    name = args.workload if args.workload in PREFILL_WORKLOADS else "prefill_fp8"
+    w = PREFILL_WORKLOADS[name]
+    inp = make_prefill_workload(name, device=dev)
+    g = inp.to(dev)
+    pre = mla.MlaPrefill(g.batch, g.max_q_len, g.heads, g.max_seq_len, g.dtype, dev)
+    out = torch.empty((g.total_q, g.heads, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((g.total_q, g.heads), dtype=torch.float32, device=dev)
+    cu = inp.cu_seqlens_q.tolist()
+    flops = prefill_flops(cu, inp.seq_lens.tolist(), g.heads)
+    esize = 1 if g.dtype == "fp8" else 2
+    kv_bytes = int(inp.seq_lens.sum()) * 576 * esize
+    alg_bytes = kv_bytes + g.q.numel() * esize + out.numel() * 2 + lse.numel() * 4
+    pool_bytes = g.kv_cache.numel() * esize
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # the cache pool fits in L2
+    call = (g.q, g.cu_seqlens_q, g.kv_cache, g.block_tables, g.seq_lens, g.softmax_scale)
+
+    def step():
+        mla.mla_prefill(pre.plan, *call, out, lse, pre.workspace, g.q_scale, g.kv_scale)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if pre.status() != 0:
+        raise RuntimeError("device status word set during warm-up")
+    sampler = ClockSampler(local)
+    sampler.start()
+    t_end = time.perf_counter() + args.clock_window_s
+    while time.perf_counter() < t_end:
+        flush.zero_()
+        step()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for k in range(args.steps):
+        flush.zero_()
+        evs[k][0].record()
+        step()
+        evs[k][1].record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    if pre.status() != 0:
+        raise RuntimeError("device status word set during the timed steps")
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    mean_s = total_ms / args.steps / 1e3
+    value = world * flops / mean_s / 1e12
+
+    # end to end through MlaPrefill: packed q, offsets and tables from pinned host memory,
+    # out/lse back, inside the timed region
+    hq = inp.q.cpu().pin_memory()
+    hcu, hbt, hsl = (inp.cu_seqlens_q.pin_memory(), inp.block_tables.pin_memory(), inp.seq_lens.pin_memory())
+    dq, dcu, dbt, dsl = (torch.empty_like(g.q), torch.empty_like(g.cu_seqlens_q), torch.empty_like(g.block_tables),
+                         torch.empty_like(g.seq_lens))
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = hq.numel() * esize + (hcu.numel() + hbt.numel() + hsl.numel()) * 4
+    d2h = hout.numel() * 2 + hlse.numel() * 4
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dcu.copy_(hcu, non_blocking=True)
+        dbt.copy_(hbt, non_blocking=True)
+        dsl.copy_(hsl, non_blocking=True)
+        pre(dq, dcu, g.kv_cache, dbt, dsl, g.softmax_scale, g.q_scale, g.kv_scale, out=out, lse=lse)
+        hout.copy_(out, non_blocking=True)
+        hlse.copy_(lse, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for k in range(args.steps):
+        flush.zero_()
+        ev2[k][0].record()
+        e2e_step()
+        ev2[k][1].record()
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in ev2)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": round(world * flops / (e2e_ms / args.steps / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+           "ms_per_step": round(e2e_ms / args.steps, 4), "h2d_bytes_per_step": int(h2d),
+           "d2h_bytes_per_step": int(d2h)}
+
+    tpeak, tpeak_kind = measured_tensor_peak(g.dtype, sustained=True)
+    hpeak, hpeak_kind = measured_peak()
+    kname = "tc_fp8_pair_kernel" if g.dtype == "fp8" else "tc16_pair_kernel"
+    achieved_t = flops / mean_s / 1e12
+    achieved_h = alg_bytes / mean_s / 1e9
+    roofline = {"bound": "tensor", "achieved": round(achieved_t, 1), "peak": round(tpeak, 1), "unit": "TFLOP/s",
+                "frac": round(achieved_t / tpeak, 4), "peak_source": tpeak_kind, "traffic": None,
+                "kernel": kname, "scope": "whole step (partial + combine)", "alg_flops_per_step": int(flops),
+                "floor_ms": round(flops / (tpeak * 1e12) * 1e3, 4),
+                "other": {"bound": "hbm", "achieved": round(achieved_h, 1), "peak": hpeak, "unit": "GB/s",
+                          "frac": round(achieved_h / hpeak, 4), "peak_source": hpeak_kind,
+                          "floor_ms": round(alg_bytes / (hpeak * 1e9) * 1e3, 4)}}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        H = g.heads
+        toks = list(range(cu[1] - 8, cu[1])) if g.batch else []  # the last tokens of entry 0: its longest rows
+        rows = [t * H + h for t in toks for h in range(H)]
+        hcache = inp.kv_cache.cpu()
+        t0 = time.perf_counter()
+        oracle.mla_prefill(hq, inp.cu_seqlens_q, hcache, inp.block_tables, inp.seq_lens, g.softmax_scale,
+                           dtype=g.dtype, q_scale=g.q_scale, kv_scale=g.kv_scale, rows=rows)
+        dt = time.perf_counter() - t0
+        n0 = int(inp.seq_lens[0])
+        sample_flops = sum(n0 - (cu[1] - cu[0]) + (t - cu[0]) + 1 for t in toks) * H * 2 * (576 + 512)
+        cpu = {"value": round(sample_flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+               "kind": "oracle", "seconds": round(dt, 3),
+               "sample": f"{len(rows)} query rows (the last 8 tokens of entry 0, all heads); flops of those rows"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": "MLA ragged prefill TFLOP/s (algorithmic flops per step / step time) on 1 B200",
+        "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": {"fp8": "fp8_e4m3", "bf16": "bf16", "fp16": "fp16"}[g.dtype],
+        "data": "synthetic (seeded, generated on device)",
+        "config": {"workload": name, "batch": g.batch, "heads": g.heads, "total_q": g.total_q,
+                   "max_q_len": g.max_q_len, "kv_tokens": int(inp.seq_lens.sum()), "fold": pre.plan.fold,
+                   "units": pre.plan.batch * pre.plan.q_groups, "desc": w.desc,
+                   "l2": f"256 MiB buffer rewritten between steps (cache pool {pool_bytes >> 20} MiB)",
+                   "parallelism": f"replicas x{world}"},
+        "gpu_launches": 2 * args.steps,
+        "roofline": roofline, "e2e": e2e, "clocks": clocks, "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     if args.op == "kv_pack":
         run_kv_pack(args)
+        return
+    if args.op == "prefill":
+        run_prefill(args)
         return
     if args.impl == "reference":
         run_reference(args)

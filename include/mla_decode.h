@@ -73,6 +73,8 @@ typedef enum {
 #define MLA_DEV_BAD_PAGE 0x1     /* block-table entry outside [0, num_pages): keys masked */
 #define MLA_DEV_SEQ_TOO_LONG 0x2 /* seq_len above max_seq_len or the table width: clamped */
 #define MLA_DEV_TIMEOUT 0x4      /* a bounded pipeline wait gave up; outputs unspecified */
+#define MLA_DEV_BAD_QLEN 0x8     /* ragged queries: a cu_seqlens_q range decreasing, longer than the
+                                    plan's max_q_len or past total_q; that entry gets no output */
 
 typedef enum {
   MLA_KERNEL_AUTO = 0,         /* MLA_KERNEL_TCGEN05 */
@@ -88,7 +90,7 @@ typedef enum {
  * Two work schedules exist (field `schedule`):
  *   MLA_SCHEDULE_SPLITS: every unit is cut into split_kv chunks of
  *     keys_per_split keys, one CTA (pair) each; partials [B*q_len*H, S, 512].
- *   MLA_SCHEDULE_BALANCED (FP8 CTA-pair kernel): split_kv = P CTA pairs stay
+ *   MLA_SCHEDULE_BALANCED (CTA-pair kernels): split_kv = P CTA pairs stay
  *     resident; the units' 128-key tiles, counted from the device seq_lens,
  *     are dealt out as equal contiguous ranges. A unit a pair covers whole
  *     is written to out/lse directly; a unit cut between pairs leaves
@@ -97,7 +99,9 @@ typedef enum {
  *     columns][M rows][4] at partial_offset, fp32 LSE as [2P][M] at
  *     lse_offset. Between the 256-byte status header and partial_offset
  *     lie B*G + 1 int32 counters (finished pieces per unit, then a flag for
- *     the unit table at the end of the workspace), cleared with the status
+ *     the unit table at the end of the workspace; before that table, a
+ *     spill area for piece lists longer than a pair keeps in shared
+ *     memory), cleared with the status
  *     word before every launch: the combine kernel is launched as the
  *     partial kernel's programmatic dependent and merges each unit as soon
  *     as its counter is complete. keys_per_split then only
@@ -123,7 +127,7 @@ typedef struct {
   uint32_t magic;    /* set by the planner; checked by mla_decode */
   uint32_t schedule; /* MLA_SCHEDULE_* below */
   int32_t window;    /* sliding window in keys (0 = none); set with mla_decode_plan_window */
-  int32_t reserved;
+  int32_t varlen;    /* 1: ragged query lengths (mla_prefill_plan / mla_prefill), q_len = the longest */
 } mla_plan;
 
 /*
@@ -215,6 +219,58 @@ int mla_decode_combine(const mla_plan* plan, const void* q, const void* kv_cache
                        int max_pages_per_seq, const int32_t* seq_lens, float softmax_scale,
                        float q_scale, float kv_scale, void* out, float* lse, void* workspace,
                        uint64_t workspace_bytes, void* stream);
+
+/*
+ * Ragged-query (prefill) forms: chunked prefill of several sequences with
+ * different numbers of new tokens, packed without padding (tokenspeed-mla
+ * package card, "What it is and what it does": the prefill path handles
+ * ragged variable-length sequences without padding and takes FP8 inputs;
+ * TokenSpeed MLA article, section 一, its kernel table). The attention is
+ * the decode's, in the latent form over the same paged cache: entry b has
+ * q_len_b = cu_seqlens_q[b + 1] - cu_seqlens_q[b] new tokens, already
+ * written to the cache, and seq_lens[b] keys in all; its token t sees keys
+ * 0 .. seq_lens[b] - q_len_b + t.
+ *
+ * mla_prefill_plan: as mla_decode_plan with max_q_len = the most new tokens
+ * an entry may have. F is the largest fold with H * F <= 128 (need not
+ * divide max_q_len); every entry gets ceil(max_q_len / F) query groups, the
+ * ones past its tokens empty. Runs on the CTA-pair kernels (balanced
+ * schedule, at most 65536 groups in all, else MLA_ERR_UNSUPPORTED_SHAPE);
+ * mla_prefill_plan_custom also takes kernel = MLA_KERNEL_SIMT and forced
+ * split_kv / fold, like mla_decode_plan_custom. The plan's `varlen` is 1.
+ */
+int mla_prefill_plan(int batch, int max_q_len, int num_heads, int max_seq_len, int dtype, mla_plan* plan);
+int mla_prefill_plan_custom(int batch, int max_q_len, int num_heads, int max_seq_len, int dtype,
+                            int split_kv, int fold, int kernel, mla_plan* plan);
+
+/*
+ * mla_prefill: one ragged prefill step. Arguments as mla_decode, except:
+ *   plan          from mla_prefill_plan (varlen = 1)
+ *   q             device, [total_q, H, 576]: the entries' new tokens, packed
+ *   total_q       tokens in q, 0 <= total_q <= batch * max_q_len
+ *   cu_seqlens_q  device int32 [B + 1], non-decreasing, cu[0] >= 0,
+ *                 cu[B] <= total_q, each q_len_b <= max_q_len; a range that
+ *                 breaks this sets MLA_DEV_BAD_QLEN and that entry gets no
+ *                 output. Packed tokens outside every entry are not written.
+ *   out           device bf16 [total_q, H, 512]; lse fp32 [total_q, H] or NULL
+ * mla_prefill_partial / mla_prefill_combine: its two kernels, as
+ * mla_decode_partial / mla_decode_combine. A decode plan, or a null
+ * cu_seqlens_q, is refused (MLA_ERR_PLAN_MISMATCH / MLA_ERR_INVALID_ARG).
+ */
+int mla_prefill(const mla_plan* plan, const void* q, int64_t total_q, const int32_t* cu_seqlens_q,
+                const void* kv_cache, int64_t num_pages, int page_size, const int32_t* block_tables,
+                int max_pages_per_seq, const int32_t* seq_lens, float softmax_scale, float q_scale,
+                float kv_scale, void* out, float* lse, void* workspace, uint64_t workspace_bytes, void* stream);
+int mla_prefill_partial(const mla_plan* plan, const void* q, int64_t total_q, const int32_t* cu_seqlens_q,
+                        const void* kv_cache, int64_t num_pages, int page_size, const int32_t* block_tables,
+                        int max_pages_per_seq, const int32_t* seq_lens, float softmax_scale, float q_scale,
+                        float kv_scale, void* out, float* lse, void* workspace, uint64_t workspace_bytes,
+                        void* stream);
+int mla_prefill_combine(const mla_plan* plan, const void* q, int64_t total_q, const int32_t* cu_seqlens_q,
+                        const void* kv_cache, int64_t num_pages, int page_size, const int32_t* block_tables,
+                        int max_pages_per_seq, const int32_t* seq_lens, float softmax_scale, float q_scale,
+                        float kv_scale, void* out, float* lse, void* workspace, uint64_t workspace_bytes,
+                        void* stream);
 
 /*
  * mla_decode_status: synchronise `stream`, copy the device status word of

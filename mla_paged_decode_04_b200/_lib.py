@@ -22,14 +22,15 @@ MLA_KERNEL_AUTO, MLA_KERNEL_TCGEN05, MLA_KERNEL_SIMT, MLA_KERNEL_TCGEN05_SOLO = 
 KERNELS = {"auto": MLA_KERNEL_AUTO, "tcgen05": MLA_KERNEL_TCGEN05, "simt": MLA_KERNEL_SIMT,
            "tcgen05_solo": MLA_KERNEL_TCGEN05_SOLO}
 
-MLA_DEV_BAD_PAGE, MLA_DEV_SEQ_TOO_LONG, MLA_DEV_TIMEOUT = 0x1, 0x2, 0x4
+MLA_DEV_BAD_PAGE, MLA_DEV_SEQ_TOO_LONG, MLA_DEV_TIMEOUT, MLA_DEV_BAD_QLEN = 0x1, 0x2, 0x4, 0x8
 (MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED_SHAPE, MLA_ERR_WORKSPACE_TOO_SMALL, MLA_ERR_ARCH, MLA_ERR_CUDA,
  MLA_ERR_PLAN_MISMATCH) = (-1, -2, -3, -4, -5, -6)
 
 EXPORTED = ["mla_decode_plan", "mla_decode_plan_custom", "mla_decode", "mla_decode_partial",
             "mla_decode_combine", "mla_decode_status", "mla_status_string", "mla_version",
             "mla_decode_no_alloc", "mla_last_cuda_error", "mla_kv_pack", "mla_kv_amax",
-            "mla_decode_plan_window"]
+            "mla_decode_plan_window", "mla_prefill_plan", "mla_prefill_plan_custom", "mla_prefill",
+            "mla_prefill_partial", "mla_prefill_combine"]
 MLA_NO_ALLOC_SCRATCH_BYTES = 48 << 20
 
 
@@ -42,7 +43,7 @@ class MlaPlan(ctypes.Structure):
         ("kernel", ctypes.c_int32), ("num_ctas", ctypes.c_int32),
         ("workspace_bytes", ctypes.c_uint64), ("partial_offset", ctypes.c_uint64),
         ("lse_offset", ctypes.c_uint64), ("magic", ctypes.c_uint32), ("schedule", ctypes.c_uint32),
-        ("window", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("window", ctypes.c_int32), ("varlen", ctypes.c_int32),
     ]
 
     def as_dict(self):
@@ -85,6 +86,14 @@ def _load():
     lib.mla_version.restype = ctypes.c_char_p
     lib.mla_last_cuda_error.argtypes = [ctypes.POINTER(ctypes.c_char_p)]
     lib.mla_last_cuda_error.restype = i32
+    lib.mla_prefill_plan.argtypes = [i32, i32, i32, i32, i32, P]
+    lib.mla_prefill_plan.restype = i32
+    lib.mla_prefill_plan_custom.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, P]
+    lib.mla_prefill_plan_custom.restype = i32
+    for name in ("mla_prefill", "mla_prefill_partial", "mla_prefill_combine"):
+        fn = getattr(lib, name)
+        fn.argtypes = [P, vp, i64, vp, vp, i64, i32, vp, i32, vp, f32, f32, f32, vp, vp, vp, u64, vp]
+        fn.restype = i32
     lib.mla_decode_plan_window.argtypes = [P, i32]
     lib.mla_decode_plan_window.restype = i32
     lib.mla_kv_pack.argtypes = [vp, vp, i64, vp, vp, i64, i32, i32, i32, f32, vp, vp]
@@ -155,6 +164,18 @@ def mla_decode_plan_window(plan: MlaPlan, window: int) -> MlaPlan:
     return plan
 
 
+def mla_prefill_plan(batch, max_q_len, num_heads, max_seq_len, dtype, split_kv=0, fold=0,
+                     kernel="auto") -> MlaPlan:
+    """Plan of a ragged-query (prefill) shape: max_q_len = the most new tokens an entry may have."""
+    p = MlaPlan()
+    k = KERNELS[kernel] if isinstance(kernel, str) else int(kernel)
+    rc = _lib.mla_prefill_plan_custom(batch, max_q_len, num_heads, max_seq_len, _dtype_code(dtype),
+                                      split_kv, fold, k, ctypes.byref(p))
+    if rc != 0:
+        raise MlaError(rc, "mla_prefill_plan")
+    return p
+
+
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -219,6 +240,37 @@ def mla_decode_combine(plan: MlaPlan, q, kv_cache, block_tables, seq_lens, softm
     """Second kernel only (LSE merge of the partials; no-op when split_kv == 1)."""
     _call("mla_decode_combine", plan, q, kv_cache, block_tables, seq_lens, softmax_scale, out,
           lse, workspace, q_scale, kv_scale, stream)
+
+
+def _call_prefill(name, plan, q, cu_seqlens_q, kv_cache, block_tables, seq_lens, softmax_scale, out, lse,
+                  workspace, q_scale, kv_scale, stream):
+    _check_tensors(q, cu_seqlens_q=cu_seqlens_q, kv_cache=kv_cache, block_tables=block_tables,
+                   seq_lens=seq_lens, out=out, lse=lse, workspace=workspace)
+    if cu_seqlens_q is None or cu_seqlens_q.dtype != torch.int32:
+        raise ValueError("cu_seqlens_q must be an int32 CUDA tensor")
+    num_pages, page_size = int(kv_cache.shape[0]), int(kv_cache.shape[1])
+    rc = getattr(_lib, name)(ctypes.byref(plan), _ptr(q), int(q.shape[0]), _ptr(cu_seqlens_q), _ptr(kv_cache),
+                             num_pages, page_size, _ptr(block_tables), int(block_tables.shape[1]), _ptr(seq_lens),
+                             float(softmax_scale), float(q_scale), float(kv_scale), _ptr(out), _ptr(lse),
+                             _ptr(workspace), int(workspace.numel() * workspace.element_size()),
+                             ctypes.c_void_p(_stream_of(q, stream)))
+    if rc != 0:
+        raise MlaError(rc, name)
+
+
+def mla_prefill(plan: MlaPlan, q, cu_seqlens_q, kv_cache, block_tables, seq_lens, softmax_scale, out, lse,
+                workspace, q_scale=1.0, kv_scale=1.0, stream=None) -> None:
+    """Enqueue one ragged prefill step: q [total_q, H, 576] packed, cu_seqlens_q int32 [B + 1],
+    out bf16 [total_q, H, 512], lse fp32 [total_q, H] or None (include/mla_decode.h)."""
+    _call_prefill("mla_prefill", plan, q, cu_seqlens_q, kv_cache, block_tables, seq_lens, softmax_scale, out,
+                  lse, workspace, q_scale, kv_scale, stream)
+
+
+def mla_prefill_partial(plan: MlaPlan, q, cu_seqlens_q, kv_cache, block_tables, seq_lens, softmax_scale, out,
+                        lse, workspace, q_scale=1.0, kv_scale=1.0, stream=None) -> None:
+    """First kernel of mla_prefill only."""
+    _call_prefill("mla_prefill_partial", plan, q, cu_seqlens_q, kv_cache, block_tables, seq_lens, softmax_scale,
+                  out, lse, workspace, q_scale, kv_scale, stream)
 
 
 def mla_decode_status(workspace, clear=True, stream=None) -> int:
@@ -299,6 +351,33 @@ class MlaDecoder:
             lse = torch.empty((B, T, H), dtype=torch.float32, device=self.device)
         mla_decode(self.plan, q, kv_cache, block_tables, seq_lens, softmax_scale, out, lse,
                    self.workspace, q_scale, kv_scale, stream)
+        return out, lse
+
+    def status(self, clear=True) -> int:
+        return mla_decode_status(self.workspace, clear)
+
+
+class MlaPrefill:
+    """Plan + workspace for one ragged prefill shape (batch, longest entry, H, longest sequence)."""
+
+    def __init__(self, batch, max_q_len, num_heads, max_seq_len, dtype, device, split_kv=0, fold=0,
+                 kernel="auto", window=0):
+        self.plan = mla_prefill_plan(batch, max_q_len, num_heads, max_seq_len, dtype, split_kv, fold, kernel)
+        if window:
+            mla_decode_plan_window(self.plan, window)
+        self.device = torch.device(device)
+        self.workspace = alloc_workspace(self.plan, self.device)
+        self.num_heads = num_heads
+
+    def __call__(self, q, cu_seqlens_q, kv_cache, block_tables, seq_lens, softmax_scale, q_scale=1.0,
+                 kv_scale=1.0, out=None, lse=None, want_lse=True, stream=None):
+        total_q, H = int(q.shape[0]), self.num_heads
+        if out is None:
+            out = torch.empty((total_q, H, 512), dtype=torch.bfloat16, device=self.device)
+        if lse is None and want_lse:
+            lse = torch.empty((total_q, H), dtype=torch.float32, device=self.device)
+        mla_prefill(self.plan, q, cu_seqlens_q, kv_cache, block_tables, seq_lens, softmax_scale, out, lse,
+                    self.workspace, q_scale, kv_scale, stream)
         return out, lse
 
     def status(self, clear=True) -> int:

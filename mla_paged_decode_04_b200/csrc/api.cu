@@ -67,8 +67,11 @@ int check_plan(const mla_plan* p) {
       p->max_seq_len < 0)
     return MLA_ERR_PLAN_MISMATCH;
   if (p->dtype != MLA_BF16 && p->dtype != MLA_FP16 && p->dtype != MLA_FP8_E4M3) return MLA_ERR_PLAN_MISMATCH;
-  if (p->fold < 1 || p->q_len % p->fold != 0 || p->q_groups * p->fold != p->q_len ||
-      p->rows_per_unit != p->num_heads * p->fold || p->rows_per_unit > MLA_MAX_ROWS)
+  if (p->varlen != 0 && p->varlen != 1) return MLA_ERR_PLAN_MISMATCH;
+  // decode: F divides q_len; ragged queries: an entry's last group may be short
+  if (p->fold < 1 || p->fold > p->q_len || (!p->varlen && p->q_len % p->fold != 0) ||
+      p->q_groups != (p->q_len + p->fold - 1) / p->fold || p->rows_per_unit != p->num_heads * p->fold ||
+      p->rows_per_unit > MLA_MAX_ROWS)
     return MLA_ERR_PLAN_MISMATCH;
   if (p->split_kv < 1 || p->keys_per_split < kTileKeys || p->keys_per_split % kTileKeys != 0)
     return MLA_ERR_PLAN_MISMATCH;
@@ -78,19 +81,21 @@ int check_plan(const mla_plan* p) {
   if (p->kernel == MLA_KERNEL_TCGEN05_SOLO && p->dtype != MLA_FP8_E4M3) return MLA_ERR_PLAN_MISMATCH;
   if (p->schedule != MLA_SCHEDULE_SPLITS && p->schedule != MLA_SCHEDULE_BALANCED) return MLA_ERR_PLAN_MISMATCH;
   if (p->window < 0) return MLA_ERR_PLAN_MISMATCH;
-  if (p->window > 0 && !(p->kernel == MLA_KERNEL_SIMT ||
-                         (p->kernel == MLA_KERNEL_TCGEN05 && p->schedule == MLA_SCHEDULE_BALANCED)))
+  // a window and ragged queries run on the CTA-pair kernels and the SIMT kernel
+  if ((p->window > 0 || p->varlen) &&
+      !(p->kernel == MLA_KERNEL_SIMT || (p->kernel == MLA_KERNEL_TCGEN05 && p->schedule == MLA_SCHEDULE_BALANCED)))
     return MLA_ERR_PLAN_MISMATCH;
   if (p->schedule == MLA_SCHEDULE_BALANCED) {
     // CTA-pair kernels only; slots [2P, M, 512] fp32 + [2P, M] + unit table
     if (p->kernel != MLA_KERNEL_TCGEN05 || p->split_kv > kNumSMs / 2)
       return MLA_ERR_PLAN_MISMATCH;
     const int64_t units = (int64_t)p->batch * p->q_groups;
-    if (units > kMaxBalancedUnits) return MLA_ERR_PLAN_MISMATCH;
+    if (units > (p->varlen ? kMaxVarlenUnits : kMaxBalancedUnits)) return MLA_ERR_PLAN_MISMATCH;
     const uint64_t slot_rows = 2ull * p->split_kv * p->rows_per_unit;
     if (p->partial_offset < (uint64_t)kHeaderBytes + balanced_counter_bytes(units) || p->partial_offset % 256 != 0 ||
         p->lse_offset < p->partial_offset + slot_rows * MLA_D_V * 4 || p->lse_offset % 256 != 0 ||
-        p->workspace_bytes < p->lse_offset + slot_rows * 4 + balanced_table_bytes(units))
+        p->workspace_bytes < p->lse_offset + slot_rows * 4 + balanced_spill_bytes(units, p->split_kv) +
+                                 balanced_table_bytes(units))
       return MLA_ERR_PLAN_MISMATCH;
     return MLA_OK;
   }
@@ -113,13 +118,20 @@ namespace {
 
 // Validate the arguments and fill the launch description. Returns MLA_OK or
 // an error code; nothing is enqueued here.
+// cu_q: null for decode (every entry has the plan's q_len tokens); for a
+// ragged-query plan the device [B + 1] token offsets, with total_q tokens in q.
 int prepare(const mla_plan* plan, const void* q, const void* kv_cache, int64_t num_pages,
             int page_size, const int32_t* block_tables, int max_pages_per_seq,
             const int32_t* seq_lens, float softmax_scale, float q_scale, float kv_scale, void* out,
-            float* lse, void* workspace, uint64_t workspace_bytes, DecodeArgs* a) {
+            float* lse, void* workspace, uint64_t workspace_bytes, const int32_t* cu_q, int64_t total_q,
+            DecodeArgs* a) {
   int rc = check_plan(plan);
   if (rc != MLA_OK) return rc;
   const mla_plan& p = *plan;
+  if ((cu_q != nullptr) != (p.varlen != 0)) return MLA_ERR_PLAN_MISMATCH;
+  if (!p.varlen) total_q = (int64_t)p.batch * p.q_len;
+  // the fixed-split workspace holds B * q_len * H rows
+  if (total_q < 0 || total_q > (int64_t)p.batch * p.q_len) return MLA_ERR_INVALID_ARG;
   if (page_size != MLA_PAGE_SIZE) return MLA_ERR_UNSUPPORTED_SHAPE;
   if (!workspace || !aligned(workspace, 256)) return MLA_ERR_INVALID_ARG;
   if (workspace_bytes < p.workspace_bytes) return MLA_ERR_WORKSPACE_TOO_SMALL;
@@ -130,7 +142,7 @@ int prepare(const mla_plan* plan, const void* q, const void* kv_cache, int64_t n
   if (p.batch > 0) {
     if (!q || !kv_cache || !block_tables || !seq_lens || !out) return MLA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(kv_cache, 16) || !aligned(out, 16) || !aligned(block_tables, 4) ||
-        !aligned(seq_lens, 4) || (lse && !aligned(lse, 4)))
+        !aligned(seq_lens, 4) || (lse && !aligned(lse, 4)) || (cu_q && !aligned(cu_q, 4)))
       return MLA_ERR_INVALID_ARG;
     if (num_pages < 1 || max_pages_per_seq < 1) return MLA_ERR_INVALID_ARG;
     if (num_pages > (int64_t(1) << 31) / MLA_PAGE_SIZE) return MLA_ERR_UNSUPPORTED_SHAPE;
@@ -139,7 +151,7 @@ int prepare(const mla_plan* plan, const void* q, const void* kv_cache, int64_t n
     if (!device_addressable(q, dev) || !device_addressable(kv_cache, dev) ||
         !device_addressable(block_tables, dev) || !device_addressable(seq_lens, dev) ||
         !device_addressable(out, dev) || (lse && !device_addressable(lse, dev)) ||
-        !device_addressable(workspace, dev))
+        !device_addressable(workspace, dev) || (cu_q && !device_addressable(cu_q, dev)))
       return MLA_ERR_INVALID_ARG;
   }
   rc = check_device_arch();
@@ -164,10 +176,16 @@ int prepare(const mla_plan* plan, const void* q, const void* kv_cache, int64_t n
   const bool partials = p.split_kv > 1 || p.schedule == MLA_SCHEDULE_BALANCED;
   a->o_part = partials ? reinterpret_cast<float*>(ws + p.partial_offset) : nullptr;
   a->lse_part = partials ? reinterpret_cast<float*>(ws + p.lse_offset) : nullptr;
+  const int64_t units = (int64_t)p.batch * p.q_groups;
   a->sched = p.schedule == MLA_SCHEDULE_BALANCED
-                 ? reinterpret_cast<int32_t*>(ws + p.workspace_bytes -
-                                              balanced_table_bytes((int64_t)p.batch * p.q_groups))
+                 ? reinterpret_cast<int32_t*>(ws + p.workspace_bytes - balanced_table_bytes(units))
                  : nullptr;
+  a->pieces = p.schedule == MLA_SCHEDULE_BALANCED
+                  ? reinterpret_cast<int32_t*>(ws + p.workspace_bytes - balanced_table_bytes(units) -
+                                               balanced_spill_bytes(units, p.split_kv))
+                  : nullptr;
+  a->cu_q = cu_q;
+  a->total_q = total_q;
   a->unit_done = p.schedule == MLA_SCHEDULE_BALANCED ? reinterpret_cast<int32_t*>(ws + kHeaderBytes) : nullptr;
   return MLA_OK;
 }
@@ -177,7 +195,7 @@ int run_partial(const DecodeArgs& a, cudaStream_t st) {
   const size_t clear = a.unit_done ? kHeaderBytes + balanced_counter_bytes((int64_t)a.plan.batch * a.plan.q_groups)
                                    : sizeof(int32_t);
   if (cudaError_t e = cudaMemsetAsync(a.status, 0, clear, st); e != cudaSuccess) return cuda_failure(e);
-  if (a.plan.batch == 0) return MLA_OK;
+  if (a.plan.batch == 0 || a.total_q == 0) return MLA_OK;
   cudaError_t e;
   if (a.plan.kernel == MLA_KERNEL_SIMT)
     e = launch_simt_partial(a, st);
@@ -191,7 +209,7 @@ int run_partial(const DecodeArgs& a, cudaStream_t st) {
 }
 
 int run_combine(const DecodeArgs& a, cudaStream_t st) {
-  if (a.plan.batch == 0) return MLA_OK;
+  if (a.plan.batch == 0 || a.total_q == 0) return MLA_OK;
   if (a.plan.schedule == MLA_SCHEDULE_BALANCED) {
     const cudaError_t e = launch_combine_balanced(a, st);
     return e == cudaSuccess ? MLA_OK : cuda_failure(e);
@@ -211,7 +229,15 @@ int run_combine(const DecodeArgs& a, cudaStream_t st) {
       uint64_t workspace_bytes, void *stream
 #define MLA_ARGS_FWD                                                                            \
   plan, q, kv_cache, num_pages, page_size, block_tables, max_pages_per_seq, seq_lens,          \
-      softmax_scale, q_scale, kv_scale, out, lse, workspace, workspace_bytes
+      softmax_scale, q_scale, kv_scale, out, lse, workspace, workspace_bytes, nullptr, 0
+#define MLA_PREFILL_ARGS_DECL                                                                   \
+  const mla_plan *plan, const void *q, int64_t total_q, const int32_t *cu_seqlens_q,            \
+      const void *kv_cache, int64_t num_pages, int page_size, const int32_t *block_tables,      \
+      int max_pages_per_seq, const int32_t *seq_lens, float softmax_scale, float q_scale,       \
+      float kv_scale, void *out, float *lse, void *workspace, uint64_t workspace_bytes, void *stream
+#define MLA_PREFILL_ARGS_FWD                                                                    \
+  plan, q, kv_cache, num_pages, page_size, block_tables, max_pages_per_seq, seq_lens,          \
+      softmax_scale, q_scale, kv_scale, out, lse, workspace, workspace_bytes, cu_seqlens_q, total_q
 
 using namespace mla;
 
@@ -235,6 +261,36 @@ extern "C" int mla_decode_partial(MLA_ARGS_DECL) {
 extern "C" int mla_decode_combine(MLA_ARGS_DECL) {
   DecodeArgs a;
   int rc = prepare(MLA_ARGS_FWD, &a);
+  if (rc != MLA_OK) return rc;
+  return run_combine(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// Ragged-query (prefill) forms: the same kernels, entries' tokens given by
+// cu_seqlens_q. A null cu_seqlens_q is refused (it would select the decode
+// geometry).
+extern "C" int mla_prefill(MLA_PREFILL_ARGS_DECL) {
+  if (!cu_seqlens_q) return MLA_ERR_INVALID_ARG;
+  DecodeArgs a;
+  int rc = prepare(MLA_PREFILL_ARGS_FWD, &a);
+  if (rc != MLA_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  rc = run_partial(a, st);
+  if (rc != MLA_OK) return rc;
+  return run_combine(a, st);
+}
+
+extern "C" int mla_prefill_partial(MLA_PREFILL_ARGS_DECL) {
+  if (!cu_seqlens_q) return MLA_ERR_INVALID_ARG;
+  DecodeArgs a;
+  int rc = prepare(MLA_PREFILL_ARGS_FWD, &a);
+  if (rc != MLA_OK) return rc;
+  return run_partial(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int mla_prefill_combine(MLA_PREFILL_ARGS_DECL) {
+  if (!cu_seqlens_q) return MLA_ERR_INVALID_ARG;
+  DecodeArgs a;
+  int rc = prepare(MLA_PREFILL_ARGS_FWD, &a);
   if (rc != MLA_OK) return rc;
   return run_combine(a, reinterpret_cast<cudaStream_t>(stream));
 }

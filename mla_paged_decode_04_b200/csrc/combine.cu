@@ -15,13 +15,28 @@
 namespace mla {
 namespace {
 
+// Batch entry of packed query token `tok` (ragged queries: the last entry
+// whose first token is at most tok), or -1 when no entry holds the token.
+__device__ int entry_of_token(const DecodeArgs& a, int64_t tok) {
+  const mla_plan& p = a.plan;
+  if (!a.cu_q) return (int)(tok / p.q_len);
+  int lo = 0, hi = p.batch - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.cu_q[mid] <= tok) lo = mid; else hi = mid - 1;
+  }
+  const EntryQ e = entry_q(a, lo, false);
+  return (tok >= e.q0 && tok < e.q0 + e.qlen) ? lo : -1;
+}
+
 __global__ void __launch_bounds__(256) combine_kernel(const DecodeArgs a) {
   const mla_plan& p = a.plan;
-  const int64_t rows = (int64_t)p.batch * p.q_len * p.num_heads;
+  const int64_t rows = a.total_q * p.num_heads;
   const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
-  const int b = (int)(row / ((int64_t)p.q_len * p.num_heads));
+  const int b = entry_of_token(a, row / p.num_heads);
+  if (b < 0) return;  // a packed token outside every entry: no output
   const int n = effective_seq_len(a, b, false);
   const int S = p.split_kv;
   const int ns = min(S, (n + p.keys_per_split - 1) / p.keys_per_split);
@@ -72,7 +87,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const DecodeArgs a) {
 }  // namespace
 
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t stream) {
-  const int64_t rows = (int64_t)a.plan.batch * a.plan.q_len * a.plan.num_heads;
+  const int64_t rows = a.total_q * a.plan.num_heads;
   if (rows == 0) return cudaSuccess;
   combine_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(a);
   return cudaGetLastError();
@@ -142,9 +157,9 @@ __global__ void __launch_bounds__(256) combine_balanced_kernel(const DecodeArgs 
   }
   const int r = (blk % nb) * 32 + (threadIdx.x & 31);       // row within the unit
   const int c4_0 = cb * 16 + (threadIdx.x >> 5) * 2;         // first of this thread's two 16-byte chunks
-  if (r >= M) return;
-  const int b = u / p.q_groups, g = u % p.q_groups;
-  const int64_t row = (int64_t)b * p.q_len * p.num_heads + (int64_t)g * M + r;
+  const UnitGeom ug = unit_geom(a, u, false);
+  if (r >= ug.rows) return;  // past the unit's rows (an entry's last group under ragged queries)
+  const int64_t row = ug.row0 + r;
   uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + row * MLA_D_V + c4_0 * 4);
   const bool lse_writer = a.lse && cb == 0 && (threadIdx.x >> 5) == 0;
   if (end == start) {  // no key at all

@@ -41,16 +41,64 @@ __device__ __forceinline__ int effective_seq_len(const DecodeArgs& a, int b, boo
   return n;
 }
 
-// Sliding window (plan.window = W > 0): query token t of an entry with n
-// keys sees keys [n - q_len + t + 1 - W, n - q_len + t]. First key of token t,
-// and of the first token of query group g (the lowest key its unit needs).
-__device__ __forceinline__ int window_row_lo(const mla_plan& p, int t, int n) {
-  if (p.window <= 0) return 0;
-  const int lo = n - p.q_len + t + 1 - p.window;
-  return lo > 0 ? lo : 0;
+// Query tokens of batch entry b: the first one's index in the packed query
+// and how many there are. Decode: q_len tokens each, entry-major. Ragged
+// queries (prefill): entry b holds tokens [cu_q[b], cu_q[b + 1]); a range that
+// is decreasing, longer than the plan's q_len or past total_q sets
+// MLA_DEV_BAD_QLEN (when `flag` is set) and leaves the entry without tokens.
+struct EntryQ {
+  int64_t q0;
+  int qlen;
+};
+__device__ __forceinline__ EntryQ entry_q(const DecodeArgs& a, int b, bool flag) {
+  if (!a.cu_q) return {(int64_t)b * a.plan.q_len, a.plan.q_len};
+  const int s = a.cu_q[b], e = a.cu_q[b + 1];
+  if (s < 0 || e < s || e - s > a.plan.q_len || (int64_t)e > a.total_q) {
+    if (flag) atomicOr(a.status, MLA_DEV_BAD_QLEN);
+    return {0, 0};
+  }
+  return {(int64_t)s, e - s};
 }
-__device__ __forceinline__ int window_unit_lo(const mla_plan& p, int g, int n) {
-  return window_row_lo(p, g * p.fold, n);
+
+// Unit u = (entry b, query group g): tokens g*F .. g*F + F - 1 of entry b
+// (fewer in an entry's last group when queries are ragged), H rows each.
+// Token t of an entry with n keys and qlen tokens sees keys up to
+// n - qlen + t (causal, aligned to the end); with a sliding window W > 0 only
+// its last W of them, from n - qlen + t + 1 - W.
+struct UnitGeom {
+  int b, g;
+  int n;         // keys of the entry (clamped seq_len)
+  int rows;      // query rows of the unit (0: a group past the entry's tokens)
+  int nq;        // last key of the unit's first token; row r sees keys <= nq + r / H
+  int klo;       // lowest key a row of the unit sees
+  int kend;      // one past the highest key a row of the unit sees
+  int64_t row0;  // first output row (token * H + head) of the unit
+};
+__device__ __forceinline__ UnitGeom unit_geom(const DecodeArgs& a, int u, bool flag) {
+  const mla_plan& p = a.plan;
+  UnitGeom ug;
+  ug.b = u / p.q_groups;
+  ug.g = u % p.q_groups;
+  const bool first = flag && ug.g == 0;
+  ug.n = effective_seq_len(a, ug.b, first);
+  const EntryQ e = entry_q(a, ug.b, first);
+  const int t0 = ug.g * p.fold;
+  const int tu = min(p.fold, e.qlen - t0);
+  ug.rows = tu > 0 ? tu * p.num_heads : 0;
+  ug.nq = ug.n - e.qlen + t0;
+  ug.row0 = (e.q0 + t0) * p.num_heads;
+  ug.kend = tu > 0 ? max(0, ug.nq + tu) : 0;
+  ug.klo = (tu > 0 && p.window > 0) ? max(0, ug.nq + 1 - p.window) : 0;
+  return ug;
+}
+// First key of the row whose last key is `last` (its sliding window's start).
+__device__ __forceinline__ int row_key_lo(const mla_plan& p, int last) {
+  return p.window > 0 ? max(0, last + 1 - p.window) : 0;
+}
+// Tiles of kKeys keys a unit spans, from the tile of its lowest key.
+template <int kKeys>
+__device__ __forceinline__ int unit_span_tiles(const UnitGeom& ug) {
+  return ug.kend > ug.klo ? (ug.kend + kKeys - 1) / kKeys - ug.klo / kKeys : 0;
 }
 
 __device__ __forceinline__ float warp_sum(float v) {

@@ -13,7 +13,8 @@ constexpr int kNumSMs = 148;                    // B200
 constexpr int kHeaderBytes = 256;               // workspace header (status word at offset 0)
 constexpr int kTileKeys = 64;                   // keys per tile = one cache page
 constexpr int kPairTileKeys = 128;              // keys per CTA-pair tile (one page per CTA)
-constexpr int kMaxBalancedUnits = 2048;         // units (entry x query group) the balanced schedule takes
+constexpr int kMaxBalancedUnits = 2048;         // decode units (entry x query group) the balanced schedule takes
+constexpr int kMaxVarlenUnits = 1 << 16;        // units of a ragged-query (prefill) plan
 
 // Balanced schedule table at the end of the workspace: int32 start tile of
 // every unit (U + 1 entries, the last = W, the total pair tiles), then the
@@ -28,6 +29,13 @@ inline uint64_t balanced_counter_bytes(int64_t units) {
 }
 inline uint64_t balanced_table_bytes(int64_t units) {
   return ((uint64_t)(units + 2) * 4 + 255) & ~uint64_t(255);
+}
+// Piece lists too long for a CTA's shared memory go to a spill area right
+// before the unit table: per CTA rank, U + P pieces of 3 int32 (a pair's
+// pieces are the units its range meets; pair p's list starts at entry
+// first_unit(p) + p, so the lists of consecutive pairs never overlap).
+inline uint64_t balanced_spill_bytes(int64_t units, int pairs) {
+  return ((uint64_t)2 * (units + pairs) * 12 + 255) & ~uint64_t(255);
 }
 
 // Everything a launch needs, validated by the ABI layer.
@@ -48,6 +56,9 @@ struct DecodeArgs {
   float* lse_part;         // fp32 [B*T*H, S]       (split_kv > 1)
   int32_t* sched;          // balanced schedule table (MLA_SCHEDULE_BALANCED), else null
   int32_t* unit_done;      // balanced: [U] finished-piece counts, [U] table-ready flag; else null
+  int32_t* pieces;         // balanced: piece-list spill area; else null
+  const int32_t* cu_q;     // ragged queries: [B + 1] token offsets of the entries; decode: null
+  int64_t total_q;         // query tokens in q (B * q_len for decode)
 };
 
 // Pair of the balanced schedule whose range holds pair tile x (0 <= x < W):
@@ -62,7 +73,7 @@ __host__ __device__ inline int64_t balanced_lo(int p, int64_t W, int np) { retur
 int cuda_failure(cudaError_t e);
 
 int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, int split_kv,
-              int fold, int kernel, mla_plan* plan);
+              int fold, int kernel, int varlen, mla_plan* plan);
 
 cudaError_t launch_simt_partial(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_tc_partial(const DecodeArgs& a, cudaStream_t stream);      // 16-bit inputs

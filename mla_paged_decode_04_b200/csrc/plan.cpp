@@ -13,9 +13,16 @@
 // with one CTA pair per two SMs (74 pairs per wave on 148 SMs), and take the
 // cheapest. The result is memoised per shape.
 //
-// The FP8 CTA-pair kernel instead keeps all 74 pairs resident and balances
-// the work on the device (MLA_SCHEDULE_BALANCED): the plan only fixes the
-// number of pairs and sizes the partial slots and the schedule table.
+// The CTA-pair kernels instead keep all 74 pairs resident and balance the
+// work on the device (MLA_SCHEDULE_BALANCED): the plan only fixes the number
+// of pairs and sizes the partial slots, the piece spill and the schedule
+// table.
+//
+// Ragged queries (prefill; tokenspeed-mla package card, "What it is and what
+// it does": variable-length sequences without padding): q_len is the longest
+// entry's token count, F the largest fold with H * F <= 128 (it need not
+// divide q_len, an entry's last group holds the remainder) and every entry
+// gets ceil(q_len / F) groups; groups past an entry's tokens are empty.
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -65,12 +72,12 @@ void choose_split(int64_t units, int64_t tiles, int64_t slots_per_wave, int forc
 }
 
 std::mutex g_mu;
-std::map<std::tuple<int, int, int, int, int, int, int, int>, mla_plan> g_memo;
+std::map<std::tuple<int, int, int, int, int, int, int, int, int>, mla_plan> g_memo;
 
 }  // namespace
 
 int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, int split_kv,
-              int fold, int kernel, mla_plan* plan) {
+              int fold, int kernel, int varlen, mla_plan* plan) {
   if (!plan) return MLA_ERR_INVALID_ARG;
   if (batch < 0 || q_len < 1 || num_heads < 1 || max_seq_len < 0 || split_kv < 0 || fold < 0)
     return MLA_ERR_INVALID_ARG;
@@ -82,7 +89,8 @@ int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, i
   if (num_heads > MLA_MAX_ROWS) return MLA_ERR_UNSUPPORTED_SHAPE;
   if (max_seq_len > (1 << 30)) return MLA_ERR_UNSUPPORTED_SHAPE;
 
-  auto key = std::make_tuple(batch, q_len, num_heads, max_seq_len, dtype, split_kv, fold, kernel);
+  if (varlen && kernel == MLA_KERNEL_TCGEN05_SOLO) return MLA_ERR_UNSUPPORTED_SHAPE;
+  auto key = std::make_tuple(batch, q_len, num_heads, max_seq_len, dtype, split_kv, fold, kernel, varlen);
   {
     std::lock_guard<std::mutex> lk(g_mu);
     auto it = g_memo.find(key);
@@ -92,18 +100,21 @@ int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, i
     }
   }
 
+  // Ragged queries (prefill): q_len is the longest entry, and an entry's last
+  // group may hold fewer than F tokens, so F need not divide q_len.
   int F = 0;
   if (fold > 0) {
-    if (q_len % fold != 0 || num_heads * fold > MLA_MAX_ROWS) return MLA_ERR_UNSUPPORTED_SHAPE;
+    if (fold > q_len || (!varlen && q_len % fold != 0) || num_heads * fold > MLA_MAX_ROWS)
+      return MLA_ERR_UNSUPPORTED_SHAPE;
     F = fold;
   } else {
     for (int f = q_len; f >= 1; --f)
-      if (q_len % f == 0 && num_heads * f <= MLA_MAX_ROWS) {
+      if ((varlen || q_len % f == 0) && num_heads * f <= MLA_MAX_ROWS) {
         F = f;
         break;
       }
   }
-  const int G = q_len / F;
+  const int G = (q_len + F - 1) / F;
   const int M = num_heads * F;
   int kern = kernel == MLA_KERNEL_AUTO ? MLA_KERNEL_TCGEN05 : kernel;
   const int64_t units = (int64_t)batch * G;
@@ -127,10 +138,15 @@ int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, i
   // The balanced schedule (CTA-pair kernels) keeps a per-pair piece list in
   // shared memory; far more units than pairs can hold fall back to fixed
   // splits (FP8: the solo kernel; 16-bit: the exchange kernel).
-  if (kern == MLA_KERNEL_TCGEN05 && dtype == MLA_FP8_E4M3 && units > kMaxBalancedUnits)
-    kern = MLA_KERNEL_TCGEN05_SOLO;
+  p.varlen = varlen ? 1 : 0;
+  const int64_t max_units = varlen ? kMaxVarlenUnits : kMaxBalancedUnits;
+  if (kern == MLA_KERNEL_TCGEN05 && units > max_units) {
+    // ragged queries run only on the balanced schedule (or the SIMT kernel)
+    if (varlen) return MLA_ERR_UNSUPPORTED_SHAPE;
+    if (dtype == MLA_FP8_E4M3) kern = MLA_KERNEL_TCGEN05_SOLO;
+  }
   p.kernel = kern;
-  if (kern == MLA_KERNEL_TCGEN05 && units <= kMaxBalancedUnits) {
+  if (kern == MLA_KERNEL_TCGEN05 && units <= max_units) {
     const int P = split_kv > 0 ? (split_kv < kNumSMs / 2 ? split_kv : kNumSMs / 2) : kNumSMs / 2;
     p.schedule = MLA_SCHEDULE_BALANCED;
     p.split_kv = P;
@@ -144,7 +160,8 @@ int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, i
     p.lse_offset = off;
     off += slots * (uint64_t)M * sizeof(float);
     off = (off + 255) & ~uint64_t(255);
-    off += balanced_table_bytes(units);  // unit start table, at the end of the workspace
+    off += balanced_spill_bytes(units, P);  // piece lists too long for shared memory
+    off += balanced_table_bytes(units);     // unit start table, at the end of the workspace
     p.workspace_bytes = off;
   } else {
     p.schedule = MLA_SCHEDULE_SPLITS;
@@ -178,11 +195,21 @@ int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, i
 
 extern "C" int mla_decode_plan(int batch, int q_len, int num_heads, int max_seq_len, int dtype,
                                mla_plan* plan) {
-  return mla::plan_impl(batch, q_len, num_heads, max_seq_len, dtype, 0, 0, MLA_KERNEL_AUTO, plan);
+  return mla::plan_impl(batch, q_len, num_heads, max_seq_len, dtype, 0, 0, MLA_KERNEL_AUTO, 0, plan);
 }
 
 extern "C" int mla_decode_plan_custom(int batch, int q_len, int num_heads, int max_seq_len,
                                       int dtype, int split_kv, int fold, int kernel,
                                       mla_plan* plan) {
-  return mla::plan_impl(batch, q_len, num_heads, max_seq_len, dtype, split_kv, fold, kernel, plan);
+  return mla::plan_impl(batch, q_len, num_heads, max_seq_len, dtype, split_kv, fold, kernel, 0, plan);
+}
+
+extern "C" int mla_prefill_plan(int batch, int max_q_len, int num_heads, int max_seq_len, int dtype,
+                                mla_plan* plan) {
+  return mla::plan_impl(batch, max_q_len, num_heads, max_seq_len, dtype, 0, 0, MLA_KERNEL_AUTO, 1, plan);
+}
+
+extern "C" int mla_prefill_plan_custom(int batch, int max_q_len, int num_heads, int max_seq_len, int dtype,
+                                       int split_kv, int fold, int kernel, mla_plan* plan) {
+  return mla::plan_impl(batch, max_q_len, num_heads, max_seq_len, dtype, split_kv, fold, kernel, 1, plan);
 }

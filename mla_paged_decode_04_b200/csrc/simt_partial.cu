@@ -16,14 +16,14 @@ namespace {
 template <int DT>
 __global__ void __launch_bounds__(256) simt_partial_kernel(const DecodeArgs a) {
   const mla_plan& p = a.plan;
-  const int S = p.split_kv, G = p.q_groups, T = p.q_len, H = p.num_heads;
-  const int M = p.rows_per_unit;
+  const int S = p.split_kv, G = p.q_groups, H = p.num_heads;
   int idx = blockIdx.x;
   const int g = idx % G;
   idx /= G;
   const int s = idx % S;
   const int b = idx / S;
-  const int n = effective_seq_len(a, b, s == 0 && g == 0 && threadIdx.x == 0);
+  const UnitGeom ug = unit_geom(a, b * G + g, s == 0 && threadIdx.x == 0);
+  const int n = ug.n;
   const int key0 = s * p.keys_per_split;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (key0 >= n) {
@@ -31,8 +31,8 @@ __global__ void __launch_bounds__(256) simt_partial_kernel(const DecodeArgs a) {
     // written here, so an entry without keys still gets out = 0, lse = -inf.
     // (With several splits the combine kernel writes those rows.)
     if (S == 1) {
-      for (int m = warp; m < M; m += 8) {
-        const int64_t row = (int64_t)b * T * H + (int64_t)g * M + m;
+      for (int m = warp; m < ug.rows; m += 8) {
+        const int64_t row = ug.row0 + m;
         __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + row * MLA_D_V;
         for (int i = lane; i < MLA_D_V; i += 32) out[i] = __float2bfloat16_rn(0.f);
         if (a.lse && lane == 0) a.lse[row] = -INFINITY;
@@ -43,10 +43,10 @@ __global__ void __launch_bounds__(256) simt_partial_kernel(const DecodeArgs a) {
   const int key1 = min(n, key0 + p.keys_per_split);
   const int32_t* table = a.block_tables + (int64_t)b * a.max_pages_per_seq;
 
-  for (int m = warp; m < M; m += 8) {
-    const int t = g * p.fold + m / H;
-    const int64_t row = (int64_t)b * T * H + (int64_t)g * M + m;
-    const int jend = min(key1, n - T + t + 1);  // causal: keys <= n - T + t
+  for (int m = warp; m < ug.rows; m += 8) {
+    const int last = ug.nq + m / H;  // causal: keys <= last
+    const int64_t row = ug.row0 + m;
+    const int jend = min(key1, last + 1);
     float qv[MLA_D_QK / 32];
 #pragma unroll
     for (int i = 0; i < MLA_D_QK / 32; ++i) qv[i] = load_elem<DT>(a.q, row * MLA_D_QK + lane + 32 * i);
@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(256) simt_partial_kernel(const DecodeArgs a) {
     float o[MLA_D_V / 32];
 #pragma unroll
     for (int i = 0; i < MLA_D_V / 32; ++i) o[i] = 0.f;
-    for (int j = max(key0, window_row_lo(p, t, n)); j < jend; ++j) {  // sliding window: the row's last keys
+    for (int j = max(key0, row_key_lo(p, last)); j < jend; ++j) {  // sliding window: the row's last keys
       const int page = table[j / kTileKeys];
       if (page < 0 || (int64_t)page >= a.num_pages) {
         if (lane == 0) atomicOr(a.status, MLA_DEV_BAD_PAGE);

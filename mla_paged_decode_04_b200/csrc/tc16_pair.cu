@@ -32,6 +32,7 @@
 
 #include "device_common.cuh"
 #include "sm100_ptx.cuh"
+#include "pair_schedule.cuh"
 #include "tc_common.cuh"
 
 namespace mla {
@@ -41,20 +42,9 @@ using namespace ptx;
 
 constexpr float kTau = 4.f;          // lazy-rescale threshold (log2 units)
 constexpr float kSigma = 8.f;        // P <= 2^(kTau + kSigma) = 4096, inside FP16's range
-constexpr int kMaxPieces = 64;       // pieces per pair (units its range touches)
-constexpr int kMinPairTiles = 2;     // fewer tiles than this per pair: use fewer pairs
 constexpr int kHalfKeys = 32;        // keys per CTA per pair tile
 constexpr int kTile16 = 64;          // keys per pair tile (one page)
 
-struct Piece {
-  int u, t0, t1;  // pair tiles [t0, t1) of unit u
-};
-struct SchedInfo {
-  int npc;  // pieces of this pair
-  int pad;
-};
-constexpr uint32_t kSchedBytes = 1024;
-static_assert(kMaxPieces * sizeof(Piece) + sizeof(SchedInfo) <= kSchedBytes, "schedule area");
 
 struct Layout16 {
   static constexpr int NK = 3;                                  // K-ring slots: this CTA's half page
@@ -125,110 +115,30 @@ struct Pair16Params {
   DecodeArgs a;
 };
 
-// Pair tiles of unit u (= b * G + g): one per 64-key page of entry b, from
-// the page of the lowest key the group's rows see (its sliding window's start).
-__device__ __forceinline__ int unit_tiles16(const DecodeArgs& a, int u, bool flag) {
-  const int n = effective_seq_len(a, u / a.plan.q_groups, flag);
-  const int tlo = window_unit_lo(a.plan, u % a.plan.q_groups, n) / kTile16;
-  return (n + kTile16 - 1) / kTile16 - tlo;
-}
-
-// One warp: the balanced schedule of this pair (the FP8 kernel's, with
-// 64-key pair tiles). CTA 0 of pair 0 also writes the unit start table the
-// combine reads, then its ready flag.
-__device__ void build_schedule16(const DecodeArgs& a, int pair, uint32_t rank, Piece* pcs, SchedInfo* info) {
-  const mla_plan& p = a.plan;
-  const int lane = threadIdx.x & 31;
-  const int U = p.batch * p.q_groups;
-  const int per = (U + 31) / 32;
-  const int u_beg = min(U, lane * per), u_end = min(U, u_beg + per);
-  const bool writer = pair == 0 && rank == 0;
-  int run = 0;
-  for (int u = u_beg; u < u_end; ++u) run += unit_tiles16(a, u, writer && u % p.q_groups == 0);
-  int excl = run;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, excl, d);
-    if (lane >= d) excl += y;
-  }
-  const int W = __shfl_sync(0xffffffffu, excl, 31);
-  excl -= run;
-  const int np = max(1, min(p.split_kv, (W + kMinPairTiles - 1) / kMinPairTiles));
-  const int64_t lo = pair < np ? balanced_lo(pair, W, np) : W;
-  const int64_t hi = pair < np ? balanced_lo(pair + 1, W, np) : W;
-  if (writer) {
-    int start = excl;
-    for (int u = u_beg; u < u_end; ++u) {
-      a.sched[u] = start;
-      start += unit_tiles16(a, u, false);
-    }
-    if (lane == 31) {
-      a.sched[U] = W;
-      a.sched[U + 1] = np;
-    }
-    __syncwarp();
-    if (lane == 0) {
-      __threadfence();
-      st_release_gpu(a.unit_done + U, 1);
-    }
-  }
-  int cnt = 0;
-  {
-    int start = excl;
-    for (int u = u_beg; u < u_end; ++u) {
-      const int t = unit_tiles16(a, u, false);
-      if (t > 0 && start < hi && start + t > lo) ++cnt;
-      start += t;
-    }
-  }
-  int base = cnt;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, base, d);
-    if (lane >= d) base += y;
-  }
-  const int npc = __shfl_sync(0xffffffffu, base, 31);
-  base -= cnt;
-  {
-    int start = excl, k = base;
-    for (int u = u_beg; u < u_end; ++u) {
-      const int t = unit_tiles16(a, u, false);
-      if (t > 0 && start < hi && start + t > lo) {
-        if (k < kMaxPieces) {
-          pcs[k].u = u;
-          pcs[k].t0 = lo > start ? (int)(lo - start) : 0;
-          pcs[k].t1 = hi - start < t ? (int)(hi - start) : t;
-        }
-        ++k;
-      }
-      start += t;
-    }
-  }
-  if (lane == 0) info->npc = npc;
-}
-
 // Per-piece constants every role derives the same way.
 struct PieceCtx16 {
-  int b, g, n, key0, key1, n_pt, page0;
+  int b, g, n, nq, rows, key0, key1, n_pt, page0;
   int64_t row0;
   const int32_t* table;
   bool whole;  // the piece is the whole unit: final output, not a partial
 };
 
 __device__ __forceinline__ PieceCtx16 piece_ctx16(const DecodeArgs& a, const Piece& pc) {
-  const mla_plan& p = a.plan;
   PieceCtx16 c;
-  c.b = pc.u / p.q_groups;
-  c.g = pc.u % p.q_groups;
-  c.n = effective_seq_len(a, c.b, false);
-  const int tlo = window_unit_lo(p, c.g, c.n) / kTile16;  // the unit's first page
+  const UnitGeom ug = unit_geom(a, pc.u, false);
+  c.b = ug.b;
+  c.g = ug.g;
+  c.n = ug.n;
+  c.nq = ug.nq;
+  c.rows = ug.rows;
+  const int tlo = ug.klo / kTile16;  // the unit's first page
   c.key0 = (tlo + pc.t0) * kTile16;
-  c.key1 = min(c.n, (tlo + pc.t1) * kTile16);
+  c.key1 = min(ug.kend, (tlo + pc.t1) * kTile16);
   c.n_pt = pc.t1 - pc.t0;
   c.page0 = tlo + pc.t0;  // block-table index of the piece's first page
-  c.row0 = (int64_t)c.b * p.q_len * p.num_heads + (int64_t)c.g * p.rows_per_unit;
+  c.row0 = ug.row0;
   c.table = a.block_tables + (int64_t)c.b * a.max_pages_per_seq;
-  c.whole = pc.t0 == 0 && c.key1 >= c.n;
+  c.whole = pc.t0 == 0 && c.key1 >= ug.kend;
   return c;
 }
 
@@ -243,7 +153,8 @@ __device__ __forceinline__ int valid_page16(const DecodeArgs& a, int pg) {
 }
 
 template <bool kBf16>
-__device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* smem, const Piece* pcs, int npc) {
+__device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* smem, int npc,
+                                           int n_all) {
   using L = Layout16;
   constexpr int NK = L::NK, NV = L::NV, NQ = L::NQ;
   const DecodeArgs& a = prm.a;
@@ -256,7 +167,7 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();  // 0 = leader
   const int pair = blockIdx.x >> 1;
-  const int T = p.q_len, H = p.num_heads, M = p.rows_per_unit;
+  const int H = p.num_heads, M = p.rows_per_unit;
   const int box_q = M < 64 ? M : 64;  // query rows per TMA box
   auto slot_of = [&](int k) -> int64_t { return 2 * (int64_t)pair + (k == 0 ? 0 : 1); };
   auto lead = [&](int i) -> uint32_t { return mapa(bar(i), 0); };
@@ -313,8 +224,6 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
   cluster_sync();  // both CTAs' barriers and TMEM exist before any cross-CTA use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  int n_all = 0;  // pair tiles over all pieces
-  for (int k = 0; k < npc; ++k) n_all += pcs[k].t1 - pcs[k].t0;
 
   if (warp == 0) {
     // ------------------------------------------------------------ Q and K-ring loads
@@ -327,7 +236,7 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
       int jt = 0;
       bool ok = true;
       for (int k = 0; ok && k < npc; ++k) {
-        const PieceCtx16 c = piece_ctx16(a, pcs[k]);
+        const PieceCtx16 c = piece_ctx16(a, load_piece(a, smem, k));
         if (k > 0) {
           // the Q areas and the staging slots are free once every MMA of the
           // previous piece is done: its O_FINAL phase
@@ -367,7 +276,7 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
       int jt = 0;
       bool ok = true;
       for (int k = 0; ok && k < npc; ++k) {
-        const PieceCtx16 c = piece_ctx16(a, pcs[k]);
+        const PieceCtx16 c = piece_ctx16(a, load_piece(a, smem, k));
         int e_nx = piece_entry16(c, 0);
         for (int j = 0; j < c.n_pt; ++j, ++jt) {
           const int sv = jt % NV;
@@ -395,7 +304,8 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
       int jt = 0;
       bool ok = true;
       for (int k = 0; ok && k < npc; ++k) {
-        const int n_pt = pcs[k].t1 - pcs[k].t0;
+        const Piece pk = load_piece(a, smem, k);
+        const int n_pt = pk.t1 - pk.t0;
         if (!(ok = warp_wait(bar(L::B_Q_TMEM), k & 1, abort_flag, a.status))) break;
         for (int j = 0; j < n_pt; ++j, ++jt) {
           const int sk = jt % NK, buf = jt & 1;
@@ -443,7 +353,8 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
       int jt = 0;
       bool ok = true;
       for (int k = 0; ok && k < npc; ++k) {
-        const int n_pt = pcs[k].t1 - pcs[k].t0;
+        const Piece pk = load_piece(a, smem, k);
+        const int n_pt = pk.t1 - pk.t0;
         if (k > 0 && !(ok = warp_wait(bar(L::B_O_FREE), (k - 1) & 1, abort_flag, a.status))) break;
         for (int j = 0; j < n_pt; ++j, ++jt) {
           const int buf = jt & 1, sv = jt % NV;
@@ -487,10 +398,12 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
     int jt = 0;  // running index of the piece's first tile
 
     for (int k = 0; ok && k < npc; ++k) {
-      const PieceCtx16 c = piece_ctx16(a, pcs[k]);
+      const PieceCtx16 c = piece_ctx16(a, load_piece(a, smem, k));
       const bool last_piece = k == npc - 1;
-      const int limit = min((r < M) ? c.n - T + c.g * p.fold + r / H : c.n - 1, c.key1 - 1);
-      const int lower = (r < M) ? window_row_lo(p, c.g * p.fold + r / H, c.n) : 0;  // sliding window
+      // causal limit and sliding-window start of this row (rows past the
+      // unit compute on whatever Q holds and are never stored)
+      const int limit = (r < c.rows) ? min(c.nq + r / H, c.key1 - 1) : c.key1 - 1;
+      const int lower = (r < c.rows) ? row_key_lo(p, c.nq + r / H) : 0;
 
       // Q dims 0..255 (and, group 0, the rope) of local row rl into TMEM:
       // lane quarters q and q^2 both hold rows 32(q%2)..; group g copies
@@ -514,7 +427,7 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
           w[4 * u + 2] = v.z;
           w[4 * u + 3] = v.w;
         }
-        if (r >= M) {
+        if (r >= c.rows) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) w[i] = 0;
         }
@@ -679,7 +592,7 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
       tc_fence_after();
       const float inv = (le > 0.f) ? a.v_scale / le : 0.f;
       const int64_t slot = slot_of(k);
-      if (r < M && grp == 0 && hf == 0) {
+      if (r < c.rows && grp == 0 && hf == 0) {
         const float lse_val = (le > 0.f) ? (m_fin - kSigma + log2f(le)) * kLn2 : -INFINITY;
         if (c.whole) {
           if (a.lse) a.lse[c.row0 + r] = lse_val;
@@ -697,7 +610,7 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
           uint32_t o[32];
           tmem_ld32(tmem + tl + kOCol + 128u * grp + 32u * cc, o);
           tmem_wait_ld();
-          if (r >= M) continue;
+          if (r >= c.rows) continue;
           const int col = 256 * grp + 128 * hf + 32 * cc;
           if (c.whole) {
             uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + (c.row0 + r) * MLA_D_V + col);
@@ -732,7 +645,7 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
           __syncwarp();
           if (lane == 0) {
             __threadfence();
-            atomicAdd(a.unit_done + pcs[k].u, 1);
+            atomicAdd(a.unit_done + load_piece(a, smem, k).u, 1);
           }
         }
         if (!last_piece) {
@@ -771,7 +684,7 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
 #pragma unroll 1
         for (int i = 0; i < 8; ++i) {
           const int rr = 8 * w8 + i;
-          if (64 * (int)rank + rr >= M) break;  // rows past the unit belong to no output
+          if (64 * (int)rank + rr >= c.rows) break;  // rows past the unit belong to no output
           const float inv2 = rowinv[rr];
           const int rr_u = 64 * (int)rank + rr;  // row within the unit
           const float* srow = stage + rr * MLA_D_V;
@@ -844,20 +757,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     return;
   }
   uint8_t* smem = smem_raw;
-  Piece* pcs = reinterpret_cast<Piece*>(smem);
-  SchedInfo* info = reinterpret_cast<SchedInfo*>(smem + kMaxPieces * sizeof(Piece));
-  if (threadIdx.x < 32) build_schedule16(prm.a, blockIdx.x >> 1, cluster_ctarank(), pcs, info);
+  SchedInfo* info = reinterpret_cast<SchedInfo*>(smem + kMaxSmemPieces * sizeof(Piece));
+  if (threadIdx.x < 32)
+    build_schedule<kTile16>(prm.a, blockIdx.x >> 1, cluster_ctarank(), reinterpret_cast<Piece*>(smem), info, 0);
   __syncthreads();
   const int npc = info->npc;
   if (npc == 0) return;  // no work for this pair (the same in both CTAs)
-  if (npc > kMaxPieces) {  // cannot happen within the planner's unit limit
-    if (threadIdx.x == 0) atomicOr(prm.a.status, MLA_DEV_TIMEOUT);
-    return;
-  }
   if (prm.a.plan.dtype == MLA_BF16)
-    pair_cta16<true>(prm, smem, pcs, npc);
+    pair_cta16<true>(prm, smem, npc, info->tiles);
   else
-    pair_cta16<false>(prm, smem, pcs, npc);
+    pair_cta16<false>(prm, smem, npc, info->tiles);
 }
 
 }  // namespace
@@ -867,7 +776,7 @@ cudaError_t launch_tc16_pair_partial(const DecodeArgs& a, cudaStream_t stream) {
   if (p.batch == 0 || p.split_kv < 1) return cudaSuccess;
   Pair16Params prm;
   prm.a = a;
-  const uint64_t q_rows = (uint64_t)p.batch * p.q_len * p.num_heads;
+  const uint64_t q_rows = (uint64_t)a.total_q * p.num_heads;  // the packed query rows
   const uint64_t kv_rows = (uint64_t)a.num_pages * kTileKeys;
   const uint32_t box_q = p.rows_per_unit < 64 ? (uint32_t)p.rows_per_unit : 64u;
   const uint8_t* kv = static_cast<const uint8_t*>(a.kv_cache);

@@ -62,6 +62,7 @@
 #include <cuda.h>
 
 #include "device_common.cuh"
+#include "pair_schedule.cuh"
 #include "sm100_ptx.cuh"
 #include "tc_common.cuh"
 
@@ -73,20 +74,8 @@ using namespace ptx;
 constexpr int kTwoTermKeys = 16384;  // entries shorter than this use two-term P
 constexpr float kTau = 4.f;          // lazy-rescale threshold (log2 units)
 constexpr float kSigma = 4.f;        // P <= 2^(kTau + kSigma) = 256 <= 448
-constexpr int kMaxPieces = 64;       // pieces per pair (units its range touches)
-constexpr int kMinPairTiles = 2;     // fewer tiles than this per pair: use fewer pairs
-
-// One piece: pair tiles [t0, t1) of unit u.
-struct Piece {
-  int u, t0, t1;
-};
-struct SchedInfo {
-  int npc;  // pieces of this pair
-  int two;  // some piece needs two-term P
-};
-// Schedule area at the start of shared memory (the same place in both layouts).
-constexpr uint32_t kSchedBytes = 1024;
-static_assert(kMaxPieces * sizeof(Piece) + sizeof(SchedInfo) <= kSchedBytes, "schedule area");
+// The schedule area (pair_schedule.cuh) is at the start of shared memory, the
+// same place in both layouts.
 
 template <bool kTwo>
 struct PairLayout {
@@ -163,129 +152,40 @@ struct PairParams {
   DecodeArgs a;
 };
 
-// Most keys a row of an entry with n keys attends to (its window, if shorter):
-// the length the two-term P choice looks at.
-__device__ __forceinline__ int row_keys(const DecodeArgs& a, int n) {
-  return (a.plan.window > 0 && a.plan.window < n) ? a.plan.window : n;
-}
-
-// Pair tiles of unit u (= b * G + g): from the tile of the lowest key the
-// group's rows see (0, or its sliding window's start) to the entry's end.
-__device__ __forceinline__ int unit_tiles(const DecodeArgs& a, int u, bool flag) {
-  const int n = effective_seq_len(a, u / a.plan.q_groups, flag);
-  const int tlo = window_unit_lo(a.plan, u % a.plan.q_groups, n) / kPairTileKeys;
-  return (n + kPairTileKeys - 1) / kPairTileKeys - tlo;
-}
-
-// One warp: the balanced schedule of this pair. Every lane takes a run of
-// consecutive units and a warp scan gives each run's first tile; the pieces
-// of the pair's range [lo, hi) go to `pcs` in unit order. CTA 0 of pair 0
-// also writes the unit start table the combine reads.
-__device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, Piece* pcs, SchedInfo* info) {
-  const mla_plan& p = a.plan;
-  const int lane = threadIdx.x & 31;
-  const int U = p.batch * p.q_groups;
-  const int per = (U + 31) / 32;
-  const int u_beg = min(U, lane * per), u_end = min(U, u_beg + per);
-  const bool writer = pair == 0 && rank == 0;
-  int run = 0;
-  for (int u = u_beg; u < u_end; ++u) run += unit_tiles(a, u, writer && u % p.q_groups == 0);
-  int excl = run;  // inclusive prefix, then exclusive
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, excl, d);
-    if (lane >= d) excl += y;
-  }
-  const int W = __shfl_sync(0xffffffffu, excl, 31);
-  excl -= run;
-  const int np = max(1, min(p.split_kv, (W + kMinPairTiles - 1) / kMinPairTiles));
-  const int64_t lo = pair < np ? balanced_lo(pair, W, np) : W;
-  const int64_t hi = pair < np ? balanced_lo(pair + 1, W, np) : W;
-  if (writer) {
-    int start = excl;
-    for (int u = u_beg; u < u_end; ++u) {
-      a.sched[u] = start;
-      start += unit_tiles(a, u, false);
-    }
-    if (lane == 31) {
-      a.sched[U] = W;
-      a.sched[U + 1] = np;
-    }
-    // the table is complete: the combine (which may already run) reads it
-    // once this flag is set
-    __syncwarp();
-    if (lane == 0) {
-      __threadfence();
-      st_release_gpu(a.unit_done + U, 1);
-    }
-  }
-  // pieces: units of this lane's run that meet [lo, hi)
-  int cnt = 0;
-  {
-    int start = excl;
-    for (int u = u_beg; u < u_end; ++u) {
-      const int t = unit_tiles(a, u, false);
-      if (t > 0 && start < hi && start + t > lo) ++cnt;
-      start += t;
-    }
-  }
-  int base = cnt;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, base, d);
-    if (lane >= d) base += y;
-  }
-  const int npc = __shfl_sync(0xffffffffu, base, 31);
-  base -= cnt;
-  int two = 0;
-  {
-    int start = excl, k = base;
-    for (int u = u_beg; u < u_end; ++u) {
-      const int t = unit_tiles(a, u, false);
-      if (t > 0 && start < hi && start + t > lo) {
-        if (k < kMaxPieces) {
-          pcs[k].u = u;
-          pcs[k].t0 = lo > start ? (int)(lo - start) : 0;
-          pcs[k].t1 = hi - start < t ? (int)(hi - start) : t;
-          if (row_keys(a, effective_seq_len(a, u / p.q_groups, false)) < kTwoTermKeys) two = 1;
-        }
-        ++k;
-      }
-      start += t;
-    }
-  }
-  two = __any_sync(0xffffffffu, two);
-  if (lane == 0) {
-    info->npc = npc;
-    info->two = two;
-  }
-}
-
 // Per-piece constants every role derives the same way.
 struct PieceCtx {
-  int b, g, n, key0, key1, n_pt, n_tiles, tile0;
+  int b, g, n, nq, rows, key0, key1, n_pt, n_tiles, tile0;
   int64_t row0;
   const int32_t* table;
   bool whole;  // the piece is the whole unit: final output, not a partial
   bool two;    // two-term P
 };
 
+// The unit geometry as a call, not inlined into every role: the roles' code
+// stays smaller, which measured ~3% faster on the 80K-key FP8 batch (the
+// kernel is sensitive to instruction-cache layout; the 16-bit kernel measured
+// faster with it inlined).
+__device__ __noinline__ UnitGeom unit_geom_call(const DecodeArgs& a, int u) { return unit_geom(a, u, false); }
+
 __device__ __forceinline__ PieceCtx piece_ctx(const DecodeArgs& a, const Piece& pc, bool kTwo) {
   const mla_plan& p = a.plan;
   PieceCtx c;
-  c.b = pc.u / p.q_groups;
-  c.g = pc.u % p.q_groups;
-  c.n = effective_seq_len(a, c.b, false);
-  const int tlo = window_unit_lo(p, c.g, c.n) / kPairTileKeys;  // the unit's first pair tile
+  const UnitGeom ug = unit_geom_call(a, pc.u);
+  c.b = ug.b;
+  c.g = ug.g;
+  c.n = ug.n;
+  c.nq = ug.nq;
+  c.rows = ug.rows;
+  const int tlo = ug.klo / kPairTileKeys;  // the unit's first pair tile
   c.key0 = (tlo + pc.t0) * kPairTileKeys;
-  c.key1 = min(c.n, (tlo + pc.t1) * kPairTileKeys);
+  c.key1 = min(ug.kend, (tlo + pc.t1) * kPairTileKeys);
   c.n_pt = pc.t1 - pc.t0;
   c.n_tiles = (c.key1 - c.key0 + kTileKeys - 1) / kTileKeys;
   c.tile0 = c.key0 / kTileKeys;
-  c.row0 = (int64_t)c.b * p.q_len * p.num_heads + (int64_t)c.g * p.rows_per_unit;
+  c.row0 = ug.row0;
   c.table = a.block_tables + (int64_t)c.b * a.max_pages_per_seq;
-  c.whole = pc.t0 == 0 && c.key1 >= c.n;
-  c.two = kTwo && row_keys(a, c.n) < kTwoTermKeys;
+  c.whole = pc.t0 == 0 && c.key1 >= ug.kend;
+  c.two = kTwo && ((p.window > 0 && p.window < c.n) ? p.window : c.n) < kTwoTermKeys;
   return c;
 }
 
@@ -301,7 +201,8 @@ __device__ __forceinline__ int valid_page(const DecodeArgs& a, int pg) {
 }
 
 template <bool kTwo>
-__device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, const Piece* pcs, int npc) {
+__device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, int npc,
+                                         int n_all) {
   using L = PairLayout<kTwo>;
   constexpr int NK = L::NK, NV = L::NV, NQ = L::NQ;
   const DecodeArgs& a = prm.a;
@@ -314,7 +215,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();  // 0 = leader
   const int pair = blockIdx.x >> 1;
-  const int T = p.q_len, H = p.num_heads, M = p.rows_per_unit;
+  const int H = p.num_heads, M = p.rows_per_unit;
   const int box_q = M < 64 ? M : 64;  // query rows per TMA box (the tensor maps' box height)
   // slot of piece k: 2p for the pair's first piece, 2p + 1 for its last
   auto slot_of = [&](int k) -> int64_t { return 2 * (int64_t)pair + (k == 0 ? 0 : 1); };
@@ -378,8 +279,6 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
   cluster_sync();  // both CTAs' barriers and TMEM exist before any cross-CTA use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  int n_all = 0;  // pair tiles over all pieces
-  for (int k = 0; k < npc; ++k) n_all += pcs[k].t1 - pcs[k].t0;
 
   if (warp == 0) {
     // ------------------------------------------------------------ Q and K-ring loads
@@ -393,7 +292,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
       int jt = 0;     // tile counter across pieces
       bool ok = true;
       for (int k = 0; ok && k < npc; ++k) {
-        const PieceCtx c = piece_ctx(a, pcs[k], kTwo);
+        const PieceCtx c = piece_ctx(a, load_piece(a, smem, k), kTwo);
         if (k > 0) {
           // Q rope, Q in TMEM and the staging slot are free once every MMA of
           // the previous piece is done: its O_FINAL phase. (The V ring's own
@@ -435,7 +334,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
       int jt = 0;
       bool ok = true;
       for (int k = 0; ok && k < npc; ++k) {
-        const PieceCtx c = piece_ctx(a, pcs[k], kTwo);
+        const PieceCtx c = piece_ctx(a, load_piece(a, smem, k), kTwo);
         int e0_nx = piece_entry(c, 0), e1_nx = piece_entry(c, 1);
         for (int j = 0; j < c.n_pt; ++j, ++jt) {
           const int sv = jt % NV;
@@ -468,7 +367,8 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
       int jt = 0;
       bool ok = true;
       for (int k = 0; ok && k < npc; ++k) {
-        const int n_pt = pcs[k].t1 - pcs[k].t0;
+        const Piece pk = load_piece(a, smem, k);
+        const int n_pt = pk.t1 - pk.t0;
         if (!(ok = warp_wait(bar(L::B_Q_ROPE), k & 1, abort_flag, a.status) &&
                    warp_wait(bar(L::B_Q_TMEM), k & 1, abort_flag, a.status)))
           break;
@@ -504,7 +404,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
       int jt = 0;
       bool ok = true;
       for (int k = 0; ok && k < npc; ++k) {
-        const PieceCtx c = piece_ctx(a, pcs[k], kTwo);
+        const PieceCtx c = piece_ctx(a, load_piece(a, smem, k), kTwo);
         // the piece's first P.V overwrites O: the previous piece's epilogue
         // must have read it
         if (k > 0 && !(ok = warp_wait(bar(L::B_O_FREE), (k - 1) & 1, abort_flag, a.status))) break;
@@ -556,10 +456,12 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
     int jt = 0;  // running index of the piece's first tile
 
     for (int k = 0; ok && k < npc; ++k) {
-      const PieceCtx c = piece_ctx(a, pcs[k], kTwo);
+      const PieceCtx c = piece_ctx(a, load_piece(a, smem, k), kTwo);
       const bool last_piece = k == npc - 1;
-      const int limit = min((r < M) ? c.n - T + c.g * p.fold + r / H : c.n - 1, c.key1 - 1);
-      const int lower = (r < M) ? window_row_lo(p, c.g * p.fold + r / H, c.n) : 0;  // sliding window
+      // causal limit and sliding-window start of this row (rows past the
+      // unit compute on whatever Q holds and are never stored)
+      const int limit = (r < c.rows) ? min(c.nq + r / H, c.key1 - 1) : c.key1 - 1;
+      const int lower = (r < c.rows) ? row_key_lo(p, c.nq + r / H) : 0;
 
       // Q latent dims of local row rl into TMEM (A operand of S = Q.K^T): lane
       // quarters q and q^2 both hold rows 32(q%2)..; group g copies chunks
@@ -582,7 +484,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
           w[4 * u + 2] = v.z;
           w[4 * u + 3] = v.w;
         }
-        if (r >= M) {
+        if (r >= c.rows) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) w[i] = 0;
         }
@@ -765,7 +667,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
       tc_fence_after();
       const float inv = (le > 0.f) ? a.v_scale / le : 0.f;
       const int64_t slot = slot_of(k);
-      if (r < M && grp == 0 && hf == 0) {
+      if (r < c.rows && grp == 0 && hf == 0) {
         const float lse_val = (le > 0.f) ? (m_fin - kSigma + log2f(le)) * kLn2 : -INFINITY;
         if (c.whole) {
           if (a.lse) a.lse[c.row0 + r] = lse_val;
@@ -783,7 +685,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
           uint32_t o[32];
           tmem_ld32(tmem + tl + kOCol + 128u * grp + 32u * cc, o);
           tmem_wait_ld();
-          if (r >= M) continue;
+          if (r >= c.rows) continue;
           const int col = 256 * grp + 128 * hf + 32 * cc;
           if (c.whole) {
             uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + (c.row0 + r) * MLA_D_V + col);
@@ -818,7 +720,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
           __syncwarp();
           if (lane == 0) {
             __threadfence();
-            atomicAdd(a.unit_done + pcs[k].u, 1);
+            atomicAdd(a.unit_done + load_piece(a, smem, k).u, 1);
           }
         }
         if (!last_piece) {
@@ -857,7 +759,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, c
 #pragma unroll 1
         for (int i = 0; i < 8; ++i) {
           const int rr = 8 * w8 + i;
-          if (64 * (int)rank + rr >= M) break;  // rows past the unit belong to no output
+          if (64 * (int)rank + rr >= c.rows) break;  // rows past the unit belong to no output
           const float inv2 = rowinv[rr];
           const int rr_u = 64 * (int)rank + rr;  // row within the unit
           const float* srow = stage + rr * MLA_D_V;
@@ -924,22 +826,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Piece* pcs = reinterpret_cast<Piece*>(smem);
-  SchedInfo* info = reinterpret_cast<SchedInfo*>(smem + kMaxPieces * sizeof(Piece));
-  if (threadIdx.x < 32) build_schedule(prm.a, blockIdx.x >> 1, cluster_ctarank(), pcs, info);
+  SchedInfo* info = reinterpret_cast<SchedInfo*>(smem + kMaxSmemPieces * sizeof(Piece));
+  if (threadIdx.x < 32)
+    build_schedule<kPairTileKeys>(prm.a, blockIdx.x >> 1, cluster_ctarank(), reinterpret_cast<Piece*>(smem), info,
+                                  kTwoTermKeys);
   __syncthreads();
   const int npc = info->npc;
   if (npc == 0) return;  // no work for this pair (the same in both CTAs)
-  if (npc > kMaxPieces) {  // cannot happen within the planner's unit limit
-    if (threadIdx.x == 0) atomicOr(prm.a.status, MLA_DEV_TIMEOUT);
-    return;
-  }
   // Short entries send P as two E4M3 terms; a pair with any such piece takes
   // the layout with room for both planes (the choice is the same in both CTAs).
   if (info->two)
-    pair_cta<true>(prm, smem, pcs, npc);
+    pair_cta<true>(prm, smem, npc, info->tiles);
   else
-    pair_cta<false>(prm, smem, pcs, npc);
+    pair_cta<false>(prm, smem, npc, info->tiles);
 }
 
 }  // namespace
@@ -949,7 +848,7 @@ cudaError_t launch_tc_fp8_pair_partial(const DecodeArgs& a, cudaStream_t stream)
   if (p.batch == 0 || p.split_kv < 1) return cudaSuccess;
   PairParams prm;
   prm.a = a;
-  const uint64_t q_rows = (uint64_t)p.batch * p.q_len * p.num_heads;
+  const uint64_t q_rows = (uint64_t)a.total_q * p.num_heads;  // the packed query rows
   const uint64_t kv_rows = (uint64_t)a.num_pages * kTileKeys;
   const uint32_t box_q = p.rows_per_unit < 64 ? (uint32_t)p.rows_per_unit : 64u;
   if (!encode_rows_576(&prm.tm_q_main, a.q, 1, q_rows, 128, box_q, CU_TENSOR_MAP_SWIZZLE_128B) ||

@@ -226,3 +226,107 @@ def kv_bytes(inp: DecodeInputs) -> int:
     """Bytes of distinct cache rows a decode step must read (each token once)."""
     esize = 1 if inp.dtype == "fp8" else 2
     return inp.kv_tokens() * D_QK * esize
+
+
+# ---------------------------------------------------------------- ragged prefill
+@dataclasses.dataclass
+class PrefillInputs:
+    """A ragged prefill step: entry b's q_lens[b] new tokens (packed in q) extend a cached
+    prefix of prefix_lens[b] tokens; seq_lens = prefix + new, all already in the cache."""
+    q: torch.Tensor             # [total_q, H, 576]
+    cu_seqlens_q: torch.Tensor  # int32 [B + 1]
+    kv_cache: torch.Tensor
+    block_tables: torch.Tensor
+    seq_lens: torch.Tensor
+    dtype: str
+    softmax_scale: float
+    q_scale: float = 1.0
+    kv_scale: float = 1.0
+    max_q_len: int = 0
+    max_seq_len: int = 0
+    name: str = "custom"
+
+    @property
+    def batch(self) -> int:
+        return int(self.seq_lens.shape[0])
+
+    @property
+    def heads(self) -> int:
+        return int(self.q.shape[1])
+
+    @property
+    def total_q(self) -> int:
+        return int(self.q.shape[0])
+
+    def to(self, device) -> "PrefillInputs":
+        return dataclasses.replace(self, q=self.q.to(device), cu_seqlens_q=self.cu_seqlens_q.to(device),
+                                   kv_cache=self.kv_cache.to(device), block_tables=self.block_tables.to(device),
+                                   seq_lens=self.seq_lens.to(device))
+
+
+@dataclasses.dataclass(frozen=True)
+class PrefillWorkload:
+    name: str
+    seed: int
+    batch: int
+    heads: int
+    dtype: str
+    q_lens: tuple      # ("uniform", lo, hi)
+    prefix: tuple      # ("uniform", lo, hi)
+    max_q_len: int
+    max_seq_len: int
+    desc: str
+
+
+PREFILL_WORKLOADS = {
+    w.name: w
+    for w in [
+        PrefillWorkload("prefill_fp8", 2001, 8, 32, "fp8", ("uniform", 512, 4096), ("uniform", 0, 16384),
+                        4096, 16384 + 4096,
+                        "FP8 ragged prefill: B=8, H=32, new tokens U[512,4096], cached prefix U[0,16384]"),
+        PrefillWorkload("prefill_bf16", 2002, 8, 32, "bf16", ("uniform", 512, 4096), ("uniform", 0, 16384),
+                        4096, 16384 + 4096,
+                        "BF16 ragged prefill: B=8, H=32, new tokens U[512,4096], cached prefix U[0,16384]"),
+    ]
+}
+
+
+def make_prefill_inputs(q_lens: Sequence[int], prefix_lens: Sequence[int], heads: int, dtype: str, *,
+                        seed: int, pool=1.5, q_std: float = 1.0, kv_std: float = 1.0,
+                        max_q_len: Optional[int] = None, max_seq_len: Optional[int] = None,
+                        name: str = "custom", device="cpu") -> PrefillInputs:
+    """Seeded ragged prefill inputs: packed q [sum q_lens, H, 576], cu_seqlens_q, a permuted page
+    pool of `pool` x the pages needed, block tables and seq_lens = prefix + new tokens."""
+    g = torch.Generator(device=device).manual_seed(int(seed))
+    ql = [int(x) for x in q_lens]
+    sl = torch.tensor([int(a) + int(b) for a, b in zip(ql, prefix_lens)], dtype=torch.int32)
+    B = len(ql)
+    cu = torch.zeros(B + 1, dtype=torch.int32)
+    if B:
+        cu[1:] = torch.cumsum(torch.tensor(ql, dtype=torch.int64), 0).to(torch.int32)
+    pages_needed = [(int(n) + PAGE_SIZE - 1) // PAGE_SIZE for n in sl.tolist()]
+    num_pages = max(1, int(math.ceil(float(pool) * sum(pages_needed))))
+    width = max(1, max(pages_needed) if pages_needed else 1)
+    q, q_scale = _draw((max(int(cu[-1]), 0), heads, D_QK), g, q_std, dtype)
+    cache, kv_scale = _draw((num_pages, PAGE_SIZE, D_QK), g, kv_std, dtype)
+    perm = torch.randperm(num_pages, generator=g, device=g.device).to(torch.int32).cpu()
+    bt = torch.full((B, width), -1, dtype=torch.int32)
+    off = 0
+    for b, npg in enumerate(pages_needed):
+        bt[b, :npg] = perm[off:off + npg]
+        off += npg
+    return PrefillInputs(q=q, cu_seqlens_q=cu, kv_cache=cache, block_tables=bt, seq_lens=sl, dtype=dtype,
+                         softmax_scale=D_QK ** -0.5, q_scale=q_scale, kv_scale=kv_scale,
+                         max_q_len=int(max_q_len if max_q_len is not None else max(ql + [1])),
+                         max_seq_len=int(max_seq_len if max_seq_len is not None else (int(sl.max()) if B else 0)),
+                         name=name)
+
+
+def make_prefill_workload(name: str, device="cpu") -> PrefillInputs:
+    """Inputs of a named ragged prefill workload (lengths from its seed, on the CPU)."""
+    w = PREFILL_WORKLOADS[name]
+    gl = torch.Generator().manual_seed(w.seed)
+    ql = torch.randint(w.q_lens[1], w.q_lens[2] + 1, (w.batch,), generator=gl).tolist()
+    pre = torch.randint(w.prefix[1], w.prefix[2] + 1, (w.batch,), generator=gl).tolist()
+    return make_prefill_inputs(ql, pre, w.heads, w.dtype, seed=w.seed + 1, pool=1.5, max_q_len=w.max_q_len,
+                               max_seq_len=w.max_seq_len, name=name, device=device)

@@ -156,6 +156,44 @@ def mla_decode(q, kv_cache, block_tables, seq_lens, softmax_scale, *, dtype,
     return out, lse
 
 
+def mla_prefill(q, cu_seqlens_q, kv_cache, block_tables, seq_lens, softmax_scale, *, dtype,
+                q_scale=1.0, kv_scale=1.0, rows=None, window=0):
+    """Oracle ragged (prefill) attention over the paged cache.
+
+    tokenspeed-mla package card, "What it is and what it does": prefill of
+    variable-length sequences packed without padding. Entry b's new tokens
+    are q[cu[b]:cu[b+1]] (q: [total_q, H, D]); token t of the entry sees keys
+    0 .. seq_lens[b] - q_len_b + t, which is the decode definition with
+    q_len = q_len_b, so each entry is one call of `mla_decode`.
+    rows: optional packed row indices token*H + h (each inside some entry).
+    Returns (out [n_rows, 512] float64, lse [n_rows] float64).
+    """
+    cu = [int(x) for x in np.asarray(cu_seqlens_q).reshape(-1)]
+    total_q, H, D = (int(x) for x in q.shape)
+    B = len(cu) - 1
+    bt = np.asarray(block_tables, dtype=np.int32)
+    sl = np.asarray(seq_lens, dtype=np.int32)
+    all_rows = np.arange(total_q * H) if rows is None else np.asarray(rows, dtype=np.int64).reshape(-1)
+    out = np.zeros((all_rows.size, 512))
+    lse = np.zeros(all_rows.size)
+    tok = all_rows // H
+    done = np.zeros(all_rows.size, dtype=bool)
+    for b in range(B):
+        s, e = cu[b], cu[b + 1]
+        sel = np.nonzero((tok >= s) & (tok < e))[0]
+        if sel.size == 0:
+            continue
+        qb = q[s:e].reshape(1, e - s, H, D)
+        o, l = mla_decode(qb, kv_cache, bt[b:b + 1], sl[b:b + 1], softmax_scale, dtype=dtype,
+                          q_scale=q_scale, kv_scale=kv_scale, rows=all_rows[sel] - s * H, window=window)
+        out[sel] = o
+        lse[sel] = l
+        done[sel] = True
+    if not done.all():
+        raise ValueError("a requested row lies outside every entry")
+    return out, lse
+
+
 def lse_merge(o_parts, lse_parts):
     """Merge per-split partials of one row: returns (out [Dv], lse)."""
     o = np.ascontiguousarray(np.asarray(o_parts, dtype=np.float64))

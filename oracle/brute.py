@@ -52,3 +52,34 @@ def mla_decode_brute(q, kv_cache, block_tables, seq_lens, softmax_scale,
                 outs.append([math.fsum(w[j] * keys[j][d] for j in range(len(keys))) for d in range(Dv)])
                 lses.append(lse)
     return outs, lses
+
+
+def mla_prefill_brute(q, cu_seqlens_q, kv_cache, block_tables, seq_lens, softmax_scale,
+                      q_scale=1.0, kv_scale=1.0):
+    """Ragged prefill written out directly: packed token i of entry b (cu[b] <= i < cu[b+1])
+    sees keys 0 .. seq_lens[b] - (cu[b+1] - cu[b]) + (i - cu[b]). q [total_q, H, D]."""
+    total_q, H, D = (int(x) for x in q.shape)
+    _, page, _ = (int(x) for x in kv_cache.shape)
+    qrows = _as_floats(q, q_scale)
+    cache_rows = _as_floats(kv_cache, kv_scale)
+    cu = [int(x) for x in cu_seqlens_q.tolist()]
+    bt = [[int(x) for x in row] for row in block_tables.tolist()]
+    sl = [int(x) for x in seq_lens.tolist()]
+    outs, lses = {}, {}
+    for b in range(len(cu) - 1):
+        qlen = cu[b + 1] - cu[b]
+        for i in range(cu[b], cu[b + 1]):
+            last = sl[b] - qlen + (i - cu[b])  # highest visible key
+            for h in range(H):
+                qv = qrows[i * H + h]
+                if last < 0:
+                    outs[i * H + h], lses[i * H + h] = [0.0] * 512, -math.inf
+                    continue
+                keys = [cache_rows[bt[b][j // page] * page + j % page] for j in range(last + 1)]
+                s = [softmax_scale * math.fsum(qv[d] * k[d] for d in range(D)) for k in keys]
+                m = max(s)
+                lse = m + math.log(math.fsum(math.exp(x - m) for x in s))
+                w = [math.exp(x - lse) for x in s]
+                outs[i * H + h] = [math.fsum(w[j] * keys[j][d] for j in range(len(keys))) for d in range(512)]
+                lses[i * H + h] = lse
+    return outs, lses

@@ -126,3 +126,31 @@ def test_decode_rejects_a_window_the_plan_cannot_run():
     bad = _lib.MlaPlan.from_buffer_copy(solo)
     bad.window = 64
     assert _call(bad) == -6
+
+
+def _prefill_call(plan, cu=FAKE, total_q=8, **kw):
+    args = dict(q=FAKE, kv=FAKE, num_pages=8, page_size=64, bt=FAKE, maxp=4, sl=FAKE,
+                scale=0.04, qs=1.0, ks=1.0, out=FAKE, lse=FAKE, ws=FAKE, ws_bytes=1 << 30)
+    args.update(kw)
+    vp = ctypes.c_void_p
+    return _lib.lib().mla_prefill(ctypes.byref(plan), vp(args["q"]), total_q, vp(cu), vp(args["kv"]),
+                                  args["num_pages"], args["page_size"], vp(args["bt"]), args["maxp"],
+                                  vp(args["sl"]), args["scale"], args["qs"], args["ks"], vp(args["out"]),
+                                  vp(args["lse"]), vp(args["ws"]), args["ws_bytes"], None)
+
+
+def test_prefill_and_decode_refuse_each_others_plans():
+    pre = mla.mla_prefill_plan(2, 4, 32, 256, "fp8")
+    dec = mla.mla_decode_plan(2, 4, 32, 256, "fp8")
+    assert _call(pre) == -6                  # a ragged plan needs cu_seqlens_q
+    assert _prefill_call(dec) == -6          # a decode plan has no ragged queries
+    assert _prefill_call(pre, cu=0) == -1    # null cu_seqlens_q
+    assert _prefill_call(pre, total_q=9) == -1   # more tokens than batch x max_q_len
+    assert _prefill_call(pre, total_q=-1) == -1
+    assert _prefill_call(pre, cu=FAKE + 2) == -1  # cu_seqlens_q not 4-byte aligned
+    bad = _lib.MlaPlan.from_buffer_copy(pre)
+    bad.varlen = 2
+    assert _prefill_call(bad) == -6
+    bad = _lib.MlaPlan.from_buffer_copy(pre)
+    bad.kernel = 3  # the solo kernel has no ragged form
+    assert _prefill_call(bad) == -6

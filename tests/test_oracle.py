@@ -364,3 +364,57 @@ def test_window_ignores_keys_before_its_start():
         inp.kv_cache[int(bt[j // 64]), j % 64] = 7.0
     o1, l1 = _decode(inp, window=50)
     assert np.array_equal(o0, o1) and np.array_equal(l0, l1)
+
+
+# ---------------------------------------------------------------- ragged prefill
+# tokenspeed-mla package card, "What it is and what it does": prefill of
+# variable-length sequences packed without padding. Entry b's token t sees keys
+# 0 .. seq_lens[b] - q_len_b + t.
+
+from oracle.brute import mla_prefill_brute  # noqa: E402
+from mla_paged_decode_04_b200.inputs import make_prefill_inputs  # noqa: E402
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_prefill_matches_the_brute_force_loop(dtype):
+    # an empty entry, one token, a new sequence (no prefix), tokens spanning two pages
+    inp = make_prefill_inputs([3, 0, 1, 5], [2, 4, 0, 60], 2, dtype, seed=71, pool=2.0)
+    o, l = oracle.mla_prefill(inp.q, inp.cu_seqlens_q, inp.kv_cache, inp.block_tables, inp.seq_lens,
+                              inp.softmax_scale, dtype=dtype, q_scale=inp.q_scale, kv_scale=inp.kv_scale)
+    bo, bl = mla_prefill_brute(inp.q, inp.cu_seqlens_q, inp.kv_cache, inp.block_tables, inp.seq_lens,
+                               inp.softmax_scale, inp.q_scale, inp.kv_scale)
+    assert sorted(bo) == list(range(inp.total_q * inp.heads))
+    for r in range(inp.total_q * inp.heads):
+        assert np.allclose(o[r], bo[r], rtol=0, atol=1e-12)
+        assert abs(l[r] - bl[r]) <= 1e-12
+
+
+def test_prefill_token_is_a_single_token_decode_of_its_prefix():
+    """Each new token's row equals a q_len = 1 decode over the keys up to its own position."""
+    inp = make_prefill_inputs([4, 2, 7], [0, 9, 130], 3, "fp16", seed=72, pool=1.5)
+    o, l = oracle.mla_prefill(inp.q, inp.cu_seqlens_q, inp.kv_cache, inp.block_tables, inp.seq_lens,
+                              inp.softmax_scale, dtype="fp16")
+    cu, H = inp.cu_seqlens_q.tolist(), inp.heads
+    for b in range(inp.batch):
+        qlen = cu[b + 1] - cu[b]
+        for i in range(cu[b], cu[b + 1]):
+            n_i = int(inp.seq_lens[b]) - qlen + (i - cu[b]) + 1
+            d_o, d_l = oracle.mla_decode(inp.q[i].reshape(1, 1, H, 576), inp.kv_cache, inp.block_tables[b:b + 1],
+                                         torch.tensor([n_i], dtype=torch.int32), inp.softmax_scale, dtype="fp16")
+            assert np.allclose(o[i * H:(i + 1) * H], d_o, rtol=0, atol=1e-12)
+            assert np.allclose(l[i * H:(i + 1) * H], d_l, rtol=0, atol=1e-12)
+
+
+def test_prefill_rows_before_any_key_are_empty_and_rows_subset_matches():
+    inp = make_prefill_inputs([5, 3], [0, 40], 2, "bf16", seed=73)
+    sl = inp.seq_lens.clone()
+    sl[0] = 2  # fewer keys than new tokens: the first three tokens see nothing
+    o, l = oracle.mla_prefill(inp.q, inp.cu_seqlens_q, inp.kv_cache, inp.block_tables, sl, inp.softmax_scale,
+                              dtype="bf16")
+    H = inp.heads
+    assert (o[:3 * H] == 0).all() and np.isneginf(l[:3 * H]).all()
+    assert np.isfinite(l[3 * H:]).all()
+    rows = [15, 0, 9, 3]
+    so, sl_ = oracle.mla_prefill(inp.q, inp.cu_seqlens_q, inp.kv_cache, inp.block_tables, sl, inp.softmax_scale,
+                                 dtype="bf16", rows=rows)
+    assert np.array_equal(so, o[rows]) and np.array_equal(sl_, l[rows])

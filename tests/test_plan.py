@@ -214,3 +214,38 @@ def test_window_is_set_only_on_plans_whose_kernels_support_it():
     with pytest.raises(mla.MlaError) as e:
         mla.mla_decode_plan_window(forged, 8)
     assert e.value.code == -6
+
+
+def test_prefill_plan_folds_without_dividing_and_counts_groups():
+    # ragged queries: the largest F with H * F <= 128, whether or not it divides max_q_len
+    p = mla.mla_prefill_plan(3, 5, 48, 1000, "bf16")
+    assert (p.varlen, p.fold, p.q_groups, p.rows_per_unit, p.schedule) == (1, 2, 3, 96, 1)
+    p = mla.mla_prefill_plan(2, 4096, 32, 20480, "fp8")
+    assert (p.fold, p.q_groups, p.kernel, p.schedule, p.split_kv) == (4, 1024, 1, 1, 74)
+    p = mla.mla_prefill_plan(2, 3, 16, 100, "fp16")  # F = 3 <= max_q_len
+    assert (p.fold, p.q_groups) == (3, 1)
+    # the SIMT cross-check takes fixed splits; the solo FP8 kernel has no ragged form
+    p = mla.mla_prefill_plan(2, 100, 16, 5000, "fp8", kernel="simt")
+    assert (p.varlen, p.schedule, p.kernel) == (1, 0, 2)
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_prefill_plan(2, 100, 16, 5000, "fp8", kernel="tcgen05_solo")
+    assert e.value.code == -2
+    # more than 65536 groups in all
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_prefill_plan(17, 4096, 128, 8192, "bf16")
+    assert e.value.code == -2
+    # a decode plan of the same numbers is not ragged
+    assert mla.mla_decode_plan(2, 4, 32, 100, "bf16").varlen == 0
+
+
+def test_balanced_workspace_holds_the_piece_spill():
+    for units, pairs in ((4, 74), (2048, 74), (65536, 74), (7, 3)):
+        spill = (2 * (units + pairs) * 12 + 255) // 256 * 256
+        table = ((units + 2) * 4 + 255) // 256 * 256
+        assert spill >= 2 * (units + pairs) * 12
+        del table
+    p = mla.mla_prefill_plan(8, 4096, 32, 20480, "fp8")
+    units = 8 * 1024
+    need = (p.lse_offset + 2 * p.split_kv * p.rows_per_unit * 4
+            + (2 * (units + p.split_kv) * 12 + 255) // 256 * 256 + ((units + 2) * 4 + 255) // 256 * 256)
+    assert p.workspace_bytes >= need
