@@ -47,6 +47,8 @@ def parse_args():
     ap.add_argument("--op", default="decode", choices=["decode", "kv_pack", "prefill"],
                     help="decode (the headline) or the fused K/V pack + FP8 quantise kernel")
     ap.add_argument("--kernel", default="auto", choices=["auto", "tcgen05", "simt", "tcgen05_solo"])
+    ap.add_argument("--batch", type=int, default=0,
+                    help="draw the workload with this many entries instead (small cases for ncu captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--clock-window-s", type=float, default=1.5,
@@ -198,7 +200,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
 
     w = WORKLOADS[args.workload]
-    inp = make_inputs(args.workload, device=dev)
+    inp = make_inputs(args.workload, device=dev, batch=args.batch or None)
     g = inp.to(dev)
     B, T, H = g.batch, g.q_len, g.heads
     dec = mla.MlaDecoder(B, T, H, g.max_seq_len, g.dtype, dev, kernel=args.kernel)
@@ -556,7 +558,7 @@ def run_prefill(args):
     dev = torch.device("cuda", local)
     name = args.workload if args.workload in PREFILL_WORKLOADS else "prefill_fp8"
     w = PREFILL_WORKLOADS[name]
-    inp = make_prefill_workload(name, device=dev)
+    inp = make_prefill_workload(name, device=dev, batch=args.batch or None)
     g = inp.to(dev)
     pre = mla.MlaPrefill(g.batch, g.max_q_len, g.heads, g.max_seq_len, g.dtype, dev)
     out = torch.empty((g.total_q, g.heads, 512), dtype=torch.bfloat16, device=dev)

@@ -10,6 +10,7 @@
 // never written and are skipped; a split whose lse is -inf (no visible key)
 // has weight 0; a row with no visible key at all gets out = 0, lse = -inf.
 #include "device_common.cuh"
+#include "pair_schedule.cuh"
 #include "sm100_ptx.cuh"
 
 namespace mla {
@@ -145,8 +146,10 @@ __global__ void __launch_bounds__(256) combine_balanced_kernel(const DecodeArgs 
   const int32_t* tbl = a.sched;
   const int64_t start = tbl[u], end = tbl[u + 1], W = tbl[U];
   const int np = tbl[U + 1];
+  const UnitGeom ug = unit_geom(a, u, false);
+  // pairs holding the unit's first and last tiles (tile starts are weighted)
   const int p0 = end > start ? balanced_pair_of(start, W, np) : 0;
-  const int p1 = end > start ? balanced_pair_of(end - 1, W, np) : 0;
+  const int p1 = end > start ? balanced_pair_of(end - tile_weight(p, ug), W, np) : 0;
   if (end > start && p0 == p1) return;  // a whole unit: written by its pair
   if (end > start) {
     __syncthreads();  // every thread has read s_ok
@@ -157,7 +160,6 @@ __global__ void __launch_bounds__(256) combine_balanced_kernel(const DecodeArgs 
   }
   const int r = (blk % nb) * 32 + (threadIdx.x & 31);       // row within the unit
   const int c4_0 = cb * 16 + (threadIdx.x >> 5) * 2;         // first of this thread's two 16-byte chunks
-  const UnitGeom ug = unit_geom(a, u, false);
   if (r >= ug.rows) return;  // past the unit's rows (an entry's last group under ragged queries)
   const int64_t row = ug.row0 + r;
   uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + row * MLA_D_V + c4_0 * 4);
@@ -167,9 +169,11 @@ __global__ void __launch_bounds__(256) combine_balanced_kernel(const DecodeArgs 
     if (lse_writer) a.lse[row] = -INFINITY;
     return;
   }
-  // The unit is pair p0's first unit only if p0's range starts exactly at
-  // it; every later pair's range starts inside the unit (slot 2q).
-  const int64_t first_slot = balanced_lo(p0, W, np) == start ? 2 * (int64_t)p0 : 2 * (int64_t)p0 + 1;
+  // Pair p0 kept the unit in slot 2p0 if it was its first piece (each pair
+  // records its first unit in the table), else in 2p0 + 1; every later pair
+  // starts inside the unit (slot 2q). Pair p0's record precedes its piece
+  // arrivals, which the counter wait above acquired.
+  const int64_t first_slot = tbl[U + 2 + p0] == u ? 2 * (int64_t)p0 : 2 * (int64_t)p0 + 1;
 
   auto slot = [&](int q) -> int64_t { return q == p0 ? first_slot : 2 * (int64_t)q; };
 

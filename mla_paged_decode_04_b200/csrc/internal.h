@@ -16,10 +16,10 @@ constexpr int kPairTileKeys = 128;              // keys per CTA-pair tile (one p
 constexpr int kMaxBalancedUnits = 2048;         // decode units (entry x query group) the balanced schedule takes
 constexpr int kMaxVarlenUnits = 1 << 16;        // units of a ragged-query (prefill) plan
 
-// Balanced schedule table at the end of the workspace: int32 start tile of
-// every unit (U + 1 entries, the last = W, the total pair tiles), then the
-// number of pairs that have work. Written by the partial kernel, read by the
-// combine.
+// Balanced schedule table at the end of the workspace: int32 weighted start
+// of every unit (U + 1 entries, the last = W, the total tile weight), the
+// number of pairs that have work, then each pair's first unit (-1: none).
+// Written by the partial kernel, read by the combine.
 // Balanced schedule: per-unit counts of finished partial pieces, then the
 // unit table's ready flag; right after the status header, and cleared with it
 // before every launch of the partial kernel.
@@ -28,8 +28,11 @@ inline uint64_t balanced_counter_bytes(int64_t units) {
   return ((uint64_t)(units + 1) * 4 + 255) & ~uint64_t(255);
 }
 inline uint64_t balanced_table_bytes(int64_t units) {
-  return ((uint64_t)(units + 2) * 4 + 255) & ~uint64_t(255);
+  return ((uint64_t)(units + 2 + kNumSMs / 2) * 4 + 255) & ~uint64_t(255);
 }
+// FP8 rows that see fewer keys than this send P as two E4M3 terms (the P.V
+// MMAs run twice); the balanced schedule weighs such tiles 3 against 2.
+constexpr int kTwoTermKeys = 16384;
 // Piece lists too long for a CTA's shared memory go to a spill area right
 // before the unit table: per CTA rank, U + P pieces of 3 int32 (a pair's
 // pieces are the units its range meets; pair p's list starts at entry

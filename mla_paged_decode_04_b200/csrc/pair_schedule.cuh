@@ -2,10 +2,12 @@
 //
 // Every unit (entry, query group) is a run of pair tiles counted from the
 // device seq_lens (and, for ragged queries, cu_q): from the tile of the
-// lowest key a row of the unit sees to the tile of the highest. The units'
-// runs, in unit order, form one sequence of W tiles; pair p takes the
-// contiguous range [floor(W p / np), floor(W (p + 1) / np)) and walks it as a
-// list of pieces (the units its range meets, each cut to the range).
+// lowest key a row of the unit sees to the tile of the highest. A tile
+// weighs 2, or 3 when its P.V runs twice (FP8 two-term P), so that pairs get
+// equal work rather than equal tiles. The units' runs, in unit order, form one
+// sequence of total weight W; pair p takes the tiles whose start lies in
+// [floor(W p / np), floor(W (p + 1) / np)) and walks them as a list of pieces
+// (the units its range meets, each cut to the range).
 #pragma once
 
 #include "device_common.cuh"
@@ -19,31 +21,48 @@ struct Piece {
 };
 struct SchedInfo {
   int npc;         // pieces of this pair
-  int tiles;       // pair tiles of this pair (its range's length)
-  int two;         // some piece's entry is shorter than the two-term threshold
+  int tiles;       // pair tiles of this pair
+  int two;         // some piece has two-term P
   int spill_base;  // piece k >= kMaxSmemPieces is entry spill_base + k of the spill area
 };
 constexpr int kMaxSmemPieces = 64;  // pieces a pair keeps in shared memory; the rest go to the spill area
 constexpr uint32_t kSchedBytes = 1024;
 static_assert(kMaxSmemPieces * sizeof(Piece) + sizeof(SchedInfo) <= kSchedBytes, "schedule area");
-constexpr int kMinPairTiles = 2;  // fewer tiles than this per pair: use fewer pairs
+constexpr int kMinPairWeight = 4;  // pairs get at least this much weight (>= the heaviest tile)
 
-// Pair tiles (of kKeys keys) of unit u.
-template <int kKeys>
-__device__ __forceinline__ int unit_tiles(const DecodeArgs& a, int u, bool flag) {
-  return unit_span_tiles<kKeys>(unit_geom(a, u, flag));
+// Weight of one tile of a unit: 3 when its rows' P goes as two E4M3 terms
+// (FP8 rows that see fewer than kTwoTermKeys keys), else 2.
+__device__ __forceinline__ int tile_weight(const mla_plan& p, const UnitGeom& ug) {
+  if (p.dtype != MLA_FP8_E4M3) return 2;
+  const int seen = (p.window > 0 && p.window < ug.n) ? p.window : ug.n;
+  return seen < kTwoTermKeys ? 3 : 2;
+}
+
+// Tiles [i0, i1) of a unit with `t` tiles of weight `w` starting at weighted
+// position `start` whose own start positions lie in [lo, hi).
+__device__ __forceinline__ void tiles_in_range(int64_t start, int t, int w, int64_t lo, int64_t hi, int& i0,
+                                               int& i1) {
+  const int64_t a0 = lo > start ? (lo - start + w - 1) / w : 0;
+  const int64_t a1 = hi > start ? (hi - start + w - 1) / w : 0;
+  i0 = (int)(a0 < t ? a0 : t);
+  i1 = (int)(a1 < t ? a1 : t);
+}
+
+__device__ __forceinline__ int warp_sum_int(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
 }
 
 // One warp: the schedule of this pair. Every lane takes a run of consecutive
-// units and a warp scan gives each run's first tile; the pieces of the pair's
-// range [lo, hi) are written in unit order, the first kMaxSmemPieces to shared
+// units and a warp scan gives each run's weighted start; the pieces of the
+// pair's range are written in unit order, the first kMaxSmemPieces to shared
 // memory and, when there are more, all of them to this CTA's part of the
 // spill area (read back by load_piece). CTA 0 of pair 0 also writes the unit
-// start table the combine reads, then its ready flag.
-// `two_keys` > 0: report whether a piece's entry lets a row see fewer keys.
+// start table the combine reads, then its ready flag; CTA 0 of every pair
+// records its first unit there (the combine's slot rule).
 template <int kKeys>
-__device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, Piece* smem_list, SchedInfo* info,
-                               int two_keys) {
+__device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, Piece* smem_list, SchedInfo* info) {
   const mla_plan& p = a.plan;
   const int lane = threadIdx.x & 31;
   const int U = p.batch * p.q_groups;
@@ -51,7 +70,10 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, Pie
   const int u_beg = min(U, lane * per), u_end = min(U, u_beg + per);
   const bool writer = pair == 0 && rank == 0;
   int run = 0;
-  for (int u = u_beg; u < u_end; ++u) run += unit_tiles<kKeys>(a, u, writer);
+  for (int u = u_beg; u < u_end; ++u) {
+    const UnitGeom ug = unit_geom(a, u, writer);
+    run += unit_span_tiles<kKeys>(ug) * tile_weight(p, ug);
+  }
   int excl = run;  // inclusive prefix, then exclusive
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
@@ -60,14 +82,15 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, Pie
   }
   const int W = __shfl_sync(0xffffffffu, excl, 31);
   excl -= run;
-  const int np = max(1, min(p.split_kv, (W + kMinPairTiles - 1) / kMinPairTiles));
+  const int np = max(1, min(p.split_kv, W / kMinPairWeight));
   const int64_t lo = pair < np ? balanced_lo(pair, W, np) : W;
   const int64_t hi = pair < np ? balanced_lo(pair + 1, W, np) : W;
   if (writer) {
     int start = excl;
     for (int u = u_beg; u < u_end; ++u) {
       a.sched[u] = start;
-      start += unit_tiles<kKeys>(a, u, false);
+      const UnitGeom ug = unit_geom(a, u, false);
+      start += unit_span_tiles<kKeys>(ug) * tile_weight(p, ug);
     }
     if (lane == 31) {
       a.sched[U] = W;
@@ -81,17 +104,20 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, Pie
       ptx::st_release_gpu(a.unit_done + U, 1);
     }
   }
-  // pieces: units of this lane's run that meet [lo, hi)
+  // pieces: units of this lane's run with tiles in the range
   int cnt = 0, u_first_lane = 0;
   {
     int start = excl;
     for (int u = u_beg; u < u_end; ++u) {
-      const int t = unit_tiles<kKeys>(a, u, false);
-      if (t > 0 && start < hi && start + t > lo) {
+      const UnitGeom ug = unit_geom(a, u, false);
+      const int t = unit_span_tiles<kKeys>(ug), w = tile_weight(p, ug);
+      int i0, i1;
+      tiles_in_range(start, t, w, lo, hi, i0, i1);
+      if (i1 > i0) {
         if (cnt == 0) u_first_lane = u;
         ++cnt;
       }
-      start += t;
+      start += t * w;
     }
   }
   int base = cnt;
@@ -106,32 +132,36 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, Pie
   const int u_first = has ? __shfl_sync(0xffffffffu, u_first_lane, __ffs(has) - 1) : 0;
   const int spill_base = (int)rank * (U + p.split_kv) + u_first + pair;
   Piece* spill = npc > kMaxSmemPieces ? reinterpret_cast<Piece*>(a.pieces) + spill_base : nullptr;
-  int two = 0;
+  int two = 0, tiles = 0;
   {
     int start = excl, k = base;
     for (int u = u_beg; u < u_end; ++u) {
       const UnitGeom ug = unit_geom(a, u, false);
-      const int t = unit_span_tiles<kKeys>(ug);
-      if (t > 0 && start < hi && start + t > lo) {
+      const int t = unit_span_tiles<kKeys>(ug), w = tile_weight(p, ug);
+      int i0, i1;
+      tiles_in_range(start, t, w, lo, hi, i0, i1);
+      if (i1 > i0) {
         Piece pc;
         pc.u = u;
-        pc.t0 = lo > start ? (int)(lo - start) : 0;
-        pc.t1 = hi - start < t ? (int)(hi - start) : t;
+        pc.t0 = i0;
+        pc.t1 = i1;
         if (k < kMaxSmemPieces) smem_list[k] = pc;
         if (spill) spill[k] = pc;
-        const int seen = (p.window > 0 && p.window < ug.n) ? p.window : ug.n;
-        if (two_keys > 0 && seen < two_keys) two = 1;
+        if (w == 3) two = 1;
+        tiles += i1 - i0;
         ++k;
       }
-      start += t;
+      start += t * w;
     }
   }
   two = __any_sync(0xffffffffu, two);
+  tiles = warp_sum_int(tiles);
   if (lane == 0) {
     info->spill_base = spill_base;
     info->npc = npc;
-    info->tiles = (int)(hi - lo);
+    info->tiles = tiles;
     info->two = two;
+    if (rank == 0 && pair < p.split_kv) a.sched[U + 2 + pair] = npc > 0 ? u_first : -1;
   }
 }
 

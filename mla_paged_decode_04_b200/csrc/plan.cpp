@@ -23,6 +23,7 @@
 // entry's token count, F the largest fold with H * F <= 128 (it need not
 // divide q_len, an entry's last group holds the remainder) and every entry
 // gets ceil(q_len / F) groups; groups past an entry's tokens are empty.
+#include <climits>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -139,7 +140,9 @@ int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, i
   // shared memory; far more units than pairs can hold fall back to fixed
   // splits (FP8: the solo kernel; 16-bit: the exchange kernel).
   p.varlen = varlen ? 1 : 0;
-  const int64_t max_units = varlen ? kMaxVarlenUnits : kMaxBalancedUnits;
+  // the balanced schedule's int32 tile weights (3 per 64 keys at most) must fit
+  const bool weights_fit = units * tiles * 3 < (int64_t)INT32_MAX;
+  const int64_t max_units = weights_fit ? (varlen ? kMaxVarlenUnits : kMaxBalancedUnits) : 0;
   if (kern == MLA_KERNEL_TCGEN05 && units > max_units) {
     // ragged queries run only on the balanced schedule (or the SIMT kernel)
     if (varlen) return MLA_ERR_UNSUPPORTED_SHAPE;

@@ -759,7 +759,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw;
   SchedInfo* info = reinterpret_cast<SchedInfo*>(smem + kMaxSmemPieces * sizeof(Piece));
   if (threadIdx.x < 32)
-    build_schedule<kTile16>(prm.a, blockIdx.x >> 1, cluster_ctarank(), reinterpret_cast<Piece*>(smem), info, 0);
+    build_schedule<kTile16>(prm.a, blockIdx.x >> 1, cluster_ctarank(), reinterpret_cast<Piece*>(smem), info);
   __syncthreads();
   const int npc = info->npc;
   if (npc == 0) return;  // no work for this pair (the same in both CTAs)

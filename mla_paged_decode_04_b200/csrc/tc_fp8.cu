@@ -48,7 +48,6 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kTwoTermKeys = 16384;        // entries shorter than this use two-term P
 constexpr float kTau = 2.f;                // lazy-rescale threshold (log2 units)
 constexpr float kSigma = 6.f;              // P <= 2^(kTau + kSigma) = 256 <= 448
 

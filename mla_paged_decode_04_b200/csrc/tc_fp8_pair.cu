@@ -71,7 +71,6 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kTwoTermKeys = 16384;  // entries shorter than this use two-term P
 constexpr float kTau = 4.f;          // lazy-rescale threshold (log2 units)
 constexpr float kSigma = 4.f;        // P <= 2^(kTau + kSigma) = 256 <= 448
 // The schedule area (pair_schedule.cuh) is at the start of shared memory, the
@@ -828,8 +827,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   SchedInfo* info = reinterpret_cast<SchedInfo*>(smem + kMaxSmemPieces * sizeof(Piece));
   if (threadIdx.x < 32)
-    build_schedule<kPairTileKeys>(prm.a, blockIdx.x >> 1, cluster_ctarank(), reinterpret_cast<Piece*>(smem), info,
-                                  kTwoTermKeys);
+    build_schedule<kPairTileKeys>(prm.a, blockIdx.x >> 1, cluster_ctarank(), reinterpret_cast<Piece*>(smem), info);
   __syncthreads();
   const int npc = info->npc;
   if (npc == 0) return;  // no work for this pair (the same in both CTAs)

@@ -182,14 +182,18 @@ def make_inputs_custom(batch: int, q_len: int, heads: int, dtype: str,
                   max_pages, name, softmax_scale)
 
 
-def make_inputs(name: str, device="cpu") -> DecodeInputs:
+def make_inputs(name: str, device="cpu", batch: Optional[int] = None) -> DecodeInputs:
     """Inputs of a named workload (see WORKLOADS), seed 1000 + config number.
 
     The generator lives on ``device``: the bytes are reproducible per device
     type, and the oracle always consumes the same bytes as the GPU path.
-    Small tensors (block tables, seq_lens) are returned on the CPU.
+    Small tensors (block tables, seq_lens) are returned on the CPU. `batch`
+    draws the same distributions with that many entries (a smaller case of
+    the workload, e.g. for profiler captures).
     """
     w = WORKLOADS[name]
+    if batch is not None:
+        w = dataclasses.replace(w, batch=int(batch))
     g = torch.Generator(device=device).manual_seed(1000 + w.config)
     sl = draw_seq_lens(w, g)
     return _build(w.batch, w.q_len, w.heads, w.dtype, sl, g, w.pool, w.q_std, w.kv_std,
@@ -322,9 +326,12 @@ def make_prefill_inputs(q_lens: Sequence[int], prefix_lens: Sequence[int], heads
                          name=name)
 
 
-def make_prefill_workload(name: str, device="cpu") -> PrefillInputs:
-    """Inputs of a named ragged prefill workload (lengths from its seed, on the CPU)."""
+def make_prefill_workload(name: str, device="cpu", batch: Optional[int] = None) -> PrefillInputs:
+    """Inputs of a named ragged prefill workload (lengths from its seed, on the CPU); `batch`
+    draws that many entries of the same distributions instead."""
     w = PREFILL_WORKLOADS[name]
+    if batch is not None:
+        w = dataclasses.replace(w, batch=int(batch))
     gl = torch.Generator().manual_seed(w.seed)
     ql = torch.randint(w.q_lens[1], w.q_lens[2] + 1, (w.batch,), generator=gl).tolist()
     pre = torch.randint(w.prefix[1], w.prefix[2] + 1, (w.batch,), generator=gl).tolist()

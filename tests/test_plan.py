@@ -85,40 +85,56 @@ def test_balanced_plan_uses_every_sm_and_caps_units():
     assert big16.schedule == 0 and big16.kernel == 1
 
 
-def _balanced_schedule(tiles, P, min_tiles=2):
-    """Host model of the device schedule: unit starts, pairs with work, each pair's pieces."""
+def _balanced_schedule(tiles, P, weights=None, min_weight=4):
+    """Host model of the device schedule: a tile weighs 2, or 3 with FP8 two-term P; pair p takes
+    the tiles whose weighted start lies in [W p / np, W (p + 1) / np). Returns unit starts, W,
+    np, each pair's pieces (u, t0, t1) and each pair's first unit (-1: none)."""
+    weights = weights or [2] * len(tiles)
     starts = [0]
-    for t in tiles:
-        starts.append(starts[-1] + t)
+    for t, w in zip(tiles, weights):
+        starts.append(starts[-1] + t * w)
     W = starts[-1]
-    np_ = max(1, min(P, -(-W // min_tiles)))
+    np_ = max(1, min(P, W // min_weight))
     pieces = []
     for p in range(P):
         lo, hi = (W * p // np_, W * (p + 1) // np_) if p < np_ else (W, W)
         pp = []
-        for u, t in enumerate(tiles):
-            if t > 0 and starts[u] < hi and starts[u] + t > lo:
-                pp.append((u, max(lo - starts[u], 0), min(hi - starts[u], t)))
+        for u, (t, w) in enumerate(zip(tiles, weights)):
+            s0 = starts[u]
+            i0 = min(t, -(-(lo - s0) // w)) if lo > s0 else 0
+            i1 = min(t, -(-(hi - s0) // w)) if hi > s0 else 0
+            if i1 > i0:
+                pp.append((u, i0, i1))
         pieces.append(pp)
-    return starts, W, np_, pieces
+    first = [pp[0][0] if pp else -1 for pp in pieces]
+    return starts, W, np_, pieces, first
 
 
 def _pair_of(x, W, np_):
     return ((x + 1) * np_ + W - 1) // W - 1
 
 
-@pytest.mark.parametrize("tiles", [[640] * 16, [1, 0, 3, 2], [2] * 2048, [190, 3, 0, 640, 1, 1, 77] * 9,
-                                   [5], [0, 0, 4]])
-def test_balanced_schedule_covers_each_tile_once(tiles):
+_rng = __import__("random").Random(5)
+_MIXED = [_rng.choice([0, 1, 2, 7, 130, 640]) for _ in range(300)]
+
+
+@pytest.mark.parametrize("tiles,weights", [
+    ([640] * 16, None), ([1, 0, 3, 2], None), ([2] * 2048, None), ([190, 3, 0, 640, 1, 1, 77] * 9, None),
+    ([5], None), ([0, 0, 4], None), ([1] * 250 + [157] * 50, None),
+    ([640] * 16, [2, 3] * 8), ([1, 0, 3, 2], [3, 3, 2, 3]), (_MIXED, [_rng.choice([2, 3]) for _ in _MIXED]),
+    ([3] * 1000 + [400] * 7, [3] * 1000 + [2] * 7),
+])
+def test_balanced_schedule_covers_each_tile_once(tiles, weights):
     """Every tile of every unit lies in exactly one piece; a pair leaves at most two partial
-    pieces (its first and last), in slots 2p and 2p + 1; the combine's rule (unit u is pair q's
-    first unit iff q's range starts at or after u) finds the same slots; pieces fit the list."""
+    pieces (its first and last), in slots 2p and 2p + 1; the combine's rule (the pairs of the
+    unit's first and last tile starts; slot 2p0 iff the unit is p0's recorded first unit) finds
+    the same slots, and every pair it waits for holds a piece of the unit."""
     P = 74
-    starts, W, np_, pieces = _balanced_schedule(tiles, P)
+    w_of = weights or [2] * len(tiles)
+    starts, W, np_, pieces, first = _balanced_schedule(tiles, P, weights)
     seen = {}
     slot_of_piece = {}
     for p, pp in enumerate(pieces):
-        assert len(pp) <= 64
         for k, (u, t0, t1) in enumerate(pp):
             for t in range(t0, t1):
                 assert (u, t) not in seen
@@ -133,13 +149,25 @@ def test_balanced_schedule_covers_each_tile_once(tiles):
     for u, t in enumerate(tiles):
         if t == 0:
             continue
-        p0, p1 = _pair_of(starts[u], W, np_), _pair_of(starts[u] + t - 1, W, np_)
+        p0 = _pair_of(starts[u], W, np_)
+        p1 = _pair_of(starts[u + 1] - w_of[u], W, np_)
+        assert seen[(u, 0)] == p0 and seen[(u, t - 1)] == p1
         if p0 == p1:
             assert (u, p0) not in slot_of_piece  # whole: written directly
             continue
         for q in range(p0, p1 + 1):
-            slot = 2 * q if W * q // np_ >= starts[u] else 2 * q + 1
+            assert any(pu == u for pu, _, _ in pieces[q])  # the combine's wait ends
+            slot = (2 * q if first[q] == u else 2 * q + 1) if q == p0 else 2 * q
             assert slot_of_piece[(u, q)] == slot
+
+
+def test_weighted_schedule_evens_out_two_term_work():
+    # half the units have two-term tiles (weight 3): per-pair weight stays within one tile
+    tiles = [100] * 40
+    weights = [3] * 20 + [2] * 20
+    starts, W, np_, pieces, _ = _balanced_schedule(tiles, 74, weights)
+    work = [sum((t1 - t0) * weights[u] for u, t0, t1 in pp) for pp in pieces]
+    assert max(work) - min(work) <= 2 * 3
 
 
 def test_split_fills_the_gpu_for_the_long_fp8_case():
