@@ -61,6 +61,26 @@ def dist_env():
             int(os.environ.get("LOCAL_RANK", "0")))
 
 
+def init_dist(world, dev, backend="nccl", timeout_s=180):
+    """One process per GPU (replicas): a process group only for the barrier and the timing
+    reduction; nothing on the data path crosses ranks."""
+    if world > 1:
+        import torch.distributed as dist
+        kw = {"device_id": dev} if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+
+
+def max_over_ranks(x, world, dev):
+    """The largest of the ranks' values (every rank gets it); x itself on one rank."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------- helpers
 
 def measured_peak():
@@ -196,8 +216,7 @@ def run_ours(args):
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+    init_dist(world, dev)
 
     w = WORKLOADS[args.workload]
     inp = make_inputs(args.workload, device=dev, batch=args.batch or None)
@@ -286,11 +305,7 @@ def run_ours(args):
         raise RuntimeError("device status word set during the timed steps")
     step_ms = [e0.elapsed_time(e1) for e0, e1 in evs]
     part_ms = [e0.elapsed_time(e1) for e0, e1 in pevs]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = total_ms / args.steps
     value = world * kv_bytes * args.steps / (total_ms / 1e3) / 1e9
 
@@ -326,10 +341,7 @@ def run_ours(args):
             ev2[k][1].record()
         torch.cuda.synchronize()
         e2e_ms = sum(a.elapsed_time(b) for a, b in ev2)
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e2e_ms, world, dev)
         e2e = {"value": round(world * kv_bytes * args.steps / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
                "us_per_step": round(e2e_ms / args.steps * 1e3, 2),
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
@@ -481,9 +493,12 @@ def run_kv_pack(args):
     import torch
     import mla_paged_decode_04_b200 as mla
 
+    import torch.distributed as dist
+
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    init_dist(world, dev)
     n = 16 * 81920
     num_pages = 2 * n // 64
     g = torch.Generator(device=dev).manual_seed(4242)
@@ -503,23 +518,30 @@ def run_kv_pack(args):
         for _ in range(20):
             mla.kv_pack(latent, rope, slots, cache, kv_scale=scale)
         torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     for k in range(args.steps):
         evs[k][0].record()
         mla.kv_pack(latent, rope, slots, cache, kv_scale=scale)
         evs[k][1].record()
     torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
     clocks = sampler.stop()
     ms = [a.elapsed_time(b) for a, b in evs]
-    mean_s = statistics.mean(ms) / 1e3
+    mean_s = max_over_ranks(statistics.mean(ms), world, dev) / 1e3
     peak, peak_kind = measured_peak()
     achieved = alg / mean_s / 1e9
+    if world > 1:
+        dist.destroy_process_group()
     if rank != 0:
         return
     line = {
         "metric": "fused K/V pack + FP8 quantise GB/s (inputs + FP8 rows + slots per call)",
-        "value": round(achieved, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(statistics.mean(ms), 5), "higher_is_better": True, "scaling": "weak",
+        "value": round(world * achieved, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(mean_s * 1e3, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16->fp8_e4m3", "data": "synthetic (seeded, generated on device)",
         "config": {"workload": "kv_pack_bf16_fp8", "tokens": n, "num_pages": num_pages,
                    "l2": "inputs larger than L2 (1.5 GB read, 755 MB written per call), no flush"},
@@ -553,9 +575,12 @@ def run_prefill(args):
     import mla_paged_decode_04_b200 as mla
     from mla_paged_decode_04_b200.inputs import PREFILL_WORKLOADS, make_prefill_workload
 
+    import torch.distributed as dist
+
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    init_dist(world, dev)
     name = args.workload if args.workload in PREFILL_WORKLOADS else "prefill_fp8"
     w = PREFILL_WORKLOADS[name]
     inp = make_prefill_workload(name, device=dev, batch=args.batch or None)
@@ -604,10 +629,7 @@ def run_prefill(args):
         raise RuntimeError("device status word set during the timed steps")
     step_ms = [a.elapsed_time(b) for a, b in evs]
     total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     mean_s = total_ms / args.steps / 1e3
     value = world * flops / mean_s / 1e12
 
@@ -642,10 +664,7 @@ def run_prefill(args):
         ev2[k][1].record()
     torch.cuda.synchronize()
     e2e_ms = sum(a.elapsed_time(b) for a, b in ev2)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
     e2e = {"value": round(world * flops / (e2e_ms / args.steps / 1e3) / 1e12, 2), "unit": "TFLOP/s",
            "ms_per_step": round(e2e_ms / args.steps, 4), "h2d_bytes_per_step": int(h2d),
            "d2h_bytes_per_step": int(d2h)}
