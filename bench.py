@@ -380,7 +380,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(args.workload, rows_per_sample=64, repeats=1)
+        cpu = cpu_baseline(args.workload)
 
     if world > 1:
         dist.barrier()
@@ -417,31 +417,33 @@ def run_ours(args):
 
 # ---------------------------------------------------------------- oracle timing
 
-def _oracle_sample_inputs(workload):
+def _oracle_sample_inputs(workload, index=0):
     """One batch entry of the workload, same shape and distributions, drawn on the CPU."""
     from mla_paged_decode_04_b200.inputs import WORKLOADS, make_inputs_custom
     w = WORKLOADS[workload]
     n = w.max_seq_len if w.seq[0] == "fixed" else int(w.seq[1]) if w.seq[0] == "lognormal" else (w.seq[1] + w.seq[2]) // 2
-    return make_inputs_custom(1, w.q_len, w.heads, w.dtype, [n], seed=2000 + w.config,
+    return make_inputs_custom(1, w.q_len, w.heads, w.dtype, [n], seed=2000 + 97 * index + w.config,
                               pool="exact", q_std=w.q_std, kv_std=w.kv_std), n
 
 
-def cpu_baseline(workload, rows_per_sample, repeats):
+def cpu_baseline(workload, target_s=10.0, max_entries=16):
+    """The oracle on the host cores over a bounded sample: whole batch entries of the workload (all
+    their query rows), drawn one at a time until about target_s seconds of oracle time."""
     import oracle
-    inp, n = _oracle_sample_inputs(workload)
-    rows_total = inp.q_len * inp.heads
-    rows = list(range(0, rows_total, max(1, rows_total // rows_per_sample)))[:rows_per_sample]
-    esize = 1 if inp.dtype == "fp8" else 2
-    t0 = time.perf_counter()
-    for _ in range(repeats):
+    t_total, work_bytes, entries, rows_total, n = 0.0, 0, 0, 0, 0
+    while entries < max_entries and (entries == 0 or t_total < target_s):
+        inp, n = _oracle_sample_inputs(workload, entries)
+        rows_total = inp.q_len * inp.heads
+        t0 = time.perf_counter()
         oracle.mla_decode(inp.q, inp.kv_cache, inp.block_tables, inp.seq_lens, inp.softmax_scale,
-                          dtype=inp.dtype, q_scale=inp.q_scale, kv_scale=inp.kv_scale, rows=rows)
-    dt = (time.perf_counter() - t0) / repeats
-    work_bytes = n * 576 * esize * len(rows) / rows_total
-    return {"value": round(work_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
-            "kind": "oracle", "seconds": round(dt, 3),
-            "sample": f"{len(rows)} of the {rows_total} query rows of one batch entry "
-                      f"({n} keys, {inp.dtype}); KV bytes scaled by the row fraction"}
+                          dtype=inp.dtype, q_scale=inp.q_scale, kv_scale=inp.kv_scale)
+        t_total += time.perf_counter() - t0
+        work_bytes += n * 576 * (1 if inp.dtype == "fp8" else 2)
+        entries += 1
+    return {"value": round(work_bytes / t_total / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "seconds": round(t_total, 3),
+            "sample": f"{entries} batch entries of the workload ({n} keys, all {rows_total} query rows each); "
+                      f"KV bytes of those entries over the oracle's time"}
 
 
 def run_reference(args):
@@ -685,18 +687,22 @@ def run_prefill(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         H = g.heads
-        toks = list(range(cu[1] - 8, cu[1])) if g.batch else []  # the last tokens of entry 0: its longest rows
-        rows = [t * H + h for t in toks for h in range(H)]
         hcache = inp.kv_cache.cpu()
-        t0 = time.perf_counter()
-        oracle.mla_prefill(hq, inp.cu_seqlens_q, hcache, inp.block_tables, inp.seq_lens, g.softmax_scale,
-                           dtype=g.dtype, q_scale=g.q_scale, kv_scale=g.kv_scale, rows=rows)
-        dt = time.perf_counter() - t0
-        n0 = int(inp.seq_lens[0])
-        sample_flops = sum(n0 - (cu[1] - cu[0]) + (t - cu[0]) + 1 for t in toks) * H * 2 * (576 + 512)
+        n0, q0 = int(inp.seq_lens[0]), cu[1] - cu[0]
+        dt, sample_flops, ntok, end = 0.0, 0, 0, cu[1]
+        while end > cu[0] and (ntok == 0 or dt < 10.0):  # the last tokens of entry 0 (its longest rows), 8 at a time
+            toks = list(range(max(cu[0], end - 8), end))
+            rows = [t * H + h for t in toks for h in range(H)]
+            t0 = time.perf_counter()
+            oracle.mla_prefill(hq, inp.cu_seqlens_q, hcache, inp.block_tables, inp.seq_lens, g.softmax_scale,
+                               dtype=g.dtype, q_scale=g.q_scale, kv_scale=g.kv_scale, rows=rows)
+            dt += time.perf_counter() - t0
+            sample_flops += sum(n0 - q0 + (t - cu[0]) + 1 for t in toks) * H * 2 * (576 + 512)
+            ntok += len(toks)
+            end -= 8
         cpu = {"value": round(sample_flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
                "kind": "oracle", "seconds": round(dt, 3),
-               "sample": f"{len(rows)} query rows (the last 8 tokens of entry 0, all heads); flops of those rows"}
+               "sample": f"{ntok * H} query rows (the last {ntok} tokens of entry 0, all heads); flops of those rows"}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
