@@ -126,23 +126,12 @@ __device__ bool wait_count(const int32_t* ctr, int target, int32_t* status) {
   return true;
 }
 
-__global__ void __launch_bounds__(256) combine_balanced_kernel(const DecodeArgs a) {
+// Merge of one unit's rows [32 rb, 32 rb + 32) x column block cb (block-
+// uniform u, so every thread takes the same path through the barriers).
+__device__ __forceinline__ void combine_unit(const DecodeArgs& a, int u, int rb, int cb, int* s_ok) {
   const mla_plan& p = a.plan;
   const int M = p.rows_per_unit;
   const int U = p.batch * p.q_groups;
-  // Launched as the partial kernel's programmatic dependent, this block may
-  // start while pairs still run: it waits for the unit table, then for
-  // every piece of its unit (kPieceArrivals arrivals each). Each thread then
-  // acquires the counter itself before reading what it guards.
-  __shared__ int s_ok;
-  if (threadIdx.x == 0) s_ok = wait_count(a.unit_done + U, 1, a.status);
-  __syncthreads();
-  if (!s_ok) return;
-  (void)ptx::ld_acquire_gpu(a.unit_done + U);
-  const int nb = (M + 31) / 32;
-  const int cb = blockIdx.x % kCombineColBlocks;
-  const int blk = blockIdx.x / kCombineColBlocks;
-  const int u = blk / nb;  // the same for the whole block
   const int32_t* tbl = a.sched;
   const int64_t start = tbl[u], end = tbl[u + 1], W = tbl[U];
   const int np = tbl[U + 1];
@@ -153,12 +142,12 @@ __global__ void __launch_bounds__(256) combine_balanced_kernel(const DecodeArgs 
   if (end > start && p0 == p1) return;  // a whole unit: written by its pair
   if (end > start) {
     __syncthreads();  // every thread has read s_ok
-    if (threadIdx.x == 0) s_ok = wait_count(a.unit_done + u, kPieceArrivals * (p1 - p0 + 1), a.status);
+    if (threadIdx.x == 0) *s_ok = wait_count(a.unit_done + u, kPieceArrivals * (p1 - p0 + 1), a.status);
     __syncthreads();
-    if (!s_ok) return;
+    if (!*s_ok) return;
     (void)ptx::ld_acquire_gpu(a.unit_done + u);
   }
-  const int r = (blk % nb) * 32 + (threadIdx.x & 31);       // row within the unit
+  const int r = rb * 32 + (threadIdx.x & 31);       // row within the unit
   const int c4_0 = cb * 16 + (threadIdx.x >> 5) * 2;         // first of this thread's two 16-byte chunks
   if (r >= ug.rows) return;  // past the unit's rows (an entry's last group under ragged queries)
   const int64_t row = ug.row0 + r;
@@ -235,6 +224,34 @@ __global__ void __launch_bounds__(256) combine_balanced_kernel(const DecodeArgs 
   if (lse_writer) a.lse[row] = L;
 }
 
+__global__ void __launch_bounds__(256) combine_balanced_kernel(const DecodeArgs a, int units_per_block) {
+  const mla_plan& p = a.plan;
+  const int M = p.rows_per_unit;
+  const int U = p.batch * p.q_groups;
+  // Launched as the partial kernel's programmatic dependent, this block may
+  // start while pairs still run: it waits for the unit table, then, per unit
+  // of its share, for every piece of the unit (kPieceArrivals arrivals each).
+  // Each thread then acquires the counter itself before reading what it
+  // guards. A block takes units_per_block consecutive units (more than one
+  // only for large unit counts, e.g. ragged prefill), so that blocks of whole
+  // units, which have nothing to merge, do not dominate the grid.
+  __shared__ int s_ok;
+  if (threadIdx.x == 0) s_ok = wait_count(a.unit_done + U, 1, a.status);
+  __syncthreads();
+  if (!s_ok) return;
+  (void)ptx::ld_acquire_gpu(a.unit_done + U);
+  const int nb = (M + 31) / 32;
+  const int cb = blockIdx.x % kCombineColBlocks;
+  const int blk = blockIdx.x / kCombineColBlocks;
+  const int rb = blk % nb;
+  const int u0 = (blk / nb) * units_per_block;
+  for (int u = u0; u < U && u < u0 + units_per_block; ++u) {
+    combine_unit(a, u, rb, cb, &s_ok);
+    __syncthreads();
+    if (!s_ok) return;  // a wait gave up (the same in every thread)
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_combine_balanced(const DecodeArgs& a, cudaStream_t stream) {
@@ -244,8 +261,11 @@ cudaError_t launch_combine_balanced(const DecodeArgs& a, cudaStream_t stream) {
   // programmatic dependent of the partial kernel: blocks take the SMs of
   // pairs that are done and wait for their own unit (the partial kernel
   // never waits for this grid)
+  // about 4096 unit blocks at most: beyond that a block takes several units
+  const int64_t per = (units + 4095) / 4096;
+  const int64_t unit_blocks = (units + per - 1) / per;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(units * nb * kCombineColBlocks));
+  cfg.gridDim = dim3((unsigned)(unit_blocks * nb * kCombineColBlocks));
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
@@ -254,7 +274,7 @@ cudaError_t launch_combine_balanced(const DecodeArgs& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, combine_balanced_kernel, a);
+  return cudaLaunchKernelEx(&cfg, combine_balanced_kernel, a, (int)per);
 }
 
 }  // namespace mla

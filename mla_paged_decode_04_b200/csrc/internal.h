@@ -13,7 +13,7 @@ constexpr int kNumSMs = 148;                    // B200
 constexpr int kHeaderBytes = 256;               // workspace header (status word at offset 0)
 constexpr int kTileKeys = 64;                   // keys per tile = one cache page
 constexpr int kPairTileKeys = 128;              // keys per CTA-pair tile (one page per CTA)
-constexpr int kMaxBalancedUnits = 2048;         // decode units (entry x query group) the balanced schedule takes
+constexpr int kMaxBalancedUnits = 16384;        // decode units (entry x query group) the balanced schedule takes
 constexpr int kMaxVarlenUnits = 1 << 16;        // units of a ragged-query (prefill) plan
 
 // Balanced schedule table at the end of the workspace: int32 weighted start

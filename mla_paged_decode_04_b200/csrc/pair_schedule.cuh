@@ -48,40 +48,59 @@ __device__ __forceinline__ void tiles_in_range(int64_t start, int t, int w, int6
   i1 = (int)(a1 < t ? a1 : t);
 }
 
-__device__ __forceinline__ int warp_sum_int(int v) {
+// Scratch of the block-wide scans, after the piece list and SchedInfo: one int
+// per warp for the first scan, four per warp for the second.
+constexpr int kMaxSchedWarps = 12;  // the CTA-pair kernels run 384 threads
+constexpr uint32_t kSchedScratchOff = 784;
+static_assert(kSchedScratchOff >= kMaxSmemPieces * sizeof(Piece) + sizeof(SchedInfo) &&
+                  kSchedScratchOff + 4 * 5 * kMaxSchedWarps <= kSchedBytes,
+              "schedule scratch");
+
+__device__ __forceinline__ int warp_incl_scan(int v) {
+  const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  for (int d = 1; d < 32; d <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, v, d);
+    if (lane >= d) v += y;
+  }
   return v;
 }
 
-// One warp: the schedule of this pair. Every lane takes a run of consecutive
-// units and a warp scan gives each run's weighted start; the pieces of the
+// The whole block: the schedule of this pair. Every thread takes a run of
+// consecutive units; block scans (two barriers in all) give each run's
+// weighted start and each thread's first piece index. The pieces of the
 // pair's range are written in unit order, the first kMaxSmemPieces to shared
 // memory and, when there are more, all of them to this CTA's part of the
 // spill area (read back by load_piece). CTA 0 of pair 0 also writes the unit
 // start table the combine reads, then its ready flag; CTA 0 of every pair
 // records its first unit there (the combine's slot rule).
 template <int kKeys>
-__device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, Piece* smem_list, SchedInfo* info) {
+__device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uint8_t* sched_area) {
   const mla_plan& p = a.plan;
-  const int lane = threadIdx.x & 31;
+  Piece* smem_list = reinterpret_cast<Piece*>(sched_area);
+  SchedInfo* info = reinterpret_cast<SchedInfo*>(sched_area + kMaxSmemPieces * sizeof(Piece));
+  int* scan1 = reinterpret_cast<int*>(sched_area + kSchedScratchOff);  // [warp]
+  int4* scan2 = reinterpret_cast<int4*>(scan1 + kMaxSchedWarps);       // [warp]: pieces, tiles, two, first unit
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = (int)(blockDim.x >> 5);
   const int U = p.batch * p.q_groups;
-  const int per = (U + 31) / 32;
-  const int u_beg = min(U, lane * per), u_end = min(U, u_beg + per);
+  const int per = (U + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int u_beg = min(U, tid * per), u_end = min(U, u_beg + per);
   const bool writer = pair == 0 && rank == 0;
+  // scan 1: the weighted start of this thread's run
   int run = 0;
   for (int u = u_beg; u < u_end; ++u) {
     const UnitGeom ug = unit_geom(a, u, writer);
     run += unit_span_tiles<kKeys>(ug) * tile_weight(p, ug);
   }
-  int excl = run;  // inclusive prefix, then exclusive
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, excl, d);
-    if (lane >= d) excl += y;
+  int incl = warp_incl_scan(run);
+  if (lane == 31) scan1[warp] = incl;
+  __syncthreads();
+  int W = 0, excl = incl - run;
+  for (int w = 0; w < nw; ++w) {
+    const int x = scan1[w];
+    if (w < warp) excl += x;
+    W += x;
   }
-  const int W = __shfl_sync(0xffffffffu, excl, 31);
-  excl -= run;
   const int np = max(1, min(p.split_kv, W / kMinPairWeight));
   const int64_t lo = pair < np ? balanced_lo(pair, W, np) : W;
   const int64_t hi = pair < np ? balanced_lo(pair + 1, W, np) : W;
@@ -92,20 +111,13 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, Pie
       const UnitGeom ug = unit_geom(a, u, false);
       start += unit_span_tiles<kKeys>(ug) * tile_weight(p, ug);
     }
-    if (lane == 31) {
+    if (tid == 0) {
       a.sched[U] = W;
       a.sched[U + 1] = np;
     }
-    // the table is complete: the combine (which may already run) reads it
-    // once this flag is set
-    __syncwarp();
-    if (lane == 0) {
-      __threadfence();
-      ptx::st_release_gpu(a.unit_done + U, 1);
-    }
   }
-  // pieces: units of this lane's run with tiles in the range
-  int cnt = 0, u_first_lane = 0;
+  // scan 2: this thread's pieces (units of its run with tiles in the range)
+  int cnt = 0, tiles = 0, two = 0, u_first_t = 0;
   {
     int start = excl;
     for (int u = u_beg; u < u_end; ++u) {
@@ -114,26 +126,40 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, Pie
       int i0, i1;
       tiles_in_range(start, t, w, lo, hi, i0, i1);
       if (i1 > i0) {
-        if (cnt == 0) u_first_lane = u;
+        if (cnt == 0) u_first_t = u;
         ++cnt;
+        tiles += i1 - i0;
+        if (w == 3) two = 1;
       }
       start += t * w;
     }
   }
-  int base = cnt;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, base, d);
-    if (lane >= d) base += y;
-  }
-  const int npc = __shfl_sync(0xffffffffu, base, 31);
-  base -= cnt;
+  const int cnt_incl = warp_incl_scan(cnt);
+  const int tiles_w = warp_incl_scan(tiles);
   const unsigned has = __ballot_sync(0xffffffffu, cnt > 0);
-  const int u_first = has ? __shfl_sync(0xffffffffu, u_first_lane, __ffs(has) - 1) : 0;
+  const int two_w = __any_sync(0xffffffffu, two);
+  const int first_w = has ? __shfl_sync(0xffffffffu, u_first_t, __ffs(has) - 1) : -1;
+  if (lane == 31) scan2[warp] = make_int4(cnt_incl, tiles_w, two_w, first_w);
+  __syncthreads();
+  int base = cnt_incl - cnt, npc = 0, all_tiles = 0, any_two = 0, u_first = -1;
+  for (int w = 0; w < nw; ++w) {
+    const int4 x = scan2[w];
+    if (w < warp) base += x.x;
+    npc += x.x;
+    all_tiles += x.y;
+    any_two |= x.z;
+    if (u_first < 0 && x.x > 0) u_first = x.w;
+  }
+  // the table is complete (every thread wrote its units before the barrier):
+  // the combine, which may already run, reads it once the flag is set
+  if (writer && tid == 0) {
+    __threadfence();
+    ptx::st_release_gpu(a.unit_done + U, 1);
+  }
+  if (u_first < 0) u_first = 0;
   const int spill_base = (int)rank * (U + p.split_kv) + u_first + pair;
   Piece* spill = npc > kMaxSmemPieces ? reinterpret_cast<Piece*>(a.pieces) + spill_base : nullptr;
-  int two = 0, tiles = 0;
-  {
+  if (cnt > 0) {
     int start = excl, k = base;
     for (int u = u_beg; u < u_end; ++u) {
       const UnitGeom ug = unit_geom(a, u, false);
@@ -147,20 +173,16 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, Pie
         pc.t1 = i1;
         if (k < kMaxSmemPieces) smem_list[k] = pc;
         if (spill) spill[k] = pc;
-        if (w == 3) two = 1;
-        tiles += i1 - i0;
         ++k;
       }
       start += t * w;
     }
   }
-  two = __any_sync(0xffffffffu, two);
-  tiles = warp_sum_int(tiles);
-  if (lane == 0) {
+  if (tid == 0) {
     info->spill_base = spill_base;
     info->npc = npc;
-    info->tiles = tiles;
-    info->two = two;
+    info->tiles = all_tiles;
+    info->two = any_two;
     if (rank == 0 && pair < p.split_kv) a.sched[U + 2 + pair] = npc > 0 ? u_first : -1;
   }
 }

@@ -103,6 +103,7 @@ constexpr int kSoftmaxWarp0 = 4;
 constexpr int kSoftmaxWarps = 8;
 static_assert(2 * kSoftmaxWarps == kPieceArrivals, "unit counter arrivals per piece");
 constexpr int kThreads = 32 * (kSoftmaxWarp0 + kSoftmaxWarps);
+static_assert(kThreads <= 32 * kMaxSchedWarps, "the schedule build's scratch");
 
 // tensor memory columns (per CTA)
 constexpr uint32_t kOCol = 0;       // O: column half h at [128h, 128h + 128)
@@ -758,8 +759,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
   uint8_t* smem = smem_raw;
   SchedInfo* info = reinterpret_cast<SchedInfo*>(smem + kMaxSmemPieces * sizeof(Piece));
-  if (threadIdx.x < 32)
-    build_schedule<kTile16>(prm.a, blockIdx.x >> 1, cluster_ctarank(), reinterpret_cast<Piece*>(smem), info);
+  build_schedule<kTile16>(prm.a, blockIdx.x >> 1, cluster_ctarank(), smem);  // every thread
   __syncthreads();
   const int npc = info->npc;
   if (npc == 0) return;  // no work for this pair (the same in both CTAs)

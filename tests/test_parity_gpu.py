@@ -255,15 +255,30 @@ def test_balanced_schedule_many_ragged_units(dtype):
 
 
 def test_past_the_balanced_unit_limit_16bit_takes_fixed_splits():
-    """More units than the balanced schedule's piece list: 16-bit inputs go to the
+    """More units than the balanced decode schedule takes (16384): 16-bit inputs go to the
     fixed-split exchange kernel, still exact against the oracle (sampled rows)."""
     g = torch.Generator().manual_seed(35)
-    sl = torch.randint(1, 200, (2100,), generator=g).tolist()
-    inp = make_inputs_custom(2100, 1, 16, "bf16", sl, seed=36, pool=1.2)
+    sl = torch.randint(1, 200, (16400,), generator=g).tolist()
+    inp = make_inputs_custom(16400, 1, 16, "bf16", sl, seed=36, pool=1.2)
     out, lse, status, dec = run(inp, "tcgen05")
     assert dec.plan.schedule == 0 and dec.plan.kernel == 1 and status == 0
-    ref_o, ref_l = oracle_rows(inp)
-    compare(out, lse, ref_o, ref_l, "bf16", what="2100 units, fixed splits")
+    rows = sample_rows(16400, 1, 16, n=400, seed=37)
+    ref_o, ref_l = oracle_rows(inp, rows)
+    compare(out, lse, ref_o, ref_l, "bf16", rows=rows, what="16400 units, fixed splits")
+
+
+@pytest.mark.parametrize("dtype", ["fp8", "bf16"])
+def test_thousands_of_short_units_on_the_balanced_schedule(dtype):
+    """4000 one-token entries of 1..300 keys: far more units than pairs, every pair's piece list
+    spills past shared memory, and the combine's blocks take several units each."""
+    g = torch.Generator().manual_seed(38)
+    sl = torch.randint(0, 300, (4000,), generator=g).tolist()
+    inp = make_inputs_custom(4000, 1, 16, dtype, sl, seed=39, pool=1.2)
+    out, lse, status, dec = run(inp, "tcgen05")
+    assert dec.plan.schedule == 1 and status == 0
+    rows = sample_rows(4000, 1, 16, n=400, seed=40)
+    ref_o, ref_l = oracle_rows(inp, rows)
+    compare(out, lse, ref_o, ref_l, dtype, rows=rows, what="4000 short units, balanced")
 
 
 # ---------------------------------------------------------------- sliding window

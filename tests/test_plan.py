@@ -75,13 +75,13 @@ def test_balanced_plan_uses_every_sm_and_caps_units():
     assert mla.mla_decode_plan_custom(16, 4, 32, 81920, "fp8", split_kv=5).split_kv == 5
     assert mla.mla_decode_plan_custom(16, 4, 32, 81920, "fp8", split_kv=1000).split_kv == 74
     # more units than the per-pair piece list can hold: fixed splits, solo kernel
-    big = mla.mla_decode_plan(4096, 1, 16, 1024, "fp8")
+    big = mla.mla_decode_plan(20000, 1, 16, 1024, "fp8")
     assert big.schedule == 0 and big.kernel == 3
     # 16-bit inputs take the balanced schedule too (16-bit CTA-pair kernel),
     # and past the unit limit fixed splits on the exchange kernel
     assert mla.mla_decode_plan(16, 4, 32, 81920, "bf16").schedule == 1
     assert mla.mla_decode_plan(128, 2, 128, 81920, "bf16").schedule == 1
-    big16 = mla.mla_decode_plan(4096, 1, 16, 1024, "fp16")
+    big16 = mla.mla_decode_plan(20000, 1, 16, 1024, "fp16")
     assert big16.schedule == 0 and big16.kernel == 1
 
 
@@ -227,7 +227,7 @@ def test_window_is_set_only_on_plans_whose_kernels_support_it():
     # fixed-split tensor-core plans (the FP8 solo kernel, the 16-bit exchange
     # kernel past the balanced unit limit) do not take a window
     solo = mla.mla_decode_plan_custom(2, 4, 32, 4096, "fp8", kernel="tcgen05_solo")
-    big16 = mla.mla_decode_plan_custom(2100, 1, 16, 256, "bf16")
+    big16 = mla.mla_decode_plan_custom(17000, 1, 16, 256, "bf16")
     assert big16.schedule == 0
     for q in (solo, big16):
         with pytest.raises(mla.MlaError) as e:
