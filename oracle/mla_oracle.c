@@ -23,8 +23,14 @@
  * kv_cache [num_pages, page_size, D_total], block_tables) and section 一
  * (the latent cache shared by all heads: K is the whole 576-wide latent+rope
  * row, V its first 512 entries). Causal masking among the q_len tokens and
- * the per-row LSE are the options named in section 四. The seq_len reading
- * (it counts this step's q_len tokens) is stated in the design notes.
+ * the per-row LSE are the options named in section 四. The pages do not say
+ * whether seq_len counts this step's q_len tokens; this oracle takes that it
+ * does (token t of q_len sees keys up to seq_len - q_len + t).
+ *
+ * Also here: the same decode restricted to a sliding window (each row's last
+ * W visible keys), and the fused K/V pack with the E4M3 encoder it uses.
+ * Ragged prefill, in the Python wrapper, calls this decode once per entry
+ * with that entry's query length.
  *
  * Inputs are the raw element bytes the GPU path also receives; this file
  * decodes them itself from the published encodings (IEEE 754 binary16,
