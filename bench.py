@@ -2,18 +2,26 @@
 """Bench: MLA paged decode on B200 -- µs per decode step and effective KV GB/s.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                [--op decode|prefill|kv_pack] [--batch B]
 
 One step = one decode call (split-KV partial kernel + combine kernel) over a
 resident synthetic workload (default: FP8 E4M3 cache, q_len 4, 32 heads,
 81,920 keys, batch 16). Each timed step is bracketed by CUDA events on the
-launching stream; a 256 MiB buffer is rewritten between steps so no step
-starts from a warm L2 (the cache pool is larger than L2 anyway). With N > 1
-(torchrun) every rank runs an independent replica on its own GPU ("replicas
-only": the decode has no exchange step); the time is the max over ranks and
-the value the KV bytes of all ranks over that time.
+launching stream, after a loaded window that brings the clocks to those of
+continuous decoding. When the cache pool is smaller than twice the L2, a
+256 MiB buffer is rewritten between steps; otherwise the inputs are larger
+than L2 and nothing is flushed. With N > 1 (torchrun) every rank runs an
+independent replica on its own GPU ("replicas only": the decode has no
+exchange step); the time is the max over ranks and the value the KV bytes of
+all ranks over that time.
 
---impl reference times the fp64 CPU oracle (the only reference this build
-has) on the host cores, one bounded sample of the workload per step.
+--op prefill times a ragged prefill step (TFLOP/s) and --op kv_pack the fused
+K/V pack + FP8 quantise (GB/s), with the same JSON keys. --batch draws a
+smaller case of a workload (for profiler captures).
+
+--impl reference times the fp64 CPU oracle (no other implementation of this
+path is available to run) on the host cores, one bounded sample of the
+workload per step.
 """
 from __future__ import annotations
 

@@ -1,6 +1,6 @@
 """Shared test helpers: run the oracle on chosen rows and compare with the GPU.
 
-Tolerances (stated by the target of this build, written here in the tests):
+Tolerances (the accuracy bar for the GPU path against the fp64 oracle):
   out (BF16):  |gpu - ref| <= 1e-2 + 2e-2 * |ref| elementwise, and a
                relative L2 error <= 1e-2 (16-bit P) / 3e-2 (E4M3 P), since
                decode outputs are small and the absolute bound alone is weak;
