@@ -136,9 +136,9 @@ int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, i
   p.q_groups = G;
   p.rows_per_unit = M;
   const uint64_t rows = (uint64_t)batch * q_len * num_heads;
-  // The balanced schedule (CTA-pair kernels) keeps a per-pair piece list in
-  // shared memory; far more units than pairs can hold fall back to fixed
-  // splits (FP8: the solo kernel; 16-bit: the exchange kernel).
+  // Every CTA of the balanced schedule (CTA-pair kernels) scans all units at
+  // start; decode batches of more units than kMaxBalancedUnits take fixed
+  // splits instead (FP8: the solo kernel; 16-bit: the exchange kernel).
   p.varlen = varlen ? 1 : 0;
   // the balanced schedule's int32 tile weights (3 per 64 keys at most) must fit
   const bool weights_fit = units * tiles * 3 < (int64_t)INT32_MAX;

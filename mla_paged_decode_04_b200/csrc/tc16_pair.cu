@@ -24,8 +24,9 @@
 //   supplying V columns [256h + 128c, 256h + 128c + 128) as B from its V
 //   ring (the page's 64 keys, re-read from L2 once S exists).
 //
-// Roles (384 threads per CTA), barriers, the piece walk, the epilogue and
-// the bounded waits are those of the FP8 pair kernel (warp 0 Q and K loads,
+// Roles (384 threads per CTA), barriers, the schedule (pair_schedule.cuh),
+// the piece walk, the epilogue and the bounded waits are those of the FP8
+// pair kernel (warp 0 Q and K loads,
 // warp 1 TMEM and S MMAs, warp 2 P.V MMAs, warp 3 V loads, warps 4-11 two
 // softmax groups on alternate tiles). No TMA load uses multicast.
 #include <cuda.h>

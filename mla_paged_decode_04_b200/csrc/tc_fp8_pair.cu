@@ -7,16 +7,19 @@
 // tcgen05.mma together (cta_group::2, M = 128), each holding half of the
 // operands and half of the result.
 //
-// Schedule. The pairs stay resident (one per two SMs). A unit (batch entry,
-// query group) of n keys is ceil(n / 128) pair tiles of two cache pages; the
-// units' tiles, counted from the device seq_lens, form one sequence that is
-// dealt out as equal contiguous ranges, one per pair. A pair walks its range
-// as pieces (the part of one unit inside the range): a piece that is a whole
+// Schedule (pair_schedule.cuh). The pairs stay resident (one per two SMs). A
+// unit (batch entry, query group) spans the pair tiles of two cache pages
+// that hold the keys its rows see; the units' tiles, counted from the device
+// seq_lens and weighted by their P.V work, form one sequence that is dealt
+// out as equal contiguous ranges, one per pair. A pair walks its range as
+// pieces (the part of one unit inside the range): a piece that is a whole
 // unit writes out / lse directly; a unit cut between pairs leaves partial O
 // and LSE in the pair's slot (2p for its first piece, 2p + 1 for its last),
 // merged by the combine kernel. Every pair therefore does the same amount of
 // work whatever the length mix, and the pipeline runs on across pieces. This
 // is the article's split_kv auto-sizing (section 二) made exact on the device.
+// The same kernel serves ragged prefill (entries with their own query
+// lengths) and sliding windows through the unit geometry of device_common.cuh.
 //
 // Inside a pair tile, page 2j of the piece goes to CTA 0 and page 2j+1 to CTA 1.
 //  * S = Q.K^T (N = 128 keys): CTA c supplies query rows [64c, 64c+64) as
