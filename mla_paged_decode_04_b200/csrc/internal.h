@@ -32,7 +32,11 @@ inline uint64_t balanced_table_bytes(int64_t units) {
 }
 // FP8 rows that see fewer keys than this send P as two E4M3 terms (the P.V
 // MMAs run twice); the balanced schedule weighs such tiles 3 against 2.
-constexpr int kTwoTermKeys = 16384;
+// Measured with one E4M3 term on N(0,1) inputs, the output's relative L2
+// error is 2.3e-2 at 256 keys, 1.3e-2 at 4096, 1.0e-2 at 8192 and 7.7e-3 at
+// 16384 (the bound is 3e-2), and the worst element uses 1.04, 0.26, 0.20 and
+// 0.15 of its tolerance; with two terms both stay at 1.7e-3 and 0.11.
+constexpr int kTwoTermKeys = 8192;
 // Piece lists too long for a CTA's shared memory go to a spill area right
 // before the unit table: per CTA rank, U + P pieces of 3 int32 (a pair's
 // pieces are the units its range meets; pair p's list starts at entry
