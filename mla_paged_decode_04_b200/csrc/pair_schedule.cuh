@@ -30,12 +30,19 @@ constexpr uint32_t kSchedBytes = 1024;
 static_assert(kMaxSmemPieces * sizeof(Piece) + sizeof(SchedInfo) <= kSchedBytes, "schedule area");
 constexpr int kMinPairWeight = 4;  // pairs get at least this much weight (>= the heaviest tile)
 
+// Keys the unit's first row sees: the fewest of any of its rows (ragged
+// prefill units early in an entry see only a few keys even when the entry
+// has many).
+__device__ __forceinline__ int unit_min_keys(const mla_plan& p, const UnitGeom& ug) {
+  const int n = ug.nq + 1;
+  return (p.window > 0 && p.window < n) ? p.window : n;
+}
+
 // Weight of one tile of a unit: 3 when its rows' P goes as two E4M3 terms
-// (FP8 rows that see fewer than kTwoTermKeys keys), else 2.
+// (FP8 units whose first row sees fewer than kTwoTermKeys keys), else 2.
 __device__ __forceinline__ int tile_weight(const mla_plan& p, const UnitGeom& ug) {
   if (p.dtype != MLA_FP8_E4M3) return 2;
-  const int seen = (p.window > 0 && p.window < ug.n) ? p.window : ug.n;
-  return seen < kTwoTermKeys ? 3 : 2;
+  return unit_min_keys(p, ug) < kTwoTermKeys ? 3 : 2;
 }
 
 // Tiles [i0, i1) of a unit with `t` tiles of weight `w` starting at weighted

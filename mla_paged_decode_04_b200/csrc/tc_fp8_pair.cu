@@ -188,7 +188,7 @@ __device__ __forceinline__ PieceCtx piece_ctx(const DecodeArgs& a, const Piece& 
   c.row0 = ug.row0;
   c.table = a.block_tables + (int64_t)c.b * a.max_pages_per_seq;
   c.whole = pc.t0 == 0 && c.key1 >= ug.kend;
-  c.two = kTwo && ((p.window > 0 && p.window < c.n) ? p.window : c.n) < kTwoTermKeys;
+  c.two = kTwo && tile_weight(p, ug) == 3;  // the same rule as the schedule's weights
   return c;
 }
 

@@ -281,6 +281,17 @@ def test_thousands_of_short_units_on_the_balanced_schedule(dtype):
     compare(out, lse, ref_o, ref_l, dtype, rows=rows, what="4000 short units, balanced")
 
 
+@pytest.mark.parametrize("kernel", ["tcgen05", "tcgen05_solo"])
+def test_fp8_entries_around_the_two_term_threshold(kernel):
+    """FP8 rows just below and above 8192 visible keys: two-term P below, one E4M3 term above;
+    every row within the tolerances."""
+    inp = make_inputs_custom(4, 4, 32, "fp8", [8190, 8196, 12000, 16383], seed=45, pool=1.2)
+    out, lse, status, dec = run(inp, kernel)
+    assert status == 0
+    ref_o, ref_l = oracle_rows(inp)
+    compare(out, lse, ref_o, ref_l, "fp8", what=f"threshold {kernel}")
+
+
 # ---------------------------------------------------------------- sliding window
 # A row with n visible keys attends to keys [max(0, n - W), n) (a decode option
 # the TokenSpeed MLA article lists among its tests, section 六). The CTA-pair

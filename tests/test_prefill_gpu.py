@@ -129,3 +129,18 @@ def test_skewed_decode_batch_spills_long_piece_lists(dtype):
                                                                                             False))))
     ref_o, ref_l = oracle_rows(inp, rows)
     compare(out, lse, ref_o, ref_l, dtype, rows=rows, what="skewed decode batch")
+
+
+def test_long_fresh_prefill_keeps_two_term_p_for_its_early_rows():
+    """9000 new tokens with no cached prefix (FP8): the entry has more keys than the two-term
+    threshold, but its first tokens see only a few keys; their units must still send P as
+    two E4M3 terms (the choice follows the unit's fewest visible keys, not the entry's)."""
+    inp = make_prefill_inputs([9000], [0], 16, "fp8", seed=216, pool=1.1)
+    out, lse, status, p = run_prefill(inp)
+    assert status == 0
+    H = inp.heads
+    rng = np.random.default_rng(9)
+    toks = sorted(set(range(0, 40)) | set(range(8950, 9000)) | set(int(x) for x in rng.choice(9000, 60, False)))
+    rows = np.array([t * H + h for t in toks for h in range(H)], dtype=np.int64)
+    ref_o, ref_l = prefill_oracle(inp, rows=rows)
+    compare(out, lse, ref_o, ref_l, "fp8", rows=rows, what="9000 fresh tokens")
