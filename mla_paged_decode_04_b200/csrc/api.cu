@@ -371,6 +371,18 @@ extern "C" int mla_kv_amax(const void* latent, const void* rope, int64_t n_token
   return e == cudaSuccess ? MLA_OK : cuda_failure(e);
 }
 
+namespace mla {
+cudaError_t set_max_dynamic_smem(const void* func, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+}  // namespace mla
+
 extern "C" int mla_decode_plan_window(mla_plan* plan, int window) {
   if (!plan || window < 0) return MLA_ERR_INVALID_ARG;
   mla_plan p = *plan;

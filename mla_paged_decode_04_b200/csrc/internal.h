@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "mla_decode.h"
 
 namespace mla {
@@ -78,6 +80,13 @@ __host__ __device__ inline int64_t balanced_lo(int p, int64_t W, int np) { retur
 // Records `e` as this thread's last CUDA error (read by mla_last_cuda_error)
 // and returns MLA_ERR_CUDA.
 int cuda_failure(cudaError_t e);
+
+// Raises a kernel's dynamic shared memory limit to `bytes` on the current
+// device, once per device: the attribute belongs to each device's context, so
+// a process that drives several GPUs needs it on every one. `done` is the
+// caller's per-kernel bitmask of devices already set (devices >= 64 are set
+// on every call).
+cudaError_t set_max_dynamic_smem(const void* func, int bytes, std::atomic<uint64_t>& done);
 
 int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, int split_kv,
               int fold, int kernel, int varlen, mla_plan* plan);

@@ -787,13 +787,10 @@ cudaError_t launch_tc16_pair_partial(const DecodeArgs& a, cudaStream_t stream) {
       !encode_rows_576_chunks(&prm.tm_v[0], kv, 2, kv_rows, 6, 128, kTile16, 2) ||
       !encode_rows_576_chunks(&prm.tm_v[1], kv + 256, 2, kv_rows, 6, 128, kTile16, 2))
     return cudaErrorInvalidValue;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(tc16_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)Layout16::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_max_dynamic_smem((const void*)tc16_pair_kernel, (int)Layout16::kSmemBytes, smem_set);
+      e != cudaSuccess)
+    return e;
   tc16_pair_kernel<<<(unsigned)(2 * p.split_kv), kThreads, Layout16::kSmemBytes, stream>>>(prm);
   return cudaGetLastError();
 }

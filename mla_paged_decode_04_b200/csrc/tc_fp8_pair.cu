@@ -857,13 +857,10 @@ cudaError_t launch_tc_fp8_pair_partial(const DecodeArgs& a, cudaStream_t stream)
       !encode_rows_576(&prm.tm_kv_main, a.kv_cache, 1, kv_rows, 128, kTileKeys, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_rows_576(&prm.tm_kv_rope, a.kv_cache, 1, kv_rows, 64, kTileKeys, CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(tc_fp8_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_max_dynamic_smem((const void*)tc_fp8_pair_kernel, (int)kPairSmemBytes, smem_set);
+      e != cudaSuccess)
+    return e;
   tc_fp8_pair_kernel<<<(unsigned)(2 * p.split_kv), kThreads, kPairSmemBytes, stream>>>(prm);
   return cudaGetLastError();
 }

@@ -576,13 +576,10 @@ cudaError_t launch_dt(const DecodeArgs& a, cudaStream_t stream) {
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_rows_576(&prm.tm_kv_rope, a.kv_cache, C::E, kv_rows, 32, kTileKeys, rope_sw))
     return cudaErrorInvalidValue;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(tc_partial_kernel<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_max_dynamic_smem((const void*)tc_partial_kernel<DT>, (int)C::SMEM_BYTES, smem_set);
+      e != cudaSuccess)
+    return e;
   const uint64_t pairs = (uint64_t)p.batch * p.q_groups * p.split_kv;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
