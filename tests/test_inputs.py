@@ -53,3 +53,26 @@ def test_tiny_workload_layout():
     assert inp.num_pages == 4 and inp.block_tables.shape == (1, 4)
     assert sorted(inp.block_tables[0].tolist()) == [0, 1, 2, 3]
     assert inp.q.shape == (1, 1, 16, 576) and inp.kv_cache.shape == (4, 64, 576)
+
+
+def test_prefill_inputs_are_seeded_and_consistent():
+    from mla_paged_decode_04_b200.inputs import make_prefill_inputs, make_prefill_workload, PREFILL_WORKLOADS
+    a = make_prefill_inputs([5, 0, 70], [3, 9, 0], 16, "fp8", seed=3)
+    b = make_prefill_inputs([5, 0, 70], [3, 9, 0], 16, "fp8", seed=3)
+    assert torch.equal(a.q.view(torch.uint8), b.q.view(torch.uint8))
+    assert torch.equal(a.kv_cache.view(torch.uint8), b.kv_cache.view(torch.uint8))
+    assert a.cu_seqlens_q.tolist() == [0, 5, 5, 75] and a.seq_lens.tolist() == [8, 9, 70]
+    assert a.total_q == 75 and a.max_q_len == 70 and a.q.shape == (75, 16, 576)
+    # every page an entry needs is a distinct page of the pool; unused table slots are -1
+    used = []
+    for bi, n in enumerate(a.seq_lens.tolist()):
+        npg = (n + 63) // 64
+        row = a.block_tables[bi].tolist()
+        assert all(0 <= pg < a.kv_cache.shape[0] for pg in row[:npg]) and all(pg == -1 for pg in row[npg:])
+        used += row[:npg]
+    assert len(used) == len(set(used))
+    w = PREFILL_WORKLOADS["prefill_bf16"]
+    small = make_prefill_workload("prefill_bf16", batch=2)
+    assert small.batch == 2 and small.max_q_len == w.max_q_len and small.dtype == "bf16"
+    ql = [small.cu_seqlens_q[i + 1] - small.cu_seqlens_q[i] for i in range(2)]
+    assert all(w.q_lens[1] <= int(q) <= w.q_lens[2] for q in ql)
