@@ -497,6 +497,46 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_reference_prefill(args):
+    """--op prefill --impl reference: the oracle's ragged prefill on the host cores, each step a
+    bounded sample (the last 8 tokens of entry 0 of the workload, all heads), flops of those rows."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    from mla_paged_decode_04_b200.inputs import PREFILL_WORKLOADS, make_prefill_workload
+    name = args.workload if args.workload in PREFILL_WORKLOADS else "prefill_fp8"
+    inp = make_prefill_workload(name)
+    cu, H = inp.cu_seqlens_q.tolist(), inp.heads
+    toks = list(range(max(cu[0], cu[1] - 8), cu[1]))
+    rows = [t * H + h for t in toks for h in range(H)]
+    n0, q0 = int(inp.seq_lens[0]), cu[1] - cu[0]
+    flops = sum(n0 - q0 + (t - cu[0]) + 1 for t in toks) * H * 2 * (576 + 512)
+
+    def one():
+        oracle.mla_prefill(inp.q, inp.cu_seqlens_q, inp.kv_cache, inp.block_tables, inp.seq_lens,
+                           inp.softmax_scale, dtype=inp.dtype, q_scale=inp.q_scale, kv_scale=inp.kv_scale, rows=rows)
+
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    dt = time.perf_counter() - t0
+    value = flops * args.steps / dt / 1e12
+    sample = f"{len(rows)} query rows per step (the last {len(toks)} tokens of entry 0, all heads); flops of those rows"
+    line = {"impl": "reference", "metric": "MLA ragged prefill TFLOP/s (algorithmic flops per step / step time) on 1 B200",
+            "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": {"fp8": "fp8_e4m3", "bf16": "bf16", "fp16": "fp16"}[inp.dtype], "data": "synthetic (seeded)",
+            "config": {"workload": name, "batch": inp.batch, "heads": H, "total_q": inp.total_q},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
 def run_kv_pack(args):
     """Fused K/V pack + FP8 quantise on a prefill-sized write: 16 x 81,920 BF16 tokens into an
     FP8 cache of twice the pages (permuted slots). One JSON line; HBM roofline."""
@@ -736,10 +776,17 @@ def run_prefill(args):
 def main():
     args = parse_args()
     if args.op == "kv_pack":
-        run_kv_pack(args)
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the K/V pack reference arm is not timed; "
+                              "its oracle is checked byte for byte in tests/test_kv_pack.py"}), flush=True)
+        else:
+            run_kv_pack(args)
         return
     if args.op == "prefill":
-        run_prefill(args)
+        if args.impl == "reference":
+            run_reference_prefill(args)
+        else:
+            run_prefill(args)
         return
     if args.impl == "reference":
         run_reference(args)
