@@ -55,9 +55,10 @@ def mla_decode_brute(q, kv_cache, block_tables, seq_lens, softmax_scale,
 
 
 def mla_prefill_brute(q, cu_seqlens_q, kv_cache, block_tables, seq_lens, softmax_scale,
-                      q_scale=1.0, kv_scale=1.0):
+                      q_scale=1.0, kv_scale=1.0, window=0):
     """Ragged prefill written out directly: packed token i of entry b (cu[b] <= i < cu[b+1])
-    sees keys 0 .. seq_lens[b] - (cu[b+1] - cu[b]) + (i - cu[b]). q [total_q, H, D]."""
+    sees keys 0 .. seq_lens[b] - (cu[b+1] - cu[b]) + (i - cu[b]); with window W > 0 only the
+    last W of them. q [total_q, H, D]."""
     total_q, H, D = (int(x) for x in q.shape)
     _, page, _ = (int(x) for x in kv_cache.shape)
     qrows = _as_floats(q, q_scale)
@@ -75,7 +76,8 @@ def mla_prefill_brute(q, cu_seqlens_q, kv_cache, block_tables, seq_lens, softmax
                 if last < 0:
                     outs[i * H + h], lses[i * H + h] = [0.0] * 512, -math.inf
                     continue
-                keys = [cache_rows[bt[b][j // page] * page + j % page] for j in range(last + 1)]
+                first = max(0, last + 1 - window) if window > 0 else 0
+                keys = [cache_rows[bt[b][j // page] * page + j % page] for j in range(first, last + 1)]
                 s = [softmax_scale * math.fsum(qv[d] * k[d] for d in range(D)) for k in keys]
                 m = max(s)
                 lse = m + math.log(math.fsum(math.exp(x - m) for x in s))

@@ -418,3 +418,15 @@ def test_prefill_rows_before_any_key_are_empty_and_rows_subset_matches():
     so, sl_ = oracle.mla_prefill(inp.q, inp.cu_seqlens_q, inp.kv_cache, inp.block_tables, sl, inp.softmax_scale,
                                  dtype="bf16", rows=rows)
     assert np.array_equal(so, o[rows]) and np.array_equal(sl_, l[rows])
+
+
+@pytest.mark.parametrize("window", [1, 3, 50])
+def test_prefill_with_a_window_matches_the_brute_force_loop(window):
+    inp = make_prefill_inputs([4, 6], [20, 0], 2, "bf16", seed=74, pool=1.5)
+    o, l = oracle.mla_prefill(inp.q, inp.cu_seqlens_q, inp.kv_cache, inp.block_tables, inp.seq_lens,
+                              inp.softmax_scale, dtype="bf16", window=window)
+    bo, bl = mla_prefill_brute(inp.q, inp.cu_seqlens_q, inp.kv_cache, inp.block_tables, inp.seq_lens,
+                               inp.softmax_scale, window=window)
+    for r in range(inp.total_q * inp.heads):
+        assert np.allclose(o[r], bo[r], rtol=0, atol=1e-12)
+        assert abs(l[r] - bl[r]) <= 1e-12
