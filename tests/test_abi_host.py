@@ -106,6 +106,15 @@ def test_python_wrapper_refuses_host_tensors():
                        0.04, t, None, torch.empty(0, dtype=torch.uint8))
 
 
+def test_prefill_wrapper_refuses_host_tensors():
+    torch = pytest.importorskip("torch")
+    p = mla.mla_prefill_plan(1, 4, 16, 256, "bf16")
+    t = torch.empty(0)
+    with pytest.raises(ValueError, match="q must be a CUDA tensor"):
+        mla.mla_prefill(p, t, torch.zeros(2, dtype=torch.int32), torch.empty(1, 64, 576),
+                        torch.empty(1, 4, dtype=torch.int32), t, 0.04, t, None, torch.empty(0, dtype=torch.uint8))
+
+
 def test_last_cuda_error_starts_clean():
     """No CUDA failure has been recorded on a fresh thread: code 0, name cudaSuccess."""
     import threading
