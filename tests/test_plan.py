@@ -273,3 +273,14 @@ def test_balanced_workspace_holds_the_piece_spill():
     need = (p.lse_offset + 2 * p.split_kv * p.rows_per_unit * 4
             + (2 * (units + p.split_kv) * 12 + 255) // 256 * 256 + ((units + 2) * 4 + 255) // 256 * 256)
     assert p.workspace_bytes >= need
+
+
+def test_window_applies_to_prefill_plans():
+    p = mla.mla_prefill_plan(2, 500, 32, 5000, "fp8")
+    ws = p.workspace_bytes
+    assert mla.mla_decode_plan_window(p, 256).window == 256 and p.varlen == 1 and p.workspace_bytes == ws
+    s = mla.mla_prefill_plan(2, 500, 32, 5000, "bf16", kernel="simt")
+    assert mla.mla_decode_plan_window(s, 1).window == 1
+    # the fixed-split workspace of a ragged plan holds batch x max_q_len x H rows of partials
+    if s.split_kv > 1:
+        assert s.lse_offset - s.partial_offset >= 2 * 500 * 32 * s.split_kv * 512 * 4
