@@ -284,3 +284,24 @@ def test_window_applies_to_prefill_plans():
     # the fixed-split workspace of a ragged plan holds batch x max_q_len x H rows of partials
     if s.split_kv > 1:
         assert s.lse_offset - s.partial_offset >= 2 * 500 * 32 * s.split_kv * 512 * 4
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_spilled_piece_lists_of_different_pairs_never_overlap(seed):
+    """A pair's spill list starts at entry u_first + p (per CTA rank, U + P entries each) and
+    holds one piece per unit its range meets: the lists of all pairs fit and never overlap."""
+    import random
+    rnd = random.Random(seed)
+    U, P = rnd.choice([50, 300, 3000]), 74
+    tiles = [rnd.choice([0, 0, 1, 1, 2, 5, 40, 300]) for _ in range(U)]
+    weights = [rnd.choice([2, 3]) for _ in range(U)]
+    _, _, _, pieces, first = _balanced_schedule(tiles, P, weights)
+    used = set()
+    for p, pp in enumerate(pieces):
+        if not pp:
+            continue
+        base = first[p] + p
+        for k in range(len(pp)):
+            idx = base + k
+            assert 0 <= idx < U + P and idx not in used
+            used.add(idx)
