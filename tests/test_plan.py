@@ -305,3 +305,37 @@ def test_spilled_piece_lists_of_different_pairs_never_overlap(seed):
             idx = base + k
             assert 0 <= idx < U + P and idx not in used
             used.add(idx)
+
+
+def _unit_span(n, qlen, g, F, window):
+    """The unit geometry's key span [klo, kend) restated: rows of tokens g*F .. of an entry with
+    n keys and qlen new tokens (token t sees keys up to n - qlen + t, its last `window` if set)."""
+    t0 = g * F
+    tu = min(F, qlen - t0)
+    if tu <= 0:
+        return 0, 0, 0
+    nq = n - qlen + t0
+    kend = max(0, nq + tu)
+    klo = max(0, nq + 1 - window) if window > 0 else 0
+    return tu, klo, kend
+
+
+@pytest.mark.parametrize("window", [0, 1, 7, 100])
+def test_unit_span_is_the_union_of_its_rows_visible_keys(window):
+    import random
+    rnd = random.Random(window)
+    for _ in range(300):
+        F = rnd.choice([1, 2, 4, 8])
+        qlen = rnd.randint(0, 40)
+        n = rnd.randint(0, 200)
+        for g in range((max(qlen, 1) + F - 1) // F + 1):
+            tu, klo, kend = _unit_span(n, qlen, g, F, window)
+            keys = set()
+            for t in range(g * F, g * F + max(tu, 0)):
+                last = n - qlen + t
+                first = max(0, last + 1 - window) if window > 0 else 0
+                keys |= set(range(first, last + 1))
+            if keys:
+                assert (klo, kend) == (min(keys), max(keys) + 1)
+            else:
+                assert kend <= klo or tu <= 0
