@@ -294,18 +294,33 @@ int mla_decode_status(void* workspace, void* stream, int clear, int32_t* device_
  *     workspace_bytes. A plan whose workspace_bytes exceeds
  *     MLA_NO_ALLOC_SCRATCH_BYTES is rejected with MLA_ERR_WORKSPACE_TOO_SMALL
  *     before anything is enqueued (use fewer splits or mla_decode).
- *   - The first call on a device looks up the scratch array's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture on the device.
+ *   - Every call looks up the scratch array's device address in the current
+ *     device's context (cudaGetSymbolAddress, a host-side query), so a
+ *     context that was reset and created again gets the array's new address.
+ *     The first lookup on a device loads the library's device code there:
+ *     make the first call on a device before any stream capture on it.
  *   - Every call on a device shares the one scratch array and it keeps the
  *     last call's contents: calls that overlap on the GPU (different streams
  *     without ordering) race on it and must not be issued. The status word
- *     it holds is reset by each call.
+ *     it holds is reset by each call; read it with
+ *     mla_decode_no_alloc_status.
  */
 int mla_decode_no_alloc(const mla_plan* plan, const void* q, const void* kv_cache,
                         int64_t num_pages, int page_size, const int32_t* block_tables,
                         int max_pages_per_seq, const int32_t* seq_lens, float softmax_scale,
                         float q_scale, float kv_scale, void* out, float* lse, void* stream);
+
+/*
+ * mla_decode_no_alloc_status: mla_decode_status for the scratch array of
+ * mla_decode_no_alloc on the current device (no counterpart on the pages).
+ * Synchronises `stream`, copies the status word (MLA_DEV_* bits of the last
+ * mla_decode_no_alloc on this device) into *device_status and clears it when
+ * `clear` is non-zero. A caller of mla_decode_no_alloc never sees the
+ * scratch address, so this is its only way to learn of bad pages, over-long
+ * sequences or a wait that ran out. MLA_ERR_INVALID_ARG for a null
+ * device_status; MLA_ERR_CUDA if the synchronise or the copy fails.
+ */
+int mla_decode_no_alloc_status(void* stream, int clear, int32_t* device_status);
 
 /* Human-readable name of an mla_status code (static storage, never NULL). */
 const char* mla_status_string(int code);

@@ -28,7 +28,7 @@ MLA_DEV_BAD_PAGE, MLA_DEV_SEQ_TOO_LONG, MLA_DEV_TIMEOUT, MLA_DEV_BAD_QLEN = 0x1,
 
 EXPORTED = ["mla_decode_plan", "mla_decode_plan_custom", "mla_decode", "mla_decode_partial",
             "mla_decode_combine", "mla_decode_status", "mla_status_string", "mla_version",
-            "mla_decode_no_alloc", "mla_last_cuda_error", "mla_kv_pack", "mla_kv_amax",
+            "mla_decode_no_alloc", "mla_decode_no_alloc_status", "mla_last_cuda_error", "mla_kv_pack", "mla_kv_amax",
             "mla_decode_plan_window", "mla_prefill_plan", "mla_prefill_plan_custom", "mla_prefill",
             "mla_prefill_partial", "mla_prefill_combine"]
 MLA_NO_ALLOC_SCRATCH_BYTES = 48 << 20

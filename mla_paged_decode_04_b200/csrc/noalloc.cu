@@ -10,35 +10,26 @@
 // memory: a file-scope array of MLA_NO_ALLOC_SCRATCH_BYTES, reserved on every
 // GPU that loads the library and held until the process exits.
 //
-// The array's name is only a host-side stand-in; its device address is looked
-// up once per device with cudaGetSymbolAddress (with that device current, on
-// the first call on the device) and then passed to the kernels like any
-// workspace. Nothing here calls cudaMalloc or cudaFree.
-#include <mutex>
-
+// The array's name is only a host-side stand-in. Its device address is looked
+// up with cudaGetSymbolAddress on every call, with the calling device current,
+// and then passed to the kernels like any workspace. The lookup is a host-side
+// table query, so it costs little, and it always names the array of the
+// current context: after a cudaDeviceReset the module is loaded again and the
+// array may sit at another address. The first lookup on a device loads the
+// module there (lazy loading), so the first call on a device should come
+// before any stream capture on it. Nothing here calls cudaMalloc or cudaFree.
 #include "internal.h"
 
 namespace {
 
 __device__ __align__(256) unsigned char g_no_alloc_scratch[MLA_NO_ALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {nullptr};
-
-// Device address of the scratch array on the current device (looked up once).
+// Device address of the scratch array in the current device's context.
 int scratch_address(void** out) {
-  int dev = 0;
-  if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return mla::cuda_failure(e);
-  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaError_t e = cudaGetSymbolAddress(&p, g_no_alloc_scratch); e != cudaSuccess) return mla::cuda_failure(e);
-    if (p == nullptr) return mla::cuda_failure(cudaErrorInvalidSymbol);
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
+  void* p = nullptr;
+  if (cudaError_t e = cudaGetSymbolAddress(&p, g_no_alloc_scratch); e != cudaSuccess) return mla::cuda_failure(e);
+  if (p == nullptr) return mla::cuda_failure(cudaErrorInvalidSymbol);
+  *out = p;
   return MLA_OK;
 }
 
@@ -56,4 +47,12 @@ extern "C" int mla_decode_no_alloc(const mla_plan* plan, const void* q, const vo
   return mla_decode(plan, q, kv_cache, num_pages, page_size, block_tables, max_pages_per_seq, seq_lens,
                     softmax_scale, q_scale, kv_scale, out, lse, scratch, (uint64_t)MLA_NO_ALLOC_SCRATCH_BYTES,
                     stream);
+}
+
+extern "C" int mla_decode_no_alloc_status(void* stream, int clear, int32_t* device_status) {
+  if (!device_status) return MLA_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  const int rc = scratch_address(&scratch);
+  if (rc != MLA_OK) return rc;
+  return mla_decode_status(scratch, stream, clear, device_status);
 }
