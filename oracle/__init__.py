@@ -76,6 +76,8 @@ def _load():
         lib.oracle_decode_buffer.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = i32
+        lib.oracle_set_num_threads.argtypes = [i32]
+        lib.oracle_set_num_threads.restype = None
         lib.oracle_encode_e4m3_buffer.argtypes = [vp, ctypes.c_size_t, vp]
         lib.oracle_encode_e4m3_buffer.restype = None
         lib.oracle_kv_pack.argtypes = [i32, i32, vp, vp, i64, vp, ctypes.c_float, vp, i64]
@@ -88,6 +90,12 @@ def _load():
 
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of the oracle's parallel loops from now on (timing only: a row is always
+    computed by one thread, so results do not depend on it)."""
+    _load().oracle_set_num_threads(int(n))
 
 
 def _raw_bytes(t) -> np.ndarray:

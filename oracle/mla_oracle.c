@@ -327,6 +327,16 @@ int oracle_num_threads(void) {
 #endif
 }
 
+/* Threads the parallel loops use from now on (n >= 1; timing only, the
+   results do not depend on it: every row is computed by one thread). */
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n >= 1) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 /*
  * Fused K/V pack + FP8 quantise (the cache-writing step before decode).
  * Sources: tokenspeed-mla package card, "What it is and what it does" (a
