@@ -6,10 +6,13 @@ python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ou
 
 One step = one decode call (split-KV partial kernel + combine kernel) over a
 resident synthetic workload (default: FP8 E4M3 cache, q_len 4, 32 heads,
-81,920 keys, batch 16). Each timed step is bracketed by CUDA events on the
-launching stream, after a loaded window that brings the clocks to those of
-continuous decoding. When the cache pool is smaller than twice the L2, a
-256 MiB buffer is rewritten between steps; otherwise the inputs are larger
+81,920 keys, batch 16). After W warm-up steps, exactly K steps are timed, each
+bracketed by CUDA events on the launching stream, with the SM clock read
+through NVML during them. The same K steps are then timed again after a
+loaded window (--clock-window-s seconds of back-to-back steps, which bring the
+clocks to those of continuous decoding under the power cap) and reported
+beside them as "sustained". When the cache pool is smaller than twice the L2,
+a 256 MiB buffer is rewritten between steps; otherwise the inputs are larger
 than L2 and nothing is flushed. With N > 1 (torchrun) every rank runs an
 independent replica on its own GPU ("replicas only": the decode has no
 exchange step); the time is the max over ranks and the value the KV bytes of
@@ -60,7 +63,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--clock-window-s", type=float, default=1.5,
-                    help="seconds of untimed decode steps run while clocks are sampled")
+                    help="seconds of back-to-back steps before the sustained timing (0: no sustained timing)")
     return ap.parse_args()
 
 
@@ -212,6 +215,89 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+class NvmlClockPoller:
+    """SM clock and clock-event reasons read through NVML about every 0.5 ms from a host thread,
+    so that a timed region of a few milliseconds still gets samples (nvidia-smi's loop samples
+    every 100 ms at best). Read-only: nothing is set. window(t0, t1) summarises the samples
+    taken between two host perf_counter() times."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+    def __init__(self, device_index):
+        import threading
+        self.samples = []  # (perf_counter, sm_mhz, reason bits)
+        self.ok = False
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self.nv = pynvml
+            self.bits = {name: getattr(pynvml, attr, 0) for name, attr in self.REASONS}
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv, h = self.nv, self.h
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((time.perf_counter(), float(mhz), int(rs)))
+            except Exception:
+                pass
+            time.sleep(0.0005)
+
+    def start(self):
+        if self.ok:
+            import threading
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+
+    def window(self, t0, t1):
+        sel = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not sel:
+            return None
+        reasons = sorted({name for _, _, rs in sel for name, bit in self.bits.items() if bit and rs & bit})
+        return {"sm_mhz": statistics.median(s[1] for s in sel), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(sel), "source": "nvml, ~0.5 ms polling during the timed steps"}
+
+
+def roofline_fields(alg_bytes, flops, seconds, hbm_peak, hbm_kind, dtype, sustained):
+    """Roofline of one partial-kernel launch of `seconds`: the HBM side (algorithmic bytes at the
+    measured copy bandwidth) and the tensor side (algorithmic flops at the measured cuBLAS peak,
+    burst or sustained), `bound` being the side with the higher floor. hbm_frac is always given:
+    decode reads the KV cache once, so HBM is the yardstick of the workloads the cache dominates."""
+    tpeak, tkind = measured_tensor_peak(dtype, sustained=sustained)
+    t_hbm = alg_bytes / (hbm_peak * 1e9)
+    t_tensor = flops / (tpeak * 1e12)
+    hbm_ach = alg_bytes / seconds / 1e9
+    ten_ach = flops / seconds / 1e12
+    hbm = {"bound": "hbm", "achieved": round(hbm_ach, 1), "peak": hbm_peak, "unit": "GB/s",
+           "frac": round(hbm_ach / hbm_peak, 4), "peak_source": f"{hbm_kind} (of measured copy bandwidth)"
+           if hbm_kind == "measured" else hbm_kind, "floor_us": round(t_hbm * 1e6, 2)}
+    ten = {"bound": "tensor", "achieved": round(ten_ach, 1), "peak": round(tpeak, 1), "unit": "TFLOP/s",
+           "frac": round(ten_ach / tpeak, 4), "peak_source": tkind, "floor_us": round(t_tensor * 1e6, 2)}
+    bind, other = (ten, hbm) if t_tensor > t_hbm else (hbm, ten)
+    out = dict(bind)
+    out.update({"hbm_frac": hbm["frac"], "tensor_frac": ten["frac"], "tensor_peak": ten["peak"], "other": other})
+    return out
+
+
 # ---------------------------------------------------------------- our arm
 
 def run_ours(args):
@@ -265,54 +351,80 @@ def run_ours(args):
         # one call: the combine is launched as the partial kernel's dependent
         mla.mla_decode(plan, *call)
 
+    poller = NvmlClockPoller(local)
+    poller.start()
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize()
     if dec.status() != 0:
         raise RuntimeError("device status word set during warm-up")
 
-    sampler = ClockSampler(local)
-    sampler.start()
-    # keep the GPU busy for ~1.5 s so the clock samples see the kernel under load
-    t_end = time.perf_counter() + args.clock_window_s
-    while time.perf_counter() < t_end:
-        for _ in range(20):
-            flush.zero_()
-            step()
+    def timed(fn, n):
+        """n steps, each bracketed by CUDA events on the launching stream; returns per-step ms
+        and the host time window the steps ran in."""
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+        if world > 1:
+            dist.barrier()
         torch.cuda.synchronize()
+        h0 = time.perf_counter()
+        for k in range(n):
+            flush.zero_()
+            evs[k][0].record()
+            fn()
+            evs[k][1].record()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        return [e0.elapsed_time(e1) for e0, e1 in evs], h0, time.perf_counter()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    wall0 = time.perf_counter()
-    for k in range(args.steps):
-        flush.zero_()
-        e0, e1 = evs[k]
-        e0.record()
-        step()
-        e1.record()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    wall1 = time.perf_counter()
-    # The partial kernel alone, for its roofline: an event between the two
-    # launches (which also serialises them) marks its end. Same number of
-    # steps, still under load.
-    pevs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    for k in range(args.steps):
-        flush.zero_()
-        e0, e1 = pevs[k]
+    def partial_only():
+        # the partial kernel alone: an event between the two launches (which also serialises
+        # them) marks its end
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         mla.mla_decode_partial(plan, *call)
         e1.record()
         mla.mla_decode_combine(plan, *call)
-    torch.cuda.synchronize()
-    clocks = sampler.stop()
+        part_events.append((e0, e1))
+
+    # (1) the timed steps: W warm-up steps above, then exactly K steps
+    step_ms, wall0, wall1 = timed(step, args.steps)
+    clocks = poller.window(wall0, wall1)
+    part_events = []
+    _, p0, p1 = timed(partial_only, args.steps)
+    part_ms = [a.elapsed_time(b) for a, b in part_events]
     if dec.status() != 0:
         raise RuntimeError("device status word set during the timed steps")
-    step_ms = [e0.elapsed_time(e1) for e0, e1 in evs]
-    part_ms = [e0.elapsed_time(e1) for e0, e1 in pevs]
+
+    # (2) the same K steps after a loaded window (continuous decoding: the clocks settle under
+    # the power cap), reported beside the timed steps
+    sustained = None
+    if args.clock_window_s > 0:
+        sampler = ClockSampler(local)
+        sampler.start()
+        t_end = time.perf_counter() + args.clock_window_s
+        while time.perf_counter() < t_end:
+            for _ in range(20):
+                flush.zero_()
+                step()
+            torch.cuda.synchronize()
+        sus_ms, s0, s1 = timed(step, args.steps)
+        part_events = []
+        _, _, _ = timed(partial_only, args.steps)
+        sus_part_ms = [a.elapsed_time(b) for a, b in part_events]
+        smi = sampler.stop()
+        sus_clocks = poller.window(s0, s1) or smi
+        if sus_clocks is not None and smi is not None:
+            sus_clocks = dict(sus_clocks, loaded_window_nvidia_smi=smi)
+        if dec.status() != 0:
+            raise RuntimeError("device status word set during the sustained steps")
+        sustained = {"us_per_step": round(statistics.mean(sus_ms) * 1e3, 2),
+                     "value": round(world * kv_bytes / (max_over_ranks(statistics.mean(sus_ms), world, dev) / 1e3)
+                                    / 1e9, 2),
+                     "partial_us": round(statistics.mean(sus_part_ms) * 1e3, 2),
+                     "clocks": sus_clocks,
+                     "how": f"the same {args.steps} steps after {args.clock_window_s} s of back-to-back steps"}
+    poller.stop()
     total_ms = max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = total_ms / args.steps
     value = world * kv_bytes * args.steps / (total_ms / 1e3) / 1e9
@@ -357,14 +469,7 @@ def run_ours(args):
             raise RuntimeError("e2e read-back differs from the device result")
 
     peak, peak_kind = measured_peak()
-    part_avg_s = statistics.mean(part_ms) / 1e3
-    achieved = alg_bytes_partial / part_avg_s / 1e9
-    # binding roofline: the larger of (bytes at HBM bandwidth) and (flops at tensor peak); the
-    # kernel runs inside a seconds-long loaded window, so the tensor peak is the sustained one
     flops = algorithmic_flops(inp.seq_lens.tolist(), T, H)
-    tpeak, tpeak_kind = measured_tensor_peak(g.dtype, sustained=True)
-    t_hbm = alg_bytes_partial / (peak * 1e9)
-    t_tensor = flops / (tpeak * 1e12)
     # the partial kernel's function name, as ncu lists it
     if plan.kernel == 2:
         kname = "simt_partial_kernel"
@@ -372,19 +477,20 @@ def run_ours(args):
         kname = "tc_fp8_pair_kernel" if plan.kernel == 1 else "tc_fp8_partial_kernel"
     else:
         kname = "tc16_pair_kernel" if plan.schedule == 1 else "tc_partial_kernel"
-    hbm_side = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "peak_source": peak_kind,
-                "floor_us": round(t_hbm * 1e6, 2)}
-    tensor_side = {"bound": "tensor", "achieved": round(flops / part_avg_s / 1e12, 1), "peak": round(tpeak, 1),
-                   "unit": "TFLOP/s", "frac": round(flops / part_avg_s / 1e12 / tpeak, 4),
-                   "peak_source": tpeak_kind, "floor_us": round(t_tensor * 1e6, 2)}
-    bind, other = (tensor_side, hbm_side) if t_tensor > t_hbm else (hbm_side, tensor_side)
-    roofline = dict(bind)
+    # The timed steps are a few milliseconds of work after a short warm-up: the tensor side is
+    # taken against the measured burst peak. The sustained block (after the loaded window, under
+    # the power cap) is taken against the measured sustained peak.
+    roofline = roofline_fields(alg_bytes_partial, flops, statistics.mean(part_ms) / 1e3, peak, peak_kind,
+                               g.dtype, sustained=False)
     roofline.update({"traffic": traffic_from_profile(args.workload, kname), "kernel": kname,
                      "alg_bytes_per_launch": int(alg_bytes_partial), "alg_flops_per_launch": int(flops),
                      "partial_us": round(statistics.mean(part_ms) * 1e3, 2),
-                     "combine_tail_us": round((statistics.mean(step_ms) - statistics.mean(part_ms)) * 1e3, 2),
-                     "other": other})
+                     "combine_tail_us": round((statistics.mean(step_ms) - statistics.mean(part_ms)) * 1e3, 2)})
+    if sustained is not None:
+        r2 = roofline_fields(alg_bytes_partial, flops, sustained["partial_us"] / 1e6, peak, peak_kind, g.dtype,
+                             sustained=True)
+        sustained["roofline"] = {"bound": r2["bound"], "frac": r2["frac"], "hbm_frac": r2["hbm_frac"],
+                                 "tensor_frac": r2["tensor_frac"], "tensor_peak": r2["tensor_peak"]}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -418,7 +524,7 @@ def run_ours(args):
                    "parallelism": f"replicas x{world}"},
         "gpu_launches": kernels_per_step * args.steps,
         "wall_s_timed": round(wall1 - wall0, 4),
-        "roofline": roofline, "e2e": e2e, "clocks": clocks, "cpu_baseline": cpu,
+        "roofline": roofline, "e2e": e2e, "clocks": clocks, "sustained": sustained, "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
 
@@ -448,10 +554,39 @@ def cpu_baseline(workload, target_s=10.0, max_entries=16):
         t_total += time.perf_counter() - t0
         work_bytes += n * 576 * (1 if inp.dtype == "fp8" else 2)
         entries += 1
-    return {"value": round(work_bytes / t_total / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+    cores = oracle.num_threads()
+    one = cpu_baseline_one_core(workload)
+    return {"value": round(work_bytes / t_total / 1e9, 4), "unit": "GB/s", "cores": cores,
             "kind": "oracle", "seconds": round(t_total, 3),
             "sample": f"{entries} batch entries of the workload ({n} keys, all {rows_total} query rows each); "
-                      f"KV bytes of those entries over the oracle's time"}
+                      f"KV bytes of those entries over the oracle's time",
+            "one_core": one}
+
+
+def cpu_baseline_one_core(workload, target_s=5.0):
+    """The oracle on one host core: query rows of the workload's first entry, 32 at a time, until
+    about target_s seconds; KV bytes counted per row (the fraction of the entry's rows done)."""
+    import oracle
+    inp, n = _oracle_sample_inputs(workload, 0)
+    rows_total = inp.q_len * inp.heads
+    esize = 1 if inp.dtype == "fp8" else 2
+    cores = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        t_total, done = 0.0, 0
+        while done < rows_total and (done == 0 or t_total < target_s):
+            rows = list(range(done, min(rows_total, done + 32)))
+            t0 = time.perf_counter()
+            oracle.mla_decode(inp.q, inp.kv_cache, inp.block_tables, inp.seq_lens, inp.softmax_scale,
+                              dtype=inp.dtype, q_scale=inp.q_scale, kv_scale=inp.kv_scale, rows=rows)
+            t_total += time.perf_counter() - t0
+            done += len(rows)
+    finally:
+        oracle.set_num_threads(cores)
+    work_bytes = n * 576 * esize * done / rows_total
+    return {"value": round(work_bytes / t_total / 1e9, 5), "unit": "GB/s", "cores": 1, "seconds": round(t_total, 3),
+            "sample": f"{done} of the {rows_total} query rows of one batch entry ({n} keys); "
+                      f"KV bytes scaled by the row fraction"}
 
 
 def run_reference(args):
