@@ -48,25 +48,6 @@ def _headers():
 _SPILL = re.compile(r"(\d+) bytes spill stores, (\d+) bytes spill loads")
 
 
-# Kernels that split registers with setmaxnreg must be launched with exactly
-# the register count their split was computed for (a smaller pool could make
-# setmaxnreg.inc wait forever).
-_EXACT_REGS = {}
-
-
-def _check_regs(log: str, src: str) -> None:
-    fn = None
-    for line in log.splitlines():
-        m = re.search(r"Compiling entry function '([^']+)'", line)
-        if m:
-            fn = m.group(1)
-        m = re.search(r"Used (\d+) registers", line)
-        if m and fn:
-            for name, regs in _EXACT_REGS.items():
-                if name in fn and int(m.group(1)) != regs:
-                    raise RuntimeError(f"{fn} uses {m.group(1)} registers, its register split needs {regs}")
-
-
 def _check_spills(log: str, src: str) -> None:
     fn = None
     for line in log.splitlines():
@@ -102,7 +83,6 @@ def build(force: bool = False, verbose: bool = False) -> str:
         if verbose:
             print(log)
         _check_spills(log, src)
-        _check_regs(log, src)
         changed = True
     if changed or os.path.getmtime(LIB_PATH) < max(os.path.getmtime(o) for o in objs):
         tmp = LIB_PATH + f".tmp{os.getpid()}"

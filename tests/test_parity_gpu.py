@@ -332,13 +332,14 @@ def test_window_past_every_length_is_bitwise_full_attention(dtype):
     assert torch.equal(o0, ow) and torch.equal(l0, lw)
 
 
-@pytest.mark.parametrize("name", ["fp8_long_b16", "fold_fp16_h16"])
-def test_window_full_size_sampled_rows(name):
-    """Full-size workloads with an 8192-key window (for FP8 entries this also takes
-    the two-term P encoding, which the kernel picks for rows of fewer than 16384 keys)."""
+@pytest.mark.parametrize("name,window", [("fp8_long_b16", 8192), ("fp8_long_b16", 4096), ("fold_fp16_h16", 8192)])
+def test_window_full_size_sampled_rows(name, window):
+    """Full-size workloads with a sliding window. An FP8 row then attends to min(n, W) keys, so
+    W = 8192 keeps the single-term P encoding (two terms are taken below 8192 keys) and W = 4096
+    takes the two-term encoding on every row of the 80K-key entries."""
     inp = make_inputs(name, device=torch.device("cuda", 0))
-    out, lse, status, dec = run(inp, "auto", window=8192)
-    assert dec.plan.window == 8192 and status == 0
+    out, lse, status, dec = run(inp, "auto", window=window)
+    assert dec.plan.window == window and status == 0
     rows = sample_rows(inp.batch, inp.q_len, inp.heads, n=48, seed=45)
-    ref_o, ref_l = oracle_rows(inp, rows, window=8192)
-    compare(out, lse, ref_o, ref_l, inp.dtype, rows=rows, what=f"{name} W=8192")
+    ref_o, ref_l = oracle_rows(inp, rows, window=window)
+    compare(out, lse, ref_o, ref_l, inp.dtype, rows=rows, what=f"{name} W={window}")
