@@ -133,11 +133,14 @@ __device__ __forceinline__ void combine_unit(const DecodeArgs& a, int u, int rb,
   const int M = p.rows_per_unit;
   const int U = p.batch * p.q_groups;
   const int32_t* tbl = a.sched;
-  const int64_t start = tbl[u], end = tbl[u + 1], W = tbl[U];
+  const int sl = sched_slot(p, u);  // the unit's position in the schedule's sequence
+  const int64_t start = tbl[sl], end = tbl[sl + 1], W = tbl[U];
   const int np = tbl[U + 1];
   const UnitGeom ug = unit_geom(a, u, false);
-  // pairs holding the unit's first and last tiles (tile starts are weighted)
-  const int p0 = end > start ? balanced_pair_of(start, W, np) : 0;
+  // pairs holding the unit's first and last tiles (tile starts are weighted;
+  // the first follows the unit's lead-in)
+  const int lead = end > start ? unit_lead_weight(sl, 1) : 0;
+  const int p0 = end > start ? balanced_pair_of(start + lead, W, np) : 0;
   const int p1 = end > start ? balanced_pair_of(end - tile_weight(p, ug), W, np) : 0;
   if (end > start && p0 == p1) return;  // a whole unit: written by its pair
   if (end > start) {
@@ -159,10 +162,10 @@ __device__ __forceinline__ void combine_unit(const DecodeArgs& a, int u, int rb,
     return;
   }
   // Pair p0 kept the unit in slot 2p0 if it was its first piece (each pair
-  // records its first unit in the table), else in 2p0 + 1; every later pair
-  // starts inside the unit (slot 2q). Pair p0's record precedes its piece
-  // arrivals, which the counter wait above acquired.
-  const int64_t first_slot = tbl[U + 2 + p0] == u ? 2 * (int64_t)p0 : 2 * (int64_t)p0 + 1;
+  // records the schedule position of its first unit in the table), else in
+  // 2p0 + 1; every later pair starts inside the unit (slot 2q). Pair p0's
+  // record precedes its piece arrivals, which the counter wait above acquired.
+  const int64_t first_slot = tbl[U + 2 + p0] == sl ? 2 * (int64_t)p0 : 2 * (int64_t)p0 + 1;
 
   auto slot = [&](int q) -> int64_t { return q == p0 ? first_slot : 2 * (int64_t)q; };
 

@@ -19,9 +19,10 @@ constexpr int kMaxBalancedUnits = 16384;        // decode units (entry x query g
 constexpr int kMaxVarlenUnits = 1 << 16;        // units of a ragged-query (prefill) plan
 
 // Balanced schedule table at the end of the workspace: int32 weighted start
-// of every unit (U + 1 entries, the last = W, the total tile weight), the
-// number of pairs that have work, then each pair's first unit (-1: none).
-// Written by the partial kernel, read by the combine.
+// of every schedule slot (U + 1 entries, the last = W, the total weight; slot
+// s holds unit sched_unit(s), see pair_schedule.cuh), the number of pairs that
+// have work, then the slot of each pair's first unit (-1: none). Written by
+// the partial kernel, read by the combine.
 // Balanced schedule: per-unit counts of finished partial pieces, then the
 // unit table's ready flag; right after the status header, and cleared with it
 // before every launch of the partial kernel.
@@ -39,10 +40,24 @@ inline uint64_t balanced_table_bytes(int64_t units) {
 // 16384 (the bound is 3e-2), and the worst element uses 1.04, 0.26, 0.20 and
 // 0.15 of its tolerance; with two terms both stay at 1.7e-3 and 0.11.
 constexpr int kTwoTermKeys = 8192;
+// A piece transition (a pair moving on to a new unit) costs about as much as
+// 8 pair tiles: the cut piece's epilogue, the drain of its last MMAs before the
+// next unit's query block can be loaded, and the refill. Measured on the 80K-key
+// FP8 batch of 16 entries, pairs whose range crosses an entry boundary finished
+// 8.3 us (~8 tiles) after the others. The balanced schedule therefore charges
+// every unit with tiles but the first of the sequence a lead-in of this
+// weight (a tile weighs 2 or 3) at its weighted start, ahead of its first
+// tile, so that a pair whose range holds a unit start takes correspondingly
+// fewer tiles. `slot` is the unit's position in the schedule's sequence.
+constexpr int kPieceLeadWeight = 16;
+__host__ __device__ inline int unit_lead_weight(int slot, int tiles) {
+  return (tiles > 0 && slot > 0) ? kPieceLeadWeight : 0;
+}
 // Piece lists too long for a CTA's shared memory go to a spill area right
 // before the unit table: per CTA rank, U + P pieces of 3 int32 (a pair's
-// pieces are the units its range meets; pair p's list starts at entry
-// first_unit(p) + p, so the lists of consecutive pairs never overlap).
+// pieces are the units its range meets, consecutive in the schedule's
+// sequence; pair p's list starts at entry first_slot(p) + p, so the lists of
+// consecutive pairs never overlap).
 inline uint64_t balanced_spill_bytes(int64_t units, int pairs) {
   return ((uint64_t)2 * (units + pairs) * 12 + 255) & ~uint64_t(255);
 }

@@ -4,10 +4,23 @@
 // device seq_lens (and, for ragged queries, cu_q): from the tile of the
 // lowest key a row of the unit sees to the tile of the highest. A tile
 // weighs 2, or 3 when its P.V runs twice (FP8 two-term P), so that pairs get
-// equal work rather than equal tiles. The units' runs, in unit order, form one
-// sequence of total weight W; pair p takes the tiles whose start lies in
-// [floor(W p / np), floor(W (p + 1) / np)) and walks them as a list of pieces
-// (the units its range meets, each cut to the range).
+// equal work rather than equal tiles, and every unit with tiles but the first
+// starts with a lead-in of kPieceLeadWeight, the cost of a piece transition.
+// The units' runs form one sequence of total weight W; pair p takes the tiles
+// whose start lies in [floor(W p / np), floor(W (p + 1) / np)) and walks them
+// as a list of pieces (the units its range meets, each cut to the range).
+//
+// Order of the sequence. A decode entry with G > 1 query groups (more query
+// tokens than fit one 128-row tile) has G units over the same pages. In entry
+// order they sit next to each other and the same pair reads the entry's pages
+// once per group, far apart in time, so each page comes from DRAM G times.
+// Decode plans with G > 1 therefore take the units group-major (group 0 of
+// every entry, then group 1, ...): with equal ranges, pair p and the pair
+// W / G weight further on walk the same pages at about the same time, and the
+// later read is served by L2. Ragged prefill keeps entry order (its groups
+// see different key spans and its pool is mostly L2-resident). Positions in
+// the sequence are schedule slots; sched_unit / sched_slot map between them
+// and units.
 #pragma once
 
 #include "device_common.cuh"
@@ -29,6 +42,17 @@ constexpr int kMaxSmemPieces = 64;  // pieces a pair keeps in shared memory; the
 constexpr uint32_t kSchedBytes = 1024;
 static_assert(kMaxSmemPieces * sizeof(Piece) + sizeof(SchedInfo) <= kSchedBytes, "schedule area");
 constexpr int kMinPairWeight = 4;  // pairs get at least this much weight (>= the heaviest tile)
+
+// Unit at schedule slot s, and the slot of unit u (u = entry * G + group).
+__host__ __device__ __forceinline__ bool sched_group_major(const mla_plan& p) {
+  return !p.varlen && p.q_groups > 1;
+}
+__host__ __device__ __forceinline__ int sched_unit(const mla_plan& p, int s) {
+  return sched_group_major(p) ? (s % p.batch) * p.q_groups + s / p.batch : s;
+}
+__host__ __device__ __forceinline__ int sched_slot(const mla_plan& p, int u) {
+  return sched_group_major(p) ? (u % p.q_groups) * p.batch + u / p.q_groups : u;
+}
 
 // Keys the unit's first row sees: the fewest of any of its rows (ragged
 // prefill units early in an entry see only a few keys even when the entry
@@ -74,30 +98,31 @@ __device__ __forceinline__ int warp_incl_scan(int v) {
 }
 
 // The whole block: the schedule of this pair. Every thread takes a run of
-// consecutive units; block scans (two barriers in all) give each run's
-// weighted start and each thread's first piece index. The pieces of the
-// pair's range are written in unit order, the first kMaxSmemPieces to shared
+// consecutive schedule slots; block scans (two barriers in all) give each
+// run's weighted start and each thread's first piece index. The pieces of the
+// pair's range are written in slot order, the first kMaxSmemPieces to shared
 // memory and, when there are more, all of them to this CTA's part of the
-// spill area (read back by load_piece). CTA 0 of pair 0 also writes the unit
+// spill area (read back by load_piece). CTA 0 of pair 0 also writes the slot
 // start table the combine reads, then its ready flag; CTA 0 of every pair
-// records its first unit there (the combine's slot rule).
+// records its first slot there (the combine's slot rule).
 template <int kKeys>
 __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uint8_t* sched_area) {
   const mla_plan& p = a.plan;
   Piece* smem_list = reinterpret_cast<Piece*>(sched_area);
   SchedInfo* info = reinterpret_cast<SchedInfo*>(sched_area + kMaxSmemPieces * sizeof(Piece));
   int* scan1 = reinterpret_cast<int*>(sched_area + kSchedScratchOff);  // [warp]
-  int4* scan2 = reinterpret_cast<int4*>(scan1 + kMaxSchedWarps);       // [warp]: pieces, tiles, two, first unit
+  int4* scan2 = reinterpret_cast<int4*>(scan1 + kMaxSchedWarps);       // [warp]: pieces, tiles, two, first slot
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = (int)(blockDim.x >> 5);
   const int U = p.batch * p.q_groups;
   const int per = (U + (int)blockDim.x - 1) / (int)blockDim.x;
-  const int u_beg = min(U, tid * per), u_end = min(U, u_beg + per);
+  const int s_beg = min(U, tid * per), s_end = min(U, s_beg + per);  // this thread's schedule slots
   const bool writer = pair == 0 && rank == 0;
   // scan 1: the weighted start of this thread's run
   int run = 0;
-  for (int u = u_beg; u < u_end; ++u) {
-    const UnitGeom ug = unit_geom(a, u, writer);
-    run += unit_span_tiles<kKeys>(ug) * tile_weight(p, ug);
+  for (int sl = s_beg; sl < s_end; ++sl) {
+    const UnitGeom ug = unit_geom(a, sched_unit(p, sl), writer);
+    const int t = unit_span_tiles<kKeys>(ug);
+    run += unit_lead_weight(sl, t) + t * tile_weight(p, ug);
   }
   int incl = warp_incl_scan(run);
   if (lane == 31) scan1[warp] = incl;
@@ -113,10 +138,11 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uin
   const int64_t hi = pair < np ? balanced_lo(pair + 1, W, np) : W;
   if (writer) {
     int start = excl;
-    for (int u = u_beg; u < u_end; ++u) {
-      a.sched[u] = start;
-      const UnitGeom ug = unit_geom(a, u, false);
-      start += unit_span_tiles<kKeys>(ug) * tile_weight(p, ug);
+    for (int sl = s_beg; sl < s_end; ++sl) {
+      a.sched[sl] = start;
+      const UnitGeom ug = unit_geom(a, sched_unit(p, sl), false);
+      const int t = unit_span_tiles<kKeys>(ug);
+      start += unit_lead_weight(sl, t) + t * tile_weight(p, ug);
     }
     if (tid == 0) {
       a.sched[U] = W;
@@ -124,38 +150,38 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uin
     }
   }
   // scan 2: this thread's pieces (units of its run with tiles in the range)
-  int cnt = 0, tiles = 0, two = 0, u_first_t = 0;
+  int cnt = 0, tiles = 0, two = 0, s_first_t = 0;
   {
     int start = excl;
-    for (int u = u_beg; u < u_end; ++u) {
-      const UnitGeom ug = unit_geom(a, u, false);
-      const int t = unit_span_tiles<kKeys>(ug), w = tile_weight(p, ug);
+    for (int sl = s_beg; sl < s_end; ++sl) {
+      const UnitGeom ug = unit_geom(a, sched_unit(p, sl), false);
+      const int t = unit_span_tiles<kKeys>(ug), w = tile_weight(p, ug), lead = unit_lead_weight(sl, t);
       int i0, i1;
-      tiles_in_range(start, t, w, lo, hi, i0, i1);
+      tiles_in_range(start + lead, t, w, lo, hi, i0, i1);
       if (i1 > i0) {
-        if (cnt == 0) u_first_t = u;
+        if (cnt == 0) s_first_t = sl;
         ++cnt;
         tiles += i1 - i0;
         if (w == 3) two = 1;
       }
-      start += t * w;
+      start += lead + t * w;
     }
   }
   const int cnt_incl = warp_incl_scan(cnt);
   const int tiles_w = warp_incl_scan(tiles);
   const unsigned has = __ballot_sync(0xffffffffu, cnt > 0);
   const int two_w = __any_sync(0xffffffffu, two);
-  const int first_w = has ? __shfl_sync(0xffffffffu, u_first_t, __ffs(has) - 1) : -1;
+  const int first_w = has ? __shfl_sync(0xffffffffu, s_first_t, __ffs(has) - 1) : -1;
   if (lane == 31) scan2[warp] = make_int4(cnt_incl, tiles_w, two_w, first_w);
   __syncthreads();
-  int base = cnt_incl - cnt, npc = 0, all_tiles = 0, any_two = 0, u_first = -1;
+  int base = cnt_incl - cnt, npc = 0, all_tiles = 0, any_two = 0, s_first = -1;
   for (int w = 0; w < nw; ++w) {
     const int4 x = scan2[w];
     if (w < warp) base += x.x;
     npc += x.x;
     all_tiles += x.y;
     any_two |= x.z;
-    if (u_first < 0 && x.x > 0) u_first = x.w;
+    if (s_first < 0 && x.x > 0) s_first = x.w;
   }
   // the table is complete (every thread wrote its units before the barrier):
   // the combine, which may already run, reads it once the flag is set
@@ -163,16 +189,17 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uin
     __threadfence();
     ptx::st_release_gpu(a.unit_done + U, 1);
   }
-  if (u_first < 0) u_first = 0;
-  const int spill_base = (int)rank * (U + p.split_kv) + u_first + pair;
+  if (s_first < 0) s_first = 0;
+  const int spill_base = (int)rank * (U + p.split_kv) + s_first + pair;
   Piece* spill = npc > kMaxSmemPieces ? reinterpret_cast<Piece*>(a.pieces) + spill_base : nullptr;
   if (cnt > 0) {
     int start = excl, k = base;
-    for (int u = u_beg; u < u_end; ++u) {
+    for (int sl = s_beg; sl < s_end; ++sl) {
+      const int u = sched_unit(p, sl);
       const UnitGeom ug = unit_geom(a, u, false);
-      const int t = unit_span_tiles<kKeys>(ug), w = tile_weight(p, ug);
+      const int t = unit_span_tiles<kKeys>(ug), w = tile_weight(p, ug), lead = unit_lead_weight(sl, t);
       int i0, i1;
-      tiles_in_range(start, t, w, lo, hi, i0, i1);
+      tiles_in_range(start + lead, t, w, lo, hi, i0, i1);
       if (i1 > i0) {
         Piece pc;
         pc.u = u;
@@ -182,7 +209,7 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uin
         if (spill) spill[k] = pc;
         ++k;
       }
-      start += t * w;
+      start += lead + t * w;
     }
   }
   if (tid == 0) {
@@ -190,7 +217,7 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uin
     info->npc = npc;
     info->tiles = all_tiles;
     info->two = any_two;
-    if (rank == 0 && pair < p.split_kv) a.sched[U + 2 + pair] = npc > 0 ? u_first : -1;
+    if (rank == 0 && pair < p.split_kv) a.sched[U + 2 + pair] = npc > 0 ? s_first : -1;
   }
 }
 

@@ -140,8 +140,9 @@ int plan_impl(int batch, int q_len, int num_heads, int max_seq_len, int dtype, i
   // start; decode batches of more units than kMaxBalancedUnits take fixed
   // splits instead (FP8: the solo kernel; 16-bit: the exchange kernel).
   p.varlen = varlen ? 1 : 0;
-  // the balanced schedule's int32 tile weights (3 per 64 keys at most) must fit
-  const bool weights_fit = units * tiles * 3 < (int64_t)INT32_MAX;
+  // the balanced schedule's int32 weights (3 per 64 keys at most, plus a unit's
+  // lead-in) must fit
+  const bool weights_fit = units * (tiles * 3 + kPieceLeadWeight) < (int64_t)INT32_MAX;
   const int64_t max_units = weights_fit ? (varlen ? kMaxVarlenUnits : kMaxBalancedUnits) : 0;
   if (kern == MLA_KERNEL_TCGEN05 && units > max_units) {
     // ragged queries run only on the balanced schedule (or the SIMT kernel)

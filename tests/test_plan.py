@@ -85,14 +85,23 @@ def test_balanced_plan_uses_every_sm_and_caps_units():
     assert big16.schedule == 0 and big16.kernel == 1
 
 
+LEAD = 16  # weight of a piece transition, charged at the start of every unit with tiles but the first
+
+
+def _lead(u, t):
+    return LEAD if (t > 0 and u > 0) else 0
+
+
 def _balanced_schedule(tiles, P, weights=None, min_weight=4):
-    """Host model of the device schedule: a tile weighs 2, or 3 with FP8 two-term P; pair p takes
-    the tiles whose weighted start lies in [W p / np, W (p + 1) / np). Returns unit starts, W,
-    np, each pair's pieces (u, t0, t1) and each pair's first unit (-1: none)."""
+    """Host model of the device schedule: a tile weighs 2, or 3 with FP8 two-term P, and every
+    unit with tiles but the first starts with a lead-in of LEAD (the cost of moving on to a new
+    unit); pair p takes the tiles whose weighted start lies in [W p / np, W (p + 1) / np).
+    Returns unit starts, W, np, each pair's pieces (u, t0, t1) and each pair's first unit
+    (-1: none)."""
     weights = weights or [2] * len(tiles)
     starts = [0]
-    for t, w in zip(tiles, weights):
-        starts.append(starts[-1] + t * w)
+    for u, (t, w) in enumerate(zip(tiles, weights)):
+        starts.append(starts[-1] + _lead(u, t) + t * w)
     W = starts[-1]
     np_ = max(1, min(P, W // min_weight))
     pieces = []
@@ -100,7 +109,7 @@ def _balanced_schedule(tiles, P, weights=None, min_weight=4):
         lo, hi = (W * p // np_, W * (p + 1) // np_) if p < np_ else (W, W)
         pp = []
         for u, (t, w) in enumerate(zip(tiles, weights)):
-            s0 = starts[u]
+            s0 = starts[u] + _lead(u, t)  # weighted start of the unit's first tile
             i0 = min(t, -(-(lo - s0) // w)) if lo > s0 else 0
             i1 = min(t, -(-(hi - s0) // w)) if hi > s0 else 0
             if i1 > i0:
@@ -149,7 +158,7 @@ def test_balanced_schedule_covers_each_tile_once(tiles, weights):
     for u, t in enumerate(tiles):
         if t == 0:
             continue
-        p0 = _pair_of(starts[u], W, np_)
+        p0 = _pair_of(starts[u] + _lead(u, t), W, np_)
         p1 = _pair_of(starts[u + 1] - w_of[u], W, np_)
         assert seen[(u, 0)] == p0 and seen[(u, t - 1)] == p1
         if p0 == p1:
@@ -161,13 +170,38 @@ def test_balanced_schedule_covers_each_tile_once(tiles, weights):
             assert slot_of_piece[(u, q)] == slot
 
 
+def _tile_work(pp, weights):
+    return sum((t1 - t0) * weights[u] for u, t0, t1 in pp)
+
+
+def _lead_overlap(starts, tiles, W, np_, p):
+    """Weight of the units' lead-ins that lies inside pair p's range."""
+    lo, hi = W * p // np_, W * (p + 1) // np_
+    return sum(max(0, min(hi, starts[u] + _lead(u, t)) - max(lo, starts[u])) for u, t in enumerate(tiles))
+
+
 def test_weighted_schedule_evens_out_two_term_work():
     # half the units have two-term tiles (weight 3): per-pair weight stays within one tile
     tiles = [100] * 40
     weights = [3] * 20 + [2] * 20
     starts, W, np_, pieces, _ = _balanced_schedule(tiles, 74, weights)
-    work = [sum((t1 - t0) * weights[u] for u, t0, t1 in pp) for pp in pieces]
-    assert max(work) - min(work) <= 2 * 3
+    load = [_tile_work(pp, weights) + _lead_overlap(starts, tiles, W, np_, p) for p, pp in enumerate(pieces)]
+    # tile work plus the lead-in weight inside the range stays within a tile of the range size
+    assert max(load) - min(load) <= 2 * 3
+
+
+def test_lead_in_gives_pairs_that_cross_a_unit_boundary_fewer_tiles():
+    # 16 entries of 640 pair tiles (the 80K-key FP8 batch): a pair whose range holds a unit start
+    # pays a piece transition, so it takes LEAD / 2 fewer tiles; tile work plus the lead-ins a
+    # pair holds stays within one tile of every other pair's
+    tiles = [640] * 16
+    starts, W, np_, pieces, _ = _balanced_schedule(tiles, 74)
+    work = [_tile_work(pp, [2] * 16) for pp in pieces]
+    load = [w + _lead_overlap(starts, tiles, W, np_, p) for p, w in enumerate(work)]
+    assert max(load) - min(load) <= 2 * 2
+    crossing = [w for p, w in enumerate(work) if len(pieces[p]) == 2]
+    single = [w for p, w in enumerate(work) if len(pieces[p]) == 1]
+    assert crossing and max(crossing) < min(single)
 
 
 def test_split_fills_the_gpu_for_the_long_fp8_case():
@@ -305,6 +339,44 @@ def test_spilled_piece_lists_of_different_pairs_never_overlap(seed):
             idx = base + k
             assert 0 <= idx < U + P and idx not in used
             used.add(idx)
+
+
+def _sched_unit(B, G, varlen, s):
+    """Host mirror of sched_unit: decode plans with G > 1 query groups order the schedule
+    group-major (slot s = g * B + b holds unit b * G + g); ragged prefill keeps entry order."""
+    return (s % B) * G + s // B if (not varlen and G > 1) else s
+
+
+def _sched_slot(B, G, varlen, u):
+    return (u % G) * B + u // G if (not varlen and G > 1) else u
+
+
+@pytest.mark.parametrize("B,G,varlen", [(1, 1, 0), (16, 1, 0), (32, 2, 0), (128, 2, 0), (3, 4, 0), (7, 3, 1),
+                                        (5, 1024, 1)])
+def test_schedule_slot_order_is_a_bijection_and_group_major_for_decode(B, G, varlen):
+    U = B * G
+    units = [_sched_unit(B, G, varlen, s) for s in range(U)]
+    assert sorted(units) == list(range(U))
+    assert all(_sched_slot(B, G, varlen, u) == s for s, u in enumerate(units))
+    if not varlen and G > 1:
+        # the first B slots are group 0 of every entry, in entry order
+        assert units[:B] == [b * G for b in range(B)]
+    else:
+        assert units == list(range(U))
+
+
+def test_group_major_order_puts_both_groups_of_an_entry_on_pairs_half_the_sequence_apart():
+    # 128 entries x 2 groups of equal length (the high-concurrency shape): pair p and pair p + np/2
+    # cover the same entries' key tiles, so their reads of a page are close in time
+    B, G, t = 128, 2, 50
+    tiles = [t] * (B * G)  # in slot order (group-major)
+    starts, W, np_, pieces, _ = _balanced_schedule(tiles, 74)
+    half = np_ // 2
+    for p in range(half):
+        a = {(_sched_unit(B, G, 0, s) // G, i) for s, t0, t1 in pieces[p] for i in range(t0, t1)}
+        b = {(_sched_unit(B, G, 0, s) // G, i) for s, t0, t1 in pieces[p + half] for i in range(t0, t1)}
+        # (entry, key tile) sets overlap in all but a few tiles (the lead-in of slot 0 shifts one half)
+        assert len(a & b) >= 0.9 * min(len(a), len(b))
 
 
 def _unit_span(n, qlen, g, F, window):
