@@ -441,6 +441,7 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
       if (lane == 0) arrive_lead(L::B_Q_TMEM);
 
       float m_grp = -INFINITY, l_grp = 0.f;  // this group's reference and partial sum (this half row)
+      float m_last = -INFINITY;              // the reference of this group's previous tile of the piece
       const int j_first = (jt & 1) == grp ? 0 : 1;
       int pg_next = j_first < c.n_pt ? piece_entry16(c, j_first) : 0;
       for (int j = j_first; ok && j < c.n_pt; j += 2) {
@@ -483,26 +484,37 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
           }
           mt = fmaxf(m2[0], m2[1]) * sl2;
         }
-        // the other half of the row lives in the warp of quarter q^2
-        xm[((grp * 2 + ph) * 2 + hf) * 64 + rl] = mt;
+        // The other half of the row lives in the warp of quarter q^2: this
+        // half's maximum is published now and the partner's read when needed.
+        float* xm_own = xm + ((grp * 2 + ph) * 2 + hf) * 64;
+        const float* xm_other = xm + ((grp * 2 + ph) * 2 + (hf ^ 1)) * 64;
+        xm_own[rl] = mt;
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(L::B_X + grp));
-        if (!(ok = warp_wait_cta(bar(L::B_X + grp), ph, abort_flag, a.status))) break;
-        mt = fmaxf(mt, xm[((grp * 2 + ph) * 2 + (hf ^ 1)) * 64 + rl]);
-        // reference maximum after the previous tile (from the other group),
-        // lazily updated; a new piece starts afresh but takes the hand-off
-        float m_prev = -INFINITY;
-        if (jg > 0) {
-          if (!(ok = warp_wait_cta(bar(L::B_M_READY + (buf ^ 1)), ((jg - 1) >> 1) & 1, abort_flag, a.status)))
-            break;
-          if (j > 0) m_prev = mref[(buf ^ 1) * 64 + rl];
+        // The reference maximum of the tile, as in the FP8 pair kernel: in
+        // exact order (a piece's first two tiles, or a half whose scores
+        // exceed the group's last reference by more than kTau) the row
+        // maximum and the previous tile's reference (the other group's hand-
+        // off; a new piece starts afresh but takes it) come before P; in the
+        // steady state P is computed against this group's last reference and
+        // the exchange and hand-off are read afterwards to confirm it, P being
+        // computed again if the previous tile or this one moved the reference.
+        bool spec = j >= 2 && m_last != -INFINITY && mt <= m_last + kTau;
+        spec = __all_sync(0xffffffffu, spec);
+        float m_prev = -INFINITY, m_j = m_last;
+        if (!spec) {
+          if (!(ok = warp_wait_cta(bar(L::B_X + grp), ph, abort_flag, a.status))) break;
+          mt = fmaxf(mt, xm_other[rl]);
+          if (jg > 0) {
+            if (!(ok = warp_wait_cta(bar(L::B_M_READY + (buf ^ 1)), ((jg - 1) >> 1) & 1, abort_flag, a.status)))
+              break;
+            if (j > 0) m_prev = mref[(buf ^ 1) * 64 + rl];
+          }
+          m_j = (mt > m_prev + kTau) ? mt : m_prev;
+          mref[buf * 64 + rl] = m_j;  // both halves write the same value
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(L::B_M_READY + buf));
         }
-        const float m_j = (mt > m_prev + kTau) ? mt : m_prev;
-        mref[buf * 64 + rl] = m_j;  // both halves write the same value
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(L::B_M_READY + buf));
-        const float alpha = (m_j == m_prev) ? 1.f : ex2_approx(m_prev - m_j);  // O rescale for tile j
-        const float m_use = (m_j == -INFINITY) ? 0.f : m_j - kSigma;
 
         // P buffer is free once the P.V two tiles back has finished
         if (jg >= 2 && !(ok = warp_wait_cta(bar(L::B_P_EMPTY + buf), ph ^ 1, abort_flag, a.status))) break;
@@ -510,37 +522,54 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
         // P = 2^(s * sl2 - m_use) in the inputs' 16-bit type, 8 keys (one
         // 16-byte chunk) at a time; this half's 32 keys are bytes
         // [64hf, 64hf + 64) of the 128-byte P row.
-        const uint64_t sl2x2 = f2_pack(sl2, sl2), nmx2 = f2_pack(-m_use, -m_use);
-        uint64_t se2[2] = {0ull, 0ull};
+        const uint64_t sl2x2 = f2_pack(sl2, sl2);
+        uint64_t se2[2];
         uint8_t* prow = smem + L::kPOff + buf * L::kPBuf + rl * 128;
+#pragma unroll 1
+        for (;;) {
+          const float m_use = (m_j == -INFINITY) ? 0.f : m_j - kSigma;
+          const uint64_t nmx2 = f2_pack(-m_use, -m_use);
+          se2[0] = se2[1] = 0ull;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          uint32_t pk[4];
+          for (int u = 0; u < 4; ++u) {
+            uint32_t pk[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int e = 8 * u + 2 * i;
-            float a0, a1;
-            f2_unpack(fma_f32x2(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nmx2), a0, a1);
-            const float p0 = ex2_approx(a0);
-            const float p1 = ex2_approx(a1);
-            se2[i & 1] = add_f32x2(se2[i & 1], f2_pack(p0, p1));
-            if (kBf16) {
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-              pk[i] = *reinterpret_cast<uint32_t*>(&h2);
-            } else {
-              __half2 h2 = __floats2half2_rn(p0, p1);
-              pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+            for (int i = 0; i < 4; ++i) {
+              const int e = 8 * u + 2 * i;
+              float a0, a1;
+              f2_unpack(fma_f32x2(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nmx2), a0, a1);
+              const float p0 = ex2_approx(a0);
+              const float p1 = ex2_approx(a1);
+              se2[i & 1] = add_f32x2(se2[i & 1], f2_pack(p0, p1));
+              if (kBf16) {
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+              } else {
+                __half2 h2 = __floats2half2_rn(p0, p1);
+                pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+              }
             }
+            const int phys = (4 * hf + u) ^ (rl & 7);
+            *reinterpret_cast<uint4*>(prow + phys * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
-          const int phys = (4 * hf + u) ^ (rl & 7);
-          *reinterpret_cast<uint4*>(prow + phys * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          if (!spec) break;
+          // confirm the speculation (j >= 2 here, so jg > 0 and j > 0)
+          if (!(ok = warp_wait_cta(bar(L::B_X + grp), ph, abort_flag, a.status))) break;
+          mt = fmaxf(mt, xm_other[rl]);
+          if (!(ok = warp_wait_cta(bar(L::B_M_READY + (buf ^ 1)), ((jg - 1) >> 1) & 1, abort_flag, a.status)))
+            break;
+          m_prev = mref[(buf ^ 1) * 64 + rl];
+          const float m_x = (mt > m_prev + kTau) ? mt : m_prev;
+          mref[buf * 64 + rl] = m_x;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(L::B_M_READY + buf));
+          spec = false;
+          const bool redo = __any_sync(0xffffffffu, m_x != m_j);
+          m_j = m_x;
+          if (!redo) break;
         }
-        float s0, s1, s2, s3;
-        f2_unpack(se2[0], s0, s1);
-        f2_unpack(se2[1], s2, s3);
-        const float sum = (s0 + s1) + (s2 + s3);
-        l_grp = (m_grp == m_j) ? l_grp + sum : fmaf(l_grp, ex2_approx(m_grp - m_j), sum);
-        m_grp = m_j;
+        if (!ok) break;
+        const float alpha = (m_j == m_prev) ? 1.f : ex2_approx(m_prev - m_j);  // O rescale for tile j
 
         // rescale this thread's 256 O columns if the reference maximum moved
         // (not on a piece's first tile: O is reset by its first P.V)
@@ -567,6 +596,15 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
         tc_fence_before();
         __syncwarp();
         if (lane == 0) arrive_lead(L::B_P_FULL + buf);
+
+        // row-sum bookkeeping, after the hand-off (the P.V does not need it)
+        float s0, s1, s2, s3;
+        f2_unpack(se2[0], s0, s1);
+        f2_unpack(se2[1], s2, s3);
+        const float sum = (s0 + s1) + (s2 + s3);
+        l_grp = (m_grp == m_j) ? l_grp + sum : fmaf(l_grp, ex2_approx(m_grp - m_j), sum);
+        m_grp = m_j;
+        m_last = m_j;
       }
       // ---------------------------------------------------------- epilogue of the piece
       // Row sum over both groups and both key halves, relative to the final
