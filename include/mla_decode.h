@@ -128,6 +128,10 @@ typedef struct {
   uint32_t schedule; /* MLA_SCHEDULE_* below */
   int32_t window;    /* sliding window in keys (0 = none); set with mla_decode_plan_window */
   int32_t varlen;    /* 1: ragged query lengths (mla_prefill_plan / mla_prefill), q_len = the longest */
+  int32_t fault_test; /* 0, as the planner sets it. Tests of failure detection only: 1 makes the
+                         FP8 CTA-pair kernel leave the first tile of every pair unloaded, so that
+                         the wait for it runs out (MLA_DEV_TIMEOUT after its 0.5 s limit, no
+                         fault); refused on other plans */
 } mla_plan;
 
 /*

@@ -43,7 +43,7 @@ class MlaPlan(ctypes.Structure):
         ("kernel", ctypes.c_int32), ("num_ctas", ctypes.c_int32),
         ("workspace_bytes", ctypes.c_uint64), ("partial_offset", ctypes.c_uint64),
         ("lse_offset", ctypes.c_uint64), ("magic", ctypes.c_uint32), ("schedule", ctypes.c_uint32),
-        ("window", ctypes.c_int32), ("varlen", ctypes.c_int32),
+        ("window", ctypes.c_int32), ("varlen", ctypes.c_int32), ("fault_test", ctypes.c_int32),
     ]
 
     def as_dict(self):

@@ -81,6 +81,10 @@ int check_plan(const mla_plan* p) {
   if (p->kernel == MLA_KERNEL_TCGEN05_SOLO && p->dtype != MLA_FP8_E4M3) return MLA_ERR_PLAN_MISMATCH;
   if (p->schedule != MLA_SCHEDULE_SPLITS && p->schedule != MLA_SCHEDULE_BALANCED) return MLA_ERR_PLAN_MISMATCH;
   if (p->window < 0) return MLA_ERR_PLAN_MISMATCH;
+  // the failure-detection test mode exists on the FP8 CTA-pair kernel only
+  if (p->fault_test != 0 && !(p->fault_test == 1 && p->dtype == MLA_FP8_E4M3 && p->kernel == MLA_KERNEL_TCGEN05 &&
+                              p->schedule == MLA_SCHEDULE_BALANCED))
+    return MLA_ERR_PLAN_MISMATCH;
   // a window and ragged queries run on the CTA-pair kernels and the SIMT kernel
   if ((p->window > 0 || p->varlen) &&
       !(p->kernel == MLA_KERNEL_SIMT || (p->kernel == MLA_KERNEL_TCGEN05 && p->schedule == MLA_SCHEDULE_BALANCED)))
@@ -191,10 +195,17 @@ int prepare(const mla_plan* plan, const void* q, const void* kv_cache, int64_t n
 }
 
 int run_partial(const DecodeArgs& a, cudaStream_t st) {
-  // the status word, and for the balanced schedule the unit counters after it
-  const size_t clear = a.unit_done ? kHeaderBytes + balanced_counter_bytes((int64_t)a.plan.batch * a.plan.q_groups)
-                                   : sizeof(int32_t);
-  if (cudaError_t e = cudaMemsetAsync(a.status, 0, clear, st); e != cudaSuccess) return cuda_failure(e);
+  // The status word, and for the balanced schedule the unit counters after it.
+  // The balanced schedule clears them with a small kernel launched as a
+  // programmatic dependent, and the partial kernel after it is one too: both
+  // start while the kernel before them in the stream finishes (normally the
+  // previous step's combine), and wait for it before touching memory.
+  if (a.unit_done) {
+    const uint64_t clear = kHeaderBytes + balanced_counter_bytes((int64_t)a.plan.batch * a.plan.q_groups);
+    if (cudaError_t e = launch_workspace_clear(a.status, clear, st); e != cudaSuccess) return cuda_failure(e);
+  } else if (cudaError_t e = cudaMemsetAsync(a.status, 0, sizeof(int32_t), st); e != cudaSuccess) {
+    return cuda_failure(e);
+  }
   if (a.plan.batch == 0 || a.total_q == 0) return MLA_OK;
   cudaError_t e;
   if (a.plan.kernel == MLA_KERNEL_SIMT)

@@ -227,7 +227,23 @@ __device__ __forceinline__ void combine_unit(const DecodeArgs& a, int u, int rb,
   if (lse_writer) a.lse[row] = L;
 }
 
+__device__ __forceinline__ void combine_balanced_block(const DecodeArgs& a, int units_per_block);
+
 __global__ void __launch_bounds__(256) combine_balanced_kernel(const DecodeArgs a, int units_per_block) {
+  // The next step's workspace clear may be launched now: it waits for this
+  // grid's completion before touching the workspace.
+  ptx::launch_dependents();
+  combine_balanced_block(a, units_per_block);
+  // This grid completes only after the partial kernel it depends on: the
+  // partial kernel's last writes (the rows of units one pair finished whole)
+  // may come after every merge here, and work later in the stream relies on
+  // the completion of this grid alone. One block waiting for it is enough (a
+  // grid completes when its last block exits); the others leave as soon as
+  // their merges are done and make room for the rest of the grid.
+  if (blockIdx.x == 0) ptx::grid_dep_wait();
+}
+
+__device__ __forceinline__ void combine_balanced_block(const DecodeArgs& a, int units_per_block) {
   const mla_plan& p = a.plan;
   const int M = p.rows_per_unit;
   const int U = p.batch * p.q_groups;
@@ -256,6 +272,34 @@ __global__ void __launch_bounds__(256) combine_balanced_kernel(const DecodeArgs 
 }
 
 }  // namespace
+
+// Clears the status word, the unit counters and the table's ready flag of a
+// balanced-schedule workspace before the partial kernel runs. Launched as a
+// programmatic dependent of the previous kernel in the stream (normally the
+// previous step's combine, which reads these counters): it lets the partial
+// kernel start its set-up at once and waits for that kernel before writing.
+__global__ void __launch_bounds__(256) workspace_clear_kernel(uint4* ws, int64_t n16) {
+  ptx::launch_dependents();
+  ptx::grid_dep_wait();
+  for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n16; i += (int64_t)gridDim.x * 256)
+    ws[i] = make_uint4(0, 0, 0, 0);
+}
+
+cudaError_t launch_workspace_clear(void* ws, uint64_t bytes, cudaStream_t stream) {
+  const int64_t n16 = (int64_t)(bytes / 16);
+  const int64_t blocks = (n16 + 255) / 256;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(blocks < 148 ? (blocks > 0 ? blocks : 1) : 148));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, workspace_clear_kernel, reinterpret_cast<uint4*>(ws), n16);
+}
 
 cudaError_t launch_combine_balanced(const DecodeArgs& a, cudaStream_t stream) {
   const int64_t units = (int64_t)a.plan.batch * a.plan.q_groups;

@@ -41,15 +41,17 @@ inline uint64_t balanced_table_bytes(int64_t units) {
 // 0.15 of its tolerance; with two terms both stay at 1.7e-3 and 0.11.
 constexpr int kTwoTermKeys = 8192;
 // A piece transition (a pair moving on to a new unit) costs about as much as
-// 8 pair tiles: the cut piece's epilogue, the drain of its last MMAs before the
-// next unit's query block can be loaded, and the refill. Measured on the 80K-key
-// FP8 batch of 16 entries, pairs whose range crosses an entry boundary finished
-// 8.3 us (~8 tiles) after the others. The balanced schedule therefore charges
+// 8 to 12 pair tiles: the cut piece's epilogue, the drain of its last MMAs
+// before the next unit's query block can be loaded, and the refill. Measured
+// on the 80K-key FP8 batch of 16 entries, pairs whose range crosses an entry
+// boundary finished 8.3 us (~8 tiles) after the others; with a lead-in of 16
+// they still finished 5 us later, and 24 was the fastest of 8, 16, 24 and 32
+// on the 4-entry batch (74.1 against 76.1 us) and within 1% elsewhere. The balanced schedule therefore charges
 // every unit with tiles but the first of the sequence a lead-in of this
 // weight (a tile weighs 2 or 3) at its weighted start, ahead of its first
 // tile, so that a pair whose range holds a unit start takes correspondingly
 // fewer tiles. `slot` is the unit's position in the schedule's sequence.
-constexpr int kPieceLeadWeight = 16;
+constexpr int kPieceLeadWeight = 24;
 __host__ __device__ inline int unit_lead_weight(int slot, int tiles) {
   return (tiles > 0 && slot > 0) ? kPieceLeadWeight : 0;
 }
@@ -118,5 +120,8 @@ cudaError_t launch_kv_pack(const void* latent, const void* rope, int64_t n, cons
 cudaError_t launch_kv_amax(const void* latent, const void* rope, int64_t n, int in_dtype, float* amax,
                            cudaStream_t stream);
 cudaError_t launch_combine_balanced(const DecodeArgs& a, cudaStream_t stream);
+// Zeroes `bytes` (a multiple of 16) at the 16-byte aligned `ws`, as a
+// programmatic dependent of the previous kernel in the stream (see combine.cu).
+cudaError_t launch_workspace_clear(void* ws, uint64_t bytes, cudaStream_t stream);
 
 }  // namespace mla

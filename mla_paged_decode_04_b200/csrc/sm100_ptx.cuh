@@ -55,6 +55,9 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
 // Lets the grid launched after this one as its programmatic dependent be
 // scheduled once every CTA of this grid has executed it (or exited).
 __device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// Wait until the grid this one is a programmatic dependent of has completed and
+// its memory operations are visible (returns at once without such a grid).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ int ld_nc_ordered(const int* p) {
   int v;
   asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(p));

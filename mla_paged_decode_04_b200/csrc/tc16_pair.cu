@@ -180,59 +180,12 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
     if (rank == 0) mbar_arrive(bar(i)); else mbar_arrive_remote_relaxed(lead(i));
   };
 
-  // ---------------------------------------------------------------- setup
-  if (threadIdx.x == 0) {
-    mbar_init(bar(L::B_Q_MAIN), 1);
-    mbar_init(bar(L::B_Q_TMEM), 2 * kSoftmaxWarps);
-    for (int i = 0; i < NK; ++i) {
-      mbar_init(bar(L::B_K_FULL + i), 1);
-      mbar_init(bar(L::B_K_EMPTY + i), 1);
-    }
-    for (int i = 0; i < NV; ++i) {
-      mbar_init(bar(L::B_V_FULL + i), 1);
-      mbar_init(bar(L::B_V_EMPTY + i), 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(L::B_S_FULL + i), 1);
-      mbar_init(bar(L::B_S_EMPTY + i), 2 * 4);  // the tile's softmax group in each CTA
-      mbar_init(bar(L::B_P_FULL + i), 2 * 4);
-      mbar_init(bar(L::B_P_EMPTY + i), 1);
-      mbar_init(bar(L::B_M_READY + i), 4);
-      mbar_init(bar(L::B_X + i), 4);
-    }
-    mbar_init(bar(L::B_O_DONE), 1);
-    mbar_init(bar(L::B_O_FINAL), 1);
-    mbar_init(bar(L::B_FIN), kSoftmaxWarps);
-    for (int i = 0; i < NQ; ++i) mbar_init(bar(L::B_QK_DONE + i), 1);
-    mbar_init(bar(L::B_EPI), kSoftmaxWarps);
-    mbar_init(bar(L::B_O_FREE), 2 * kSoftmaxWarps);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (box_q < 64) {
-    // Rows the Q boxes do not cover are zero in the resident Q part (its
-    // rows are independent A rows of S; zero keeps them finite).
-    for (int i = threadIdx.x; i < 4 * (64 - box_q) * 8; i += blockDim.x) {
-      const int ci = i / ((64 - box_q) * 8), rem = i % ((64 - box_q) * 8);
-      reinterpret_cast<uint4*>(smem + L::kQRes + ci * 8192 + box_q * 128)[rem] = make_uint4(0, 0, 0, 0);
-    }
-    fence_proxy_async_smem();
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(smem_u32(tmem_slot), 512);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  cluster_sync();  // both CTAs' barriers and TMEM exist before any cross-CTA use
-  tc_fence_after();
+  // (barriers, TMEM and the cluster sync were set up by pair_setup16)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
     // ------------------------------------------------------------ Q and K-ring loads
     if (lane == 0) {
-      prefetch_tmap(&prm.tm_q);
-      prefetch_tmap(&prm.tm_k8);
-      prefetch_tmap(&prm.tm_kv);
       const uint64_t pol_q = policy_evict_first();
       const uint64_t pol_kv = policy_evict_last();  // read again right away for V
       int jt = 0;
@@ -784,24 +737,112 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
   }
 }
 
+// Set-up that touches no global memory, so that it runs before the kernel
+// waits for the grid it depends on: the barriers, the abort flag, the zero
+// rows of short Q boxes, the pair's tensor memory and the tensor-map
+// prefetch; then the cluster sync after which both CTAs' barriers and TMEM
+// exist.
+__device__ __forceinline__ void pair_setup16(const Pair16Params& prm, uint8_t* smem) {
+  using L = Layout16;
+  constexpr int NK = L::NK, NV = L::NV, NQ = L::NQ;
+  const uint32_t sb = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sb + L::kBarOff + 8u * (uint32_t)i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int M = prm.a.plan.rows_per_unit;
+  const int box_q = M < 64 ? M : 64;  // query rows per TMA box
+  if (threadIdx.x == 0) {
+    mbar_init(bar(L::B_Q_MAIN), 1);
+    mbar_init(bar(L::B_Q_TMEM), 2 * kSoftmaxWarps);
+    for (int i = 0; i < NK; ++i) {
+      mbar_init(bar(L::B_K_FULL + i), 1);
+      mbar_init(bar(L::B_K_EMPTY + i), 1);
+    }
+    for (int i = 0; i < NV; ++i) {
+      mbar_init(bar(L::B_V_FULL + i), 1);
+      mbar_init(bar(L::B_V_EMPTY + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(L::B_S_FULL + i), 1);
+      mbar_init(bar(L::B_S_EMPTY + i), 2 * 4);  // the tile's softmax group in each CTA
+      mbar_init(bar(L::B_P_FULL + i), 2 * 4);
+      mbar_init(bar(L::B_P_EMPTY + i), 1);
+      mbar_init(bar(L::B_M_READY + i), 4);
+      mbar_init(bar(L::B_X + i), 4);
+    }
+    mbar_init(bar(L::B_O_DONE), 1);
+    mbar_init(bar(L::B_O_FINAL), 1);
+    mbar_init(bar(L::B_FIN), kSoftmaxWarps);
+    for (int i = 0; i < NQ; ++i) mbar_init(bar(L::B_QK_DONE + i), 1);
+    mbar_init(bar(L::B_EPI), kSoftmaxWarps);
+    mbar_init(bar(L::B_O_FREE), 2 * kSoftmaxWarps);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (box_q < 64) {
+    // Rows the Q boxes do not cover are zero in the resident Q part (its
+    // rows are independent A rows of S; zero keeps them finite).
+    for (int i = threadIdx.x; i < 4 * (64 - box_q) * 8; i += blockDim.x) {
+      const int ci = i / ((64 - box_q) * 8), rem = i % ((64 - box_q) * 8);
+      reinterpret_cast<uint4*>(smem + L::kQRes + ci * 8192 + box_q * 128)[rem] = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), 512);
+    tmem_relinquish_pair();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&prm.tm_q);
+    prefetch_tmap(&prm.tm_k8);
+    prefetch_tmap(&prm.tm_kv);
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers and TMEM exist before any cross-CTA use
+  tc_fence_after();
+}
+
+// A pair with no work (the same in both CTAs) frees its tensor memory.
+__device__ __forceinline__ void pair_idle_teardown16(uint8_t* smem) {
+  __syncthreads();
+  tc_fence_before();
+  cluster_sync();
+  if ((threadIdx.x >> 5) == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(*reinterpret_cast<volatile uint32_t*>(smem + Layout16::kMiscOff), 512);
+  }
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc16_pair_kernel(const __grid_constant__ Pair16Params prm) {
-  // the combine grid may take the SMs of pairs that finish early: it waits
-  // for each unit's pieces itself
-  launch_dependents();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // The layout has no alignment slack: a base off 1024 bytes (never seen)
-  // stops both CTAs of every pair before any shared memory is used.
+  // stops both CTAs of every pair before any shared memory is used (after
+  // the dependency wait, so that the status word it sets is not cleared).
   if (smem_u32(smem_raw) & 1023u) {
+    grid_dep_wait();
+    launch_dependents();
     if (threadIdx.x == 0) atomicOr(prm.a.status, MLA_DEV_TIMEOUT);
     return;
   }
   uint8_t* smem = smem_raw;
   SchedInfo* info = reinterpret_cast<SchedInfo*>(smem + kMaxSmemPieces * sizeof(Piece));
+  // Launched as a programmatic dependent of the workspace clear: the set-up
+  // overlaps the previous step's tail, and no global memory is touched before
+  // the clear (and, through it, everything before it in the stream) is done.
+  pair_setup16(prm, smem);
+  grid_dep_wait();
+  // The combine grid may now start (the unit counters and the table's ready
+  // flag it waits on are cleared) and take the SMs of pairs that finish early.
+  launch_dependents();
   build_schedule<kTile16>(prm.a, blockIdx.x >> 1, cluster_ctarank(), smem);  // every thread
   __syncthreads();
   const int npc = info->npc;
-  if (npc == 0) return;  // no work for this pair (the same in both CTAs)
+  if (npc == 0) {  // no work for this pair (the same in both CTAs)
+    pair_idle_teardown16(smem);
+    return;
+  }
   if (prm.a.plan.dtype == MLA_BF16)
     pair_cta16<true>(prm, smem, npc, info->tiles);
   else
@@ -829,8 +870,19 @@ cudaError_t launch_tc16_pair_partial(const DecodeArgs& a, cudaStream_t stream) {
   if (cudaError_t e = set_max_dynamic_smem((const void*)tc16_pair_kernel, (int)Layout16::kSmemBytes, smem_set);
       e != cudaSuccess)
     return e;
-  tc16_pair_kernel<<<(unsigned)(2 * p.split_kv), kThreads, Layout16::kSmemBytes, stream>>>(prm);
-  return cudaGetLastError();
+  // a programmatic dependent of the previous kernel in the stream (the
+  // workspace clear): it waits for it before touching global memory
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * p.split_kv));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Layout16::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc16_pair_kernel, prm);
 }
 
 }  // namespace mla

@@ -79,14 +79,22 @@ constexpr float kSigma = 4.f;        // P <= 2^(kTau + kSigma) = 256 <= 448
 // The schedule area (pair_schedule.cuh) is at the start of shared memory, the
 // same place in both layouts.
 
+// The barriers and the TMEM slot sit at the same place in both layouts, right
+// after the schedule area, so that they are set up before the schedule (and
+// with it the layout) is known.
+constexpr uint32_t kPairBarOff = kSchedBytes;        // 64 mbarriers
+constexpr uint32_t kPairMiscOff = kPairBarOff + 512;  // TMEM address, abort flag
+
 template <bool kTwo>
 struct PairLayout {
   static constexpr int NK = 3;                                  // K-ring slots: own page
   static constexpr int NV = 2;                                  // V-ring slots: 256 V columns of both pages
-  static constexpr uint32_t kQRope = kSchedBytes;               // 64 rows x 64 B (SW64)
+  static constexpr uint32_t kBarOff = kPairBarOff;
+  static constexpr uint32_t kMiscOff = kPairMiscOff;
+  static constexpr uint32_t kQRope = kMiscOff + 512;            // 64 rows x 64 B (SW64)
   static constexpr uint32_t kPPlane = 64 * 128;                 // 64 rows x 128 keys E4M3 (SW128)
   static constexpr uint32_t kPBuf = (kTwo ? 2 : 1) * kPPlane;   // hi (and lo) plane
-  static constexpr uint32_t kPOff = kQRope + 5120;              // P[2 buffers] (1024-aligned)
+  static constexpr uint32_t kPOff = kQRope + 4096;              // P[2 buffers] (1024-aligned)
   static constexpr uint32_t kKSlot = 4 * 8192 + 64 * 64;        // 4 latent chunks (SW128) + rope (SW64)
   static constexpr uint32_t kKOff = kPOff + 2 * kPBuf;
   static constexpr uint32_t kVSlot = 4 * 8192;                  // [column half h][page] chunks (SW128)
@@ -99,7 +107,6 @@ struct PairLayout {
   static constexpr uint32_t kMOff = kVOff + NV * kVSlot;        // row reference maxima [tile parity][64]
   static constexpr uint32_t kXOff = kMOff + 512;                // half-row maxima [group][phase][half][64]
   static constexpr uint32_t kFinOff = kXOff + 2048;             // final (l, m) [l|m][group][half][64]
-  static constexpr uint32_t kBarOff = kFinOff + 2048;
   // barriers ("leader": only the leader's copy is used)
   static constexpr int B_Q_MAIN = 0;                 // local, per piece: staged Q latent landed
   static constexpr int B_Q_ROPE = 1;                 // leader, per piece: both CTAs' Q rope landed
@@ -127,8 +134,7 @@ struct PairLayout {
   static constexpr int B_O_FREE = B_EPI + 1;         // leader, per piece: both CTAs read O
   static constexpr int kNBars = B_O_FREE + 1;
   static_assert(8 * kNBars <= 512, "barrier area");
-  static constexpr uint32_t kMiscOff = kBarOff + 512;
-  static constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;
+  static constexpr uint32_t kSmemBytes = kFinOff + 2048 + 1024;  // + alignment slack of the base
   static_assert(kPOff % 1024 == 0 && kKOff % 1024 == 0 && kKSlot % 1024 == 0 && kVOff % 1024 == 0, "alignment");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   // the last piece's epilogue stages the 64 x 512 fp32 output tile in the
@@ -238,58 +244,12 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, i
     if (rank == 0) mbar_arrive(bar(i)); else mbar_arrive_remote_relaxed(lead(i));
   };
 
-  // ---------------------------------------------------------------- setup
-  if (threadIdx.x == 0) {
-    mbar_init(bar(L::B_Q_MAIN), 1);
-    mbar_init(bar(L::B_Q_ROPE), 1);
-    mbar_init(bar(L::B_Q_TMEM), 2 * kSoftmaxWarps);
-    for (int i = 0; i < NK; ++i) {
-      mbar_init(bar(L::B_K_FULL + i), 1);
-      mbar_init(bar(L::B_K_EMPTY + i), 1);
-    }
-    for (int i = 0; i < NV; ++i) {
-      mbar_init(bar(L::B_V_FULL + i), 1);
-      mbar_init(bar(L::B_V_EMPTY + i), 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(L::B_S_FULL + i), 1);
-      mbar_init(bar(L::B_S_EMPTY + i), 2 * 4);  // the tile's softmax group in each CTA
-      mbar_init(bar(L::B_P_FULL + i), 2 * 4);
-      mbar_init(bar(L::B_P_EMPTY + i), 1);
-      mbar_init(bar(L::B_M_READY + i), 4);
-      mbar_init(bar(L::B_X + i), 4);
-    }
-    mbar_init(bar(L::B_O_DONE), 1);
-    mbar_init(bar(L::B_O_FINAL), 1);
-    mbar_init(bar(L::B_FIN), kSoftmaxWarps);
-    for (int i = 0; i < NQ; ++i) mbar_init(bar(L::B_QK_DONE + i), 1);
-    mbar_init(bar(L::B_EPI), kSoftmaxWarps);
-    mbar_init(bar(L::B_O_FREE), 2 * kSoftmaxWarps);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (box_q < 64) {
-    // Q rope rows the TMA box does not cover are zero (rows are independent).
-    uint4* rb = reinterpret_cast<uint4*>(smem + L::kQRope + box_q * 64);
-    for (int i = threadIdx.x; i < (64 - box_q) * 4; i += blockDim.x) rb[i] = make_uint4(0, 0, 0, 0);
-    fence_proxy_async_smem();
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(smem_u32(tmem_slot), 512);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  cluster_sync();  // both CTAs' barriers and TMEM exist before any cross-CTA use
-  tc_fence_after();
+  // (barriers, TMEM and the cluster sync were set up by pair_setup)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
     // ------------------------------------------------------------ Q and K-ring loads
     if (lane == 0) {
-      prefetch_tmap(&prm.tm_q_main);
-      prefetch_tmap(&prm.tm_q_rope);
-      prefetch_tmap(&prm.tm_kv_main);
-      prefetch_tmap(&prm.tm_kv_rope);
       const uint64_t pol_q = policy_evict_first();
       const uint64_t pol_kv = policy_evict_last();  // read again right away for V
       int jt = 0;     // tile counter across pieces
@@ -316,6 +276,9 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, i
           const int page = valid_page(a, entry_nx);
           if (j + 1 < c.n_pt) entry_nx = piece_entry(c, 2 * (j + 1) + (int)rank);
           if (!(ok = bounded_wait_cta(bar(L::B_K_EMPTY + sk), ((jt / NK) & 1) ^ 1, abort_flag, a.status))) break;
+          // failure-detection test mode: the pair's first tile is never loaded,
+          // so the S issuer's wait for it runs out (every wait is bounded)
+          if (p.fault_test && jt == 0) continue;
           const uint32_t ks = sb + L::kKOff + sk * L::kKSlot;
           const uint32_t full = lead(L::B_K_FULL + sk);
           if (rank == 0) mbar_arrive_expect_tx(bar(L::B_K_FULL + sk), 2u * L::kKSlot);
@@ -863,18 +826,105 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, i
   }
 }
 
+// Set-up that touches no global memory, so that it runs before the kernel
+// waits for the grid it depends on: every barrier (both layouts keep them at
+// the same place), the abort flag, the zero rows of a short Q rope box, the
+// pair's tensor memory and the tensor-map prefetch; then the cluster sync
+// after which both CTAs' barriers and TMEM exist.
+__device__ __forceinline__ void pair_setup(const PairParams& prm, uint8_t* smem) {
+  using L = PairLayout<false>;
+  static_assert(PairLayout<true>::kBarOff == L::kBarOff && PairLayout<true>::kMiscOff == L::kMiscOff &&
+                    PairLayout<true>::kQRope == L::kQRope && PairLayout<true>::kNBars == L::kNBars,
+                "barriers, TMEM slot and Q rope sit at the same place in both layouts");
+  constexpr int NK = L::NK, NV = L::NV, NQ = L::NQ;
+  const uint32_t sb = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sb + L::kBarOff + 8u * (uint32_t)i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int M = prm.a.plan.rows_per_unit;
+  const int box_q = M < 64 ? M : 64;  // query rows per TMA box (the tensor maps' box height)
+  if (threadIdx.x == 0) {
+    mbar_init(bar(L::B_Q_MAIN), 1);
+    mbar_init(bar(L::B_Q_ROPE), 1);
+    mbar_init(bar(L::B_Q_TMEM), 2 * kSoftmaxWarps);
+    for (int i = 0; i < NK; ++i) {
+      mbar_init(bar(L::B_K_FULL + i), 1);
+      mbar_init(bar(L::B_K_EMPTY + i), 1);
+    }
+    for (int i = 0; i < NV; ++i) {
+      mbar_init(bar(L::B_V_FULL + i), 1);
+      mbar_init(bar(L::B_V_EMPTY + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(L::B_S_FULL + i), 1);
+      mbar_init(bar(L::B_S_EMPTY + i), 2 * 4);  // the tile's softmax group in each CTA
+      mbar_init(bar(L::B_P_FULL + i), 2 * 4);
+      mbar_init(bar(L::B_P_EMPTY + i), 1);
+      mbar_init(bar(L::B_M_READY + i), 4);
+      mbar_init(bar(L::B_X + i), 4);
+    }
+    mbar_init(bar(L::B_O_DONE), 1);
+    mbar_init(bar(L::B_O_FINAL), 1);
+    mbar_init(bar(L::B_FIN), kSoftmaxWarps);
+    for (int i = 0; i < NQ; ++i) mbar_init(bar(L::B_QK_DONE + i), 1);
+    mbar_init(bar(L::B_EPI), kSoftmaxWarps);
+    mbar_init(bar(L::B_O_FREE), 2 * kSoftmaxWarps);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (box_q < 64) {
+    // Q rope rows the TMA box does not cover are zero (rows are independent).
+    uint4* rb = reinterpret_cast<uint4*>(smem + L::kQRope + box_q * 64);
+    for (int i = threadIdx.x; i < (64 - box_q) * 4; i += blockDim.x) rb[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), 512);
+    tmem_relinquish_pair();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&prm.tm_q_main);
+    prefetch_tmap(&prm.tm_q_rope);
+    prefetch_tmap(&prm.tm_kv_main);
+    prefetch_tmap(&prm.tm_kv_rope);
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers and TMEM exist before any cross-CTA use
+  tc_fence_after();
+}
+
+// A pair with no work (the same in both CTAs) frees its tensor memory.
+__device__ __forceinline__ void pair_idle_teardown(uint8_t* smem) {
+  __syncthreads();
+  tc_fence_before();
+  cluster_sync();
+  if ((threadIdx.x >> 5) == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(*reinterpret_cast<volatile uint32_t*>(smem + kPairMiscOff), 512);
+  }
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_fp8_pair_kernel(const __grid_constant__ PairParams prm) {
-  // the combine grid may take the SMs of pairs that finish early: it waits
-  // for each unit's pieces itself
-  launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   SchedInfo* info = reinterpret_cast<SchedInfo*>(smem + kMaxSmemPieces * sizeof(Piece));
+  // Launched as a programmatic dependent of the workspace clear: the set-up
+  // overlaps the previous step's tail, and no global memory is touched before
+  // the clear (and, through it, everything before it in the stream) is done.
+  pair_setup(prm, smem);
+  grid_dep_wait();
+  // The combine grid may now start (the unit counters and the table's ready
+  // flag it waits on are cleared) and take the SMs of pairs that finish early.
+  launch_dependents();
   build_schedule<kPairTileKeys>(prm.a, blockIdx.x >> 1, cluster_ctarank(), smem);  // every thread
   __syncthreads();
   const int npc = info->npc;
-  if (npc == 0) return;  // no work for this pair (the same in both CTAs)
+  if (npc == 0) {  // no work for this pair (the same in both CTAs)
+    pair_idle_teardown(smem);
+    return;
+  }
   // Short entries send P as two E4M3 terms; a pair with any such piece takes
   // the layout with room for both planes (the choice is the same in both CTAs).
   if (info->two)
@@ -902,8 +952,19 @@ cudaError_t launch_tc_fp8_pair_partial(const DecodeArgs& a, cudaStream_t stream)
   if (cudaError_t e = set_max_dynamic_smem((const void*)tc_fp8_pair_kernel, (int)kPairSmemBytes, smem_set);
       e != cudaSuccess)
     return e;
-  tc_fp8_pair_kernel<<<(unsigned)(2 * p.split_kv), kThreads, kPairSmemBytes, stream>>>(prm);
-  return cudaGetLastError();
+  // a programmatic dependent of the previous kernel in the stream (the
+  // workspace clear): it waits for it before touching global memory
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * p.split_kv));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kPairSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc_fp8_pair_kernel, prm);
 }
 
 }  // namespace mla

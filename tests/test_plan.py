@@ -85,7 +85,7 @@ def test_balanced_plan_uses_every_sm_and_caps_units():
     assert big16.schedule == 0 and big16.kernel == 1
 
 
-LEAD = 16  # weight of a piece transition, charged at the start of every unit with tiles but the first
+LEAD = 24  # weight of a piece transition, charged at the start of every unit with tiles but the first
 
 
 def _lead(u, t):
