@@ -96,6 +96,19 @@ def test_decode_rejects_bad_arguments_before_any_launch():
     assert _call(p, scale=float("inf")) == -1
 
 
+def test_fault_test_mode_is_off_in_plans_and_refused_where_it_does_not_exist():
+    """The failure-detection test field is 0 in every plan the planner writes; 1 is accepted only on
+    the FP8 CTA-pair kernel's balanced plans, anything else is refused before any launch."""
+    fp8 = mla.mla_decode_plan(2, 4, 32, 256, "fp8")
+    bf16 = mla.mla_decode_plan(2, 4, 32, 256, "bf16")
+    simt = mla.mla_decode_plan_custom(2, 4, 32, 256, "fp8", kernel="simt")
+    assert fp8.fault_test == 0 and bf16.fault_test == 0 and simt.fault_test == 0
+    for plan, value in ((bf16, 1), (simt, 1), (fp8, 2), (fp8, -1)):
+        bad = _lib.MlaPlan.from_buffer_copy(plan)
+        bad.fault_test = value
+        assert _call(bad) == -6
+
+
 def test_python_wrapper_refuses_host_tensors():
     """The binding names the first argument that is not a CUDA tensor before calling the library."""
     torch = pytest.importorskip("torch")
