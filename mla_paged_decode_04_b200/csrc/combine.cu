@@ -139,7 +139,7 @@ __device__ __forceinline__ void combine_unit(const DecodeArgs& a, int u, int rb,
   const UnitGeom ug = unit_geom(a, u, false);
   // pairs holding the unit's first and last tiles (tile starts are weighted;
   // the first follows the unit's lead-in)
-  const int lead = end > start ? unit_lead_weight(sl, 1) : 0;
+  const int lead = end > start ? unit_lead_weight(1) : 0;
   const int p0 = end > start ? balanced_pair_of(start + lead, W, np) : 0;
   const int p1 = end > start ? balanced_pair_of(end - tile_weight(p, ug), W, np) : 0;
   if (end > start && p0 == p1) return;  // a whole unit: written by its pair

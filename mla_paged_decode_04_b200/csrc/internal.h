@@ -47,14 +47,14 @@ constexpr int kTwoTermKeys = 8192;
 // boundary finished 8.3 us (~8 tiles) after the others; with a lead-in of 16
 // they still finished 5 us later, and 24 was the fastest of 8, 16, 24 and 32
 // on the 4-entry batch (74.1 against 76.1 us) and within 1% elsewhere. The balanced schedule therefore charges
-// every unit with tiles but the first of the sequence a lead-in of this
-// weight (a tile weighs 2 or 3) at its weighted start, ahead of its first
-// tile, so that a pair whose range holds a unit start takes correspondingly
-// fewer tiles. `slot` is the unit's position in the schedule's sequence.
+// every unit with tiles a lead-in of this weight (a tile weighs 2 or 3) at its
+// weighted start, ahead of its first tile, so that a pair whose range holds a
+// unit start takes correspondingly fewer tiles. The first unit carries one
+// too: with the group-major order of pair_schedule.cuh, the halves of the
+// sequence then have equal weight and the pairs that read the same pages for
+// the two query groups of an entry stay aligned.
 constexpr int kPieceLeadWeight = 24;
-__host__ __device__ inline int unit_lead_weight(int slot, int tiles) {
-  return (tiles > 0 && slot > 0) ? kPieceLeadWeight : 0;
-}
+__host__ __device__ inline int unit_lead_weight(int tiles) { return tiles > 0 ? kPieceLeadWeight : 0; }
 // Piece lists too long for a CTA's shared memory go to a spill area right
 // before the unit table: per CTA rank, U + P pieces of 3 int32 (a pair's
 // pieces are the units its range meets, consecutive in the schedule's

@@ -4,8 +4,8 @@
 // device seq_lens (and, for ragged queries, cu_q): from the tile of the
 // lowest key a row of the unit sees to the tile of the highest. A tile
 // weighs 2, or 3 when its P.V runs twice (FP8 two-term P), so that pairs get
-// equal work rather than equal tiles, and every unit with tiles but the first
-// starts with a lead-in of kPieceLeadWeight, the cost of a piece transition.
+// equal work rather than equal tiles, and every unit with tiles starts with a
+// lead-in of kPieceLeadWeight, the cost of a piece transition.
 // The units' runs form one sequence of total weight W; pair p takes the tiles
 // whose start lies in [floor(W p / np), floor(W (p + 1) / np)) and walks them
 // as a list of pieces (the units its range meets, each cut to the range).
@@ -122,7 +122,7 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uin
   for (int sl = s_beg; sl < s_end; ++sl) {
     const UnitGeom ug = unit_geom(a, sched_unit(p, sl), writer);
     const int t = unit_span_tiles<kKeys>(ug);
-    run += unit_lead_weight(sl, t) + t * tile_weight(p, ug);
+    run += unit_lead_weight(t) + t * tile_weight(p, ug);
   }
   int incl = warp_incl_scan(run);
   if (lane == 31) scan1[warp] = incl;
@@ -142,7 +142,7 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uin
       a.sched[sl] = start;
       const UnitGeom ug = unit_geom(a, sched_unit(p, sl), false);
       const int t = unit_span_tiles<kKeys>(ug);
-      start += unit_lead_weight(sl, t) + t * tile_weight(p, ug);
+      start += unit_lead_weight(t) + t * tile_weight(p, ug);
     }
     if (tid == 0) {
       a.sched[U] = W;
@@ -155,7 +155,7 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uin
     int start = excl;
     for (int sl = s_beg; sl < s_end; ++sl) {
       const UnitGeom ug = unit_geom(a, sched_unit(p, sl), false);
-      const int t = unit_span_tiles<kKeys>(ug), w = tile_weight(p, ug), lead = unit_lead_weight(sl, t);
+      const int t = unit_span_tiles<kKeys>(ug), w = tile_weight(p, ug), lead = unit_lead_weight(t);
       int i0, i1;
       tiles_in_range(start + lead, t, w, lo, hi, i0, i1);
       if (i1 > i0) {
@@ -197,7 +197,7 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uin
     for (int sl = s_beg; sl < s_end; ++sl) {
       const int u = sched_unit(p, sl);
       const UnitGeom ug = unit_geom(a, u, false);
-      const int t = unit_span_tiles<kKeys>(ug), w = tile_weight(p, ug), lead = unit_lead_weight(sl, t);
+      const int t = unit_span_tiles<kKeys>(ug), w = tile_weight(p, ug), lead = unit_lead_weight(t);
       int i0, i1;
       tiles_in_range(start + lead, t, w, lo, hi, i0, i1);
       if (i1 > i0) {
