@@ -361,9 +361,10 @@ def run_ours(args):
 
     def timed(fn, n, per_step=False):
         """n steps back to back, timed by CUDA events on the launching stream: one pair around
-        all n steps (an event recorded between two steps widens the gap between them), or, with
-        per_step, a pair around each step (for the spread). Returns the per-step times in ms
-        (the mean n times without per_step) and the host time window the steps ran in."""
+        all n steps (an event recorded between two steps widens the gap between them; used when
+        nothing runs between steps), or, with per_step, a pair around each step (the L2 flush,
+        when there is one, runs between the pairs). Returns the per-step times in ms (the mean
+        n times without per_step) and the host time window the steps ran in."""
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
@@ -379,7 +380,6 @@ def run_ours(args):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
             for k in range(n):
-                flush.zero_()
                 fn()
             e1.record()
         torch.cuda.synchronize()
@@ -394,14 +394,16 @@ def run_ours(args):
         # the partial kernel alone: an event between the two launches (which also serialises
         # them) marks its end
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush.zero_()
         e0.record()
         mla.mla_decode_partial(plan, *call)
         e1.record()
         mla.mla_decode_combine(plan, *call)
         part_events.append((e0, e1))
 
-    # (1) the timed steps: W warm-up steps above, then exactly K steps
-    step_ms, wall0, wall1 = timed(step, args.steps)
+    # (1) the timed steps: W warm-up steps above, then exactly K steps (an event pair around each
+    # when the L2 is flushed between steps, so that the flush stays outside the timed region)
+    step_ms, wall0, wall1 = timed(step, args.steps, per_step=flush_l2)
     clocks = poller.window(wall0, wall1)
     # the same K steps with an event pair around each, for the spread only
     each_ms, _, _ = timed(step, args.steps, per_step=True)
@@ -423,7 +425,7 @@ def run_ours(args):
                 flush.zero_()
                 step()
             torch.cuda.synchronize()
-        sus_ms, s0, s1 = timed(step, args.steps)
+        sus_ms, s0, s1 = timed(step, args.steps, per_step=flush_l2)
         part_events = []
         _, _, _ = timed(partial_only, args.steps)
         sus_part_ms = [a.elapsed_time(b) for a, b in part_events]
