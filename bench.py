@@ -62,6 +62,8 @@ def parse_args():
                     help="draw the workload with this many entries instead (small cases for ncu captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--warm-l2", action="store_true",
+                    help="never flush L2 between steps (a warm-L2 line for the workloads whose pool fits in L2)")
     ap.add_argument("--clock-window-s", type=float, default=1.5,
                     help="seconds of back-to-back steps before the sustained timing (0: no sustained timing)")
     return ap.parse_args()
@@ -326,7 +328,7 @@ def run_ours(args):
     # back); a smaller pool is flushed by rewriting a 256 MB buffer.
     L2_BYTES = 126 << 20
     pool_bytes = g.kv_cache.numel() * g.kv_cache.element_size()
-    flush_l2 = pool_bytes < 2 * L2_BYTES
+    flush_l2 = pool_bytes < 2 * L2_BYTES and not args.warm_l2
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush_l2 else None
 
     class _Flush:
@@ -538,6 +540,7 @@ def run_ours(args):
                    "split_kv": plan.split_kv, "fold": plan.fold, "kernel": kname,
                    "kv_bytes_per_step": kv_bytes,
                    "l2": (f"256 MiB buffer rewritten between steps (cache pool {pool_bytes >> 20} MiB)" if flush_l2
+                          else f"warm L2: no flush between steps (cache pool {pool_bytes >> 20} MiB)" if args.warm_l2
                           else f"inputs larger than L2: cache pool {pool_bytes >> 20} MiB >= 2 x 126 MB L2, "
                                "no flush"),
                    "parallelism": f"replicas x{world}"},
