@@ -11,7 +11,9 @@ bracketed by CUDA events on the launching stream, with the SM clock read
 through NVML during them. The same K steps are then timed again after a
 loaded window (--clock-window-s seconds of back-to-back steps, which bring the
 clocks to those of continuous decoding under the power cap) and reported
-beside them as "sustained". When the cache pool is smaller than twice the L2,
+beside them as "sustained". The roofline is the partial kernel's: the same
+protocol on partial-only calls (no combine) gives its average launch duration.
+When the cache pool is smaller than twice the L2,
 a 256 MiB buffer is rewritten between steps; otherwise the inputs are larger
 than L2 and nothing is flushed. With N > 1 (torchrun) every rank runs an
 independent replica on its own GPU ("replicas only": the decode has no
@@ -347,7 +349,10 @@ def run_ours(args):
     alg_bytes_partial = kv_bytes + q_bytes + table_bytes + (out_bytes if plan.split_kv == 1 else 0)
     call = (g.q, g.kv_cache, g.block_tables, g.seq_lens, g.softmax_scale, out, lse, dec.workspace,
             g.q_scale, g.kv_scale)
-    kernels_per_step = 1 + (1 if plan.split_kv > 1 else 0)
+    # balanced schedule (plan.schedule == MLA_SCHEDULE_BALANCED = 1): the workspace-clear kernel, the
+    # partial kernel and the combine; otherwise a memset (not one of ours), the partial kernel and,
+    # with splits, the combine
+    kernels_per_step = 3 if plan.schedule == 1 else 1 + (1 if plan.split_kv > 1 else 0)
 
     def step():
         # one call: the combine is launched as the partial kernel's dependent
@@ -393,15 +398,15 @@ def run_ours(args):
         return [e0.elapsed_time(e1) / n] * n, h0, h1
 
     def partial_only():
-        # the partial kernel alone: an event between the two launches (which also serialises
-        # them) marks its end
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        flush.zero_()
-        e0.record()
+        # the partial kernel alone (after its workspace clear), without the combine
         mla.mla_decode_partial(plan, *call)
-        e1.record()
-        mla.mla_decode_combine(plan, *call)
-        part_events.append((e0, e1))
+
+    def partial_ms():
+        """Average launch duration of the partial kernel: the timed steps' protocol applied to
+        partial-only calls (K back to back under one event pair, or with the L2 flushed between
+        calls an event pair around each)."""
+        ms, _, _ = timed(partial_only, args.steps, per_step=flush_l2)
+        return ms
 
     # (1) the timed steps: W warm-up steps above, then exactly K steps (an event pair around each
     # when the L2 is flushed between steps, so that the flush stays outside the timed region)
@@ -409,9 +414,7 @@ def run_ours(args):
     clocks = poller.window(wall0, wall1)
     # the same K steps with an event pair around each, for the spread only
     each_ms, _, _ = timed(step, args.steps, per_step=True)
-    part_events = []
-    _, p0, p1 = timed(partial_only, args.steps)
-    part_ms = [a.elapsed_time(b) for a, b in part_events]
+    part_ms = partial_ms()
     if dec.status() != 0:
         raise RuntimeError("device status word set during the timed steps")
 
@@ -428,9 +431,7 @@ def run_ours(args):
                 step()
             torch.cuda.synchronize()
         sus_ms, s0, s1 = timed(step, args.steps, per_step=flush_l2)
-        part_events = []
-        _, _, _ = timed(partial_only, args.steps)
-        sus_part_ms = [a.elapsed_time(b) for a, b in part_events]
+        sus_part_ms = partial_ms()
         smi = sampler.stop()
         sus_clocks = poller.window(s0, s1) or smi
         if sus_clocks is not None and smi is not None:
@@ -504,7 +505,7 @@ def run_ours(args):
     roofline.update({"traffic": traffic_from_profile(args.workload, kname), "kernel": kname,
                      "alg_bytes_per_launch": int(alg_bytes_partial), "alg_flops_per_launch": int(flops),
                      "partial_us": round(statistics.mean(part_ms) * 1e3, 2),
-                     "partial_how": "memset + partial kernel, an event pair around each (the combine after it)"})
+                     "partial_how": ("the workspace clear and the partial kernel, " + ("an event pair around each call, the L2 flushed between calls" if flush_l2 else f"{args.steps} partial-only calls back to back under one event pair"))})
     if sustained is not None:
         r2 = roofline_fields(alg_bytes_partial, flops, sustained["partial_us"] / 1e6, peak, peak_kind, g.dtype,
                              sustained=True)
@@ -924,7 +925,7 @@ def run_prefill(args):
                    "units": pre.plan.batch * pre.plan.q_groups, "desc": w.desc,
                    "l2": f"256 MiB buffer rewritten between steps (cache pool {pool_bytes >> 20} MiB)",
                    "parallelism": f"replicas x{world}"},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": (3 if pre.plan.schedule == 1 else 2) * args.steps,  # clear, partial, combine
         "roofline": roofline, "e2e": e2e, "clocks": clocks, "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)

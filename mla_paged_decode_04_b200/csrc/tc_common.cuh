@@ -88,6 +88,34 @@ __device__ __forceinline__ void drain_phase(uint32_t bar, uint32_t parity) {
   }
 }
 
+// Teardown drain of the CTA-pair kernels (layout L, barriers at bar0 + 8 i):
+// the last phase of every barrier the leader's MMA commits arrive on, after
+// `n_all` tiles and `npc` pieces. Lane k of the calling warp waits for one
+// (barrier, parity): the last NK, NV and NQ phases of the K, V and S rings,
+// the last two of P_EMPTY and S_FULL, then O_DONE and O_FINAL, so that the
+// waits overlap instead of running one after another.
+template <class L>
+__device__ __forceinline__ void drain_pair_commits(uint32_t bar0, int lane, int n_all, int npc) {
+  static_assert(L::NK + L::NV + L::NQ + 6 <= 32, "one barrier per lane");
+  // t: the tile (or piece) whose commit completes the phase waited for, on a
+  // ring of n barriers from b; negative when there was no such tile
+  int k = lane, t = -1, n = 1, b = 0;
+  if (k < L::NK) {
+    t = n_all - 1 - k, n = L::NK, b = L::B_K_EMPTY;
+  } else if ((k -= L::NK) < L::NV) {
+    t = n_all - 1 - k, n = L::NV, b = L::B_V_EMPTY;
+  } else if ((k -= L::NV) < L::NQ) {
+    t = n_all - 1 - k, n = L::NQ, b = L::B_QK_DONE;
+  } else if ((k -= L::NQ) < 4) {
+    t = n_all - 1 - (k >> 1), n = 2, b = (k & 1) ? L::B_S_FULL : L::B_P_EMPTY;
+  } else if ((k -= 4) == 0) {
+    t = n_all - 1, n = 1, b = L::B_O_DONE;
+  } else if (k == 1) {
+    t = npc - 1, n = 1, b = L::B_O_FINAL;
+  }
+  if (t >= 0) drain_phase(bar0 + 8u * (uint32_t)(b + t % n), (uint32_t)(t / n) & 1);
+}
+
 // Write 32 output columns [col, col + 32) of flat row `rg`: BF16 to `out`
 // when there is one split, else fp32 to the split's partial. inv = 0 means the
 // row saw no key (written as exact zeros).

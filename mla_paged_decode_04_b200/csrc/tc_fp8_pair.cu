@@ -803,19 +803,10 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, i
   // shared memory after the CTA has exited. It runs once every role is done
   // (the epilogue saw the last O_FINAL, so every commit has been triggered
   // and each barrier is at most its last arrival short of its final phase).
-  // Bounded; skipped after an abort, when the phases may never complete.
+  // Each wait is bounded; all are skipped after an abort, when the phases may
+  // never complete.
   __syncthreads();
-  if (warp == 2 && lane == 0 && !*abort_flag && n_all > 0) {
-    for (int j = n_all - 1; j >= 0 && j >= n_all - NK; --j) drain_phase(bar(L::B_K_EMPTY + j % NK), (j / NK) & 1);
-    for (int j = n_all - 1; j >= 0 && j >= n_all - NV; --j) drain_phase(bar(L::B_V_EMPTY + j % NV), (j / NV) & 1);
-    for (int j = n_all - 1; j >= 0 && j >= n_all - NQ; --j) drain_phase(bar(L::B_QK_DONE + j % NQ), (j / NQ) & 1);
-    for (int j = n_all - 1; j >= 0 && j >= n_all - 2; --j) {
-      drain_phase(bar(L::B_P_EMPTY + (j & 1)), (j >> 1) & 1);
-      drain_phase(bar(L::B_S_FULL + (j & 1)), (j >> 1) & 1);
-    }
-    drain_phase(bar(L::B_O_DONE), (n_all - 1) & 1);
-    drain_phase(bar(L::B_O_FINAL), (npc - 1) & 1);
-  }
+  if (warp == 2 && !*abort_flag && n_all > 0) drain_pair_commits<L>(bar(0), lane, n_all, npc);
   __syncthreads();
   tc_fence_before();
   cluster_sync();  // the peer no longer touches this CTA's shared or tensor memory
