@@ -102,14 +102,18 @@ namespace {
 // Combine for the balanced CTA-pair schedule. Units a single pair covered
 // whole were finished by the partial kernel and are left alone; units with
 // no key get out = 0, lse = -inf; a unit cut between pairs p0 .. p1 merges
-// the pieces in their slots (pair q: slot 2q if the unit is its first, else
-// 2q + 1) as above. Slots are laid out [slot][16-byte column chunk][row]:
-// thread (row i, chunk pair c) of a block of 32 rows x 16 chunk pairs sums
-// 8 output columns of row i over the pieces, and the 32 threads of a warp
-// read 32 consecutive rows (512 contiguous bytes) per load. The grid holds
-// units x row blocks x 8 column blocks, so that even a few long units that
-// were cut into many pieces spread over the whole GPU.
-constexpr int kCombineColBlocks = 8;  // 512 columns = 8 blocks x 16 chunk pairs x 4 columns x 2
+// the pieces in their slots (pair p0: slot 2p0 + 1; every later pair q:
+// slot 2q). Slots are laid out [slot][16-byte column chunk][row]: thread
+// (row i, warp w) of a block of 32 rows x 8 warps sums kC4 chunks (4 kC4
+// output columns) of row i over the pieces, and the 32 threads of a warp read
+// 32 consecutive rows (512 contiguous bytes) per load. The grid holds
+// units x row blocks x 16 / kC4 column blocks, so that even a few long units
+// that were cut into many pieces spread over the whole GPU: plans with few
+// units take kC4 = 1 (twice the blocks, each thread half the columns and
+// twice the pieces in flight), the others kC4 = 2. At 64 registers a thread,
+// four blocks fit an SM: the grids of up to 592 blocks are resident at once
+// while their units finish, and none waits for another's slot.
+constexpr int kCombineMaxResident = 4 * 148;
 constexpr uint64_t kUnitWaitNs = 500ull * 1000 * 1000;  // per wait: 0.5 s
 
 // Bounded wait (one thread) for a counter written by the partial kernel;
@@ -128,6 +132,7 @@ __device__ bool wait_count(const int32_t* ctr, int target, int32_t* status) {
 
 // Merge of one unit's rows [32 rb, 32 rb + 32) x column block cb (block-
 // uniform u, so every thread takes the same path through the barriers).
+template <int kC4>
 __device__ __forceinline__ void combine_unit(const DecodeArgs& a, int u, int rb, int cb, int* s_ok) {
   const mla_plan& p = a.plan;
   const int M = p.rows_per_unit;
@@ -151,52 +156,59 @@ __device__ __forceinline__ void combine_unit(const DecodeArgs& a, int u, int rb,
     (void)ptx::ld_acquire_gpu(a.unit_done + u);
   }
   const int r = rb * 32 + (threadIdx.x & 31);       // row within the unit
-  const int c4_0 = cb * 16 + (threadIdx.x >> 5) * 2;         // first of this thread's two 16-byte chunks
+  const int c4_0 = (cb * 8 + (threadIdx.x >> 5)) * kC4;  // first of this thread's kC4 16-byte chunks
   if (r >= ug.rows) return;  // past the unit's rows (an entry's last group under ragged queries)
-  const int64_t row = ug.row0 + r;
-  uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + row * MLA_D_V + c4_0 * 4);
   const bool lse_writer = a.lse && cb == 0 && (threadIdx.x >> 5) == 0;
   if (end == start) {  // no key at all
-    *dst = make_uint4(0, 0, 0, 0);
+    const int64_t row = ug.row0 + r;
+    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.out) + row * MLA_D_V + c4_0 * 4;
+    if constexpr (kC4 == 2)
+      *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+    else
+      *reinterpret_cast<uint2*>(dst) = make_uint2(0, 0);
     if (lse_writer) a.lse[row] = -INFINITY;
     return;
   }
-  // Pair p0 kept the unit in slot 2p0 if it was its first piece (each pair
-  // records the schedule position of its first unit in the table), else in
-  // 2p0 + 1; every later pair starts inside the unit (slot 2q). Pair p0's
-  // record precedes its piece arrivals, which the counter wait above acquired.
-  const int64_t first_slot = tbl[U + 2 + p0] == sl ? 2 * (int64_t)p0 : 2 * (int64_t)p0 + 1;
+  // Pair p0's piece begins at the unit's start: slot 2p0 + 1. Every later
+  // pair's piece begins inside the unit: slot 2q. Slots number
+  // 2 * split_kv <= 148 of M <= MLA_MAX_ROWS rows: float offsets into the
+  // partials fit an int.
+  auto slot = [&](int q) -> int { return q == p0 ? 2 * p0 + 1 : 2 * q; };
 
-  auto slot = [&](int q) -> int64_t { return q == p0 ? first_slot : 2 * (int64_t)q; };
-
-  // The maximum piece LSE first, then the weighted sum. Pieces go in batches
-  // of kBatch whose loads are all issued before any of them is used (no
-  // branch depends on a loaded value), so their latencies overlap.
-  constexpr int kBatch = 8;
-  float m = -INFINITY;
+  // One pass over the pieces with a running maximum (the sum and the
+  // accumulators are rescaled when it grows). Pieces go in batches of kBatch
+  // whose loads are all issued before any of them is used (no branch depends
+  // on a loaded value), so their latencies overlap.
+  constexpr int kBatch = kC4 == 2 ? 3 : 6;
+  constexpr int kAcc = 4 * kC4;
+  const float* base = a.o_part + (c4_0 * M + r) * 4;
+  const int slot_stride = (MLA_D_V / 4) * M * 4;  // floats per partial slot
+  float m = -INFINITY, sum = 0.f;
+  float acc[kAcc];
+#pragma unroll
+  for (int i = 0; i < kAcc; ++i) acc[i] = 0.f;
   for (int q0 = p0; q0 <= p1; q0 += kBatch) {
-    float ls[kBatch];
-#pragma unroll
-    for (int i = 0; i < kBatch; ++i) ls[i] = q0 + i <= p1 ? a.lse_part[slot(q0 + i) * M + r] : -INFINITY;
-#pragma unroll
-    for (int i = 0; i < kBatch; ++i) m = fmaxf(m, ls[i]);
-  }
-  float sum = 0.f;
-  float acc[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  for (int q0 = p0; m != -INFINITY && q0 <= p1; q0 += kBatch) {
     float ls[kBatch];
     float4 x0[kBatch], x1[kBatch];
 #pragma unroll
     for (int i = 0; i < kBatch; ++i) {
       const bool in = q0 + i <= p1;
-      const int64_t sl = slot(in ? q0 + i : p0);
-      const float* src = a.o_part + ((sl * (MLA_D_V / 4) + c4_0) * M + r) * 4;
+      const int sl = slot(in ? q0 + i : p0);
+      const float* src = base + sl * slot_stride;
+      // past p1: slot p0 is read again and weighs 0 (lse -inf)
       ls[i] = in ? a.lse_part[sl * M + r] : -INFINITY;
-      x0[i] = in ? *reinterpret_cast<const float4*>(src) : make_float4(0.f, 0.f, 0.f, 0.f);
-      x1[i] = in ? *reinterpret_cast<const float4*>(src + (int64_t)M * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      x0[i] = *reinterpret_cast<const float4*>(src);
+      if constexpr (kC4 == 2) x1[i] = *reinterpret_cast<const float4*>(src + M * 4);
     }
+    float mb = m;
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) mb = fmaxf(mb, ls[i]);
+    if (mb == -INFINITY) continue;  // every piece so far is empty
+    const float sc = m == -INFINITY ? 0.f : expf(m - mb);
+    sum *= sc;
+#pragma unroll
+    for (int e = 0; e < kAcc; ++e) acc[e] *= sc;
+    m = mb;
 #pragma unroll
     for (int i = 0; i < kBatch; ++i) {
       // an empty piece (lse -inf) has weight 0 and may hold anything
@@ -207,33 +219,42 @@ __device__ __forceinline__ void combine_unit(const DecodeArgs& a, int u, int rb,
       acc[1] = fmaf(w, live ? x0[i].y : 0.f, acc[1]);
       acc[2] = fmaf(w, live ? x0[i].z : 0.f, acc[2]);
       acc[3] = fmaf(w, live ? x0[i].w : 0.f, acc[3]);
-      acc[4] = fmaf(w, live ? x1[i].x : 0.f, acc[4]);
-      acc[5] = fmaf(w, live ? x1[i].y : 0.f, acc[5]);
-      acc[6] = fmaf(w, live ? x1[i].z : 0.f, acc[6]);
-      acc[7] = fmaf(w, live ? x1[i].w : 0.f, acc[7]);
+      if constexpr (kC4 == 2) {
+        acc[4] = fmaf(w, live ? x1[i].x : 0.f, acc[4]);
+        acc[5] = fmaf(w, live ? x1[i].y : 0.f, acc[5]);
+        acc[6] = fmaf(w, live ? x1[i].z : 0.f, acc[6]);
+        acc[7] = fmaf(w, live ? x1[i].w : 0.f, acc[7]);
+      }
     }
   }
   const float L = m == -INFINITY ? -INFINITY : m + logf(sum);
   const float inv = m == -INFINITY ? 0.f : 1.f / sum;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] *= inv;
-  uint32_t pk[4];
+  for (int i = 0; i < kAcc; ++i) acc[i] *= inv;
+  uint32_t pk[kAcc / 2];
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
+  for (int e = 0; e < kAcc / 2; ++e) {
     __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
     pk[e] = *reinterpret_cast<uint32_t*>(&h2);
   }
-  *dst = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  const int64_t row = ug.row0 + r;
+  __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.out) + row * MLA_D_V + c4_0 * 4;
+  if constexpr (kC4 == 2)
+    *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  else
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
   if (lse_writer) a.lse[row] = L;
 }
 
+template <int kC4>
 __device__ __forceinline__ void combine_balanced_block(const DecodeArgs& a, int units_per_block);
 
-__global__ void __launch_bounds__(256) combine_balanced_kernel(const DecodeArgs a, int units_per_block) {
+template <int kC4>
+__global__ void __launch_bounds__(256, 4) combine_balanced_kernel(const DecodeArgs a, int units_per_block) {
   // The next step's workspace clear may be launched now: it waits for this
   // grid's completion before touching the workspace.
   ptx::launch_dependents();
-  combine_balanced_block(a, units_per_block);
+  combine_balanced_block<kC4>(a, units_per_block);
   // This grid completes only after the partial kernel it depends on: the
   // partial kernel's last writes (the rows of units one pair finished whole)
   // may come after every merge here, and work later in the stream relies on
@@ -243,6 +264,7 @@ __global__ void __launch_bounds__(256) combine_balanced_kernel(const DecodeArgs 
   if (blockIdx.x == 0) ptx::grid_dep_wait();
 }
 
+template <int kC4>
 __device__ __forceinline__ void combine_balanced_block(const DecodeArgs& a, int units_per_block) {
   const mla_plan& p = a.plan;
   const int M = p.rows_per_unit;
@@ -260,12 +282,13 @@ __device__ __forceinline__ void combine_balanced_block(const DecodeArgs& a, int 
   if (!s_ok) return;
   (void)ptx::ld_acquire_gpu(a.unit_done + U);
   const int nb = (M + 31) / 32;
-  const int cb = blockIdx.x % kCombineColBlocks;
-  const int blk = blockIdx.x / kCombineColBlocks;
+  constexpr int kColBlocks = 16 / kC4;
+  const int cb = blockIdx.x % kColBlocks;
+  const int blk = blockIdx.x / kColBlocks;
   const int rb = blk % nb;
   const int u0 = (blk / nb) * units_per_block;
   for (int u = u0; u < U && u < u0 + units_per_block; ++u) {
-    combine_unit(a, u, rb, cb, &s_ok);
+    combine_unit<kC4>(a, u, rb, cb, &s_ok);
     __syncthreads();
     if (!s_ok) return;  // a wait gave up (the same in every thread)
   }
@@ -311,8 +334,10 @@ cudaError_t launch_combine_balanced(const DecodeArgs& a, cudaStream_t stream) {
   // about 4096 unit blocks at most: beyond that a block takes several units
   const int64_t per = (units + 4095) / 4096;
   const int64_t unit_blocks = (units + per - 1) / per;
+  // one chunk per thread when the doubled grid is still resident at once
+  const bool narrow = unit_blocks * nb * 16 <= kCombineMaxResident;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(unit_blocks * nb * kCombineColBlocks));
+  cfg.gridDim = dim3((unsigned)(unit_blocks * nb * (narrow ? 16 : 8)));
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
@@ -321,7 +346,8 @@ cudaError_t launch_combine_balanced(const DecodeArgs& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, combine_balanced_kernel, a, (int)per);
+  return narrow ? cudaLaunchKernelEx(&cfg, combine_balanced_kernel<1>, a, (int)per)
+                : cudaLaunchKernelEx(&cfg, combine_balanced_kernel<2>, a, (int)per);
 }
 
 }  // namespace mla

@@ -20,9 +20,8 @@ constexpr int kMaxVarlenUnits = 1 << 16;        // units of a ragged-query (pref
 
 // Balanced schedule table at the end of the workspace: int32 weighted start
 // of every schedule slot (U + 1 entries, the last = W, the total weight; slot
-// s holds unit sched_unit(s), see pair_schedule.cuh), the number of pairs that
-// have work, then the slot of each pair's first unit (-1: none). Written by
-// the partial kernel, read by the combine.
+// s holds unit sched_unit(s), see pair_schedule.cuh), then the number of pairs
+// that have work. Written by the partial kernel, read by the combine.
 // Balanced schedule: per-unit counts of finished partial pieces, then the
 // unit table's ready flag; right after the status header, and cleared with it
 // before every launch of the partial kernel.
@@ -31,7 +30,7 @@ inline uint64_t balanced_counter_bytes(int64_t units) {
   return ((uint64_t)(units + 1) * 4 + 255) & ~uint64_t(255);
 }
 inline uint64_t balanced_table_bytes(int64_t units) {
-  return ((uint64_t)(units + 2 + kNumSMs / 2) * 4 + 255) & ~uint64_t(255);
+  return ((uint64_t)(units + 2) * 4 + 255) & ~uint64_t(255);
 }
 // FP8 rows that see fewer keys than this send P as two E4M3 terms (the P.V
 // MMAs run twice); the balanced schedule weighs such tiles 3 against 2.

@@ -70,13 +70,15 @@ __device__ __forceinline__ int tile_weight(const mla_plan& p, const UnitGeom& ug
 }
 
 // Tiles [i0, i1) of a unit with `t` tiles of weight `w` starting at weighted
-// position `start` whose own start positions lie in [lo, hi).
+// position `start` whose own start positions lie in [lo, hi). Positions are
+// below W < 2^31 (the plan checks the total weight), so the differences fit
+// an int.
 __device__ __forceinline__ void tiles_in_range(int64_t start, int t, int w, int64_t lo, int64_t hi, int& i0,
                                                int& i1) {
-  const int64_t a0 = lo > start ? (lo - start + w - 1) / w : 0;
-  const int64_t a1 = hi > start ? (hi - start + w - 1) / w : 0;
-  i0 = (int)(a0 < t ? a0 : t);
-  i1 = (int)(a1 < t ? a1 : t);
+  const int a0 = lo > start ? ((int)(lo - start) + w - 1) / w : 0;
+  const int a1 = hi > start ? ((int)(hi - start) + w - 1) / w : 0;
+  i0 = a0 < t ? a0 : t;
+  i1 = a1 < t ? a1 : t;
 }
 
 // Scratch of the block-wide scans, after the piece list and SchedInfo: one int
@@ -103,8 +105,7 @@ __device__ __forceinline__ int warp_incl_scan(int v) {
 // pair's range are written in slot order, the first kMaxSmemPieces to shared
 // memory and, when there are more, all of them to this CTA's part of the
 // spill area (read back by load_piece). CTA 0 of pair 0 also writes the slot
-// start table the combine reads, then its ready flag; CTA 0 of every pair
-// records its first slot there (the combine's slot rule).
+// start table the combine reads, then its ready flag.
 template <int kKeys>
 __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uint8_t* sched_area) {
   const mla_plan& p = a.plan;
@@ -117,12 +118,25 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uin
   const int per = (U + (int)blockDim.x - 1) / (int)blockDim.x;
   const int s_beg = min(U, tid * per), s_end = min(U, s_beg + per);  // this thread's schedule slots
   const bool writer = pair == 0 && rank == 0;
+  // Tiles and tile weight of slot sl. The first slot of the thread's run keeps
+  // them from the first scan (a plan of at most one slot per thread reads
+  // seq_lens once); the others read them again.
+  int t_beg = 0, w_beg = 2;
+  auto geometry = [&](int sl, int& t, int& w) {
+    if (sl == s_beg) {
+      t = t_beg, w = w_beg;
+      return;
+    }
+    const UnitGeom ug = unit_geom(a, sched_unit(p, sl), false);
+    t = unit_span_tiles<kKeys>(ug), w = tile_weight(p, ug);
+  };
   // scan 1: the weighted start of this thread's run
   int run = 0;
   for (int sl = s_beg; sl < s_end; ++sl) {
     const UnitGeom ug = unit_geom(a, sched_unit(p, sl), writer);
-    const int t = unit_span_tiles<kKeys>(ug);
-    run += unit_lead_weight(t) + t * tile_weight(p, ug);
+    const int t = unit_span_tiles<kKeys>(ug), w = tile_weight(p, ug);
+    if (sl == s_beg) t_beg = t, w_beg = w;
+    run += unit_lead_weight(t) + t * w;
   }
   int incl = warp_incl_scan(run);
   if (lane == 31) scan1[warp] = incl;
@@ -140,9 +154,9 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uin
     int start = excl;
     for (int sl = s_beg; sl < s_end; ++sl) {
       a.sched[sl] = start;
-      const UnitGeom ug = unit_geom(a, sched_unit(p, sl), false);
-      const int t = unit_span_tiles<kKeys>(ug);
-      start += unit_lead_weight(t) + t * tile_weight(p, ug);
+      int t, w;
+      geometry(sl, t, w);
+      start += unit_lead_weight(t) + t * w;
     }
     if (tid == 0) {
       a.sched[U] = W;
@@ -154,8 +168,9 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uin
   {
     int start = excl;
     for (int sl = s_beg; sl < s_end; ++sl) {
-      const UnitGeom ug = unit_geom(a, sched_unit(p, sl), false);
-      const int t = unit_span_tiles<kKeys>(ug), w = tile_weight(p, ug), lead = unit_lead_weight(t);
+      int t, w;
+      geometry(sl, t, w);
+      const int lead = unit_lead_weight(t);
       int i0, i1;
       tiles_in_range(start + lead, t, w, lo, hi, i0, i1);
       if (i1 > i0) {
@@ -196,8 +211,9 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uin
     int start = excl, k = base;
     for (int sl = s_beg; sl < s_end; ++sl) {
       const int u = sched_unit(p, sl);
-      const UnitGeom ug = unit_geom(a, u, false);
-      const int t = unit_span_tiles<kKeys>(ug), w = tile_weight(p, ug), lead = unit_lead_weight(t);
+      int t, w;
+      geometry(sl, t, w);
+      const int lead = unit_lead_weight(t);
       int i0, i1;
       tiles_in_range(start + lead, t, w, lo, hi, i0, i1);
       if (i1 > i0) {
@@ -217,7 +233,6 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uin
     info->npc = npc;
     info->tiles = all_tiles;
     info->two = any_two;
-    if (rank == 0 && pair < p.split_kv) a.sched[U + 2 + pair] = npc > 0 ? s_first : -1;
   }
 }
 

@@ -123,6 +123,7 @@ struct PieceCtx16 {
   int64_t row0;
   const int32_t* table;
   bool whole;  // the piece is the whole unit: final output, not a partial
+  bool cont;   // the piece begins inside its unit (the pair's first piece)
 };
 
 __device__ __forceinline__ PieceCtx16 piece_ctx16(const DecodeArgs& a, const Piece& pc) {
@@ -141,6 +142,7 @@ __device__ __forceinline__ PieceCtx16 piece_ctx16(const DecodeArgs& a, const Pie
   c.row0 = ug.row0;
   c.table = a.block_tables + (int64_t)c.b * a.max_pages_per_seq;
   c.whole = pc.t0 == 0 && c.key1 >= ug.kend;
+  c.cont = pc.t0 > 0;
   return c;
 }
 
@@ -171,7 +173,6 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
   const int pair = blockIdx.x >> 1;
   const int H = p.num_heads, M = p.rows_per_unit;
   const int box_q = M < 64 ? M : 64;  // query rows per TMA box
-  auto slot_of = [&](int k) -> int64_t { return 2 * (int64_t)pair + (k == 0 ? 0 : 1); };
   auto lead = [&](int i) -> uint32_t { return mapa(bar(i), 0); };
   auto arrive_lead = [&](int i) {
     if (rank == 0) mbar_arrive(bar(i)); else mbar_arrive_remote_publish_smem(lead(i));
@@ -584,7 +585,10 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
       if (!ok) break;
       tc_fence_after();
       const float inv = (le > 0.f) ? a.v_scale / le : 0.f;
-      const int64_t slot = slot_of(k);
+      // partial slot of a cut piece: 2p when it begins inside its unit (only
+      // a pair's first piece can), 2p + 1 when it begins at the unit's start
+      // (then it is cut at the end: the pair's last piece)
+      const int64_t slot = 2 * (int64_t)pair + (c.cont ? 0 : 1);
       if (r < c.rows && grp == 0 && hf == 0) {
         const float lse_val = (le > 0.f) ? (m_fin - kSigma + log2f(le)) * kLn2 : -INFINITY;
         if (c.whole) {

@@ -14,8 +14,9 @@
 // out as equal contiguous ranges, one per pair. A pair walks its range as
 // pieces (the part of one unit inside the range): a piece that is a whole
 // unit writes out / lse directly; a unit cut between pairs leaves partial O
-// and LSE in the pair's slot (2p for its first piece, 2p + 1 for its last),
-// merged by the combine kernel. Every pair therefore does the same amount of
+// and LSE in one of the pair's two slots (2p for a piece that begins inside
+// its unit, 2p + 1 for one that begins at the unit's start), merged by the
+// combine kernel. Every pair therefore does the same amount of
 // work whatever the length mix, and the pipeline runs on across pieces. This
 // is the article's split_kv auto-sizing (section 二) made exact on the device.
 // The same kernel serves ragged prefill (entries with their own query
@@ -167,6 +168,7 @@ struct PieceCtx {
   int64_t row0;
   const int32_t* table;
   bool whole;  // the piece is the whole unit: final output, not a partial
+  bool cont;   // the piece begins inside its unit (the pair's first piece)
   bool two;    // two-term P
 };
 
@@ -194,6 +196,7 @@ __device__ __forceinline__ PieceCtx piece_ctx(const DecodeArgs& a, const Piece& 
   c.row0 = ug.row0;
   c.table = a.block_tables + (int64_t)c.b * a.max_pages_per_seq;
   c.whole = pc.t0 == 0 && c.key1 >= ug.kend;
+  c.cont = pc.t0 > 0;
   c.two = kTwo && tile_weight(p, ug) == 3;  // the same rule as the schedule's weights
   return c;
 }
@@ -226,8 +229,6 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, i
   const int pair = blockIdx.x >> 1;
   const int H = p.num_heads, M = p.rows_per_unit;
   const int box_q = M < 64 ? M : 64;  // query rows per TMA box (the tensor maps' box height)
-  // slot of piece k: 2p for the pair's first piece, 2p + 1 for its last
-  auto slot_of = [&](int k) -> int64_t { return 2 * (int64_t)pair + (k == 0 ? 0 : 1); };
 
   // the leader's copy of barrier i, as a cluster address
   auto lead = [&](int i) -> uint32_t { return mapa(bar(i), 0); };
@@ -673,7 +674,10 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, i
       if (!ok) break;
       tc_fence_after();
       const float inv = (le > 0.f) ? a.v_scale / le : 0.f;
-      const int64_t slot = slot_of(k);
+      // partial slot of a cut piece: 2p when it begins inside its unit (only
+      // a pair's first piece can), 2p + 1 when it begins at the unit's start
+      // (then it is cut at the end: the pair's last piece)
+      const int64_t slot = 2 * (int64_t)pair + (c.cont ? 0 : 1);
       if (r < c.rows && grp == 0 && hf == 0) {
         const float lse_val = (le > 0.f) ? (m_fin - kSigma + log2f(le)) * kLn2 : -INFINITY;
         if (c.whole) {

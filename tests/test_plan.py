@@ -135,9 +135,11 @@ _MIXED = [_rng.choice([0, 1, 2, 7, 130, 640]) for _ in range(300)]
 ])
 def test_balanced_schedule_covers_each_tile_once(tiles, weights):
     """Every tile of every unit lies in exactly one piece; a pair leaves at most two partial
-    pieces (its first and last), in slots 2p and 2p + 1; the combine's rule (the pairs of the
-    unit's first and last tile starts; slot 2p0 iff the unit is p0's recorded first unit) finds
-    the same slots, and every pair it waits for holds a piece of the unit."""
+    pieces (its first and last): a cut piece that begins inside its unit (t0 > 0) in slot 2p,
+    one that begins at the unit's start in slot 2p + 1, never both in one slot; the combine's
+    rule (the pairs of the unit's first and last tile starts; slot 2p0 + 1 for the first, 2q for
+    every later one) finds the same slots, and every pair it waits for holds a piece of the
+    unit."""
     P = 74
     w_of = weights or [2] * len(tiles)
     starts, W, np_, pieces, first = _balanced_schedule(tiles, P, weights)
@@ -151,7 +153,9 @@ def test_balanced_schedule_covers_each_tile_once(tiles, weights):
             whole = t0 == 0 and t1 == tiles[u]
             if not whole:
                 assert k == 0 or k == len(pp) - 1
-                slot = 2 * p + (0 if k == 0 else 1)
+                assert t0 == 0 or k == 0  # only a pair's first piece begins inside its unit
+                assert t0 > 0 or k == len(pp) - 1  # a cut piece from the unit's start is the last
+                slot = 2 * p + (0 if t0 > 0 else 1)
                 assert slot not in slot_of_piece.values()
                 slot_of_piece[(u, p)] = slot
     assert len(seen) == sum(tiles)
@@ -166,7 +170,7 @@ def test_balanced_schedule_covers_each_tile_once(tiles, weights):
             continue
         for q in range(p0, p1 + 1):
             assert any(pu == u for pu, _, _ in pieces[q])  # the combine's wait ends
-            slot = (2 * q if first[q] == u else 2 * q + 1) if q == p0 else 2 * q
+            slot = 2 * q + 1 if q == p0 else 2 * q
             assert slot_of_piece[(u, q)] == slot
 
 
