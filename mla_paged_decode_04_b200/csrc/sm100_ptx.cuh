@@ -63,6 +63,11 @@ __device__ __forceinline__ int ld_nc_ordered(const int* p) {
   asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(p));
   return v;
 }
+// Drops the 128-byte L2 line at p (128-byte aligned) without writing it back:
+// its contents become undefined. For data no one reads again.
+__device__ __forceinline__ void discard_l2_line(const void* p) {
+  asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -838,6 +838,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     pair_idle_teardown16(smem);
     return;
   }
+  // The softmax warps wait for the first scores anyway: they drop the L2
+  // lines of the pair's partial slots meanwhile.
+  if (threadIdx.x >= 32 * kSoftmaxWarp0)
+    discard_pair_slots(prm.a, blockIdx.x >> 1, cluster_ctarank(), info->tiles, threadIdx.x - 32 * kSoftmaxWarp0,
+                       kThreads - 32 * kSoftmaxWarp0);
   if (prm.a.plan.dtype == MLA_BF16)
     pair_cta16<true>(prm, smem, npc, info->tiles);
   else

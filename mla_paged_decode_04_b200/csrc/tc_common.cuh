@@ -88,6 +88,34 @@ __device__ __forceinline__ void drain_phase(uint32_t bar, uint32_t parity) {
   }
 }
 
+// The pair's two partial slots hold the previous call's pieces, which its
+// combine has read (this kernel runs after it): their L2 lines are dropped
+// without a write-back, instead of being written to DRAM while this call
+// streams the cache. Each CTA drops the lines of its own 64 rows (with M a
+// multiple of 8, a 128-byte line is 8 rows of one 16-byte chunk of a slot),
+// long before its epilogue writes them again. Threads t0, t0 + nt, ... of the
+// CTA take part. Only when the call streams more cache than the L2 holds
+// (estimated from this pair's `tiles`, 72 KB of cache each in both pair
+// kernels, times the pairs): otherwise the lines are simply overwritten in L2
+// by the next call and dropping them would only cost L2 requests.
+__device__ __forceinline__ void discard_pair_slots(const DecodeArgs& a, int pair, uint32_t rank, int tiles, int t0,
+                                                   int nt) {
+  constexpr int64_t kTileBytes = 128 * MLA_D_QK;  // a pair tile: 128 FP8 or 64 16-bit keys of 576 dims
+  constexpr int64_t kL2Bytes = 126ll << 20;
+  const int M = a.plan.rows_per_unit;
+  if (!a.o_part || M % 8 != 0 || pair >= a.plan.split_kv) return;
+  if ((int64_t)tiles * a.plan.split_kv * kTileBytes < kL2Bytes) return;
+  const int groups = M / 8;                  // 8-row groups of a chunk
+  const int per_slot = (MLA_D_V / 4) * groups;  // lines of a slot
+  for (int i = t0; i < 2 * per_slot; i += nt) {
+    const int g = i % groups;
+    if (g / 8 != (int)rank) continue;  // rows [64 rank, 64 rank + 64)
+    const int c4 = (i % per_slot) / groups;
+    const int slot = 2 * pair + i / per_slot;
+    ptx::discard_l2_line(a.o_part + (((int64_t)slot * (MLA_D_V / 4) + c4) * M + 8 * g) * 4);
+  }
+}
+
 // Teardown drain of the CTA-pair kernels (layout L, barriers at bar0 + 8 i):
 // the last phase of every barrier the leader's MMA commits arrive on, after
 // `n_all` tiles and `npc` pieces. Lane k of the calling warp waits for one

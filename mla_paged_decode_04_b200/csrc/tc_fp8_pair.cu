@@ -920,6 +920,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     pair_idle_teardown(smem);
     return;
   }
+  // The softmax warps wait for the first scores anyway: they drop the L2
+  // lines of the pair's partial slots meanwhile.
+  if (threadIdx.x >= 32 * kSoftmaxWarp0)
+    discard_pair_slots(prm.a, blockIdx.x >> 1, cluster_ctarank(), info->tiles, threadIdx.x - 32 * kSoftmaxWarp0,
+                       kThreads - 32 * kSoftmaxWarp0);
   // Short entries send P as two E4M3 terms; a pair with any such piece takes
   // the layout with room for both planes (the choice is the same in both CTAs).
   if (info->two)
