@@ -108,12 +108,15 @@ namespace {
 // output columns) of row i over the pieces, and the 32 threads of a warp read
 // 32 consecutive rows (512 contiguous bytes) per load. The grid holds
 // units x row blocks x 16 / kC4 column blocks, so that even a few long units
-// that were cut into many pieces spread over the whole GPU: plans with few
-// units take kC4 = 1 (twice the blocks, each thread half the columns and
-// twice the pieces in flight), the others kC4 = 2. At 64 registers a thread,
-// four blocks fit an SM: the grids of up to 592 blocks are resident at once
-// while their units finish, and none waits for another's slot.
-constexpr int kCombineMaxResident = 4 * 148;
+// that were cut into many pieces spread over the whole GPU. The grid must be
+// resident at once while its units finish, so that no block waits for
+// another's slot: kC4 = 2 runs at 64 registers a thread (four blocks an SM,
+// grids of up to 592 blocks) and merges 3 pieces a batch; plans whose grid at
+// kC4 = 1 is at most 296 blocks (few units, each cut into many pieces) take
+// kC4 = 1 at up to 128 registers (two blocks an SM) and merge 20 pieces a
+// batch, so that the ~20 pieces of a unit spread over all 74 pairs take one
+// round of loads.
+constexpr int kCombineNarrowResident = 2 * 148;
 constexpr uint64_t kUnitWaitNs = 500ull * 1000 * 1000;  // per wait: 0.5 s
 
 // Bounded wait (one thread) for a counter written by the partial kernel;
@@ -179,7 +182,7 @@ __device__ __forceinline__ void combine_unit(const DecodeArgs& a, int u, int rb,
   // accumulators are rescaled when it grows). Pieces go in batches of kBatch
   // whose loads are all issued before any of them is used (no branch depends
   // on a loaded value), so their latencies overlap.
-  constexpr int kBatch = kC4 == 2 ? 3 : 6;
+  constexpr int kBatch = kC4 == 2 ? 3 : 20;
   constexpr int kAcc = 4 * kC4;
   const float* base = a.o_part + (c4_0 * M + r) * 4;
   const int slot_stride = (MLA_D_V / 4) * M * 4;  // floats per partial slot
@@ -250,7 +253,7 @@ template <int kC4>
 __device__ __forceinline__ void combine_balanced_block(const DecodeArgs& a, int units_per_block);
 
 template <int kC4>
-__global__ void __launch_bounds__(256, 4) combine_balanced_kernel(const DecodeArgs a, int units_per_block) {
+__global__ void __launch_bounds__(256, kC4 == 2 ? 4 : 2) combine_balanced_kernel(const DecodeArgs a, int units_per_block) {
   // The next step's workspace clear may be launched now: it waits for this
   // grid's completion before touching the workspace.
   ptx::launch_dependents();
@@ -334,8 +337,8 @@ cudaError_t launch_combine_balanced(const DecodeArgs& a, cudaStream_t stream) {
   // about 4096 unit blocks at most: beyond that a block takes several units
   const int64_t per = (units + 4095) / 4096;
   const int64_t unit_blocks = (units + per - 1) / per;
-  // one chunk per thread when the doubled grid is still resident at once
-  const bool narrow = unit_blocks * nb * 16 <= kCombineMaxResident;
+  // one chunk per thread when that grid is still resident at once
+  const bool narrow = unit_blocks * nb * 16 <= kCombineNarrowResident;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(unit_blocks * nb * (narrow ? 16 : 8)));
   cfg.blockDim = dim3(256);
