@@ -75,6 +75,9 @@ typedef enum {
 #define MLA_DEV_TIMEOUT 0x4      /* a bounded pipeline wait gave up; outputs unspecified */
 #define MLA_DEV_BAD_QLEN 0x8     /* ragged queries: a cu_seqlens_q range decreasing, longer than the
                                     plan's max_q_len or past total_q; that entry gets no output */
+#define MLA_DEV_BOUNDS 0x10      /* bounds-checking build only (mla_bounds_checked): a global
+                                    index of the CTA-pair or combine kernels fell outside its
+                                    buffer; that access was skipped, outputs unspecified */
 
 typedef enum {
   MLA_KERNEL_AUTO = 0,         /* MLA_KERNEL_TCGEN05 */
@@ -131,7 +134,10 @@ typedef struct {
   int32_t fault_test; /* 0, as the planner sets it. Tests of failure detection only: 1 makes the
                          FP8 CTA-pair kernel leave the first tile of every pair unloaded, so that
                          the wait for it runs out (MLA_DEV_TIMEOUT after its 0.5 s limit, no
-                         fault); refused on other plans */
+                         fault); 2, accepted by the bounds-checking build only, moves every
+                         output row and partial slot of that kernel past its buffer, so that
+                         the checks skip each store and set MLA_DEV_BOUNDS; refused on other
+                         plans */
 } mla_plan;
 
 /*
@@ -339,6 +345,18 @@ const char* mla_version(void);
  * CUDA call is made.
  */
 int mla_last_cuda_error(const char** name);
+
+/*
+ * 1 in the bounds-checking build of this library (libmla_decode_check.so,
+ * compiled with MLA_BOUNDS_CHECK=1), 0 in the normal one. The checking build
+ * tests, on the device, every global index of the CTA-pair partial kernels,
+ * their on-device schedule and the balanced combine against the extent of
+ * its buffer (block-table rows, the piece spill area, the schedule table, the
+ * unit counters, the partial slots, out and lse); an index outside sets
+ * MLA_DEV_BOUNDS in the status word and the access is skipped instead of
+ * made. It is slower and meant for debugging, not for production. Host only.
+ */
+int mla_bounds_checked(void);
 
 /*
  * mla_kv_pack: write new tokens into the paged latent cache, fused with the

@@ -4,7 +4,9 @@ The functions carry the C ABI's names (include/mla_decode.h) and pass raw
 device pointers and the current CUDA stream; every step of the decode runs
 in the library's kernels. PyTorch is used only to own device memory and
 streams. If the shared library is missing this module raises at import: there
-is no fallback path.
+is no fallback path. With MLA_DECODE_BOUNDS_CHECK=1 in the environment the
+bounds-checking build, libmla_decode_check.so, is loaded instead (slower; its
+kernels set MLA_DEV_BOUNDS instead of accessing memory outside a buffer).
 """
 from __future__ import annotations
 
@@ -14,7 +16,9 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmla_decode.so")
+NORMAL_LIB_PATH = os.path.join(_HERE, "libmla_decode.so")
+CHECK_LIB_PATH = os.path.join(_HERE, "libmla_decode_check.so")
+LIB_PATH = CHECK_LIB_PATH if os.environ.get("MLA_DECODE_BOUNDS_CHECK", "0") == "1" else NORMAL_LIB_PATH
 
 MLA_BF16, MLA_FP16, MLA_FP8_E4M3 = 0, 1, 2
 DTYPES = {"bf16": MLA_BF16, "fp16": MLA_FP16, "fp8": MLA_FP8_E4M3}
@@ -22,7 +26,7 @@ MLA_KERNEL_AUTO, MLA_KERNEL_TCGEN05, MLA_KERNEL_SIMT, MLA_KERNEL_TCGEN05_SOLO = 
 KERNELS = {"auto": MLA_KERNEL_AUTO, "tcgen05": MLA_KERNEL_TCGEN05, "simt": MLA_KERNEL_SIMT,
            "tcgen05_solo": MLA_KERNEL_TCGEN05_SOLO}
 
-MLA_DEV_BAD_PAGE, MLA_DEV_SEQ_TOO_LONG, MLA_DEV_TIMEOUT, MLA_DEV_BAD_QLEN = 0x1, 0x2, 0x4, 0x8
+MLA_DEV_BAD_PAGE, MLA_DEV_SEQ_TOO_LONG, MLA_DEV_TIMEOUT, MLA_DEV_BAD_QLEN, MLA_DEV_BOUNDS = 0x1, 0x2, 0x4, 0x8, 0x10
 (MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED_SHAPE, MLA_ERR_WORKSPACE_TOO_SMALL, MLA_ERR_ARCH, MLA_ERR_CUDA,
  MLA_ERR_PLAN_MISMATCH) = (-1, -2, -3, -4, -5, -6)
 
@@ -30,7 +34,7 @@ EXPORTED = ["mla_decode_plan", "mla_decode_plan_custom", "mla_decode", "mla_deco
             "mla_decode_combine", "mla_decode_status", "mla_status_string", "mla_version",
             "mla_decode_no_alloc", "mla_decode_no_alloc_status", "mla_last_cuda_error", "mla_kv_pack", "mla_kv_amax",
             "mla_decode_plan_window", "mla_prefill_plan", "mla_prefill_plan_custom", "mla_prefill",
-            "mla_prefill_partial", "mla_prefill_combine"]
+            "mla_prefill_partial", "mla_prefill_combine", "mla_bounds_checked"]
 MLA_NO_ALLOC_SCRATCH_BYTES = 48 << 20
 
 
@@ -61,12 +65,13 @@ class MlaError(RuntimeError):
         self.code = code
 
 
-def _load():
-    if not os.path.exists(LIB_PATH):
+def load_library(path):
+    """The library at `path` (the normal or the bounds-checking build) with its argument types set."""
+    if not os.path.exists(path):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python mla_paged_decode_04_b200/build.py` "
-            "(there is no non-CUDA fallback)")
-    lib = ctypes.CDLL(LIB_PATH)
+            f"{path} is missing: build it with `python mla_paged_decode_04_b200/build.py"
+            f"{' --check' if path == CHECK_LIB_PATH else ''}` (there is no non-CUDA fallback)")
+    lib = ctypes.CDLL(path)
     i32, i64, u64, f32, vp = (ctypes.c_int, ctypes.c_int64, ctypes.c_uint64, ctypes.c_float,
                               ctypes.c_void_p)
     P = ctypes.POINTER(MlaPlan)
@@ -100,10 +105,17 @@ def _load():
     lib.mla_kv_pack.restype = i32
     lib.mla_kv_amax.argtypes = [vp, vp, i64, i32, vp, vp]
     lib.mla_kv_amax.restype = i32
+    lib.mla_bounds_checked.argtypes = []
+    lib.mla_bounds_checked.restype = i32
     return lib
 
 
-_lib = _load()
+_lib = load_library(LIB_PATH)
+
+
+def bounds_checked() -> bool:
+    """True when the loaded library is the bounds-checking build."""
+    return bool(_lib.mla_bounds_checked())
 
 
 def lib():

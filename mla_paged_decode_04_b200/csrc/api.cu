@@ -81,9 +81,12 @@ int check_plan(const mla_plan* p) {
   if (p->kernel == MLA_KERNEL_TCGEN05_SOLO && p->dtype != MLA_FP8_E4M3) return MLA_ERR_PLAN_MISMATCH;
   if (p->schedule != MLA_SCHEDULE_SPLITS && p->schedule != MLA_SCHEDULE_BALANCED) return MLA_ERR_PLAN_MISMATCH;
   if (p->window < 0) return MLA_ERR_PLAN_MISMATCH;
-  // the failure-detection test mode exists on the FP8 CTA-pair kernel only
-  if (p->fault_test != 0 && !(p->fault_test == 1 && p->dtype == MLA_FP8_E4M3 && p->kernel == MLA_KERNEL_TCGEN05 &&
-                              p->schedule == MLA_SCHEDULE_BALANCED))
+  // the failure-detection test modes exist on the FP8 CTA-pair kernel only;
+  // mode 2 (stores past the buffers, caught by the checks) in the checking
+  // build only
+  if (p->fault_test != 0 &&
+      !((p->fault_test == 1 || (p->fault_test == 2 && MLA_BOUNDS_CHECK)) && p->dtype == MLA_FP8_E4M3 &&
+        p->kernel == MLA_KERNEL_TCGEN05 && p->schedule == MLA_SCHEDULE_BALANCED))
     return MLA_ERR_PLAN_MISMATCH;
   // a window and ragged queries run on the CTA-pair kernels and the SIMT kernel
   if ((p->window > 0 || p->varlen) &&
@@ -334,6 +337,8 @@ extern "C" const char* mla_status_string(int code) {
 }
 
 extern "C" const char* mla_version(void) { return "0.1.0"; }
+
+extern "C" int mla_bounds_checked(void) { return MLA_BOUNDS_CHECK ? 1 : 0; }
 
 extern "C" int mla_last_cuda_error(const char** name) {
   if (name) *name = cudaGetErrorName(g_last_cuda_error);

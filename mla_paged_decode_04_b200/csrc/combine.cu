@@ -142,6 +142,7 @@ __device__ __forceinline__ void combine_unit(const DecodeArgs& a, int u, int rb,
   const int U = p.batch * p.q_groups;
   const int32_t* tbl = a.sched;
   const int sl = sched_slot(p, u);  // the unit's position in the schedule's sequence
+  if (!in_bounds(a, sl, U)) return;  // block-uniform
   const int64_t start = tbl[sl], end = tbl[sl + 1], W = tbl[U];
   const int np = tbl[U + 1];
   const UnitGeom ug = unit_geom(a, u, false);
@@ -151,6 +152,8 @@ __device__ __forceinline__ void combine_unit(const DecodeArgs& a, int u, int rb,
   const int p0 = end > start ? balanced_pair_of(start + lead, W, np) : 0;
   const int p1 = end > start ? balanced_pair_of(end - tile_weight(p, ug), W, np) : 0;
   if (end > start && p0 == p1) return;  // a whole unit: written by its pair
+  // (block-uniform: every thread leaves together)
+  if (end > start && !(in_bounds(a, 2 * p0 + 1, balanced_slots(a)) && in_bounds(a, 2 * p1, balanced_slots(a)))) return;
   if (end > start) {
     __syncthreads();  // every thread has read s_ok
     if (threadIdx.x == 0) *s_ok = wait_count(a.unit_done + u, kPieceArrivals * (p1 - p0 + 1), a.status);
@@ -161,6 +164,7 @@ __device__ __forceinline__ void combine_unit(const DecodeArgs& a, int u, int rb,
   const int r = rb * 32 + (threadIdx.x & 31);       // row within the unit
   const int c4_0 = (cb * 8 + (threadIdx.x >> 5)) * kC4;  // first of this thread's kC4 16-byte chunks
   if (r >= ug.rows) return;  // past the unit's rows (an entry's last group under ragged queries)
+  if (!in_bounds(a, ug.row0 + r, out_rows(a)) || !in_bounds(a, r, M)) return;
   const bool lse_writer = a.lse && cb == 0 && (threadIdx.x >> 5) == 0;
   if (end == start) {  // no key at all
     const int64_t row = ug.row0 + r;

@@ -12,6 +12,33 @@ namespace mla {
 
 constexpr float kLn2 = 0.6931471805599453f;
 
+// Device bounds checks of the checking build (compiled with
+// MLA_BOUNDS_CHECK=1): in_bounds(a, i, n) is false when i lies outside
+// [0, n), after setting MLA_DEV_BOUNDS in the status word, and the caller
+// then skips the access. In the normal build it is always true and every
+// check compiles away.
+__device__ __forceinline__ bool in_bounds(const DecodeArgs& a, int64_t i, int64_t n) {
+#if MLA_BOUNDS_CHECK
+  if (i >= 0 && i < n) return true;
+  atomicOr(a.status, MLA_DEV_BOUNDS);
+  return false;
+#else
+  (void)a, (void)i, (void)n;
+  return true;
+#endif
+}
+// Extents the checks compare against: rows of out / lse, the balanced
+// schedule's partial slots, its piece spill entries (both CTA ranks) and its
+// units.
+__device__ __forceinline__ int64_t out_rows(const DecodeArgs& a) { return a.total_q * a.plan.num_heads; }
+__device__ __forceinline__ int64_t balanced_slots(const DecodeArgs& a) { return 2 * (int64_t)a.plan.split_kv; }
+__device__ __forceinline__ int64_t balanced_units(const DecodeArgs& a) {
+  return (int64_t)a.plan.batch * a.plan.q_groups;
+}
+__device__ __forceinline__ int64_t spill_entries(const DecodeArgs& a) {
+  return 2 * (balanced_units(a) + a.plan.split_kv);
+}
+
 // Element of a q / cache buffer as float (FP8 stays in code units; the
 // caller applies the per-tensor scale once).
 template <int DT>
@@ -30,6 +57,7 @@ __device__ __forceinline__ float load_elem(const void* base, int64_t idx) {
 // block table can cover. Out-of-contract lengths set MLA_DEV_SEQ_TOO_LONG
 // (when `flag` is set) and are clamped, so no read leaves the table.
 __device__ __forceinline__ int effective_seq_len(const DecodeArgs& a, int b, bool flag) {
+  if (!in_bounds(a, b, a.plan.batch)) return 0;
   int n = a.seq_lens[b];
   const int64_t cap_split = (int64_t)a.plan.split_kv * a.plan.keys_per_split;
   const int64_t cap_table = (int64_t)a.max_pages_per_seq * kTileKeys;
@@ -52,6 +80,7 @@ struct EntryQ {
 };
 __device__ __forceinline__ EntryQ entry_q(const DecodeArgs& a, int b, bool flag) {
   if (!a.cu_q) return {(int64_t)b * a.plan.q_len, a.plan.q_len};
+  if (!in_bounds(a, b, a.plan.batch)) return {0, 0};
   const int s = a.cu_q[b], e = a.cu_q[b + 1];
   if (s < 0 || e < s || e - s > a.plan.q_len || (int64_t)e > a.total_q) {
     if (flag) atomicOr(a.status, MLA_DEV_BAD_QLEN);

@@ -8,6 +8,11 @@
 
 #include "mla_decode.h"
 
+// 1 in the bounds-checking build (libmla_decode_check.so), 0 otherwise.
+#ifndef MLA_BOUNDS_CHECK
+#define MLA_BOUNDS_CHECK 0
+#endif
+
 namespace mla {
 
 constexpr uint32_t kPlanMagic = 0x4d4c4131u;  // "MLA1"

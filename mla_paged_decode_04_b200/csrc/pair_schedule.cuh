@@ -153,7 +153,7 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uin
   if (writer) {
     int start = excl;
     for (int sl = s_beg; sl < s_end; ++sl) {
-      a.sched[sl] = start;
+      if (in_bounds(a, sl, U)) a.sched[sl] = start;
       int t, w;
       geometry(sl, t, w);
       start += unit_lead_weight(t) + t * w;
@@ -222,7 +222,7 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uin
         pc.t0 = i0;
         pc.t1 = i1;
         if (k < kMaxSmemPieces) smem_list[k] = pc;
-        if (spill) spill[k] = pc;
+        if (spill && in_bounds(a, spill_base + k, spill_entries(a))) spill[k] = pc;
         ++k;
       }
       start += lead + t * w;
@@ -242,6 +242,7 @@ __device__ void build_schedule(const DecodeArgs& a, int pair, uint32_t rank, uin
 __device__ __forceinline__ Piece load_piece(const DecodeArgs& a, const uint8_t* smem, int k) {
   if (k < kMaxSmemPieces) return reinterpret_cast<const Piece*>(smem)[k];
   const SchedInfo* info = reinterpret_cast<const SchedInfo*>(smem + kMaxSmemPieces * sizeof(Piece));
+  if (!in_bounds(a, info->spill_base + k, spill_entries(a))) return Piece{0, 0, 0};
   return reinterpret_cast<const Piece*>(a.pieces)[info->spill_base + k];
 }
 

@@ -124,6 +124,9 @@ struct PieceCtx16 {
   const int32_t* table;
   bool whole;  // the piece is the whole unit: final output, not a partial
   bool cont;   // the piece begins inside its unit (the pair's first piece)
+#if MLA_BOUNDS_CHECK
+  bool table_ok;  // the piece's block-table entries lie inside row b of the table
+#endif
 };
 
 __device__ __forceinline__ PieceCtx16 piece_ctx16(const DecodeArgs& a, const Piece& pc) {
@@ -143,12 +146,19 @@ __device__ __forceinline__ PieceCtx16 piece_ctx16(const DecodeArgs& a, const Pie
   c.table = a.block_tables + (int64_t)c.b * a.max_pages_per_seq;
   c.whole = pc.t0 == 0 && c.key1 >= ug.kend;
   c.cont = pc.t0 > 0;
+#if MLA_BOUNDS_CHECK
+  c.table_ok = c.n_pt <= 0 || (in_bounds(a, c.b, a.plan.batch) && in_bounds(a, c.page0, a.max_pages_per_seq) &&
+                               in_bounds(a, (int64_t)c.page0 + c.n_pt - 1, a.max_pages_per_seq));
+#endif
   return c;
 }
 
 // Block-table entry of pair tile j of the piece, read one tile ahead of its
 // use with a load kept ahead of the next barrier wait.
 __device__ __forceinline__ int piece_entry16(const PieceCtx16& c, int j) {
+#if MLA_BOUNDS_CHECK
+  if (!c.table_ok) return 0;  // outputs unspecified: MLA_DEV_BOUNDS is set
+#endif
   return j < c.n_pt ? ld_nc_ordered(c.table + c.page0 + j) : 0;
 }
 // an entry outside the cache reads page 0 (its keys are masked by the softmax)
@@ -592,8 +602,8 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
       if (r < c.rows && grp == 0 && hf == 0) {
         const float lse_val = (le > 0.f) ? (m_fin - kSigma + log2f(le)) * kLn2 : -INFINITY;
         if (c.whole) {
-          if (a.lse) a.lse[c.row0 + r] = lse_val;
-        } else {
+          if (a.lse && in_bounds(a, c.row0 + r, out_rows(a))) a.lse[c.row0 + r] = lse_val;
+        } else if (in_bounds(a, slot * M + r, balanced_slots(a) * M)) {
           a.lse_part[slot * M + r] = lse_val;
         }
       }
@@ -609,6 +619,8 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
           tmem_wait_ld();
           if (r >= c.rows) continue;
           const int col = 256 * grp + 128 * hf + 32 * cc;
+          if (c.whole ? !in_bounds(a, c.row0 + r, out_rows(a)) : !in_bounds(a, slot * M + r, balanced_slots(a) * M))
+            continue;
           if (c.whole) {
             uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + (c.row0 + r) * MLA_D_V + col);
 #pragma unroll
@@ -642,7 +654,8 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
           __syncwarp();
           if (lane == 0) {
             __threadfence();
-            atomicAdd(a.unit_done + load_piece(a, smem, k).u, 1);
+            const int u = load_piece(a, smem, k).u;
+            if (in_bounds(a, u, balanced_units(a))) atomicAdd(a.unit_done + u, 1);
           }
         }
         if (!last_piece) {
@@ -684,6 +697,7 @@ __device__ __forceinline__ void pair_cta16(const Pair16Params& prm, uint8_t* sme
           if (64 * (int)rank + rr >= c.rows) break;  // rows past the unit belong to no output
           const float inv2 = rowinv[rr];
           const int rr_u = 64 * (int)rank + rr;  // row within the unit
+          if (!in_bounds(a, c.row0 + rr_u, out_rows(a))) continue;
           const float* srow = stage + rr * MLA_D_V;
           {
             // BF16: a lane writes 8 consecutive values (16 bytes) per step

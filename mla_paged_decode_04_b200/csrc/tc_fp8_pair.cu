@@ -193,11 +193,19 @@ __device__ __forceinline__ PieceCtx piece_ctx(const DecodeArgs& a, const Piece& 
   c.n_pt = pc.t1 - pc.t0;
   c.n_tiles = (c.key1 - c.key0 + kTileKeys - 1) / kTileKeys;
   c.tile0 = c.key0 / kTileKeys;
-  c.row0 = ug.row0;
+  // (test mode 2 of the checking build: every output row past out's end)
+  c.row0 = ug.row0 + (MLA_BOUNDS_CHECK && p.fault_test == 2 ? out_rows(a) : 0);
   c.table = a.block_tables + (int64_t)c.b * a.max_pages_per_seq;
   c.whole = pc.t0 == 0 && c.key1 >= ug.kend;
   c.cont = pc.t0 > 0;
   c.two = kTwo && tile_weight(p, ug) == 3;  // the same rule as the schedule's weights
+#if MLA_BOUNDS_CHECK
+  // the piece's block-table entries [tile0, tile0 + n_tiles) of row b; if any
+  // lies outside, none is read and every key of the piece is masked
+  if (c.n_tiles > 0 && !(in_bounds(a, c.b, p.batch) && in_bounds(a, c.tile0, a.max_pages_per_seq) &&
+                         in_bounds(a, (int64_t)c.tile0 + c.n_tiles - 1, a.max_pages_per_seq)))
+    c.n_tiles = 0;
+#endif
   return c;
 }
 
@@ -279,7 +287,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, i
           if (!(ok = bounded_wait_cta(bar(L::B_K_EMPTY + sk), ((jt / NK) & 1) ^ 1, abort_flag, a.status))) break;
           // failure-detection test mode: the pair's first tile is never loaded,
           // so the S issuer's wait for it runs out (every wait is bounded)
-          if (p.fault_test && jt == 0) continue;
+          if (p.fault_test == 1 && jt == 0) continue;
           const uint32_t ks = sb + L::kKOff + sk * L::kKSlot;
           const uint32_t full = lead(L::B_K_FULL + sk);
           if (rank == 0) mbar_arrive_expect_tx(bar(L::B_K_FULL + sk), 2u * L::kKSlot);
@@ -677,12 +685,14 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, i
       // partial slot of a cut piece: 2p when it begins inside its unit (only
       // a pair's first piece can), 2p + 1 when it begins at the unit's start
       // (then it is cut at the end: the pair's last piece)
-      const int64_t slot = 2 * (int64_t)pair + (c.cont ? 0 : 1);
+      // (test mode 2 of the checking build: every slot past the partials' end)
+      const int64_t slot =
+          2 * (int64_t)pair + (c.cont ? 0 : 1) + (MLA_BOUNDS_CHECK && p.fault_test == 2 ? balanced_slots(a) : 0);
       if (r < c.rows && grp == 0 && hf == 0) {
         const float lse_val = (le > 0.f) ? (m_fin - kSigma + log2f(le)) * kLn2 : -INFINITY;
         if (c.whole) {
-          if (a.lse) a.lse[c.row0 + r] = lse_val;
-        } else {
+          if (a.lse && in_bounds(a, c.row0 + r, out_rows(a))) a.lse[c.row0 + r] = lse_val;
+        } else if (in_bounds(a, slot * M + r, balanced_slots(a) * M)) {
           a.lse_part[slot * M + r] = lse_val;
         }
       }
@@ -698,6 +708,8 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, i
           tmem_wait_ld();
           if (r >= c.rows) continue;
           const int col = 256 * grp + 128 * hf + 32 * cc;
+          if (c.whole ? !in_bounds(a, c.row0 + r, out_rows(a)) : !in_bounds(a, slot * M + r, balanced_slots(a) * M))
+            continue;
           if (c.whole) {
             uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + (c.row0 + r) * MLA_D_V + col);
 #pragma unroll
@@ -731,7 +743,8 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, i
           __syncwarp();
           if (lane == 0) {
             __threadfence();
-            atomicAdd(a.unit_done + load_piece(a, smem, k).u, 1);
+            const int u = load_piece(a, smem, k).u;
+            if (in_bounds(a, u, balanced_units(a))) atomicAdd(a.unit_done + u, 1);
           }
         }
         if (!last_piece) {
@@ -773,6 +786,7 @@ __device__ __forceinline__ void pair_cta(const PairParams& prm, uint8_t* smem, i
           if (64 * (int)rank + rr >= c.rows) break;  // rows past the unit belong to no output
           const float inv2 = rowinv[rr];
           const int rr_u = 64 * (int)rank + rr;  // row within the unit
+          if (!in_bounds(a, c.row0 + rr_u, out_rows(a))) continue;
           const float* srow = stage + rr * MLA_D_V;
           {
             // BF16: a lane writes 8 consecutive values (16 bytes) per step

@@ -35,6 +35,33 @@ def test_library_exports_every_declared_symbol():
     assert set(names) <= set(_lib.EXPORTED)
 
 
+def test_bounds_checking_build_exports_the_same_symbols():
+    """libmla_decode_check.so (MLA_BOUNDS_CHECK=1) declares nothing else and says which it is."""
+    names = _declared_functions()
+    check = _lib.load_library(_lib.CHECK_LIB_PATH)
+    for n in names:
+        assert hasattr(check, n), n
+    assert check.mla_bounds_checked() == 1
+    assert _lib.load_library(_lib.NORMAL_LIB_PATH).mla_bounds_checked() == 0
+    assert "mla_bounds_checked" in names
+
+
+def test_store_fault_mode_exists_in_the_checking_build_only():
+    """fault_test = 2 (stores past the buffers) is refused before any launch by the normal build;
+    the checking build accepts it on the FP8 CTA-pair kernel's balanced plans only."""
+    fp8 = mla.mla_decode_plan(2, 4, 32, 256, "fp8")
+    bf16 = mla.mla_decode_plan(2, 4, 32, 256, "bf16")
+    bad = _lib.MlaPlan.from_buffer_copy(fp8)
+    bad.fault_test = 2
+    assert _call(bad, lib=_lib.load_library(_lib.NORMAL_LIB_PATH)) == -6
+    check = _lib.load_library(_lib.CHECK_LIB_PATH)
+    bad16 = _lib.MlaPlan.from_buffer_copy(bf16)
+    bad16.fault_test = 2
+    assert _call(bad16, lib=check) == -6
+    # accepted: the call then fails only on the fake (host-side refused) workspace size
+    assert _call(bad, lib=check, ws_bytes=0) == -3
+
+
 def test_library_is_built_for_sm100a():
     # the build records ptxas reports per translation unit
     build = os.path.join(ROOT, "_build")
@@ -57,8 +84,8 @@ FAKE = 1 << 20  # 256-byte aligned, never dereferenced
 def _call(plan, **kw):
     args = dict(q=FAKE, kv=FAKE, num_pages=8, page_size=64, bt=FAKE, maxp=4, sl=FAKE,
                 scale=0.04, qs=1.0, ks=1.0, out=FAKE, lse=FAKE, ws=FAKE, ws_bytes=1 << 30)
+    L = kw.pop("lib", None) or _lib.lib()
     args.update(kw)
-    L = _lib.lib()
     vp = ctypes.c_void_p
     return L.mla_decode(ctypes.byref(plan) if plan is not None else None, vp(args["q"]),
                         vp(args["kv"]), args["num_pages"], args["page_size"], vp(args["bt"]),
