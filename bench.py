@@ -278,7 +278,9 @@ class NvmlClockPoller:
             return None
         reasons = sorted({name for _, _, rs in sel for name, bit in self.bits.items() if bit and rs & bit})
         return {"sm_mhz": statistics.median(s[1] for s in sel), "sm_max_mhz": self.max_mhz, "reasons": reasons,
-                "samples": len(sel), "source": "nvml, ~0.5 ms polling during the timed steps"}
+                "samples": len(sel), "source": "nvml, ~0.5 ms polling during the timed steps",
+                "caveat": "NVML's SM clock lags power capping over regions of a few ms; inside the kernels "
+                          "(clock64 against globaltimer) back-to-back calls run below it"}
 
 
 def roofline_fields(alg_bytes, flops, seconds, hbm_peak, hbm_kind, dtype, sustained):
