@@ -122,6 +122,15 @@ def test_kv_pack_host_errors_before_any_launch():
 
 # ---------------------------------------------------------------- GPU parity (bit-exact)
 
+def _assert_same_codes(got, ref):
+    """Byte for byte, except that a NaN may come out as either E4M3 NaN code: the sign of a NaN that a
+    division produces is unspecified (IEEE 754, section 6.3), and S.1111.111 is NaN for either S. The
+    GPU's division returns its canonical (positive) NaN, the host's keeps the operand's sign."""
+    diff = got != ref
+    nan_pair = ((got & 0x7F) == 0x7F) & ((ref & 0x7F) == 0x7F)
+    assert not (diff & ~nan_pair).any(), f"{int((diff & ~nan_pair).sum())} bytes differ"
+
+
 def _gpu_case(n, dtype, cache_dtype, num_pages, seed, skip_every=7, specials=True):
     dev = torch.device("cuda", 0)
     lat, rope = _rand_tokens(n, dtype, seed, std=2.0, specials=specials)
@@ -149,7 +158,7 @@ def test_kv_pack_fp8_matches_the_oracle_bit_for_bit(dtype):
     ref = oracle.kv_pack(lat, rope, slots.numpy(), (num_pages, 64, 576), in_dtype=dtype, cache_dtype="fp8",
                          kv_scale=scale, cache=init.numpy())
     got = cache.view(torch.uint8).reshape(-1).cpu().numpy()
-    assert np.array_equal(got, ref), f"{int((got != ref).sum())} bytes differ"
+    _assert_same_codes(got, ref)
 
 
 @pytest.mark.gpu
@@ -178,7 +187,7 @@ def test_kv_pack_bad_slot_sets_the_status_and_writes_the_rest():
     ok[5] = -1
     ref = oracle.kv_pack(lat, rope, ok.numpy(), (num_pages, 64, 576), in_dtype="bf16", cache_dtype="fp8",
                          kv_scale=0.005, cache=init.numpy())
-    assert np.array_equal(cache.view(torch.uint8).reshape(-1).cpu().numpy(), ref)
+    _assert_same_codes(cache.view(torch.uint8).reshape(-1).cpu().numpy(), ref)
 
 
 @pytest.mark.gpu
@@ -193,4 +202,34 @@ def test_kv_pack_full_size_prefill_matches_the_oracle():
     torch.cuda.synchronize()
     ref = oracle.kv_pack(lat, rope, slots.numpy(), (num_pages, 64, 576), in_dtype="bf16", cache_dtype="fp8",
                          kv_scale=scale, cache=init.numpy())
-    assert np.array_equal(cache.view(torch.uint8).reshape(-1).cpu().numpy(), ref)
+    _assert_same_codes(cache.view(torch.uint8).reshape(-1).cpu().numpy(), ref)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_kv_pack_table_path_encodes_every_bit_pattern(dtype):
+    """Calls of more than ~50K tokens encode through a per-CTA table of the non-negative input patterns. The
+    latent dims of tokens 1..128 hold every 16-bit pattern once (NaN, infinities, subnormals and -0
+    included), one token's slot is past the cache; bit-exact against the oracle (a NaN as either NaN
+    code), and the status word reports the bad slot."""
+    n, num_pages = 52000, 850
+    dev, lat, rope, slots, cache, init = _gpu_case(n, dtype, "fp8", num_pages, seed=15, skip_every=10 ** 9)
+    # tokens 1..128 (token 0's slot is the one _gpu_case always skips)
+    lat.view(torch.int16)[1:129].reshape(-1)[:] = torch.arange(-32768, 32768, dtype=torch.int32).to(torch.int16)
+    slots[200] = num_pages * 64 + 5
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    scale = 0.37
+    mla.kv_pack(lat.to(dev), rope.to(dev), slots.to(dev), cache, kv_scale=scale, device_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == mla.MLA_DEV_BAD_PAGE
+    ok = slots.clone()
+    ok[200] = -1
+    ref = oracle.kv_pack(lat, rope, ok.numpy(), (num_pages, 64, 576), in_dtype=dtype, cache_dtype="fp8",
+                         kv_scale=scale, cache=init.numpy())
+    got = cache.view(torch.uint8).reshape(-1).cpu().numpy()
+    _assert_same_codes(got, ref)
+    # every NaN input did become a NaN code
+    nan_in = np.isnan(lat[1:129].float().numpy()).reshape(-1)
+    rows = slots[1:129].numpy()
+    codes = got.reshape(-1, 576)[rows][:, :512].reshape(-1)
+    assert ((codes[nan_in] & 0x7F) == 0x7F).all()
