@@ -215,7 +215,8 @@ def lse_merge(o_parts, lse_parts):
 
 
 def encode_e4m3(values) -> np.ndarray:
-    """OCP E4M3FN codes of fp32 values: round to nearest even, saturating to +-448, NaN -> 0x7f."""
+    """OCP E4M3FN codes of fp32 values: round to nearest even, saturating to +-448, NaN -> S.1111.111
+    (0x7f, or 0xff when the NaN's sign bit is set)."""
     v = np.ascontiguousarray(np.asarray(values, dtype=np.float32).reshape(-1))
     out = np.empty(v.size, dtype=np.uint8)
     _load().oracle_encode_e4m3_buffer(v.ctypes.data, v.size, out.ctypes.data)

@@ -79,6 +79,27 @@ def _rand_tokens(n, dtype, seed, std=1.0, specials=False):
     return lat, rope
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_e4m3_of_a_quotient_is_sign_symmetric(dtype):
+    """The FP8 pack's table path encodes only the non-negative 16-bit patterns and sets the sign bit
+    for the negative ones. That holds because x / s is -(|x| / s) exactly for s > 0 and the E4M3
+    rounding is symmetric: checked here over every non-NaN 16-bit pattern, with the quotient in
+    fp32 as the kernels form it, for scales that put values in the subnormal, normal and saturating
+    ranges."""
+    pos = np.arange(0x8000, dtype=np.uint16)
+    x_pos = oracle.decode_values(dtype, pos).astype(np.float32)
+    x_neg = oracle.decode_values(dtype, pos | np.uint16(0x8000)).astype(np.float32)
+    keep = ~np.isnan(x_pos)
+    for s in (0.37, 1.0, 3.0e-3, 2.5e2, 1.0e-6):
+        with np.errstate(over="ignore"):  # large values over a small scale overflow to +-inf (saturated)
+            q_pos = x_pos / np.float32(s)
+            q_neg = x_neg / np.float32(s)
+        assert np.array_equal(q_neg[keep], -q_pos[keep])
+        c_pos = oracle.encode_e4m3(q_pos[keep])
+        c_neg = oracle.encode_e4m3(q_neg[keep])
+        assert np.array_equal(c_neg, c_pos | np.uint8(0x80))
+
+
 def test_oracle_kv_pack_row_layout_and_skipped_slots():
     lat, rope = _rand_tokens(3, "bf16", 3)
     slots = np.array([5, -1, 0], dtype=np.int64)
